@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-2 mixer core on B200: prefill tokens/s and decode steps/s
+with % of roofline, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one prefill call of the whole mixer core (conv1d+SiLU, dt softplus,
+chunked SSD scan, D skip, gated RMSNorm, final conv/SSM states) over the
+Zamba2-2.7B-shaped workload (batch 1, 4096 tokens, 80 heads x 64, d_state 64,
+chunk 256, bf16 I/O, fp32 state), on synthetic seeded inputs already resident in
+HBM.  Four input/output/workspace sets rotate so that no step finds its data in
+the 126 MB L2.  The decode workload (batch 256, 1024 consecutive single-token
+steps) is reported in the `decode` object of the same line.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
+sequence (seed = rank); there is no data-path collective (weak scaling).  The
+step time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the same workload (a bounded
+token sample per step) on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "zamba2_2p7b_prefill"
+DECODE = "zamba2_2p7b_decode"
+METRIC = "SSD mixer prefill tokens/s and decode steps/s at 1 B200; % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ROTATE = 4
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="decode steps to time (default: the workload's 1024)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- accounting
+
+def prefill_bytes(cfg) -> int:
+    """Algorithmic bytes of one prefill: every input read once, y written once,
+    final states written once (conv state also read when carried)."""
+    e = 2 if cfg.io_dtype == "bf16" else 4
+    per_token = e * (cfg.conv_dim + cfg.d_inner + cfg.nheads + cfg.d_inner)
+    states = 4 * cfg.nheads * cfg.headdim * cfg.dstate + e * cfg.conv_dim * cfg.d_conv
+    return cfg.batch * (cfg.seqlen * per_token + states)
+
+
+def prefill_flops(cfg) -> int:
+    """Algorithmic flops: causal intra-chunk (C B^T over the triangle, times X),
+    chunk states, carried-state outputs; multiply-adds count 2."""
+    Q, H, P, N, G = cfg.chunk_size, cfg.nheads, cfg.headdim, cfg.dstate, cfg.ngroups
+    tok = cfg.batch * cfg.seqlen
+    cb = G * Q * N          # C B^T, half of Q x Q x N per token pair, x2 flops
+    intra = H * Q * P       # (L o CB) X over the causal triangle
+    states = 2 * H * P * N  # chunk state
+    off = 2 * H * P * N     # C H^T
+    return tok * (cb + intra + states + off)
+
+
+def decode_bytes(cfg) -> int:
+    e = 2 if cfg.io_dtype == "bf16" else 4
+    b = cfg.batch
+    state = 2 * 4 * cfg.nheads * cfg.headdim * cfg.dstate   # read + write
+    conv = 2 * e * cfg.conv_dim * cfg.d_conv               # read + write
+    inputs = e * (cfg.conv_dim + cfg.d_inner + cfg.nheads)
+    out = e * cfg.d_inner
+    return b * (state + conv + inputs + out)
+
+
+def stage_bytes(name, cfg) -> int | None:
+    """Algorithmic bytes of one launch of a kernel stage: the compulsory reads of
+    its inputs and writes of its outputs in their stored types."""
+    e = 2 if cfg.io_dtype == "bf16" else 4
+    bL = cfg.batch * cfg.seqlen
+    nch = -(-cfg.seqlen // cfg.chunk_size)
+    st = cfg.batch * nch * cfg.nheads * cfg.headdim * cfg.dstate * 4
+    di, cd, H, GN = cfg.d_inner, cfg.conv_dim, cfg.nheads, cfg.ngroups * cfg.dstate
+    table = {
+        "conv_silu": bL * cd * (e + 4),
+        "conv_state_out": cfg.batch * cd * cfg.d_conv * e,
+        "dt_cumsum": bL * H * (e + 8),
+        "chunk_state": bL * (di + GN) * 4 + bL * H * 8 + st,
+        "state_pass": 2 * st + bL * H * 4 // cfg.chunk_size,
+        "chunk_out": bL * cd * 4 + bL * H * 8 + st + bL * di * 4,
+        "gated_norm": bL * di * (4 + e + e),
+        "ssd_step": decode_bytes(cfg),
+    }
+    return table.get(name)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d.get(k, FALLBACK_PEAKS[k])) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "mamba_ssd_scan_mixer_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, or None if there is
+    none for this kernel and workload or the kernel sources changed since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = f"/tmp/m2bench_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        busy = [s for s, p in zip(sm, pw) if p is not None and p > 200] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import mamba_ssd_scan_mixer_b200 as m2
+    from mamba_ssd_scan_mixer_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[PREFILL]
+    seed = rank
+    lib = m2.lib()
+    dims = m2.dims_from_config(cfg)
+    params = {k: v.to(dev) for k, v in W.make_params(cfg, seed).items()}
+    pp = m2.make_params(params["conv_w"], params["conv_b"], params["dt_bias"], params["A"],
+                        params["D"], params["norm_w"])
+    host_in = W.make_prefill_inputs(cfg, seed)["zxbcdt"]
+    di, cd = cfg.d_inner, cfg.conv_dim
+    ws_bytes = m2.mamba2_prefill_workspace_size(dims)
+    sets = []
+    for r in range(ROTATE):
+        packed = host_in.to(dev)
+        sets.append(dict(
+            packed=packed, z=packed[..., :di], xBC=packed[..., di:di + cd],
+            dt=packed[..., di + cd:],
+            y=torch.empty(cfg.batch, cfg.seqlen, di, dtype=cfg.torch_dtype, device=dev),
+            cs=torch.zeros(cfg.batch, cd, cfg.d_conv, dtype=cfg.torch_dtype, device=dev),
+            hs=torch.zeros(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, device=dev),
+            ws=torch.empty(ws_bytes, dtype=torch.uint8, device=dev)))
+    rot_bytes = sum(sum(t.numel() * t.element_size() for k, t in s.items()
+                        if k in ("packed", "y", "cs", "hs", "ws")) for s in sets)
+
+    names_arr = (ctypes.c_char_p * 16)()
+    nst = lib.mamba2_stage_names(0, ctypes.byref(dims), names_arr, 16)
+    stage_names = [names_arr[i].decode() for i in range(nst)]
+    stream = torch.cuda.current_stream(dev)
+
+    def call(s, events=None):
+        if events is not None:
+            arr = (ctypes.c_void_p * len(events))(*events)
+            lib.mamba2_record_stage_events(arr, len(events))
+        m2.mamba2_conv_ssd_prefill(dims, pp, s["xBC"], s["z"], s["dt"], s["y"], s["cs"],
+                                   s["hs"], False, s["ws"], stream)
+
+    def new_event():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
+
+    # warm-up, with every stage bracketed once to find the dominant kernel
+    W_ = max(3, args.warmup)
+    stage_ms = [0.0] * nst
+    for i in range(W_):
+        evs = [new_event() for _ in range(nst + 1)]
+        call(sets[i % ROTATE], [e.cuda_event for e in evs])
+        torch.cuda.synchronize(dev)
+        for j in range(nst):
+            stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
+    dom = max(range(nst), key=lambda j: stage_ms[j])
+
+    # timed region: exactly K steps; the dominant stage bracketed by its own events
+    K = args.steps
+    dom_evs = [(new_event(), new_event()) for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(K):
+        a, b = dom_evs[k]
+        evs = [None] * dom + [a.cuda_event, b.cuda_event]
+        call(sets[k % ROTATE], evs)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed = t0.elapsed_time(t1)
+    dom_ms = sum(a.elapsed_time(b) for a, b in dom_evs) / K
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+
+    peaks, peak_src = load_peaks()
+    ms = elapsed / K
+    tokens = cfg.batch * cfg.seqlen
+    value = world * tokens * K / (elapsed / 1e3)
+    path_bytes = prefill_bytes(cfg)
+    path_flops = prefill_flops(cfg)
+    t_roof = max(path_bytes / (peaks["hbm_gbs"] * 1e9), path_flops / (peaks["bf16_tflops"] * 1e12))
+    dom_name = stage_names[dom]
+    dbytes = stage_bytes(dom_name, cfg)
+    achieved = dbytes / (dom_ms * 1e-3) / 1e9 if dbytes else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": W_, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": PREFILL, "batch": cfg.batch, "seqlen": cfg.seqlen,
+                   "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
+                   "ngroups": cfg.ngroups, "chunk": cfg.chunk_size, "state_dtype": "f32",
+                   "parallelism": f"dp{world} (independent sequences)",
+                   "l2": f"{ROTATE} rotating input/output/workspace sets, "
+                         f"{rot_bytes / 1e9:.2f} GB > 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"] if achieved else None,
+                     "traffic": traffic_for(dom_name, PREFILL),
+                     "algorithmic_bytes": dbytes, "avg_launch_ms": dom_ms,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6650 GB/s"},
+        "path_roofline": {"bytes": path_bytes, "flops": path_flops,
+                          "roofline_ms": t_roof * 1e3,
+                          "achieved_gbs": path_bytes / (ms * 1e-3) / 1e9,
+                          "frac": t_roof * 1e3 / ms, "peak_source": peak_src},
+        "stages_ms_warmup_avg": {n: stage_ms[j] / W_ for j, n in enumerate(stage_names)},
+        "gpu_launches": K * nst,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_e2e:
+        line["e2e"] = run_e2e(args, cfg, dims, pp, host_in, dev, stream, m2)
+    if not args.no_decode:
+        line["decode"] = run_decode(args, dev, stream, rank, world, peaks, peak_src, m2, W)
+        line["gpu_launches"] += line["decode"]["gpu_launches"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, seconds=10.0)
+    return line
+
+
+def run_e2e(args, cfg, dims, pp, host_in, dev, stream, m2):
+    """Tokens/s through the public entry point with host buffers: each step copies
+    the packed input from pinned host memory, runs the prefill, and reads y and
+    the final states back."""
+    import torch
+    di, cd = cfg.d_inner, cfg.conv_dim
+    h_in = host_in.pin_memory()
+    d_in = torch.empty_like(h_in, device=dev)
+    h_y = torch.empty(cfg.batch, cfg.seqlen, di, dtype=cfg.torch_dtype).pin_memory()
+    h_cs = torch.empty(cfg.batch, cd, cfg.d_conv, dtype=cfg.torch_dtype).pin_memory()
+    h_hs = torch.empty(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate).pin_memory()
+    d_y = torch.empty(h_y.shape, dtype=h_y.dtype, device=dev)
+    d_cs = torch.empty(h_cs.shape, dtype=h_cs.dtype, device=dev)
+    d_hs = torch.empty(h_hs.shape, dtype=h_hs.dtype, device=dev)
+    ws = torch.empty(m2.mamba2_prefill_workspace_size(dims), dtype=torch.uint8, device=dev)
+
+    def step():
+        d_in.copy_(h_in, non_blocking=True)
+        m2.mamba2_conv_ssd_prefill(dims, pp, d_in[..., di:di + cd], d_in[..., :di],
+                                   d_in[..., di + cd:], d_y, d_cs, d_hs, False, ws, stream)
+        h_y.copy_(d_y, non_blocking=True)
+        h_cs.copy_(d_cs, non_blocking=True)
+        h_hs.copy_(d_hs, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    K = max(3, min(args.steps, 50))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / K
+    nbytes = lambda t: t.numel() * t.element_size()
+    return {"value": cfg.batch * cfg.seqlen / (ms * 1e-3), "unit": "tokens/s", "steps": K,
+            "ms_per_step": ms, "h2d_bytes_per_step": nbytes(h_in),
+            "d2h_bytes_per_step": nbytes(h_y) + nbytes(h_cs) + nbytes(h_hs)}
+
+
+def run_decode(args, dev, stream, rank, world, peaks, peak_src, m2, W):
+    """The batch-256 decode workload: consecutive single-token steps with distinct
+    per-step inputs (pre-generated on the device), states updated in place."""
+    import torch
+    import torch.distributed as dist
+    cfg = W.CONFIGS[DECODE]
+    S = args.decode_steps or cfg.decode_steps
+    dims = m2.dims_from_config(cfg)
+    params = {k: v.to(dev) for k, v in W.make_params(cfg, rank).items()}
+    pp = m2.make_params(params["conv_w"], params["conv_b"], params["dt_bias"], params["A"],
+                        params["D"], params["norm_w"])
+    st = W.make_states(cfg, rank)
+    cs = st["conv_state"].to(dev)
+    hs = st["ssm_state"].to(dev)
+    g = torch.Generator(device=dev).manual_seed(1000 + rank)
+    inputs = torch.randn(S, cfg.batch, cfg.d_in_proj, generator=g, device=dev).to(
+        cfg.torch_dtype)
+    y = torch.empty(cfg.batch, cfg.d_inner, dtype=cfg.torch_dtype, device=dev)
+    di, cd = cfg.d_inner, cfg.conv_dim
+
+    def step(k):
+        p = inputs[k]
+        m2.mamba2_ssd_step(dims, pp, p[:, di:di + cd], p[:, :di], p[:, di + cd:], y, cs, hs,
+                           stream)
+
+    for k in range(max(3, args.warmup)):
+        step(k % S)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for k in range(S):
+        step(k)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed = a.elapsed_time(b)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    ms = elapsed / S
+    nb = decode_bytes(cfg)
+    ach = nb / (ms * 1e-3) / 1e9
+    return {"value": world * S / (elapsed / 1e3), "unit": "steps/s", "steps": S,
+            "ms_per_step": ms, "tokens_per_s": world * cfg.batch * S / (elapsed / 1e3),
+            "config": {"workload": DECODE, "batch": cfg.batch, "nheads": cfg.nheads,
+                       "headdim": cfg.headdim, "dstate": cfg.dstate,
+                       "l2": "state 335 MB > 126 MB L2; distinct per-step inputs"},
+            "roofline": {"bound": "hbm", "kernel": "ssd_step", "achieved": ach,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "traffic": traffic_for("ssd_step", DECODE),
+                         "algorithmic_bytes": nb, "peak_source": peak_src},
+            "gpu_launches": S, "clocks": clocks}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def _oracle_tokens(cfg, params, inp, ntok, nthreads):
+    import oracle
+    t = time.perf_counter()
+    oracle.mixer_prefill(inp["xBC"][:, :ntok], inp["z"][:, :ntok], inp["dt_raw"][:, :ntok],
+                         params, nheads=cfg.nheads, headdim=cfg.headdim, dstate=cfg.dstate,
+                         ngroups=cfg.ngroups, eps=cfg.norm_eps,
+                         norm_before_gate=cfg.norm_before_gate, nthreads=nthreads)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(cfg, seconds=10.0):
+    """The fp64 oracle, as it stands, on the prefill workload: whole 4096-token
+    passes repeated until `seconds` of CPU time have run (at least one)."""
+    import oracle
+    from mamba_ssd_scan_mixer_b200 import workloads as W
+    params = W.make_params(cfg, 0)
+    inp = W.make_prefill_inputs(cfg, 0)
+    cores = oracle.default_threads()
+    total_t, runs = 0.0, 0
+    while runs == 0 or (total_t < seconds and runs < 20):
+        total_t += _oracle_tokens(cfg, params, inp, cfg.seqlen, cores)
+        runs += 1
+    return {"value": runs * cfg.batch * cfg.seqlen / total_t, "unit": "tokens/s",
+            "cores": cores, "kind": "oracle",
+            "sample": f"{runs} full pass(es) of the {PREFILL} workload "
+                      f"({cfg.batch}x{cfg.seqlen} tokens, all {cfg.nheads} heads), "
+                      f"{total_t:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle on the same workload and metric, each
+    step a bounded prefix of the 4096-token sequence (all heads)."""
+    from mamba_ssd_scan_mixer_b200 import workloads as W
+    import oracle
+    cfg = W.CONFIGS[PREFILL]
+    params = W.make_params(cfg, 0)
+    inp = W.make_prefill_inputs(cfg, 0)
+    cores = oracle.default_threads()
+    # size each step so that warm-up + steps take about 90 s in total
+    calib = 256
+    t_tok = _oracle_tokens(cfg, params, inp, calib, cores) / calib
+    K, Wm = args.steps, max(3, args.warmup)
+    ntok = int(max(16, min(cfg.seqlen, 90.0 / max(1, K + Wm) / max(t_tok, 1e-9))))
+    for _ in range(Wm):
+        _oracle_tokens(cfg, params, inp, ntok, cores)
+    total = sum(_oracle_tokens(cfg, params, inp, ntok, cores) for _ in range(K))
+    value = K * cfg.batch * ntok / total
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": K, "warmup": Wm, "ms_per_step": total / K * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": PREFILL, "batch": cfg.batch, "seqlen": cfg.seqlen,
+                       "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
+                       "ngroups": cfg.ngroups, "chunk": cfg.chunk_size},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"first {ntok} of {cfg.seqlen} tokens per step, "
+                                       f"all {cfg.nheads} heads"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,187 @@
+/*
+ * mamba2ssd.h -- C ABI of the B200 (sm_100a) Mamba-2 mixer core library
+ * (libmamba2ssd.so).
+ *
+ * The mixer core is the middle of a Zamba2 Mamba2 layer, between in_proj and
+ * out_proj ("Zamba2 hybrid architecture in Transformers", qwbw.cn, section 三
+ * "Mamba2 Mixer", steps 2-4):
+ *   1. causal depthwise conv1d (width d_conv = 4, with bias) + SiLU over the
+ *      x | B | C channels (conv_dim = d_inner + 2 * ngroups * d_state);
+ *   2. dt = softplus(dt_raw + dt_bias) per head;
+ *   3. the selective state-space scan of the Mamba-2 (state-space duality)
+ *      layer named on the state-spaces/mamba repository page (opendeer.net,
+ *      "About the project"):
+ *          h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t B_t^T     (h: [P, N])
+ *          y_t = C_t h_t + D_h * x_t
+ *      evaluated chunk by chunk for prefill and as a single-token update for
+ *      decode (section 三 step 3);
+ *   4. gated group RMSNorm: out = rmsnorm(y * silu(z)) * norm_w over groups
+ *      of d_inner / ngroups channels, eps from the dims (section 三 step 4,
+ *      section 五 rms_norm_eps = 1e-5); norm_before_gate = 1 selects
+ *      rmsnorm(y) * norm_w * silu(z).
+ * The conv state and SSM state that the pages keep in the model cache
+ * (section 三) are caller-owned buffers passed to every call.
+ *
+ * Conventions shared by every entry point
+ *  - All data pointers are DEVICE pointers of the current CUDA device, except
+ *    `dims` and `params` themselves (host structs; the arrays they point to
+ *    are device arrays).  The library never allocates device memory, never
+ *    synchronises the stream and keeps no pointer after a call returns.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *    the legacy default stream) and runs asynchronously: a return of
+ *    MAMBA2_OK means the arguments were valid and the launches were enqueued.
+ *  - Layouts are row-major.  Channel c of xBC is x for c < d_inner (head h,
+ *    lane p at h*P + p), then B (ngroups * d_state, group-major), then C.
+ *    Head h uses B/C group h / (nheads / ngroups).
+ *  - Outputs must not alias inputs; the conv and SSM state buffers are read
+ *    and then overwritten in place.
+ *  - Errors are returned, never thrown; on any status other than MAMBA2_OK
+ *    from argument validation nothing was enqueued.  MAMBA2_ERR_CUDA reports
+ *    a launch error (cudaGetLastError) after enqueueing.
+ */
+#ifndef MAMBA2SSD_H
+#define MAMBA2SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(_WIN32)
+#define MAMBA2_API __declspec(dllexport)
+#else
+#define MAMBA2_API __attribute__((visibility("default")))
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MAMBA2_OK = 0,
+  MAMBA2_ERR_INVALID_ARG = -1, /* null pointer, bad size, stride or alignment */
+  MAMBA2_ERR_UNSUPPORTED = -2, /* valid in principle, not built (e.g. d_conv != 4) */
+  MAMBA2_ERR_WORKSPACE = -3,   /* workspace missing or smaller than required */
+  MAMBA2_ERR_CUDA = -4         /* a CUDA launch or runtime call failed */
+} mamba2_status;
+
+typedef enum {
+  MAMBA2_F32 = 0, /* fp32 inputs, outputs and conv state */
+  MAMBA2_BF16 = 1 /* bf16 inputs, outputs and conv state */
+} mamba2_dtype;
+
+/* Problem sizes.  The SSM state is always fp32; `io_dtype` is the type of
+ * xBC, z, dt_raw, y and the conv state. */
+typedef struct {
+  int64_t batch;            /* b >= 0 */
+  int64_t seqlen;           /* L >= 0 (prefill); ignored by mamba2_ssd_step */
+  int32_t nheads;           /* H >= 1, multiple of ngroups */
+  int32_t headdim;          /* P: 16, 32 or 64 */
+  int32_t dstate;           /* N: 16, 32, 64 or 128 */
+  int32_t ngroups;          /* G >= 1: B/C groups, and the number of norm groups */
+  int32_t d_conv;           /* conv width; must be 4 */
+  int32_t chunk_size;       /* Q: 64, 128 or 256 (prefill only) */
+  int32_t io_dtype;         /* mamba2_dtype */
+  int32_t norm_before_gate; /* 0: rmsnorm(y * silu(z)) * w;  1: rmsnorm(y) * w * silu(z) */
+  float norm_eps;           /* > 0, e.g. 1e-5 */
+} mamba2_dims;
+
+/* fp32 parameters (device arrays, read only). */
+typedef struct {
+  const float *conv_w;  /* [conv_dim, d_conv]: tap k multiplies the input d_conv-1-k steps back */
+  const float *conv_b;  /* [conv_dim] */
+  const float *dt_bias; /* [nheads] */
+  const float *A;       /* [nheads], A_h < 0 (callers holding A_log pass -exp(A_log)) */
+  const float *D;       /* [nheads] */
+  const float *norm_w;  /* [d_inner] */
+} mamba2_params;
+
+/* Human-readable name of a status code (static string). */
+MAMBA2_API const char *mamba2_status_string(int status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+MAMBA2_API int mamba2_version(void);
+
+/* Bytes of device workspace that mamba2_conv_ssd_prefill needs for `dims`
+ * (0 if dims are invalid).  The caller allocates it (256-byte aligned) and
+ * may reuse it across calls that do not overlap on the GPU. */
+MAMBA2_API size_t mamba2_prefill_workspace_size(const mamba2_dims *dims);
+
+/* Prefill: run the whole mixer core over `seqlen` new tokens of each of the
+ * `batch` sequences (qwbw.cn section 三 steps 2-4, chunked scan of step 3).
+ *
+ *  xBC     [b, L, conv_dim] io_dtype; token t of row bi starts at
+ *          xBC + (bi * L + t) * xBC_row_stride elements, so it may point into
+ *          a packed in_proj output.  Row stride >= conv_dim, multiple of 8;
+ *          pointer 16-byte aligned.
+ *  z       [b, L, d_inner] io_dtype, row stride >= d_inner, multiple of 8;
+ *          16-byte aligned.  The gate.
+ *  dt_raw  [b, L, nheads] io_dtype, row stride >= nheads (any alignment of
+ *          the element type).
+ *  y       [b, L, d_inner] io_dtype, contiguous, 16-byte aligned.  Output.
+ *  conv_state  [b, conv_dim, d_conv] io_dtype, contiguous, or NULL.  When
+ *          states_in != 0 it holds the d_conv raw xBC inputs before the first
+ *          new token (oldest first) and supplies the conv's left context;
+ *          otherwise that context is zero.  On return (if not NULL) it holds
+ *          the last d_conv raw inputs of [old state | new tokens].
+ *  ssm_state   [b, nheads, headdim, dstate] fp32, contiguous, or NULL.  When
+ *          states_in != 0 it is the state h entering the first new token,
+ *          otherwise the scan starts from zero.  On return (if not NULL) it
+ *          holds the state after the last new token.
+ *  states_in   0 or 1, as above.  States must be non-NULL when it is 1.
+ *  workspace   device scratch of at least mamba2_prefill_workspace_size(dims)
+ *          bytes, 256-byte aligned; contents on entry are ignored.
+ *  stream  cudaStream_t as void*.
+ * seqlen need not be a multiple of chunk_size.  seqlen == 0 copies or zeroes
+ * the states and writes nothing else. */
+MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_params *params,
+                                       const void *xBC, int64_t xBC_row_stride, const void *z,
+                                       int64_t z_row_stride, const void *dt_raw,
+                                       int64_t dt_row_stride, void *y, void *conv_state,
+                                       float *ssm_state, int32_t states_in, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/* Decode: advance every sequence by one token (qwbw.cn section 三 step 3,
+ * the single-token recurrent update used when the cache holds the states and
+ * the new sequence length is 1).  The conv state is shifted left by one and
+ * the new xBC column appended; the conv output is its dot product with the
+ * taps; the SSM state takes one recurrence step; then D-skip and the gated
+ * norm as in prefill.  dims->seqlen and dims->chunk_size are ignored.
+ *
+ *  xBC     [b, conv_dim] io_dtype, row (batch) stride >= conv_dim, multiple
+ *          of 8, 16-byte aligned.
+ *  z       [b, d_inner] io_dtype, row stride >= d_inner, multiple of 8,
+ *          16-byte aligned.
+ *  dt_raw  [b, nheads] io_dtype, row stride >= nheads.
+ *  y       [b, d_inner] io_dtype, contiguous, 16-byte aligned.  Output.
+ *  conv_state  [b, conv_dim, d_conv] io_dtype, contiguous, updated in place.
+ *  ssm_state   [b, nheads, headdim, dstate] fp32, contiguous, 16-byte
+ *          aligned, updated in place.
+ * Uses no workspace. */
+MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *params,
+                               const void *xBC, int64_t xBC_row_stride, const void *z,
+                               int64_t z_row_stride, const void *dt_raw, int64_t dt_row_stride,
+                               void *y, void *conv_state, float *ssm_state, void *stream);
+
+/* Profiling aid (no counterpart on the pages).  Arms the calling host thread
+ * so that its NEXT call of mamba2_conv_ssd_prefill or mamba2_ssd_step records
+ * events[i] (cudaEvent_t passed as void*, created by the caller) on the
+ * call's stream just before the call's kernel stage i, and events[S] after
+ * its last stage, S being the stage count that mamba2_stage_names reports.
+ * Entries beyond n_events, and NULL entries, are not recorded, so a caller
+ * can bracket a single stage.  The call disarms the thread when it returns,
+ * whatever its status.  0 <= n_events <= 16.  Returns MAMBA2_OK or
+ * MAMBA2_ERR_INVALID_ARG (bad count, or events NULL with n_events > 0). */
+MAMBA2_API int mamba2_record_stage_events(void *const *events, int n_events);
+
+/* Number of kernel stages a call of `kind` (0 = prefill, 1 = decode step)
+ * enqueues for `dims`, or MAMBA2_ERR_INVALID_ARG; writes up to max_names
+ * static stage names to `names` (may be NULL).  A stage is one kernel launch
+ * (a stage whose work is absent for a call, e.g. the conv-state write without
+ * a conv state buffer, launches nothing but keeps its place). */
+MAMBA2_API int mamba2_stage_names(int kind, const mamba2_dims *dims, const char **names,
+                                  int max_names);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA2SSD_H */

@@ -1,0 +1,204 @@
+// C ABI of libmamba2ssd.so: argument validation and launch.  See
+// include/mamba2ssd.h for the contract of every entry point.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace m2 {
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// Validates the sizes shared by prefill and decode and fills `pr`.
+int make_problem(const mamba2_dims *d, bool prefill, Problem *pr) {
+  if (d == nullptr) return MAMBA2_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->nheads < 1 || d->ngroups < 1 || d->headdim < 1 || d->dstate < 1 ||
+      d->d_conv < 1)
+    return MAMBA2_ERR_INVALID_ARG;
+  if (prefill && d->seqlen < 0) return MAMBA2_ERR_INVALID_ARG;
+  if (d->nheads % d->ngroups != 0) return MAMBA2_ERR_INVALID_ARG;
+  if (d->io_dtype != MAMBA2_F32 && d->io_dtype != MAMBA2_BF16) return MAMBA2_ERR_INVALID_ARG;
+  if (d->norm_before_gate != 0 && d->norm_before_gate != 1) return MAMBA2_ERR_INVALID_ARG;
+  if (!(d->norm_eps > 0.0f) || !std::isfinite(d->norm_eps)) return MAMBA2_ERR_INVALID_ARG;
+  if (d->d_conv != 4) return MAMBA2_ERR_UNSUPPORTED;
+  if (!pow2_in(d->headdim, 16, 64) || !pow2_in(d->dstate, 16, 128))
+    return MAMBA2_ERR_UNSUPPORTED;
+  if (prefill && d->chunk_size != 64 && d->chunk_size != 128 && d->chunk_size != 256)
+    return MAMBA2_ERR_UNSUPPORTED;
+  if (d->batch > 65535 || d->nheads > 65535) return MAMBA2_ERR_UNSUPPORTED;  // grid y/z limits
+  pr->batch = d->batch;
+  pr->L = prefill ? d->seqlen : 1;
+  pr->H = d->nheads;
+  pr->P = d->headdim;
+  pr->N = d->dstate;
+  pr->G = d->ngroups;
+  pr->K = d->d_conv;
+  pr->Q = prefill ? d->chunk_size : 1;
+  pr->io = d->io_dtype;
+  pr->nbg = d->norm_before_gate;
+  pr->eps = d->norm_eps;
+  pr->d_inner = (int64_t)pr->H * pr->P;
+  pr->conv_dim = pr->d_inner + 2LL * pr->G * pr->N;
+  pr->nchunks = prefill ? ceil_div(pr->L, pr->Q) : 1;
+  if (prefill && pr->L > (int64_t)1 << 31) return MAMBA2_ERR_UNSUPPORTED;  // grid x limit
+  return MAMBA2_OK;
+}
+
+bool params_ok(const mamba2_params *p) {
+  return p != nullptr && p->conv_w && p->conv_b && p->dt_bias && p->A && p->D && p->norm_w;
+}
+
+// Disarms the stage events when a call returns, whatever the path taken.
+struct DisarmOnExit {
+  ~DisarmOnExit() { g_stage_events.n = 0; }
+};
+
+}  // namespace
+
+thread_local StageEvents g_stage_events = {{}, 0};
+
+}  // namespace m2
+
+using namespace m2;
+
+extern "C" {
+
+MAMBA2_API const char *mamba2_status_string(int status) {
+  switch (status) {
+    case MAMBA2_OK: return "ok";
+    case MAMBA2_ERR_INVALID_ARG: return "invalid argument";
+    case MAMBA2_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MAMBA2_ERR_WORKSPACE: return "workspace missing or too small";
+    case MAMBA2_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+MAMBA2_API int mamba2_version(void) { return 100; }
+
+MAMBA2_API int mamba2_record_stage_events(void *const *events, int n_events) {
+  if (n_events < 0 || n_events > kMaxStageEvents || (n_events > 0 && events == nullptr))
+    return MAMBA2_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i) g_stage_events.ev[i] = static_cast<cudaEvent_t>(events[i]);
+  g_stage_events.n = n_events;
+  return MAMBA2_OK;
+}
+
+MAMBA2_API int mamba2_stage_names(int kind, const mamba2_dims *dims, const char **names,
+                                  int max_names) {
+  Problem pr;
+  if (make_problem(dims, kind == 0, &pr) != MAMBA2_OK) return MAMBA2_ERR_INVALID_ARG;
+  const char *const *list = kind == 0 ? kPrefillSimtStages : kStepSimtStages;
+  const int n = kind == 0 ? kPrefillSimtStageCount : kStepSimtStageCount;
+  if (kind != 0 && kind != 1) return MAMBA2_ERR_INVALID_ARG;
+  for (int i = 0; names != nullptr && i < n && i < max_names; ++i) names[i] = list[i];
+  return n;
+}
+
+MAMBA2_API size_t mamba2_prefill_workspace_size(const mamba2_dims *dims) {
+  Problem pr;
+  if (make_problem(dims, true, &pr) != MAMBA2_OK) return 0;
+  return prefill_simt_workspace(pr);
+}
+
+MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_params *params,
+                                       const void *xBC, int64_t xBC_row_stride, const void *z,
+                                       int64_t z_row_stride, const void *dt_raw,
+                                       int64_t dt_row_stride, void *y, void *conv_state,
+                                       float *ssm_state, int32_t states_in, void *workspace,
+                                       size_t workspace_bytes, void *stream) {
+  DisarmOnExit disarm;
+  Problem pr;
+  int st = make_problem(dims, true, &pr);
+  if (st != MAMBA2_OK) return st;
+  if (!params_ok(params)) return MAMBA2_ERR_INVALID_ARG;
+  if (states_in != 0 && states_in != 1) return MAMBA2_ERR_INVALID_ARG;
+  if (states_in && (conv_state == nullptr || ssm_state == nullptr)) return MAMBA2_ERR_INVALID_ARG;
+  if (ssm_state != nullptr && !aligned(ssm_state, 16)) return MAMBA2_ERR_INVALID_ARG;
+  const size_t esz = pr.io == MAMBA2_BF16 ? 2 : 4;
+  if (conv_state != nullptr && !aligned(conv_state, esz)) return MAMBA2_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pr.batch == 0) return MAMBA2_OK;
+  if (pr.L > 0) {
+    if (xBC == nullptr || z == nullptr || dt_raw == nullptr || y == nullptr)
+      return MAMBA2_ERR_INVALID_ARG;
+    if (xBC_row_stride < pr.conv_dim || z_row_stride < pr.d_inner || dt_row_stride < pr.H)
+      return MAMBA2_ERR_INVALID_ARG;
+    if (xBC_row_stride % 8 != 0 || z_row_stride % 8 != 0) return MAMBA2_ERR_INVALID_ARG;
+    if (!aligned(xBC, 16) || !aligned(z, 16) || !aligned(y, 16) || !aligned(dt_raw, esz))
+      return MAMBA2_ERR_INVALID_ARG;
+    const size_t need = prefill_simt_workspace(pr);
+    if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
+      return MAMBA2_ERR_WORKSPACE;
+  } else {
+    // no new tokens: the states pass through, or start (and stay) at zero
+    if (!states_in) {
+      if (conv_state != nullptr &&
+          cudaMemsetAsync(conv_state, 0, (size_t)pr.batch * pr.conv_dim * pr.K * esz, s) !=
+              cudaSuccess)
+        return MAMBA2_ERR_CUDA;
+      if (ssm_state != nullptr &&
+          cudaMemsetAsync(ssm_state, 0, (size_t)pr.batch * pr.H * pr.P * pr.N * 4, s) !=
+              cudaSuccess)
+        return MAMBA2_ERR_CUDA;
+    }
+    return MAMBA2_OK;
+  }
+  PrefillArgs a;
+  a.pr = pr;
+  a.prm = *params;
+  a.xBC = xBC;
+  a.ld_xbc = xBC_row_stride;
+  a.z = z;
+  a.ld_z = z_row_stride;
+  a.dt_raw = dt_raw;
+  a.ld_dt = dt_row_stride;
+  a.y = y;
+  a.conv_state = conv_state;
+  a.ssm_state = ssm_state;
+  a.states_in = states_in;
+  a.ws = static_cast<char *>(workspace);
+  a.stream = s;
+  return prefill_simt(a) == cudaSuccess ? MAMBA2_OK : MAMBA2_ERR_CUDA;
+}
+
+MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *params,
+                               const void *xBC, int64_t xBC_row_stride, const void *z,
+                               int64_t z_row_stride, const void *dt_raw, int64_t dt_row_stride,
+                               void *y, void *conv_state, float *ssm_state, void *stream) {
+  DisarmOnExit disarm;
+  Problem pr;
+  int st = make_problem(dims, false, &pr);
+  if (st != MAMBA2_OK) return st;
+  if (!params_ok(params)) return MAMBA2_ERR_INVALID_ARG;
+  if (pr.batch == 0) return MAMBA2_OK;
+  if (xBC == nullptr || z == nullptr || dt_raw == nullptr || y == nullptr ||
+      conv_state == nullptr || ssm_state == nullptr)
+    return MAMBA2_ERR_INVALID_ARG;
+  const size_t esz = pr.io == MAMBA2_BF16 ? 2 : 4;
+  if (xBC_row_stride < pr.conv_dim || z_row_stride < pr.d_inner || dt_row_stride < pr.H)
+    return MAMBA2_ERR_INVALID_ARG;
+  if (xBC_row_stride % 8 != 0 || z_row_stride % 8 != 0) return MAMBA2_ERR_INVALID_ARG;
+  if (!aligned(xBC, 16) || !aligned(z, 16) || !aligned(y, 16) || !aligned(ssm_state, 16) ||
+      !aligned(conv_state, esz) || !aligned(dt_raw, esz))
+    return MAMBA2_ERR_INVALID_ARG;
+  StepArgs a;
+  a.pr = pr;
+  a.prm = *params;
+  a.xBC = xBC;
+  a.ld_xbc = xBC_row_stride;
+  a.z = z;
+  a.ld_z = z_row_stride;
+  a.dt_raw = dt_raw;
+  a.ld_dt = dt_row_stride;
+  a.y = y;
+  a.conv_state = conv_state;
+  a.ssm_state = ssm_state;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return step_simt(a) == cudaSuccess ? MAMBA2_OK : MAMBA2_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+"""GPU parity at the full benchmark sizes, through the same C-ABI calls and launch
+configuration the benchmark times.
+
+Prefill workloads are compared element by element over every output (the
+oracle finishes them in seconds to a minute on the host cores).  The decode
+workload (batch 256, 1024 steps) is compared on the rows the oracle can follow
+one by one: batch rows {0, 1, 127, 255} for all 1024 steps, and every row for
+the first 8 steps; y on every checked step, the states after step 8 and after
+step 1024.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import mamba_ssd_scan_mixer_b200 as m2
+import oracle
+from mamba_ssd_scan_mixer_b200 import workloads as W
+
+from harness import (check_bf16_out, check_exact, check_rms, compare_prefill, dev_params,
+                     gpu_prefill, oracle_prefill)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["zamba2_2p7b_prefill", "zamba2_1p2b_prefill",
+                                  "zamba2_7b_long_prefill"])
+def test_full_size_prefill(name):
+    cfg = W.CONFIGS[name]
+    params = W.make_params(cfg, 0)
+    inp = W.make_prefill_inputs(cfg, 0)
+    got = gpu_prefill(cfg, inp, params)
+    t = time.time()
+    ref = oracle_prefill(cfg, inp, params)
+    rep = compare_prefill(cfg, got, ref)
+    print(name, rep, f"oracle {time.time() - t:.1f}s")
+
+
+def test_full_size_decode_1024_steps():
+    cfg = W.CONFIGS["zamba2_2p7b_decode"]
+    seed = 0
+    params = W.make_params(cfg, seed)
+    st = W.make_states(cfg, seed)
+    dims = m2.dims_from_config(cfg)
+    pt, pp = dev_params(params)
+    cs = st["conv_state"].cuda().contiguous()
+    hs = st["ssm_state"].cuda().contiguous()
+    y = torch.empty(cfg.batch, cfg.d_inner, dtype=cfg.torch_dtype, device="cuda")
+    rows = [0, 1, 127, 255]
+    odims = dict(nheads=cfg.nheads, headdim=cfg.headdim, dstate=cfg.dstate,
+                 ngroups=cfg.ngroups)
+    o_cs, o_hs = st["conv_state"], st["ssm_state"]            # all rows, first 8 steps
+    s_cs, s_hs = st["conv_state"][rows], st["ssm_state"][rows]  # checked rows, all steps
+    di, cd = cfg.d_inner, cfg.conv_dim
+    worst = 0.0
+    for s in range(cfg.decode_steps):
+        si = W.make_step_inputs(cfg, seed, s)
+        packed = si["zxbcdt"].cuda(non_blocking=True)
+        m2.mamba2_ssd_step(dims, pp, packed[:, di:di + cd], packed[:, :di], packed[:, di + cd:],
+                           y, cs, hs)
+        yg = y.cpu()
+        if s < 8:
+            o = oracle.mixer_step(si["xBC"], si["z"], si["dt_raw"], params, o_cs, o_hs, **odims)
+            o_cs, o_hs = o["conv_state"], o["ssm_state"]
+            worst = max(worst, check_bf16_out(yg, o["y"], f"y step {s} (all rows)")[0])
+            if s == 7:
+                check_exact(cs.cpu(), o_cs, "conv_state after 8 steps")
+                check_rms(hs.cpu(), o_hs, "ssm_state after 8 steps")
+        o = oracle.mixer_step(si["xBC"][rows], si["z"][rows], si["dt_raw"][rows], params, s_cs,
+                              s_hs, **odims)
+        s_cs, s_hs = o["conv_state"], o["ssm_state"]
+        worst = max(worst, check_bf16_out(yg[rows], o["y"], f"y step {s} rows {rows}")[0])
+    check_exact(cs.cpu()[rows], s_cs, "conv_state after 1024 steps")
+    e = check_rms(hs.cpu()[rows], s_hs, "ssm_state after 1024 steps")
+    print("decode worst y error beyond bf16 rounding", worst, "state", e)
