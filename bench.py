@@ -220,9 +220,9 @@ def run_ours(args, rank, world, local_rank):
     sets = []
     for r in range(ROTATE):
         packed = host_in.to(dev)
+        v = W.split_packed(cfg, packed)
         sets.append(dict(
-            packed=packed, z=packed[..., :di], xBC=packed[..., di:di + cd],
-            dt=packed[..., di + cd:],
+            packed=packed, z=v["z"], xBC=v["xBC"], dt=v["dt_raw"],
             y=torch.empty(cfg.batch, cfg.seqlen, di, dtype=cfg.torch_dtype, device=dev),
             cs=torch.zeros(cfg.batch, cd, cfg.d_conv, dtype=cfg.torch_dtype, device=dev),
             hs=torch.zeros(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, device=dev),
@@ -348,10 +348,13 @@ def run_e2e(args, cfg, dims, pp, host_in, dev, stream, m2):
     d_hs = torch.empty(h_hs.shape, dtype=h_hs.dtype, device=dev)
     ws = torch.empty(m2.mamba2_prefill_workspace_size(dims), dtype=torch.uint8, device=dev)
 
+    from mamba_ssd_scan_mixer_b200 import workloads as W
+    v = W.split_packed(cfg, d_in)
+
     def step():
         d_in.copy_(h_in, non_blocking=True)
-        m2.mamba2_conv_ssd_prefill(dims, pp, d_in[..., di:di + cd], d_in[..., :di],
-                                   d_in[..., di + cd:], d_y, d_cs, d_hs, False, ws, stream)
+        m2.mamba2_conv_ssd_prefill(dims, pp, v["xBC"], v["z"], v["dt_raw"], d_y, d_cs, d_hs,
+                                   False, ws, stream)
         h_y.copy_(d_y, non_blocking=True)
         h_cs.copy_(d_cs, non_blocking=True)
         h_hs.copy_(d_hs, non_blocking=True)
@@ -388,15 +391,14 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, m2, W):
     cs = st["conv_state"].to(dev)
     hs = st["ssm_state"].to(dev)
     g = torch.Generator(device=dev).manual_seed(1000 + rank)
-    inputs = torch.randn(S, cfg.batch, cfg.d_in_proj, generator=g, device=dev).to(
+    inputs = torch.randn(S, cfg.batch, cfg.packed_width, generator=g, device=dev).to(
         cfg.torch_dtype)
     y = torch.empty(cfg.batch, cfg.d_inner, dtype=cfg.torch_dtype, device=dev)
     di, cd = cfg.d_inner, cfg.conv_dim
 
     def step(k):
-        p = inputs[k]
-        m2.mamba2_ssd_step(dims, pp, p[:, di:di + cd], p[:, :di], p[:, di + cd:], y, cs, hs,
-                           stream)
+        v = W.split_packed(cfg, inputs[k])
+        m2.mamba2_ssd_step(dims, pp, v["xBC"], v["z"], v["dt_raw"], y, cs, hs, stream)
 
     for k in range(max(3, args.warmup)):
         step(k % S)

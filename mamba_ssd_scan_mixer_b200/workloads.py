@@ -59,6 +59,12 @@ class MixerConfig:
         return self.d_inner + self.conv_dim + self.nheads
 
     @property
+    def packed_width(self) -> int:
+        """Row width of the packed [z | xBC | dt] buffer, padded to a multiple of 8
+        elements (16 bytes in bf16) as the library's row strides require."""
+        return -(-self.d_in_proj // 8) * 8
+
+    @property
     def torch_dtype(self) -> torch.dtype:
         return torch.float32 if self.io_dtype == "f32" else torch.bfloat16
 
@@ -104,18 +110,19 @@ def make_params(cfg: MixerConfig, seed: int = 0) -> dict:
             "norm_w": norm_w}
 
 
-def _split_packed(cfg: MixerConfig, packed: torch.Tensor) -> dict:
-    di, cd = cfg.d_inner, cfg.conv_dim
+def split_packed(cfg: MixerConfig, packed: torch.Tensor) -> dict:
+    """Views z, xBC, dt_raw of a packed [..., packed_width] buffer (pad columns unused)."""
+    di, cd, H = cfg.d_inner, cfg.conv_dim, cfg.nheads
     return {"zxbcdt": packed, "z": packed[..., :di], "xBC": packed[..., di:di + cd],
-            "dt_raw": packed[..., di + cd:]}
+            "dt_raw": packed[..., di + cd:di + cd + H]}
 
 
 def make_prefill_inputs(cfg: MixerConfig, seed: int = 0) -> dict:
     """Packed [b, L, d_in_proj] buffer in the I/O dtype and its views z, xBC, dt_raw.
     All entries ~ N(0, 1) (x, B, C, z and dt_raw alike)."""
     g = generator(seed, _S_INPUTS)
-    packed = torch.randn(cfg.batch, cfg.seqlen, cfg.d_in_proj, generator=g)
-    return _split_packed(cfg, packed.to(cfg.torch_dtype))
+    packed = torch.randn(cfg.batch, cfg.seqlen, cfg.packed_width, generator=g)
+    return split_packed(cfg, packed.to(cfg.torch_dtype))
 
 
 def make_states(cfg: MixerConfig, seed: int = 0) -> dict:
@@ -135,5 +142,5 @@ def zero_states(cfg: MixerConfig) -> dict:
 def make_step_inputs(cfg: MixerConfig, seed: int, step: int) -> dict:
     """Inputs of decode step `step`: packed [b, d_in_proj] and its views."""
     g = generator(seed, _S_STEP0 + step)
-    packed = torch.randn(cfg.batch, cfg.d_in_proj, generator=g)
-    return _split_packed(cfg, packed.to(cfg.torch_dtype))
+    packed = torch.randn(cfg.batch, cfg.packed_width, generator=g)
+    return split_packed(cfg, packed.to(cfg.torch_dtype))

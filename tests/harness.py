@@ -35,9 +35,9 @@ def dev_params(params, device="cuda"):
 def gpu_prefill(cfg, inp, params, states=None, states_in=False, want_states=True):
     """Run the library's prefill on cfg-shaped inputs (CPU tensors); returns CPU tensors."""
     dims = m2.dims_from_config(cfg)
-    packed = inp["zxbcdt"].cuda()
-    di, cd = cfg.d_inner, cfg.conv_dim
-    z, xBC, dt = packed[..., :di], packed[..., di:di + cd], packed[..., di + cd:]
+    v = W.split_packed(cfg, inp["zxbcdt"].cuda())
+    z, xBC, dt = v["z"], v["xBC"], v["dt_raw"]
+    cd = cfg.conv_dim
     pt, pp = dev_params(params)
     if states is not None:
         cs = states["conv_state"].cuda().contiguous()

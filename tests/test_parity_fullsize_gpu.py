@@ -52,13 +52,11 @@ def test_full_size_decode_1024_steps():
                  ngroups=cfg.ngroups)
     o_cs, o_hs = st["conv_state"], st["ssm_state"]            # all rows, first 8 steps
     s_cs, s_hs = st["conv_state"][rows], st["ssm_state"][rows]  # checked rows, all steps
-    di, cd = cfg.d_inner, cfg.conv_dim
     worst = 0.0
     for s in range(cfg.decode_steps):
         si = W.make_step_inputs(cfg, seed, s)
-        packed = si["zxbcdt"].cuda(non_blocking=True)
-        m2.mamba2_ssd_step(dims, pp, packed[:, di:di + cd], packed[:, :di], packed[:, di + cd:],
-                           y, cs, hs)
+        v = W.split_packed(cfg, si["zxbcdt"].cuda(non_blocking=True))
+        m2.mamba2_ssd_step(dims, pp, v["xBC"], v["z"], v["dt_raw"], y, cs, hs)
         yg = y.cpu()
         if s < 8:
             o = oracle.mixer_step(si["xBC"], si["z"], si["dt_raw"], params, o_cs, o_hs, **odims)

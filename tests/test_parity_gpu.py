@@ -137,10 +137,8 @@ def _gpu_steps(cfg, params, st, step_inputs):
     hs = st["ssm_state"].cuda().contiguous()
     ys = []
     for si in step_inputs:
-        packed = si["zxbcdt"].cuda()
-        di, cd = cfg.d_inner, cfg.conv_dim
-        ys.append(m2.step(dims, pp, packed[:, di:di + cd], packed[:, :di], packed[:, di + cd:],
-                          cs, hs).cpu())
+        v = W.split_packed(cfg, si["zxbcdt"].cuda())
+        ys.append(m2.step(dims, pp, v["xBC"], v["z"], v["dt_raw"], cs, hs).cpu())
     torch.cuda.synchronize()
     return ys, cs.cpu(), hs.cpu()
 
