@@ -126,7 +126,8 @@ def _rows(t, name, width, batch, rows_per_batch):
     if t.stride(-1) != 1:
         raise ValueError(f"{name}: last dimension must be contiguous")
     rs = t.stride(-2) if t.dim() >= 2 else width
-    if t.dim() == 3 and t.shape[0] > 1 and t.stride(0) != rows_per_batch * rs:
+    if (t.dim() == 3 and t.shape[0] > 1 and rows_per_batch > 0
+            and t.stride(0) != rows_per_batch * rs):
         raise ValueError(f"{name}: batch stride must be rows * row stride")
     return rs
 
