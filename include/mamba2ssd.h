@@ -161,6 +161,38 @@ MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *par
                                int64_t z_row_stride, const void *dt_raw, int64_t dt_row_stride,
                                void *y, void *conv_state, float *ssm_state, void *stream);
 
+/* Size of the fixed device scratch array used by
+ * mamba2_conv_ssd_prefill_noalloc (64 MiB). */
+#define MAMBA2_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* Prefill without a workspace argument, for callers that may not allocate
+ * device memory (for example a plugin inside a runtime whose memory pool owns
+ * every device allocation, or a latency-critical path that cannot afford
+ * cudaMalloc's implicit synchronisation).  The pages have no counterpart of
+ * this entry point.
+ *
+ * Same arguments, meaning and results as mamba2_conv_ssd_prefill, minus the
+ * workspace: the scratch comes from one array of MAMBA2_STATIC_SCRATCH_BYTES
+ * that the library holds in every GPU it is loaded on until the process
+ * exits.  The caller still allocates inputs, outputs and states.
+ *  - Problems whose mamba2_prefill_workspace_size exceeds
+ *    MAMBA2_STATIC_SCRATCH_BYTES are rejected with MAMBA2_ERR_WORKSPACE and
+ *    nothing is enqueued.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array: calls that may overlap on the GPU (other
+ *    streams, other host threads using the same device) race on it and must
+ *    be serialised by the caller.  No part of the array needs to start at
+ *    zero, so leftover contents from an earlier call are harmless.
+ *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call. */
+MAMBA2_API int mamba2_conv_ssd_prefill_noalloc(const mamba2_dims *dims,
+                                               const mamba2_params *params, const void *xBC,
+                                               int64_t xBC_row_stride, const void *z,
+                                               int64_t z_row_stride, const void *dt_raw,
+                                               int64_t dt_row_stride, void *y, void *conv_state,
+                                               float *ssm_state, int32_t states_in,
+                                               void *stream);
+
 /* Profiling aid (no counterpart on the pages).  Arms the calling host thread
  * so that its NEXT call of mamba2_conv_ssd_prefill or mamba2_ssd_step records
  * events[i] (cudaEvent_t passed as void*, created by the caller) on the

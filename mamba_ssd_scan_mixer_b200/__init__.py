@@ -20,7 +20,8 @@ import os
 __all__ = [
     "Mamba2Dims", "Mamba2Params", "Mamba2Error", "MAMBA2_F32", "MAMBA2_BF16", "lib",
     "library_path", "make_dims", "make_params", "mamba2_prefill_workspace_size",
-    "mamba2_conv_ssd_prefill", "mamba2_ssd_step", "prefill", "step", "status_string",
+    "mamba2_conv_ssd_prefill", "mamba2_conv_ssd_prefill_noalloc", "mamba2_ssd_step", "prefill",
+    "step", "status_string",
 ]
 
 MAMBA2_F32, MAMBA2_BF16 = 0, 1
@@ -72,6 +73,9 @@ def lib() -> ctypes.CDLL:
         L.mamba2_conv_ssd_prefill.restype = ctypes.c_int
         L.mamba2_conv_ssd_prefill.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp, i32,
                                               vp, sz, vp]
+        L.mamba2_conv_ssd_prefill_noalloc.restype = ctypes.c_int
+        L.mamba2_conv_ssd_prefill_noalloc.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp,
+                                                      vp, i32, vp]
         L.mamba2_ssd_step.restype = ctypes.c_int
         L.mamba2_ssd_step.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp, vp]
         _lib = L
@@ -155,6 +159,23 @@ def mamba2_conv_ssd_prefill(dims, params, xBC, z, dt_raw, y, conv_state=None, ss
         ws_bytes, _stream(stream))
     if st != 0:
         raise Mamba2Error(st, "mamba2_conv_ssd_prefill")
+
+
+def mamba2_conv_ssd_prefill_noalloc(dims, params, xBC, z, dt_raw, y, conv_state=None,
+                                    ssm_state=None, states_in=False, stream=None) -> None:
+    """Prefill without a workspace, for callers that may not allocate device memory:
+    the library's fixed device scratch array (MAMBA2_STATIC_SCRATCH_BYTES, 64 MiB)
+    is used instead.  Larger problems raise Mamba2Error (workspace status).  Calls
+    that overlap on the GPU share that array and race; serialise them."""
+    L = dims.seqlen
+    lx = _rows(xBC, "xBC", None, dims.batch, L)
+    lz = _rows(z, "z", None, dims.batch, L)
+    ld = _rows(dt_raw, "dt_raw", None, dims.batch, L)
+    st = lib().mamba2_conv_ssd_prefill_noalloc(
+        ctypes.byref(dims), ctypes.byref(params), _ptr(xBC), lx, _ptr(z), lz, _ptr(dt_raw), ld,
+        _ptr(y), _ptr(conv_state), _ptr(ssm_state), int(bool(states_in)), _stream(stream))
+    if st != 0:
+        raise Mamba2Error(st, "mamba2_conv_ssd_prefill_noalloc")
 
 
 def mamba2_ssd_step(dims, params, xBC, z, dt_raw, y, conv_state, ssm_state, stream=None) -> None:
