@@ -141,6 +141,29 @@ def traffic_for(kernel, workload):
     return e.get("bytes_per_launch")
 
 
+# ---------------------------------------------------------------- ranks
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own independent sequence (weak scaling)."""
+    return rank
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time: all-reduce MAX (every rank must call this)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank_step: int, steps: int, max_elapsed_ms: float, world: int) -> float:
+    """Whole-job throughput: units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_elapsed_ms / 1e3)
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -208,7 +231,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cfg = W.CONFIGS[PREFILL]
-    seed = rank
+    seed = rank_seed(rank)
     lib = m2.lib()
     dims = m2.dims_from_config(cfg)
     params = {k: v.to(dev) for k, v in W.make_params(cfg, seed).items()}
@@ -282,15 +305,12 @@ def run_ours(args, rank, world, local_rank):
     elapsed = t0.elapsed_time(t1)
     dom_ms = sum(a.elapsed_time(b) for a, b in dom_evs) / K
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, world, dev)
 
     peaks, peak_src = load_peaks()
     ms = elapsed / K
     tokens = cfg.batch * cfg.seqlen
-    value = world * tokens * K / (elapsed / 1e3)
+    value = job_rate(tokens, K, elapsed, world)
     path_bytes = prefill_bytes(cfg)
     path_flops = prefill_flops(cfg)
     t_roof = max(path_bytes / (peaks["hbm_gbs"] * 1e9), path_flops / (peaks["bf16_tflops"] * 1e12))
@@ -384,10 +404,10 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, m2, W):
     cfg = W.CONFIGS[DECODE]
     S = args.decode_steps or cfg.decode_steps
     dims = m2.dims_from_config(cfg)
-    params = {k: v.to(dev) for k, v in W.make_params(cfg, rank).items()}
+    params = {k: v.to(dev) for k, v in W.make_params(cfg, rank_seed(rank)).items()}
     pp = m2.make_params(params["conv_w"], params["conv_b"], params["dt_bias"], params["A"],
                         params["D"], params["norm_w"])
-    st = W.make_states(cfg, rank)
+    st = W.make_states(cfg, rank_seed(rank))
     cs = st["conv_state"].to(dev)
     hs = st["ssm_state"].to(dev)
     g = torch.Generator(device=dev).manual_seed(1000 + rank)
@@ -420,15 +440,12 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, m2, W):
         dist.barrier()
     elapsed = a.elapsed_time(b)
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, world, dev)
     ms = elapsed / S
     nb = decode_bytes(cfg)
     ach = nb / (ms * 1e-3) / 1e9
-    return {"value": world * S / (elapsed / 1e3), "unit": "steps/s", "steps": S,
-            "ms_per_step": ms, "tokens_per_s": world * cfg.batch * S / (elapsed / 1e3),
+    return {"value": job_rate(1, S, elapsed, world), "unit": "steps/s", "steps": S,
+            "ms_per_step": ms, "tokens_per_s": job_rate(cfg.batch, S, elapsed, world),
             "config": {"workload": DECODE, "batch": cfg.batch, "nheads": cfg.nheads,
                        "headdim": cfg.headdim, "dstate": cfg.dstate,
                        "l2": "state 335 MB > 126 MB L2; distinct per-step inputs"},
