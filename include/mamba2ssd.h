@@ -161,6 +161,16 @@ MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *par
                                int64_t z_row_stride, const void *dt_raw, int64_t dt_row_stride,
                                void *y, void *conv_state, float *ssm_state, void *stream);
 
+/* Device-side error flags (no counterpart on the pages).  Kernels that wait
+ * for asynchronous copies give every wait a time limit (2 s); when one runs
+ * out the kernel stops using the data, lets its own copies in flight land,
+ * sets a flag and returns, leaving the context usable and the outputs of that
+ * call undefined.  This call synchronises the current device, stores the
+ * flags raised since the previous call in *flags (0 = none; bit 0 = a wait
+ * ran out) and clears them.  Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG (flags
+ * NULL) or MAMBA2_ERR_CUDA. */
+MAMBA2_API int mamba2_device_errors(unsigned int *flags);
+
 /* Size of the fixed device scratch array used by
  * mamba2_conv_ssd_prefill_noalloc (64 MiB). */
 #define MAMBA2_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)

@@ -76,10 +76,22 @@ def lib() -> ctypes.CDLL:
         L.mamba2_conv_ssd_prefill_noalloc.restype = ctypes.c_int
         L.mamba2_conv_ssd_prefill_noalloc.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp,
                                                       vp, i32, vp]
+        L.mamba2_device_errors.restype = ctypes.c_int
+        L.mamba2_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         L.mamba2_ssd_step.restype = ctypes.c_int
         L.mamba2_ssd_step.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp, vp]
         _lib = L
     return _lib
+
+
+def device_errors() -> int:
+    """Synchronise the current device and return (and clear) the flags raised by
+    kernels whose bounded waits ran out (0 = none)."""
+    f = ctypes.c_uint(0)
+    st = lib().mamba2_device_errors(ctypes.byref(f))
+    if st != 0:
+        raise Mamba2Error(st, "mamba2_device_errors")
+    return int(f.value)
 
 
 def status_string(status: int) -> str:

@@ -87,6 +87,16 @@ MAMBA2_API int mamba2_record_stage_events(void *const *events, int n_events) {
   return MAMBA2_OK;
 }
 
+MAMBA2_API int mamba2_device_errors(unsigned int *flags) {
+  if (flags == nullptr) return MAMBA2_ERR_INVALID_ARG;
+  *flags = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MAMBA2_ERR_CUDA;
+  unsigned int f = 0;
+  if (take_step_errors(&f) != cudaSuccess) return MAMBA2_ERR_CUDA;
+  *flags |= f;
+  return MAMBA2_OK;
+}
+
 MAMBA2_API int mamba2_stage_names(int kind, const mamba2_dims *dims, const char **names,
                                   int max_names) {
   Problem pr;

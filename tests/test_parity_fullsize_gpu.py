@@ -72,3 +72,4 @@ def test_full_size_decode_1024_steps():
     check_exact(cs.cpu()[rows], s_cs, "conv_state after 1024 steps")
     e = check_rms(hs.cpu()[rows], s_hs, "ssm_state after 1024 steps")
     print("decode worst y error beyond bf16 rounding", worst, "state", e)
+    assert m2.device_errors() == 0

@@ -184,3 +184,4 @@ def test_decode_small(cfg):
             check_bf16_out(ys[s], o["y"], f"y step {s}")
     check_exact(cs, ocs, "conv_state")
     (check_f32 if cfg.io_dtype == "f32" else check_rms)(hs, ohs, "ssm_state")
+    assert m2.device_errors() == 0
