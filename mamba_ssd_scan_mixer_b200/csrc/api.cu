@@ -47,6 +47,14 @@ int make_problem(const mamba2_dims *d, bool prefill, Problem *pr) {
   return MAMBA2_OK;
 }
 
+// The prefill kernels a problem runs on: the tensor-core path for bf16 I/O at
+// headdim 64 / d_state 64, the fp32 CUDA-core path otherwise.
+bool use_tc(const Problem &pr) { return prefill_tc_supported(pr); }
+
+size_t prefill_workspace(const Problem &pr) {
+  return use_tc(pr) ? prefill_tc_workspace(pr) : prefill_simt_workspace(pr);
+}
+
 bool params_ok(const mamba2_params *p) {
   return p != nullptr && p->conv_w && p->conv_b && p->dt_bias && p->A && p->D && p->norm_w;
 }
@@ -94,6 +102,8 @@ MAMBA2_API int mamba2_device_errors(unsigned int *flags) {
   unsigned int f = 0;
   if (take_step_errors(&f) != cudaSuccess) return MAMBA2_ERR_CUDA;
   *flags |= f;
+  if (take_prefill_tc_errors(&f) != cudaSuccess) return MAMBA2_ERR_CUDA;
+  *flags |= f;
   return MAMBA2_OK;
 }
 
@@ -101,9 +111,10 @@ MAMBA2_API int mamba2_stage_names(int kind, const mamba2_dims *dims, const char 
                                   int max_names) {
   Problem pr;
   if (make_problem(dims, kind == 0, &pr) != MAMBA2_OK) return MAMBA2_ERR_INVALID_ARG;
-  const char *const *list = kind == 0 ? kPrefillSimtStages : kStepSimtStages;
-  const int n = kind == 0 ? kPrefillSimtStageCount : kStepSimtStageCount;
   if (kind != 0 && kind != 1) return MAMBA2_ERR_INVALID_ARG;
+  const bool tc = kind == 0 && use_tc(pr);
+  const char *const *list = kind == 1 ? kStepSimtStages : tc ? kPrefillTcStages : kPrefillSimtStages;
+  const int n = kind == 1 ? kStepSimtStageCount : tc ? kPrefillTcStageCount : kPrefillSimtStageCount;
   for (int i = 0; names != nullptr && i < n && i < max_names; ++i) names[i] = list[i];
   return n;
 }
@@ -111,7 +122,7 @@ MAMBA2_API int mamba2_stage_names(int kind, const mamba2_dims *dims, const char 
 MAMBA2_API size_t mamba2_prefill_workspace_size(const mamba2_dims *dims) {
   Problem pr;
   if (make_problem(dims, true, &pr) != MAMBA2_OK) return 0;
-  return prefill_simt_workspace(pr);
+  return prefill_workspace(pr);
 }
 
 MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_params *params,
@@ -140,7 +151,7 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
     if (xBC_row_stride % 8 != 0 || z_row_stride % 8 != 0) return MAMBA2_ERR_INVALID_ARG;
     if (!aligned(xBC, 16) || !aligned(z, 16) || !aligned(y, 16) || !aligned(dt_raw, esz))
       return MAMBA2_ERR_INVALID_ARG;
-    const size_t need = prefill_simt_workspace(pr);
+    const size_t need = prefill_workspace(pr);
     if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
       return MAMBA2_ERR_WORKSPACE;
   } else {
@@ -172,7 +183,8 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
   a.states_in = states_in;
   a.ws = static_cast<char *>(workspace);
   a.stream = s;
-  return prefill_simt(a) == cudaSuccess ? MAMBA2_OK : MAMBA2_ERR_CUDA;
+  return (use_tc(pr) ? prefill_tc(a) : prefill_simt(a)) == cudaSuccess ? MAMBA2_OK
+                                                                      : MAMBA2_ERR_CUDA;
 }
 
 MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *params,

@@ -1,0 +1,835 @@
+// Prefill of the Mamba-2 mixer core on the 5th-generation tensor cores
+// (tcgen05.mma, accumulators in tensor memory), for bf16 I/O with headdim 64
+// and d_state 64.
+//
+// It evaluates the chunked state-space-duality form of the scan (the Mamba-2
+// layer named on the state-spaces/mamba repository page, opendeer.net, "About
+// the project"; chunked prefill per "Zamba2 hybrid architecture in
+// Transformers", qwbw.cn, section 三 step 3) with 128-token chunks, one chunk
+// per CTA so that the token dimension is the MMA's M = 128:
+//
+//   tc_chunk_state  conv+SiLU of x (two heads) and B, dt/cumsum, then
+//                   S_c = (x o w)^T B with w_s = exp(cum_end - cum_s) dt_s:
+//                   M = 128 (2 heads x 64 lanes), N = 64, K = 128 tokens.
+//   tc_state_pass   H_{c+1} = exp(cum_end) H_c + S_c over chunks in fp32; the
+//                   state entering each chunk is kept as the fp16 MMA operand,
+//                   the final state in fp32.
+//   tc_chunk_out    per chunk, a cluster of CTAs splits the heads of one B/C
+//                   group: CB = C B^T (M = N = 128, K = 64) once; per head the
+//                   operand [CB o exp(cum_t - cum_s) dt_s (causal) | C o exp(cum_t)]
+//                   times [x ; H_c] gives y_pre (K = 128 + 64) in TMEM; D x,
+//                   the silu(z) gate and sums of squares follow, the per-token
+//                   sums are exchanged through distributed shared memory, and
+//                   the normalised output is written in bf16.
+//
+// Operands are fp16 (11-bit significand; bf16's 8 bits cannot meet the output
+// tolerance on these workloads), accumulation is fp32.  The chunk-state
+// product uses a two-term fp16 split of both operands (hi*hi + hi*lo + lo*hi),
+// because the returned final state must hold 2e-2 of its RMS.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace m2 {
+namespace {
+
+constexpr int kQ = 128;          // tokens per chunk = MMA M
+constexpr int kThreads = 256;    // 8 warps
+constexpr int kHP = 64;          // headdim
+constexpr int kNS = 64;          // d_state
+constexpr int kMaxHeadsPerCta = 6;  // TMEM: 128 (CB) + 6 x 64 (y) <= 512 columns
+constexpr float kLog2e = 1.4426950408889634f;
+
+static __device__ unsigned int g_tc_errors = 0;
+
+struct TcArgs {
+  Problem pr;
+  mamba2_params prm;
+  const __nv_bfloat16 *xBC;
+  int64_t ld_x;
+  const __nv_bfloat16 *z;
+  int64_t ld_z;
+  const __nv_bfloat16 *dt_raw;
+  int64_t ld_dt;
+  __nv_bfloat16 *y;
+  const __nv_bfloat16 *conv_in;  // conv state read for the left context (or null)
+  float *ssm_state;              // in (if states_in) / out (may be null)
+  int states_in;
+  int nch;                       // chunks of kQ tokens
+  float *S;                      // [b][nch][H][64][64] chunk states
+  float *cum_end;                // [b][nch][H] chunk sum of dt*A
+  __half *Hc;                    // [b][nch][H][64][64] state entering each chunk
+  int hpc;                       // max heads per CTA in tc_chunk_out
+};
+
+// silu with the fast reciprocal: __fdividef returns 0 once 1 + e^-v passes
+// 2^126, which is the limit silu(v) -> 0 for very negative v.
+__device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Inclusive prefix sum over the 32 lanes of a warp.
+__device__ __forceinline__ float warp_scan(float v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// 8 consecutive bf16 channels of raw input token `tau` (sequence row bi): the
+// token itself for 0 <= tau < L, the carried conv state for tau < 0 when
+// states_in, zeros otherwise (left padding, or past the end of the sequence).
+__device__ __forceinline__ void load_row8(const TcArgs &a, int64_t bi, int64_t tau, int64_t ch,
+                                          float (&v)[8]) {
+  if (tau >= 0 && tau < a.pr.L) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a.xBC + (bi * a.pr.L + tau) * a.ld_x + ch));
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  } else if (tau < 0 && a.states_in) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = __bfloat162float(a.conv_in[(bi * a.pr.conv_dim + ch + i) * 4 + 4 + tau]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+  }
+}
+
+// conv1d + SiLU of 8 channels [ch, ch+8) for 4 tokens t0..t0+3 (absolute).
+__device__ __forceinline__ void conv8x4(const TcArgs &a, int64_t bi, int64_t t0, int64_t ch,
+                                        float (&out)[4][8]) {
+  float w[8][4], bias[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 wv = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch + i);
+    w[i][0] = wv.x;
+    w[i][1] = wv.y;
+    w[i][2] = wv.z;
+    w[i][3] = wv.w;
+    bias[i] = __ldg(a.prm.conv_b + ch + i);
+  }
+  float rows[7][8];
+#pragma unroll
+  for (int r = 0; r < 7; ++r) load_row8(a, bi, t0 - 3 + r, ch, rows[r]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float pre = bias[i] + w[i][0] * rows[k][i] + w[i][1] * rows[k + 1][i] +
+                        w[i][2] * rows[k + 2][i] + w[i][3] * rows[k + 3][i];
+      out[k][i] = silu_fast(pre);
+    }
+}
+
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// Block-uniform bounded wait on an mbarrier phase.
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, bool ok) {
+  bool got = ok ? mbar_wait_bounded(bar, parity, &g_tc_errors) : false;
+  return __syncthreads_and(got) != 0;
+}
+
+// ============================================================== chunk states
+// grid (nch, G * pairs_per_group, b); 256 threads.  Smem (1024-aligned):
+// A_hi, A_lo [2 k-blocks][128 rows][128 B]; B_hi, B_lo [2][64][128 B].
+constexpr uint32_t kK1A = 2 * 128 * 128, kK1B = 2 * 64 * 128;
+
+__global__ void __launch_bounds__(kThreads) tc_chunk_state_kernel(TcArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ float ws[2][kQ];
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tmem_holder;
+  const Problem &pr = a.pr;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sAhi = base, sAlo = base + kK1A, sBhi = base + 2 * kK1A,
+                 sBlo = base + 2 * kK1A + kK1B;
+  const int c = blockIdx.x;
+  const int hpg = pr.heads_per_group();
+  const int pairs = (hpg + 1) / 2;
+  const int g = blockIdx.y / pairs, pair = blockIdx.y % pairs;
+  const int64_t bi = blockIdx.z;
+  const int hA = g * hpg + 2 * pair;
+  const bool hasB = 2 * pair + 1 < hpg;
+  const int64_t c0 = (int64_t)c * kQ;
+
+  if (warp == 0) tmem_alloc(&tmem_holder, 64);
+  if (tid == 0) {
+    mbar_init(&mbar, 1);
+    fence_mbar_init();
+  }
+
+  // dt, chunk-local cumsum of dt*A, weights w_s = exp(cum_end - cum_s) dt_s:
+  // warp 0 for head A, warp 1 for head B, 4 consecutive tokens per lane
+  if (warp < 2) {
+    const int half = warp;
+    const bool hv = half == 0 || hasB;
+    const int h = hA + half;
+    float dt4[4], a4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t tt = c0 + 4 * lane + k;
+      dt4[k] = (hv && tt < pr.L)
+                   ? softplus_f(__bfloat162float(a.dt_raw[(bi * pr.L + tt) * a.ld_dt + h]) +
+                                a.prm.dt_bias[h])
+                   : 0.0f;
+      a4[k] = hv ? dt4[k] * a.prm.A[h] : 0.0f;
+    }
+    const float tot = a4[0] + a4[1] + a4[2] + a4[3];
+    float run = warp_scan(tot, lane) - tot;
+    const float cum_end = __shfl_sync(0xffffffffu, run + tot, 31);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      run += a4[k];
+      ws[half][4 * lane + k] = expf(cum_end - run) * dt4[k];
+    }
+    if (lane == 0 && hv) a.cum_end[(bi * a.nch + c) * pr.H + h] = cum_end;
+  }
+  __syncthreads();
+
+  // conv + SiLU: 24 groups of 8 channels (x of head A, x of head B, B) x 32
+  // ranges of 4 tokens; results split into fp16 hi + lo operands.
+  for (int item = tid; item < 24 * 32; item += kThreads) {
+    const int cgp = item >> 5, tr = item & 31;
+    const int s0 = tr * 4;
+    uint32_t hi[8][2], lo[8][2];
+    if (cgp < 16 && (cgp < 8 || hasB)) {
+      const int half = cgp >> 3, p0 = (cgp & 7) * 8;
+      float v[4][8];
+      conv8x4(a, bi, c0 + s0, (int64_t)(hA + half) * kHP + p0, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float q[4], r[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float x = v[k][i] * ws[half][s0 + k];
+          q[k] = __half2float(__float2half_rn(x));
+          r[k] = x - q[k];
+        }
+        hi[i][0] = pack_half2(q[0], q[1]);
+        hi[i][1] = pack_half2(q[2], q[3]);
+        lo[i][0] = pack_half2(r[0], r[1]);
+        lo[i][1] = pack_half2(r[2], r[3]);
+      }
+      const int blk = s0 >> 6;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int m = half * 64 + p0 + i;
+        const uint32_t off = blk * 16384 + sw128_off(m, s0 & 63);
+        st_shared_v2(sAhi + off, hi[i][0], hi[i][1]);
+        st_shared_v2(sAlo + off, lo[i][0], lo[i][1]);
+      }
+    } else if (cgp < 16) {  // missing second head: zero rows 64..127
+      const int p0 = (cgp & 7) * 8, blk = s0 >> 6;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t off = blk * 16384 + sw128_off(64 + p0 + i, s0 & 63);
+        st_shared_v2(sAhi + off, 0u, 0u);
+        st_shared_v2(sAlo + off, 0u, 0u);
+      }
+    } else {
+      const int n0 = (cgp - 16) * 8;
+      float v[4][8];
+      conv8x4(a, bi, c0 + s0, pr.d_inner + (int64_t)g * kNS + n0, v);
+      const int blk = s0 >> 6;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float q[4], r[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          q[k] = __half2float(__float2half_rn(v[k][i]));
+          r[k] = v[k][i] - q[k];
+        }
+        const uint32_t off = blk * 8192 + sw128_off(n0 + i, s0 & 63);
+        st_shared_v2(sBhi + off, pack_half2(q[0], q[1]), pack_half2(q[2], q[3]));
+        st_shared_v2(sBlo + off, pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_holder;
+
+  if (tid == 0) {
+    const uint32_t idesc = umma_idesc_f16(128, 64);
+    const uint32_t As[3] = {sAhi, sAhi, sAlo}, Bs[3] = {sBhi, sBlo, sBhi};
+    for (int prod = 0; prod < 3; ++prod)
+      for (int ks = 0; ks < 8; ++ks) {
+        const int blk = ks >> 2, kin = ks & 3;
+        umma_f16(tmem, umma_desc_sw128(As[prod] + blk * 16384 + kin * 32),
+                 umma_desc_sw128(Bs[prod] + blk * 8192 + kin * 32), idesc,
+                 (prod > 0 || ks > 0) ? 1u : 0u);
+      }
+    umma_commit(&mbar);
+  }
+  const bool ok = wait_all(&mbar, 0, true);
+  tc_fence_after();
+  if (ok) {
+    // rows m = 32*(warp%4) + lane; warps 0-3 columns 0-31, warps 4-7 columns 32-63
+    const int m = 32 * (warp & 3) + lane, half = m >> 6, p = m & 63, cb = 32 * (warp >> 2);
+    float v[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, v);
+    if (half == 0 || hasB) {
+      float4 *dst = reinterpret_cast<float4 *>(
+          a.S + (((bi * a.nch + c) * pr.H + hA + half) * kHP + p) * kNS + cb);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+// ============================================================== state passing
+// grid (P*N/256, H, b): one thread per state element, sequential over chunks.
+__global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a) {
+  const Problem &pr = a.pr;
+  const int e = blockIdx.x * 256 + threadIdx.x;  // p * 64 + n
+  const int h = blockIdx.y;
+  const int64_t bi = blockIdx.z;
+  const int64_t hs = (bi * pr.H + h) * (int64_t)(kHP * kNS) + e;
+  float hc = a.states_in ? a.ssm_state[hs] : 0.0f;
+  const int64_t stride = (int64_t)pr.H * kHP * kNS;
+  const float *S = a.S + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
+  __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
+  const float *ce = a.cum_end + bi * a.nch * pr.H + h;
+  int c = 0;
+  for (; c + 4 <= a.nch; c += 4) {
+    float s[4], d[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      s[k] = S[(c + k) * stride];
+      d[k] = ce[(int64_t)(c + k) * pr.H];
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      Hc[(c + k) * stride] = __float2half_rn(hc);
+      hc = expf(d[k]) * hc + s[k];
+    }
+  }
+  for (; c < a.nch; ++c) {
+    Hc[c * stride] = __float2half_rn(hc);
+    hc = expf(ce[(int64_t)c * pr.H]) * hc + S[c * stride];
+  }
+  if (a.ssm_state != nullptr) a.ssm_state[hs] = hc;
+}
+
+// ============================================================== chunk output
+// grid (cs, nch, G * b), cluster (cs, 1, 1); 256 threads.  Smem (1024-aligned):
+constexpr uint32_t kCt = 0;                      // C  [128 t][64 n]        16 KB
+constexpr uint32_t kBt = kCt + 16384;            // B  [128 s][64 n]        16 KB
+constexpr uint32_t kXt = kBt + 16384;            // x  2 x [2][64 p][64 s]  2 x 16 KB
+constexpr uint32_t kHt = kXt + 2 * 16384;        // Hc 2 x [64 p][64 n]     2 x 8 KB
+constexpr uint32_t kAt = kHt + 2 * 8192;         // A  [3][128 t][64 k]     48 KB
+constexpr uint32_t kTcOutTiles = kAt + 3 * 16384;  // 128 KB
+
+struct OutShared {
+  float cum2[kMaxHeadsPerCta][kQ];  // cumsum * log2(e)
+  float dt[kMaxHeadsPerCta][kQ];
+  float beta[kMaxHeadsPerCta][kQ];  // exp(cum_r - cum_s) dt_s, r = end of s's 32-token group
+  float ecum[kMaxHeadsPerCta][kQ];  // exp(cumsum)
+  float ss[2][kQ];
+  float part[16][kQ];               // per-rank partial sums of squares (rank 0's is read)
+  float inv[kQ];
+  float scan[8];
+  uint64_t mbar_cb, mbar_mma;
+  uint32_t tmem_holder;
+};
+
+__global__ void __launch_bounds__(kThreads) tc_chunk_out_kernel(TcArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int cs = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const Problem &pr = a.pr;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  OutShared &sh = *reinterpret_cast<OutShared *>(smem_raw + (base - smem_u32(smem_raw)) +
+                                                 kTcOutTiles);
+  const int c = blockIdx.y;
+  const int g = (int)(blockIdx.z % pr.G);
+  const int64_t bi = blockIdx.z / pr.G;
+  const int hpg = pr.heads_per_group();
+  const int lh0 = rank * a.hpc;
+  const int nh = max(0, min(a.hpc, hpg - lh0));  // heads of this CTA
+  const int h0 = g * hpg + lh0;
+  const int64_t c0 = (int64_t)c * kQ;
+
+  if (warp == 0) tmem_alloc(&sh.tmem_holder, 512);
+  if (tid == 0) {
+    mbar_init(&sh.mbar_cb, 1);
+    mbar_init(&sh.mbar_mma, 1);
+    fence_mbar_init();
+  }
+
+  // dt / cumsum for the CTA's heads: one warp per head, 4 consecutive tokens
+  // per lane.  beta_s = exp(cum_r - cum_s) dt_s with r the last token of the
+  // 32-token group of s (the column factor of the masked decay, see below).
+  if (warp < nh) {
+    const int j = warp, h = h0 + j;
+    float dt4[4], a4[4];
+    const float dtb = a.prm.dt_bias[h], Ah = a.prm.A[h];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t tt = c0 + 4 * lane + k;
+      dt4[k] = tt < pr.L ? softplus_f(__bfloat162float(a.dt_raw[(bi * pr.L + tt) * a.ld_dt + h]) + dtb)
+                         : 0.0f;
+      a4[k] = dt4[k] * Ah;
+    }
+    const float tot = a4[0] + a4[1] + a4[2] + a4[3];
+    float run = warp_scan(tot, lane) - tot;  // exclusive prefix of this lane's 4 tokens
+    float c2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      run += a4[k];
+      c2[k] = run * kLog2e;
+      sh.cum2[j][4 * lane + k] = c2[k];
+      sh.dt[j][4 * lane + k] = dt4[k];
+      sh.ecum[j][4 * lane + k] = ex2_approx(c2[k]);
+    }
+    // the group of 32 tokens ends at lane 8*(lane/8) + 7, token 4*that + 3
+    const float c2r = __shfl_sync(0xffffffffu, c2[3], (lane | 7));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sh.beta[j][4 * lane + k] = ex2_approx(c2r - c2[k]) * dt4[k];
+  }
+
+  // conv + SiLU of the group's B and C channels: 16 groups of 8 x 32 ranges of 4
+  for (int item = tid; item < 16 * 32; item += kThreads) {
+    const int cgp = item >> 5, tr = item & 31, s0 = tr * 4;
+    const bool isC = cgp >= 8;
+    const int n0 = (cgp & 7) * 8;
+    float v[4][8];
+    conv8x4(a, bi, c0 + s0, pr.d_inner + (int64_t)(isC ? pr.G : 0) * kNS + (int64_t)g * kNS + n0,
+            v);
+    const uint32_t tile = base + (isC ? kCt : kBt);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      st_shared_v4(tile + sw128_chunk(s0 + k, n0), pack_half2(v[k][0], v[k][1]),
+                   pack_half2(v[k][2], v[k][3]), pack_half2(v[k][4], v[k][5]),
+                   pack_half2(v[k][6], v[k][7]));
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_holder;
+  if (tid == 0) {  // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
+    const uint32_t idesc = umma_idesc_f16(128, 128);
+    for (int kin = 0; kin < 4; ++kin)
+      umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32), umma_desc_sw128(base + kBt + kin * 32),
+               idesc, kin > 0 ? 1u : 0u);
+    umma_commit(&sh.mbar_cb);
+  }
+
+  // this thread's TMEM lane (row t) and column half
+  const int t = 32 * (warp & 3) + lane, hf = warp >> 2;
+  const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+  const bool t_valid = c0 + t < pr.L;
+  float ss_acc = 0.0f;
+  bool ok = true;
+
+  // per-head epilogue, part 1: y_pre = Y + D x, gate, sum of squares; g -> TMEM
+  auto epilogue1 = [&](int j) {
+    const int h = h0 + j;
+    float v[32];
+    const uint32_t col = 128 + 64 * j + 32 * hf;
+    tmem_ld32(tmem + lane_off + col, v);
+    const float Dh = a.prm.D[h];
+    const uint32_t xt = base + kXt + (j & 1) * 16384 + (t >> 6) * 8192;
+    float zv[32];
+    if (t_valid) {
+      const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (bi * pr.L + c0 + t) * a.ld_z +
+                                                        (int64_t)h * kHP + 32 * hf);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 raw = __ldg(zp + q);
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h2[i]);
+          zv[8 * q + 2 * i] = f.x;
+          zv[8 * q + 2 * i + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) zv[i] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int p = 32 * hf + i;
+      unsigned short xs;
+      asm volatile("ld.shared.u16 %0, [%1];" : "=h"(xs) : "r"(xt + sw128_off(p, t & 63)));
+      const float xv = __half2float(__ushort_as_half(xs));
+      const float yp = v[i] + Dh * xv;
+      const float gv = pr.nbg ? yp : yp * silu_fast(zv[i]);
+      ss_acc += gv * gv;
+      v[i] = gv;
+    }
+    tmem_st32(tmem + lane_off + col, v);
+  };
+
+  for (int j = 0; j < nh && ok; ++j) {
+    const int h = h0 + j;
+    // x_j: conv + SiLU of 64 channels x 128 tokens -> [64 p][128 s] K-major, fp16
+    {
+      const int cgp = tid >> 5, tr = tid & 31, s0 = tr * 4, p0 = cgp * 8;
+      float v[4][8];
+      conv8x4(a, bi, c0 + s0, (int64_t)h * kHP + p0, v);
+      const uint32_t xt = base + kXt + (j & 1) * 16384 + (s0 >> 6) * 8192;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        st_shared_v2(xt + sw128_off(p0 + i, s0 & 63), pack_half2(v[0][i], v[1][i]),
+                     pack_half2(v[2][i], v[3][i]));
+    }
+    // H_c of head h -> [64 p][64 n] K-major, fp16
+    {
+      const uint4 *src = reinterpret_cast<const uint4 *>(
+          a.Hc + ((bi * a.nch + c) * pr.H + h) * (int64_t)(kHP * kNS));
+      const uint32_t ht = base + kHt + (j & 1) * 8192;
+      for (int q = tid; q < 512; q += kThreads) {
+        const uint4 v = src[q];
+        st_shared_v4(ht + sw128_chunk(q >> 3, (q & 7) * 8), v.x, v.y, v.z, v.w);
+      }
+    }
+    // wait for CB (first head) or for the previous head's MMA (A buffer free)
+    ok = (j == 0) ? wait_all(&sh.mbar_cb, 0, ok) : wait_all(&sh.mbar_mma, (j - 1) & 1, ok);
+    if (!ok) break;
+    tc_fence_after();
+    // A_j = [CB o exp(cum_t - cum_s) dt_s for s <= t | C o exp(cum_t)] in fp16.
+    // The warp owns rows t in quarter q = warp % 4 and the 32-column groups
+    // k = 2 hf, 2 hf + 1.  Group k > q lies above the diagonal (zeros); group
+    // k < q lies below it, where exp(cum_t - cum_s) = exp(cum_t - cum_r)
+    // exp(cum_r - cum_s) with r = 32 k + 31 and s <= r < t, both factors <= 1
+    // (alpha per row, beta per column); the diagonal group k == q takes the
+    // exponential of each difference directly.
+    {
+      const int q = warp & 3;
+      const uint32_t at = base + kAt + hf * 16384;
+      const float c2t = sh.cum2[j][t];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const int k = 2 * hf + part, s0 = 32 * k;
+        if (k > q) {
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq)
+            st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), 0u, 0u, 0u, 0u);
+          continue;
+        }
+        float cb[32];
+        tmem_ld32(tmem + lane_off + s0, cb);
+        if (k < q) {
+          const float alpha = ex2_approx(c2t - sh.cum2[j][s0 + 31]);
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int sl = 8 * qq + 2 * e;
+              w4[e] = pack_half2(cb[sl] * alpha * sh.beta[j][s0 + sl],
+                                 cb[sl + 1] * alpha * sh.beta[j][s0 + sl + 1]);
+            }
+            st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+          }
+        } else {
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float val[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
+                val[u] = (s <= t) ? cb[sl] * ex2_approx(c2t - sh.cum2[j][s]) * sh.dt[j][s] : 0.0f;
+              }
+              w4[e] = pack_half2(val[0], val[1]);
+            }
+            st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+      }
+      // K block 2: C scaled by exp(cum_t); this half does n in [32 hf, 32 hf + 32)
+      const float ec = sh.ecum[j][t];
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        const int n0 = 32 * hf + 8 * qq;
+        const uint4 cv = ld_shared_v4(base + kCt + sw128_chunk(t, n0));
+        const uint32_t in[4] = {cv.x, cv.y, cv.z, cv.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_half2(in[e]);
+          o[e] = pack_half2(f.x * ec, f.y * ec);
+        }
+        st_shared_v4(base + kAt + 2 * 16384 + sw128_chunk(t, n0), o[0], o[1], o[2], o[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t idesc = umma_idesc_f16(128, 64);
+      const uint32_t xt = base + kXt + (j & 1) * 16384, ht = base + kHt + (j & 1) * 8192;
+      for (int ks = 0; ks < 12; ++ks) {
+        const int blk = ks >> 2, kin = ks & 3;
+        const uint64_t ad = umma_desc_sw128(base + kAt + blk * 16384 + kin * 32);
+        const uint64_t bd = blk < 2 ? umma_desc_sw128(xt + blk * 8192 + kin * 32)
+                                    : umma_desc_sw128(ht + kin * 32);
+        umma_f16(tmem + 128 + 64 * j, ad, bd, idesc, ks > 0 ? 1u : 0u);
+      }
+      umma_commit(&sh.mbar_mma);
+    }
+    if (j > 0) epilogue1(j - 1);  // overlaps the MMA of head j
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (ok && nh > 0) {
+    ok = wait_all(&sh.mbar_mma, (nh - 1) & 1, ok);
+    tc_fence_after();
+    if (ok) epilogue1(nh - 1);
+  }
+  if (!ok && tid == 0) {
+    // a wait ran out: let the MMAs already issued finish before TMEM is freed
+    mbar_wait_bounded(&sh.mbar_cb, 0, &g_tc_errors);
+  }
+
+  // per-token sums of squares of this CTA -> rank 0's table; totals; scale
+  sh.ss[hf][t] = ss_acc;
+  __syncthreads();
+  float *part0 = cluster.map_shared_rank(&sh.part[0][0], 0);
+  if (tid < kQ) part0[rank * kQ + tid] = sh.ss[0][tid] + sh.ss[1][tid];
+  cluster.sync();
+  if (tid < kQ) {
+    float tot = 0.0f;
+    for (int r = 0; r < cs; ++r) tot += part0[r * kQ + tid];
+    sh.inv[tid] = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (ok) {
+    const float sc = sh.inv[t];
+    for (int j = 0; j < nh; ++j) {
+      const int h = h0 + j;
+      float v[32];
+      tmem_ld32(tmem + lane_off + 128 + 64 * j + 32 * hf, v);
+      if (!t_valid) continue;
+      const float *nw = a.prm.norm_w + (int64_t)h * kHP + 32 * hf;
+      const int64_t row = (bi * pr.L + c0 + t);
+      if (pr.nbg) {
+        const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 32 * hf);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 raw = __ldg(zp + q);
+          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h2[i]);
+            v[8 * q + 2 * i] *= silu_fast(f.x);
+            v[8 * q + 2 * i + 1] *= silu_fast(f.y);
+          }
+        }
+      }
+      uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * pr.d_inner + (int64_t)h * kHP + 32 * hf);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 8 * q + 2 * e;
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i] * sc * __ldg(nw + i),
+                                                          v[i + 1] * sc * __ldg(nw + i + 1));
+          o[e] = *reinterpret_cast<const uint32_t *>(&b2);
+        }
+        dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+  cluster.sync();  // rank 0's table stays alive until every CTA has read it
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// Final conv state = last 4 raw inputs of [old state | new tokens], in place.
+__global__ void tc_conv_state_kernel(TcArgs a, __nv_bfloat16 *cs) {
+  const Problem &pr = a.pr;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= pr.batch * pr.conv_dim) return;
+  const int64_t bi = i / pr.conv_dim, ch = i % pr.conv_dim;
+  __nv_bfloat16 v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t tau = pr.L - 4 + k;
+    if (tau >= 0) v[k] = a.xBC[(bi * pr.L + tau) * a.ld_x + ch];
+    else v[k] = a.states_in ? cs[i * 4 + 4 + tau] : __float2bfloat16(0.0f);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) cs[i * 4 + k] = v[k];
+}
+
+// Heads per CTA and cluster size of tc_chunk_out for hpg heads per group.
+void out_split(int hpg, int *cs, int *hpc) {
+  const int lo = (hpg + kMaxHeadsPerCta - 1) / kMaxHeadsPerCta;
+  for (int c = lo; c <= 16; ++c)
+    if (hpg % c == 0) {
+      *cs = c;
+      *hpc = hpg / c;
+      return;
+    }
+  *cs = lo;
+  *hpc = (hpg + lo - 1) / lo;
+}
+
+struct TcWorkspace {
+  float *S, *cum_end;
+  __half *Hc;
+};
+
+TcWorkspace tc_carve(const Problem &pr, char *base) {
+  const int64_t nch = ceil_div(pr.L, kQ);
+  const size_t st = (size_t)pr.batch * nch * pr.H * kHP * kNS;
+  TcWorkspace w;
+  size_t off = 0;
+  w.S = reinterpret_cast<float *>(base + off);
+  off += align_up(st * 4, 256);
+  w.cum_end = reinterpret_cast<float *>(base + off);
+  off += align_up((size_t)pr.batch * nch * pr.H * 4, 256);
+  w.Hc = reinterpret_cast<__half *>(base + off);
+  return w;
+}
+
+constexpr size_t kK1Smem = 2 * kK1A + 2 * kK1B + 1024;
+constexpr size_t kK3Smem = kTcOutTiles + sizeof(OutShared) + 1024;
+
+}  // namespace
+
+const char *const kPrefillTcStages[] = {"tc_chunk_state", "tc_state_pass", "tc_chunk_out",
+                                        "tc_conv_state"};
+const int kPrefillTcStageCount = 4;
+
+bool prefill_tc_supported(const Problem &pr) {
+  return pr.io == MAMBA2_BF16 && pr.P == kHP && pr.N == kNS && pr.K == 4 &&
+         pr.heads_per_group() <= 16 * kMaxHeadsPerCta && pr.L > 0 &&
+         ceil_div(pr.L, kQ) <= 65535;
+}
+
+size_t prefill_tc_workspace(const Problem &pr) {
+  const int64_t nch = ceil_div(pr.L, kQ);
+  const size_t st = (size_t)pr.batch * nch * pr.H * kHP * kNS;
+  return align_up(st * 4, 256) + align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
+         align_up(st * 2, 256);
+}
+
+cudaError_t take_prefill_tc_errors(unsigned int *out) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_tc_errors, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_tc_errors, &zero, sizeof(zero));
+  *out = v;
+  return e;
+}
+
+cudaError_t prefill_tc(const PrefillArgs &pa) {
+  const Problem &pr = pa.pr;
+  cudaStream_t st = pa.stream;
+  TcArgs a;
+  a.pr = pr;
+  a.prm = pa.prm;
+  a.xBC = static_cast<const __nv_bfloat16 *>(pa.xBC);
+  a.ld_x = pa.ld_xbc;
+  a.z = static_cast<const __nv_bfloat16 *>(pa.z);
+  a.ld_z = pa.ld_z;
+  a.dt_raw = static_cast<const __nv_bfloat16 *>(pa.dt_raw);
+  a.ld_dt = pa.ld_dt;
+  a.y = static_cast<__nv_bfloat16 *>(pa.y);
+  a.conv_in = static_cast<const __nv_bfloat16 *>(pa.conv_state);
+  a.ssm_state = pa.ssm_state;
+  a.states_in = pa.states_in;
+  a.nch = (int)ceil_div(pr.L, kQ);
+  TcWorkspace w = tc_carve(pr, pa.ws);
+  a.S = w.S;
+  a.cum_end = w.cum_end;
+  a.Hc = w.Hc;
+  const int hpg = pr.heads_per_group();
+  int cs = 1, hpc = 1;
+  out_split(hpg, &cs, &hpc);
+  a.hpc = hpc;
+
+  cudaError_t e;
+  e = cudaFuncSetAttribute(tc_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kK1Smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kK3Smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
+
+  stage_mark(st, 0);
+  dim3 g1((unsigned)a.nch, (unsigned)(pr.G * ((hpg + 1) / 2)), (unsigned)pr.batch);
+  tc_chunk_state_kernel<<<g1, kThreads, kK1Smem, st>>>(a);
+  stage_mark(st, 1);
+  dim3 g2((kHP * kNS) / 256, (unsigned)pr.H, (unsigned)pr.batch);
+  tc_state_pass_kernel<<<g2, 256, 0, st>>>(a);
+  stage_mark(st, 2);
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cs, (unsigned)a.nch, (unsigned)(pr.G * pr.batch));
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kK3Smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a);
+    if (e != cudaSuccess) return e;
+  }
+  stage_mark(st, 3);
+  if (pa.conv_state != nullptr) {
+    const int64_t n = pr.batch * pr.conv_dim;
+    tc_conv_state_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(
+        a, static_cast<__nv_bfloat16 *>(pa.conv_state));
+  }
+  stage_mark(st, 4);
+  return cudaGetLastError();
+}
+
+}  // namespace m2

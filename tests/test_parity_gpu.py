@@ -37,6 +37,12 @@ def test_tiny_f32_config():
     case("zamba2_2p7b_prefill", batch=1, seqlen=333, nheads=4, chunk_size=64),
     case("zamba2_2p7b_prefill", batch=3, seqlen=129, nheads=6, ngroups=3, chunk_size=128),
     case("zamba2_2p7b_prefill", batch=2, seqlen=300, nheads=4, norm_before_gate=True),
+    # head splits of the tensor-core output kernel: odd heads per group (a lone head in
+    # the last pair), a cluster of 13 CTAs, an uneven 6/6/5 split, four CTAs of 4 heads
+    case("zamba2_2p7b_prefill", batch=1, seqlen=300, nheads=6, ngroups=2),
+    case("zamba2_2p7b_prefill", batch=1, seqlen=260, nheads=13),
+    case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=17),
+    case("zamba2_2p7b_prefill", batch=2, seqlen=256, nheads=32, ngroups=2),
     case("zamba2_2p7b_prefill", batch=1, seqlen=257, nheads=4, headdim=32, dstate=128),
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=4, headdim=16, dstate=32),
     case("tiny_f32", batch=2, seqlen=517, nheads=6, ngroups=2, headdim=64, dstate=64,
