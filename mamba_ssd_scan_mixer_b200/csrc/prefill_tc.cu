@@ -27,6 +27,8 @@
 // product uses a two-term fp16 split of both operands (hi*hi + hi*lo + lo*hi),
 // because the returned final state must hold 2e-2 of its RMS.
 #include <cooperative_groups.h>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 
@@ -63,12 +65,21 @@ struct TcArgs {
   float *S;                      // [b][nch][H][64][64] chunk states
   float *cum_end;                // [b][nch][H] chunk sum of dt*A
   __half *Hc;                    // [b][nch][H][64][64] state entering each chunk
+  __half *u;                     // [b][L][conv_dim] post-conv x | B | C, fp16
   int hpc;                       // max heads per CTA in tc_chunk_out
 };
 
-// silu with the fast reciprocal: __fdividef returns 0 once 1 + e^-v passes
-// 2^126, which is the limit silu(v) -> 0 for very negative v.
-__device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
+// silu(v) = v * sigmoid(v) with sigmoid(v) = (1 + tanh(v / 2)) / 2, using the
+// hardware tanh approximation (one special-function op per element).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float silu_fast(float v) {
+  const float h = 0.5f * v;
+  return fmaf(h, tanh_approx(h), h);
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -134,6 +145,23 @@ __device__ __forceinline__ void conv8x4(const TcArgs &a, int64_t bi, int64_t t0,
                         w[i][2] * rows[k + 2][i] + w[i][3] * rows[k + 3][i];
       out[k][i] = silu_fast(pre);
     }
+}
+
+// Post-conv activations of 8 channels x 4 tokens -> u (fp16), tokens < L only.
+__device__ __forceinline__ void store_u(const TcArgs &a, int64_t bi, int64_t t0, int64_t ch,
+                                        const float (&v)[4][8]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t t = t0 + k;
+    if (t < a.pr.L) {
+      uint4 o;
+      o.x = pack_half2(v[k][0], v[k][1]);
+      o.y = pack_half2(v[k][2], v[k][3]);
+      o.z = pack_half2(v[k][4], v[k][5]);
+      o.w = pack_half2(v[k][6], v[k][7]);
+      *reinterpret_cast<uint4 *>(a.u + (bi * a.pr.L + t) * a.pr.conv_dim + ch) = o;
+    }
+  }
 }
 
 __device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
@@ -217,16 +245,21 @@ __global__ void __launch_bounds__(kThreads) tc_chunk_state_kernel(TcArgs a) {
   }
   __syncthreads();
 
-  // conv + SiLU: 24 groups of 8 channels (x of head A, x of head B, B) x 32
-  // ranges of 4 tokens; results split into fp16 hi + lo operands.
-  for (int item = tid; item < 24 * 32; item += kThreads) {
+  // conv + SiLU: groups of 8 channels (x of head A, x of head B, B, and for the
+  // group's first pair also C) x 32 ranges of 4 tokens.  Post-conv values go
+  // to u (fp16) for the output kernel; x o w and B are split into fp16 hi + lo
+  // operands of the chunk-state product.
+  const int ncg = pair == 0 ? 32 : 24;
+  for (int item = tid; item < ncg * 32; item += kThreads) {
     const int cgp = item >> 5, tr = item & 31;
     const int s0 = tr * 4;
     uint32_t hi[8][2], lo[8][2];
     if (cgp < 16 && (cgp < 8 || hasB)) {
       const int half = cgp >> 3, p0 = (cgp & 7) * 8;
       float v[4][8];
-      conv8x4(a, bi, c0 + s0, (int64_t)(hA + half) * kHP + p0, v);
+      const int64_t ch = (int64_t)(hA + half) * kHP + p0;
+      conv8x4(a, bi, c0 + s0, ch, v);
+      store_u(a, bi, c0 + s0, ch, v);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float q[4], r[4];
@@ -257,10 +290,12 @@ __global__ void __launch_bounds__(kThreads) tc_chunk_state_kernel(TcArgs a) {
         st_shared_v2(sAhi + off, 0u, 0u);
         st_shared_v2(sAlo + off, 0u, 0u);
       }
-    } else {
+    } else if (cgp < 24) {
       const int n0 = (cgp - 16) * 8;
       float v[4][8];
-      conv8x4(a, bi, c0 + s0, pr.d_inner + (int64_t)g * kNS + n0, v);
+      const int64_t ch = pr.d_inner + (int64_t)g * kNS + n0;
+      conv8x4(a, bi, c0 + s0, ch, v);
+      if (pair == 0) store_u(a, bi, c0 + s0, ch, v);
       const int blk = s0 >> 6;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -274,6 +309,12 @@ __global__ void __launch_bounds__(kThreads) tc_chunk_state_kernel(TcArgs a) {
         st_shared_v2(sBhi + off, pack_half2(q[0], q[1]), pack_half2(q[2], q[3]));
         st_shared_v2(sBlo + off, pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
       }
+    } else {  // C channels (first pair of the group only): post-conv values to u
+      const int n0 = (cgp - 24) * 8;
+      float v[4][8];
+      const int64_t ch = pr.d_inner + (int64_t)(pr.G + g) * kNS + n0;
+      conv8x4(a, bi, c0 + s0, ch, v);
+      store_u(a, bi, c0 + s0, ch, v);
     }
   }
   fence_proxy_async_smem();
@@ -348,13 +389,17 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a) {
 }
 
 // ============================================================== chunk output
-// grid (cs, nch, G * b), cluster (cs, 1, 1); 256 threads.  Smem (1024-aligned):
-constexpr uint32_t kCt = 0;                      // C  [128 t][64 n]        16 KB
-constexpr uint32_t kBt = kCt + 16384;            // B  [128 s][64 n]        16 KB
-constexpr uint32_t kXt = kBt + 16384;            // x  2 x [2][64 p][64 s]  2 x 16 KB
-constexpr uint32_t kHt = kXt + 2 * 16384;        // Hc 2 x [64 p][64 n]     2 x 8 KB
-constexpr uint32_t kAt = kHt + 2 * 8192;         // A  [3][128 t][64 k]     48 KB
-constexpr uint32_t kTcOutTiles = kAt + 3 * 16384;  // 128 KB
+// grid (cs, nch, G * b), cluster (cs, 1, 1); 8 compute warps + 1 TMA producer
+// warp.  Tiles arrive by TMA in 128-byte-swizzled layouts (1024-aligned):
+constexpr uint32_t kCt = 0;                      // C   [128 t][64 n] fp16     16 KB (u)
+constexpr uint32_t kBt = kCt + 16384;            // B   [128 s][64 n] fp16     16 KB (u)
+constexpr uint32_t kXt = kBt + 16384;            // x   2 x [128 s][64 p] fp16 2 x 16 KB (u)
+constexpr uint32_t kHt = kXt + 2 * 16384;        // H_c 2 x [64 p][64 n] fp16  2 x 8 KB
+constexpr uint32_t kZt = kHt + 2 * 8192;         // z   2 x [128 t][64 p] bf16 2 x 16 KB
+constexpr uint32_t kAt = kZt + 2 * 16384;        // A   [3][128 t][64 k] fp16  48 KB
+constexpr uint32_t kTcOutTiles = kAt + 3 * 16384;  // 160 KB
+constexpr int kOutThreads = kThreads + 32;       // + producer warp
+constexpr uint32_t kHeadBytes = 16384 + 8192 + 16384;  // x + H_c + z per head
 
 struct OutShared {
   float cum2[kMaxHeadsPerCta][kQ];  // cumsum * log2(e)
@@ -364,12 +409,66 @@ struct OutShared {
   float ss[2][kQ];
   float part[16][kQ];               // per-rank partial sums of squares (rank 0's is read)
   float inv[kQ];
-  float scan[8];
-  uint64_t mbar_cb, mbar_mma;
+  uint64_t full_cb, full[2], empty[2], mbar_cb, mbar_mma;
   uint32_t tmem_holder;
+  int ok_flag;
 };
 
-__global__ void __launch_bounds__(kThreads) tc_chunk_out_kernel(TcArgs a) {
+struct OutMaps {
+  CUtensorMap u;   // [b][L][conv_dim] fp16, box 64 ch x 128 tokens
+  CUtensorMap z;   // [b][L][d_inner] bf16 (row stride ld_z), box 64 x 128
+  CUtensorMap hc;  // [rows][64] fp16, box 64 x 64
+};
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// barrier over the 256 compute threads only (the producer warp never joins)
+__device__ __forceinline__ void compute_sync() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+__device__ __forceinline__ bool compute_all(bool v) {
+  int r;
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.and.pred q, 1, 256, p;\n"
+               " selp.s32 %0, 1, 0, q;\n}"
+               : "=r"(r)
+               : "r"((int)v)
+               : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool wait_compute(uint64_t *bar, uint32_t parity, bool ok) {
+  const bool got = ok ? mbar_wait_bounded(bar, parity, &g_tc_errors) : false;
+  return compute_all(got);
+}
+// Smem descriptor for an MN-major SW128 operand: 8-row (K) atoms of 64
+// elements (N) x 128 B, K atoms 1024 B apart (SBO), N atoms `lbo` apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+__global__ void __launch_bounds__(kOutThreads, 1)
+    tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = (int)cluster.num_blocks();
@@ -390,247 +489,233 @@ __global__ void __launch_bounds__(kThreads) tc_chunk_out_kernel(TcArgs a) {
 
   if (warp == 0) tmem_alloc(&sh.tmem_holder, 512);
   if (tid == 0) {
+    mbar_init(&sh.full_cb, 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&sh.full[k], 1);
+      mbar_init(&sh.empty[k], 1);
+    }
     mbar_init(&sh.mbar_cb, 1);
     mbar_init(&sh.mbar_mma, 1);
     fence_mbar_init();
   }
-
-  // dt / cumsum for the CTA's heads: one warp per head, 4 consecutive tokens
-  // per lane.  beta_s = exp(cum_r - cum_s) dt_s with r the last token of the
-  // 32-token group of s (the column factor of the masked decay, see below).
-  if (warp < nh) {
-    const int j = warp, h = h0 + j;
-    float dt4[4], a4[4];
-    const float dtb = a.prm.dt_bias[h], Ah = a.prm.A[h];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t tt = c0 + 4 * lane + k;
-      dt4[k] = tt < pr.L ? softplus_f(__bfloat162float(a.dt_raw[(bi * pr.L + tt) * a.ld_dt + h]) + dtb)
-                         : 0.0f;
-      a4[k] = dt4[k] * Ah;
-    }
-    const float tot = a4[0] + a4[1] + a4[2] + a4[3];
-    float run = warp_scan(tot, lane) - tot;  // exclusive prefix of this lane's 4 tokens
-    float c2[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      run += a4[k];
-      c2[k] = run * kLog2e;
-      sh.cum2[j][4 * lane + k] = c2[k];
-      sh.dt[j][4 * lane + k] = dt4[k];
-      sh.ecum[j][4 * lane + k] = ex2_approx(c2[k]);
-    }
-    // the group of 32 tokens ends at lane 8*(lane/8) + 7, token 4*that + 3
-    const float c2r = __shfl_sync(0xffffffffu, c2[3], (lane | 7));
-#pragma unroll
-    for (int k = 0; k < 4; ++k) sh.beta[j][4 * lane + k] = ex2_approx(c2r - c2[k]) * dt4[k];
-  }
-
-  // conv + SiLU of the group's B and C channels: 16 groups of 8 x 32 ranges of 4
-  for (int item = tid; item < 16 * 32; item += kThreads) {
-    const int cgp = item >> 5, tr = item & 31, s0 = tr * 4;
-    const bool isC = cgp >= 8;
-    const int n0 = (cgp & 7) * 8;
-    float v[4][8];
-    conv8x4(a, bi, c0 + s0, pr.d_inner + (int64_t)(isC ? pr.G : 0) * kNS + (int64_t)g * kNS + n0,
-            v);
-    const uint32_t tile = base + (isC ? kCt : kBt);
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      st_shared_v4(tile + sw128_chunk(s0 + k, n0), pack_half2(v[k][0], v[k][1]),
-                   pack_half2(v[k][2], v[k][3]), pack_half2(v[k][4], v[k][5]),
-                   pack_half2(v[k][6], v[k][7]));
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_holder;
-  if (tid == 0) {  // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
-    const uint32_t idesc = umma_idesc_f16(128, 128);
-    for (int kin = 0; kin < 4; ++kin)
-      umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32), umma_desc_sw128(base + kBt + kin * 32),
-               idesc, kin > 0 ? 1u : 0u);
-    umma_commit(&sh.mbar_cb);
-  }
 
-  // this thread's TMEM lane (row t) and column half
-  const int t = 32 * (warp & 3) + lane, hf = warp >> 2;
-  const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-  const bool t_valid = c0 + t < pr.L;
-  float ss_acc = 0.0f;
-  bool ok = true;
-
-  // per-head epilogue, part 1: y_pre = Y + D x, gate, sum of squares; g -> TMEM
-  auto epilogue1 = [&](int j) {
-    const int h = h0 + j;
-    float v[32];
-    const uint32_t col = 128 + 64 * j + 32 * hf;
-    tmem_ld32(tmem + lane_off + col, v);
-    const float Dh = a.prm.D[h];
-    const uint32_t xt = base + kXt + (j & 1) * 16384 + (t >> 6) * 8192;
-    float zv[32];
-    if (t_valid) {
-      const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (bi * pr.L + c0 + t) * a.ld_z +
-                                                        (int64_t)h * kHP + 32 * hf);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 raw = __ldg(zp + q);
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(h2[i]);
-          zv[8 * q + 2 * i] = f.x;
-          zv[8 * q + 2 * i + 1] = f.y;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) zv[i] = 0.0f;
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int p = 32 * hf + i;
-      unsigned short xs;
-      asm volatile("ld.shared.u16 %0, [%1];" : "=h"(xs) : "r"(xt + sw128_off(p, t & 63)));
-      const float xv = __half2float(__ushort_as_half(xs));
-      const float yp = v[i] + Dh * xv;
-      const float gv = pr.nbg ? yp : yp * silu_fast(zv[i]);
-      ss_acc += gv * gv;
-      v[i] = gv;
-    }
-    tmem_st32(tmem + lane_off + col, v);
-  };
-
-  for (int j = 0; j < nh && ok; ++j) {
-    const int h = h0 + j;
-    // x_j: conv + SiLU of 64 channels x 128 tokens -> [64 p][128 s] K-major, fp16
-    {
-      const int cgp = tid >> 5, tr = tid & 31, s0 = tr * 4, p0 = cgp * 8;
-      float v[4][8];
-      conv8x4(a, bi, c0 + s0, (int64_t)h * kHP + p0, v);
-      const uint32_t xt = base + kXt + (j & 1) * 16384 + (s0 >> 6) * 8192;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        st_shared_v2(xt + sw128_off(p0 + i, s0 & 63), pack_half2(v[0][i], v[1][i]),
-                     pack_half2(v[2][i], v[3][i]));
-    }
-    // H_c of head h -> [64 p][64 n] K-major, fp16
-    {
-      const uint4 *src = reinterpret_cast<const uint4 *>(
-          a.Hc + ((bi * a.nch + c) * pr.H + h) * (int64_t)(kHP * kNS));
-      const uint32_t ht = base + kHt + (j & 1) * 8192;
-      for (int q = tid; q < 512; q += kThreads) {
-        const uint4 v = src[q];
-        st_shared_v4(ht + sw128_chunk(q >> 3, (q & 7) * 8), v.x, v.y, v.z, v.w);
+  if (warp == kThreads / 32) {
+    // ---------------- producer: C, B tiles, then x, H_c, z of each head
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sh.full_cb, 2 * 16384);
+      tma_load_3d(base + kCt, &maps.u, (int)(pr.d_inner + (int64_t)(pr.G + g) * kNS), (int)c0,
+                  (int)bi, &sh.full_cb);
+      tma_load_3d(base + kBt, &maps.u, (int)(pr.d_inner + (int64_t)g * kNS), (int)c0, (int)bi,
+                  &sh.full_cb);
+      for (int j = 0; j < nh; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait_bounded(&sh.empty[st], (uint32_t)(((j >> 1) - 1) & 1),
+                                         &g_tc_errors))
+          break;
+        const int h = h0 + j;
+        mbar_arrive_expect_tx(&sh.full[st], kHeadBytes);
+        tma_load_3d(base + kXt + st * 16384, &maps.u, h * kHP, (int)c0, (int)bi, &sh.full[st]);
+        tma_load_2d(base + kHt + st * 8192, &maps.hc, 0,
+                    (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full[st]);
+        tma_load_3d(base + kZt + st * 16384, &maps.z, h * kHP, (int)c0, (int)bi, &sh.full[st]);
       }
     }
-    // wait for CB (first head) or for the previous head's MMA (A buffer free)
-    ok = (j == 0) ? wait_all(&sh.mbar_cb, 0, ok) : wait_all(&sh.mbar_mma, (j - 1) & 1, ok);
-    if (!ok) break;
+  } else {
+    // ---------------- compute warps
+    // dt / cumsum: one warp per head, 4 consecutive tokens per lane
+    if (warp < nh) {
+      const int j = warp, h = h0 + j;
+      float dt4[4], a4[4];
+      const float dtb = a.prm.dt_bias[h], Ah = a.prm.A[h];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t tt = c0 + 4 * lane + k;
+        dt4[k] = tt < pr.L ? softplus_f(__bfloat162float(a.dt_raw[(bi * pr.L + tt) * a.ld_dt + h]) +
+                                        dtb)
+                           : 0.0f;
+        a4[k] = dt4[k] * Ah;
+      }
+      const float tot = a4[0] + a4[1] + a4[2] + a4[3];
+      float run = warp_scan(tot, lane) - tot;
+      float c2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        run += a4[k];
+        c2[k] = run * kLog2e;
+        sh.cum2[j][4 * lane + k] = c2[k];
+        sh.dt[j][4 * lane + k] = dt4[k];
+        sh.ecum[j][4 * lane + k] = ex2_approx(c2[k]);
+      }
+      const float c2r = __shfl_sync(0xffffffffu, c2[3], (lane | 7));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sh.beta[j][4 * lane + k] = ex2_approx(c2r - c2[k]) * dt4[k];
+    }
+    bool ok = wait_compute(&sh.full_cb, 0, true);
     tc_fence_after();
-    // A_j = [CB o exp(cum_t - cum_s) dt_s for s <= t | C o exp(cum_t)] in fp16.
-    // The warp owns rows t in quarter q = warp % 4 and the 32-column groups
-    // k = 2 hf, 2 hf + 1.  Group k > q lies above the diagonal (zeros); group
-    // k < q lies below it, where exp(cum_t - cum_s) = exp(cum_t - cum_r)
-    // exp(cum_r - cum_s) with r = 32 k + 31 and s <= r < t, both factors <= 1
-    // (alpha per row, beta per column); the diagonal group k == q takes the
-    // exponential of each difference directly.
-    {
-      const int q = warp & 3;
-      const uint32_t at = base + kAt + hf * 16384;
-      const float c2t = sh.cum2[j][t];
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const int k = 2 * hf + part, s0 = 32 * k;
-        if (k > q) {
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq)
-            st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), 0u, 0u, 0u, 0u);
-          continue;
-        }
-        float cb[32];
-        tmem_ld32(tmem + lane_off + s0, cb);
-        if (k < q) {
-          const float alpha = ex2_approx(c2t - sh.cum2[j][s0 + 31]);
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int sl = 8 * qq + 2 * e;
-              w4[e] = pack_half2(cb[sl] * alpha * sh.beta[j][s0 + sl],
-                                 cb[sl + 1] * alpha * sh.beta[j][s0 + sl + 1]);
-            }
-            st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
-          }
-        } else {
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float val[2];
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
-                val[u] = (s <= t) ? cb[sl] * ex2_approx(c2t - sh.cum2[j][s]) * sh.dt[j][s] : 0.0f;
-              }
-              w4[e] = pack_half2(val[0], val[1]);
-            }
-            st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
-          }
-        }
-      }
-      // K block 2: C scaled by exp(cum_t); this half does n in [32 hf, 32 hf + 32)
-      const float ec = sh.ecum[j][t];
-#pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        const int n0 = 32 * hf + 8 * qq;
-        const uint4 cv = ld_shared_v4(base + kCt + sw128_chunk(t, n0));
-        const uint32_t in[4] = {cv.x, cv.y, cv.z, cv.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack_half2(in[e]);
-          o[e] = pack_half2(f.x * ec, f.y * ec);
-        }
-        st_shared_v4(base + kAt + 2 * 16384 + sw128_chunk(t, n0), o[0], o[1], o[2], o[3]);
-      }
+    if (ok && tid == 0) {  // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
+      const uint32_t idesc = umma_idesc_f16(128, 128);
+      for (int kin = 0; kin < 4; ++kin)
+        umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32),
+                 umma_desc_sw128(base + kBt + kin * 32), idesc, kin > 0 ? 1u : 0u);
+      umma_commit(&sh.mbar_cb);
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
+
+    const int t = 32 * (warp & 3) + lane, hf = warp >> 2, q = warp & 3;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    float ss_acc = 0.0f;
+
+    // epilogue, part 1: gate with silu(z) (z tile in smem), sum of squares, g -> TMEM
+    auto epilogue1 = [&](int j) {
+      float v[32];
+      const uint32_t col = 128 + 64 * j + 32 * hf;
+      tmem_ld32(tmem + lane_off + col, v);
+      if (!pr.nbg) {
+        const uint32_t zt = base + kZt + (j & 1) * 16384;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const uint4 raw = ld_shared_v4(zt + sw128_chunk(t, 32 * hf + 8 * qq));
+          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h2[i]);
+            v[8 * qq + 2 * i] *= silu_fast(f.x);
+            v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss_acc = fmaf(v[i], v[i], ss_acc);
+      if (!pr.nbg) tmem_st32(tmem + lane_off + col, v);
+    };
+
+    for (int j = 0; j < nh && ok; ++j) {
+      const int h = h0 + j;
+      ok = wait_compute(&sh.full[j & 1], (uint32_t)((j >> 1) & 1), ok);
+      ok = (j == 0) ? wait_compute(&sh.mbar_cb, 0, ok) : wait_compute(&sh.mbar_mma, (j - 1) & 1, ok);
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t idesc = umma_idesc_f16(128, 64);
-      const uint32_t xt = base + kXt + (j & 1) * 16384, ht = base + kHt + (j & 1) * 8192;
-      for (int ks = 0; ks < 12; ++ks) {
-        const int blk = ks >> 2, kin = ks & 3;
-        const uint64_t ad = umma_desc_sw128(base + kAt + blk * 16384 + kin * 32);
-        const uint64_t bd = blk < 2 ? umma_desc_sw128(xt + blk * 8192 + kin * 32)
-                                    : umma_desc_sw128(ht + kin * 32);
-        umma_f16(tmem + 128 + 64 * j, ad, bd, idesc, ks > 0 ? 1u : 0u);
+      // A_j = [CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal | C o exp(cum_t)];
+      // 32-column groups k above the row quarter q are zero, below it the decay
+      // factorises as alpha_t beta_s (both <= 1), on it exponentials are direct.
+      {
+        const uint32_t at = base + kAt + hf * 16384;
+        const float c2t = sh.cum2[j][t];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const int k = 2 * hf + part, s0 = 32 * k;
+          if (k > q) {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+              st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), 0u, 0u, 0u, 0u);
+            continue;
+          }
+          float cb[32];
+          tmem_ld32(tmem + lane_off + s0, cb);
+          if (k < q) {
+            const float alpha = ex2_approx(c2t - sh.cum2[j][s0 + 31]);
+            const float4 *b4 = reinterpret_cast<const float4 *>(&sh.beta[j][s0]);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const float4 bA = b4[2 * qq], bB = b4[2 * qq + 1];
+              const float bb[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+              uint32_t w4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int sl = 8 * qq + 2 * e;
+                w4[e] = pack_half2(cb[sl] * alpha * bb[2 * e], cb[sl + 1] * alpha * bb[2 * e + 1]);
+              }
+              st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+            }
+          } else {
+            const float Dh = a.prm.D[h];
+            const float4 *c4 = reinterpret_cast<const float4 *>(&sh.cum2[j][s0]);
+            const float4 *d4 = reinterpret_cast<const float4 *>(&sh.dt[j][s0]);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const float4 cA = c4[2 * qq], cB = c4[2 * qq + 1];
+              const float4 dA = d4[2 * qq], dB = d4[2 * qq + 1];
+              const float cc[8] = {cA.x, cA.y, cA.z, cA.w, cB.x, cB.y, cB.z, cB.w};
+              const float dd[8] = {dA.x, dA.y, dA.z, dA.w, dB.x, dB.y, dB.z, dB.w};
+              uint32_t w4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float val[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
+                  float vv = cb[sl] * ex2_approx(fminf(c2t - cc[2 * e + u], 0.0f)) * dd[2 * e + u];
+                  if (s == t) vv += Dh;
+                  val[u] = (s <= t) ? vv : 0.0f;
+                }
+                w4[e] = pack_half2(val[0], val[1]);
+              }
+              st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+            }
+          }
+        }
+        const float ec = sh.ecum[j][t];
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const int n0 = 32 * hf + 8 * qq;
+          const uint4 cv = ld_shared_v4(base + kCt + sw128_chunk(t, n0));
+          const uint32_t in[4] = {cv.x, cv.y, cv.z, cv.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_half2(in[e]);
+            o[e] = pack_half2(f.x * ec, f.y * ec);
+          }
+          st_shared_v4(base + kAt + 2 * 16384 + sw128_chunk(t, n0), o[0], o[1], o[2], o[3]);
+        }
       }
-      umma_commit(&sh.mbar_mma);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      compute_sync();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc_k = umma_idesc_f16(128, 64);
+        const uint32_t idesc_mn = idesc_k | (1u << 16);  // B operand MN-major (x tile)
+        const uint32_t xt = base + kXt + (j & 1) * 16384, ht = base + kHt + (j & 1) * 8192;
+        for (int ks = 0; ks < 12; ++ks) {
+          const int blk = ks >> 2, kin = ks & 3;
+          const uint64_t ad = umma_desc_sw128(base + kAt + blk * 16384 + kin * 32);
+          if (ks < 8)
+            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn,
+                     ks > 0 ? 1u : 0u);
+          else
+            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128(ht + kin * 32), idesc_k, 1u);
+        }
+        umma_commit(&sh.mbar_mma);
+      }
+      if (j > 0) {
+        epilogue1(j - 1);  // overlaps the MMA of head j
+        compute_sync();
+        if (tid == 0) mbar_arrive(&sh.empty[(j - 1) & 1]);
+      }
+      tc_fence_before();
+      compute_sync();
     }
-    if (j > 0) epilogue1(j - 1);  // overlaps the MMA of head j
-    tc_fence_before();
-    __syncthreads();
+    if (ok && nh > 0) {
+      ok = wait_compute(&sh.mbar_mma, (nh - 1) & 1, ok);
+      tc_fence_after();
+      if (ok) epilogue1(nh - 1);
+    }
+    if (!ok && tid == 0) {
+      // a wait ran out: let issued MMAs and tile copies land before the CTA exits
+      mbar_wait_bounded(&sh.mbar_cb, 0, &g_tc_errors);
+      mbar_wait_bounded(&sh.full_cb, 0, &g_tc_errors);
+      for (int k = 0; k < 2; ++k) mbar_wait_bounded(&sh.full[k], 0, &g_tc_errors);
+    }
+    sh.ss[hf][t] = ss_acc;
+    sh.ok_flag = ok;
   }
-  if (ok && nh > 0) {
-    ok = wait_all(&sh.mbar_mma, (nh - 1) & 1, ok);
-    tc_fence_after();
-    if (ok) epilogue1(nh - 1);
-  }
-  if (!ok && tid == 0) {
-    // a wait ran out: let the MMAs already issued finish before TMEM is freed
-    mbar_wait_bounded(&sh.mbar_cb, 0, &g_tc_errors);
-  }
+  __syncthreads();  // producer joins here
 
   // per-token sums of squares of this CTA -> rank 0's table; totals; scale
-  sh.ss[hf][t] = ss_acc;
-  __syncthreads();
   float *part0 = cluster.map_shared_rank(&sh.part[0][0], 0);
   if (tid < kQ) part0[rank * kQ + tid] = sh.ss[0][tid] + sh.ss[1][tid];
   cluster.sync();
@@ -641,7 +726,10 @@ __global__ void __launch_bounds__(kThreads) tc_chunk_out_kernel(TcArgs a) {
   }
   __syncthreads();
   tc_fence_after();
-  if (ok) {
+  if (sh.ok_flag && warp < kThreads / 32) {
+    const int t = 32 * (warp & 3) + lane, hf = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const bool t_valid = c0 + t < pr.L;
     const float sc = sh.inv[t];
     for (int j = 0; j < nh; ++j) {
       const int h = h0 + j;
@@ -649,33 +737,34 @@ __global__ void __launch_bounds__(kThreads) tc_chunk_out_kernel(TcArgs a) {
       tmem_ld32(tmem + lane_off + 128 + 64 * j + 32 * hf, v);
       if (!t_valid) continue;
       const float *nw = a.prm.norm_w + (int64_t)h * kHP + 32 * hf;
-      const int64_t row = (bi * pr.L + c0 + t);
+      const int64_t row = bi * pr.L + c0 + t;
       if (pr.nbg) {
-        const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 32 * hf);
+        const uint4 *zp =
+            reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 32 * hf);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 raw = __ldg(zp + q);
+        for (int qq = 0; qq < 4; ++qq) {
+          const uint4 raw = __ldg(zp + qq);
           const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 f = __bfloat1622float2(h2[i]);
-            v[8 * q + 2 * i] *= silu_fast(f.x);
-            v[8 * q + 2 * i + 1] *= silu_fast(f.y);
+            v[8 * qq + 2 * i] *= silu_fast(f.x);
+            v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
           }
         }
       }
       uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * pr.d_inner + (int64_t)h * kHP + 32 * hf);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int qq = 0; qq < 4; ++qq) {
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i = 8 * q + 2 * e;
+          const int i = 8 * qq + 2 * e;
           const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i] * sc * __ldg(nw + i),
                                                           v[i + 1] * sc * __ldg(nw + i + 1));
           o[e] = *reinterpret_cast<const uint32_t *>(&b2);
         }
-        dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[qq] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
   }
@@ -717,7 +806,7 @@ void out_split(int hpg, int *cs, int *hpc) {
 
 struct TcWorkspace {
   float *S, *cum_end;
-  __half *Hc;
+  __half *Hc, *u;
 };
 
 TcWorkspace tc_carve(const Problem &pr, char *base) {
@@ -730,7 +819,42 @@ TcWorkspace tc_carve(const Problem &pr, char *base) {
   w.cum_end = reinterpret_cast<float *>(base + off);
   off += align_up((size_t)pr.batch * nch * pr.H * 4, 256);
   w.Hc = reinterpret_cast<__half *>(base + off);
+  off += align_up(st * 2, 256);
+  w.u = reinterpret_cast<__half *>(base + off);
   return w;
+}
+
+// cuTensorMapEncodeTiled, fetched once through the runtime (no libcuda link-time dependency).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 3-D (channel, token, batch) or 2-D (column, row) map of a 16-bit array with
+// 128-byte swizzle; out-of-range boxes read zeros.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank,
+              const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t d[3], st[2];
+  cuuint32_t b[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
+  return enc(m, dt, (cuuint32_t)rank, const_cast<void *>(base), d, st, b, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 constexpr size_t kK1Smem = 2 * kK1A + 2 * kK1B + 1024;
@@ -743,16 +867,17 @@ const char *const kPrefillTcStages[] = {"tc_chunk_state", "tc_state_pass", "tc_c
 const int kPrefillTcStageCount = 4;
 
 bool prefill_tc_supported(const Problem &pr) {
+  const int64_t nch = ceil_div(pr.L, kQ);
   return pr.io == MAMBA2_BF16 && pr.P == kHP && pr.N == kNS && pr.K == 4 &&
-         pr.heads_per_group() <= 16 * kMaxHeadsPerCta && pr.L > 0 &&
-         ceil_div(pr.L, kQ) <= 65535;
+         pr.heads_per_group() <= 16 * kMaxHeadsPerCta && pr.L > 0 && nch <= 65535 &&
+         pr.L < ((int64_t)1 << 31) && pr.batch * nch * pr.H * kHP < ((int64_t)1 << 31);
 }
 
 size_t prefill_tc_workspace(const Problem &pr) {
   const int64_t nch = ceil_div(pr.L, kQ);
   const size_t st = (size_t)pr.batch * nch * pr.H * kHP * kNS;
   return align_up(st * 4, 256) + align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
-         align_up(st * 2, 256);
+         align_up(st * 2, 256) + align_up((size_t)pr.batch * pr.L * pr.conv_dim * 2, 256);
 }
 
 cudaError_t take_prefill_tc_errors(unsigned int *out) {
@@ -784,6 +909,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.S = w.S;
   a.cum_end = w.cum_end;
   a.Hc = w.Hc;
+  a.u = w.u;
   const int hpg = pr.heads_per_group();
   int cs = 1, hpc = 1;
   out_split(hpg, &cs, &hpc);
@@ -809,7 +935,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cs, (unsigned)a.nch, (unsigned)(pr.G * pr.batch));
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kOutThreads, 1, 1);
     cfg.dynamicSmemBytes = kK3Smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -819,7 +945,22 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a);
+    OutMaps maps;
+    {
+      const uint64_t du[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
+      const uint64_t su[2] = {(uint64_t)pr.conv_dim * 2, (uint64_t)pr.L * pr.conv_dim * 2};
+      const uint32_t bu[3] = {64, kQ, 1};
+      const uint64_t dz[3] = {(uint64_t)pr.d_inner, (uint64_t)pr.L, (uint64_t)pr.batch};
+      const uint64_t sz[2] = {(uint64_t)pa.ld_z * 2, (uint64_t)pr.L * pa.ld_z * 2};
+      const uint64_t dh[2] = {(uint64_t)kNS, (uint64_t)pr.batch * a.nch * pr.H * kHP};
+      const uint64_t shc[1] = {(uint64_t)kNS * 2};
+      const uint32_t bh[2] = {64, 64};
+      if (!make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.u, 3, du, su, bu) ||
+          !make_map(&maps.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.z, 3, dz, sz, bu) ||
+          !make_map(&maps.hc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Hc, 2, dh, shc, bh))
+        return cudaErrorInvalidValue;
+    }
+    e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps);
     if (e != cudaSuccess) return e;
   }
   stage_mark(st, 3);
