@@ -40,7 +40,8 @@ namespace m2 {
 namespace {
 
 constexpr int kQ = 128;          // tokens per chunk = MMA M
-constexpr int kThreads = 256;    // 8 warps
+constexpr int kThreads = 512;    // 16 compute warps
+constexpr int kOutThreads = kThreads + 32;  // + one TMA producer warp
 constexpr int kHP = 64;          // headdim
 constexpr int kNS = 64;          // d_state
 constexpr int kMaxHeadsPerCta = 6;  // TMEM: 128 (CB) + 6 x 64 (y) <= 512 columns
@@ -97,56 +98,6 @@ __device__ __forceinline__ float warp_scan(float v, int lane) {
   return v;
 }
 
-// 8 consecutive bf16 channels of raw input token `tau` (sequence row bi): the
-// token itself for 0 <= tau < L, the carried conv state for tau < 0 when
-// states_in, zeros otherwise (left padding, or past the end of the sequence).
-__device__ __forceinline__ void load_row8(const TcArgs &a, int64_t bi, int64_t tau, int64_t ch,
-                                          float (&v)[8]) {
-  if (tau >= 0 && tau < a.pr.L) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(a.xBC + (bi * a.pr.L + tau) * a.ld_x + ch));
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h[i]);
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
-    }
-  } else if (tau < 0 && a.states_in) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      v[i] = __bfloat162float(a.conv_in[(bi * a.pr.conv_dim + ch + i) * 4 + 4 + tau]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-  }
-}
-
-// conv1d + SiLU of 8 channels [ch, ch+8) for 4 tokens t0..t0+3 (absolute).
-__device__ __forceinline__ void conv8x4(const TcArgs &a, int64_t bi, int64_t t0, int64_t ch,
-                                        float (&out)[4][8]) {
-  float w[8][4], bias[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 wv = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch + i);
-    w[i][0] = wv.x;
-    w[i][1] = wv.y;
-    w[i][2] = wv.z;
-    w[i][3] = wv.w;
-    bias[i] = __ldg(a.prm.conv_b + ch + i);
-  }
-  float rows[7][8];
-#pragma unroll
-  for (int r = 0; r < 7; ++r) load_row8(a, bi, t0 - 3 + r, ch, rows[r]);
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float pre = bias[i] + w[i][0] * rows[k][i] + w[i][1] * rows[k + 1][i] +
-                        w[i][2] * rows[k + 2][i] + w[i][3] * rows[k + 3][i];
-      out[k][i] = silu_fast(pre);
-    }
-}
-
 // Post-conv activations of 8 channels x 4 tokens -> u (fp16), tokens < L only.
 __device__ __forceinline__ void store_u(const TcArgs &a, int64_t bi, int64_t t0, int64_t ch,
                                         const float (&v)[4][8]) {
@@ -181,172 +132,345 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
-// Block-uniform bounded wait on an mbarrier phase.
-__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, bool ok) {
-  bool got = ok ? mbar_wait_bounded(bar, parity, &g_tc_errors) : false;
-  return __syncthreads_and(got) != 0;
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// barrier over the 512 compute threads only (the producer warp never joins)
+__device__ __forceinline__ void compute_sync() {
+  asm volatile("bar.sync 1, 512;" ::: "memory");
+}
+__device__ __forceinline__ bool compute_all(bool v) {
+  int r;
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.and.pred q, 1, 512, p;\n"
+               " selp.s32 %0, 1, 0, q;\n}"
+               : "=r"(r)
+               : "r"((int)v)
+               : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool wait_compute(uint64_t *bar, uint32_t parity, bool ok) {
+  const bool got = ok ? mbar_wait_bounded(bar, parity, &g_tc_errors) : false;
+  return compute_all(got);
+}
+// Smem descriptor for an MN-major SW128 operand: 8-row (K) atoms of 64
+// elements (N) x 128 B, K atoms 1024 B apart (SBO), N atoms `lbo` apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
 }
 
 // ============================================================== chunk states
-// grid (nch, G * pairs_per_group, b); 256 threads.  Smem (1024-aligned):
-// A_hi, A_lo [2 k-blocks][128 rows][128 B]; B_hi, B_lo [2][64][128 B].
+// Persistent: grid = one CTA per SM, each looping over work items (chunk-major):
+//   pair items (b, chunk, group, head pair): conv + SiLU of x (2 heads) and B,
+//     post-conv values to u, then S = (x o w)^T B on the tensor cores;
+//   C items (b, chunk, group): conv + SiLU of the group's C channels -> u.
+// 16 compute warps + 1 producer warp.  The producer computes dt / the chunk
+// weights of the next item and TMA-loads its raw bf16 tiles [136 tokens
+// c0-3 .. c0+132][64 ch] (128-byte swizzle) into a two-stage ring while the
+// compute warps work on the current item.
+// Smem (1024-aligned): ring [2][x_A | x_B | B (a C item uses slot 0)], then the
+// operands A_hi, A_lo [2 k-blocks][128 rows][128 B] and B_hi, B_lo [2][64][128 B].
+constexpr uint32_t kRawRows = 136, kRawBytes = kRawRows * 128;  // 17 KB, 1024-multiple
+constexpr uint32_t kK1Stage = 3 * kRawBytes;
 constexpr uint32_t kK1A = 2 * 128 * 128, kK1B = 2 * 64 * 128;
+constexpr uint32_t kK1Ahi = 2 * kK1Stage, kK1Alo = kK1Ahi + kK1A, kK1Bhi = kK1Alo + kK1A,
+                   kK1Blo = kK1Bhi + kK1B, kK1Tiles = kK1Blo + kK1B;
 
-__global__ void __launch_bounds__(kThreads) tc_chunk_state_kernel(TcArgs a) {
+struct K1Maps {
+  CUtensorMap xbc;  // [b][L][conv_dim] bf16 (row stride ld_x), box 64 ch x 136 tokens
+};
+
+// conv1d + SiLU of the 8 channels in 16-byte column `cg` of a raw tile, for
+// output tokens at tile rows s0+3 .. s0+6 (inputs: rows s0 .. s0+6).
+__device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float *conv_w,
+                                             const float *conv_b, int64_t ch, float (&out)[4][8]) {
+  float w[8][4], bias[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 wv = __ldg(reinterpret_cast<const float4 *>(conv_w) + ch + i);
+    w[i][0] = wv.x;
+    w[i][1] = wv.y;
+    w[i][2] = wv.z;
+    w[i][3] = wv.w;
+    bias[i] = __ldg(conv_b + ch + i);
+  }
+  float rows[7][8];
+#pragma unroll
+  for (int r = 0; r < 7; ++r) {
+    const int R = s0 + r;
+    const uint4 raw = ld_shared_v4(tile + R * 128 + (((cg ^ R) & 7) << 4));
+    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h2[i]);
+      rows[r][2 * i] = f.x;
+      rows[r][2 * i + 1] = f.y;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float pre = bias[i] + w[i][0] * rows[k][i] + w[i][1] * rows[k + 1][i] +
+                        w[i][2] * rows[k + 2][i] + w[i][3] * rows[k + 3][i];
+      out[k][i] = silu_fast(pre);
+    }
+}
+
+struct K1Item {
+  int64_t bi;
+  int c, g, pair;
+  bool isC;
+};
+
+__device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs, int64_t it) {
+  const int per = pr.G * pairs + pr.G;  // items per (row, chunk)
+  const int64_t bc = it / per;
+  const int r = (int)(it % per);
+  K1Item w;
+  w.bi = bc / nch;
+  w.c = (int)(bc % nch);
+  if (r < pr.G * pairs) {
+    w.g = r / pairs;
+    w.pair = r % pairs;
+    w.isC = false;
+  } else {
+    w.g = r - pr.G * pairs;
+    w.pair = 0;
+    w.isC = true;
+  }
+  return w;
+}
+
+__global__ void __launch_bounds__(kOutThreads, 1)
+    tc_chunk_state_kernel(TcArgs a, const __grid_constant__ K1Maps maps, int64_t n_items) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ float ws[2][kQ];
-  __shared__ uint64_t mbar;
+  __shared__ float ws[2][2][kQ];  // [stage][head of pair][token] chunk weights
+  __shared__ uint64_t full[2], empty[2], mbar;
   __shared__ uint32_t tmem_holder;
   const Problem &pr = a.pr;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sAhi = base, sAlo = base + kK1A, sBhi = base + 2 * kK1A,
-                 sBlo = base + 2 * kK1A + kK1B;
-  const int c = blockIdx.x;
+  const uint32_t sAhi = base + kK1Ahi, sAlo = base + kK1Alo, sBhi = base + kK1Bhi,
+                 sBlo = base + kK1Blo;
   const int hpg = pr.heads_per_group();
   const int pairs = (hpg + 1) / 2;
-  const int g = blockIdx.y / pairs, pair = blockIdx.y % pairs;
-  const int64_t bi = blockIdx.z;
-  const int hA = g * hpg + 2 * pair;
-  const bool hasB = 2 * pair + 1 < hpg;
-  const int64_t c0 = (int64_t)c * kQ;
 
   if (warp == 0) tmem_alloc(&tmem_holder, 64);
   if (tid == 0) {
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], 1);
+    }
     mbar_init(&mbar, 1);
     fence_mbar_init();
   }
-
-  // dt, chunk-local cumsum of dt*A, weights w_s = exp(cum_end - cum_s) dt_s:
-  // warp 0 for head A, warp 1 for head B, 4 consecutive tokens per lane
-  if (warp < 2) {
-    const int half = warp;
-    const bool hv = half == 0 || hasB;
-    const int h = hA + half;
-    float dt4[4], a4[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t tt = c0 + 4 * lane + k;
-      dt4[k] = (hv && tt < pr.L)
-                   ? softplus_f(__bfloat162float(a.dt_raw[(bi * pr.L + tt) * a.ld_dt + h]) +
-                                a.prm.dt_bias[h])
-                   : 0.0f;
-      a4[k] = hv ? dt4[k] * a.prm.A[h] : 0.0f;
-    }
-    const float tot = a4[0] + a4[1] + a4[2] + a4[3];
-    float run = warp_scan(tot, lane) - tot;
-    const float cum_end = __shfl_sync(0xffffffffu, run + tot, 31);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      run += a4[k];
-      ws[half][4 * lane + k] = expf(cum_end - run) * dt4[k];
-    }
-    if (lane == 0 && hv) a.cum_end[(bi * a.nch + c) * pr.H + h] = cum_end;
-  }
-  __syncthreads();
-
-  // conv + SiLU: groups of 8 channels (x of head A, x of head B, B, and for the
-  // group's first pair also C) x 32 ranges of 4 tokens.  Post-conv values go
-  // to u (fp16) for the output kernel; x o w and B are split into fp16 hi + lo
-  // operands of the chunk-state product.
-  const int ncg = pair == 0 ? 32 : 24;
-  for (int item = tid; item < ncg * 32; item += kThreads) {
-    const int cgp = item >> 5, tr = item & 31;
-    const int s0 = tr * 4;
-    uint32_t hi[8][2], lo[8][2];
-    if (cgp < 16 && (cgp < 8 || hasB)) {
-      const int half = cgp >> 3, p0 = (cgp & 7) * 8;
-      float v[4][8];
-      const int64_t ch = (int64_t)(hA + half) * kHP + p0;
-      conv8x4(a, bi, c0 + s0, ch, v);
-      store_u(a, bi, c0 + s0, ch, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float q[4], r[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float x = v[k][i] * ws[half][s0 + k];
-          q[k] = __half2float(__float2half_rn(x));
-          r[k] = x - q[k];
-        }
-        hi[i][0] = pack_half2(q[0], q[1]);
-        hi[i][1] = pack_half2(q[2], q[3]);
-        lo[i][0] = pack_half2(r[0], r[1]);
-        lo[i][1] = pack_half2(r[2], r[3]);
-      }
-      const int blk = s0 >> 6;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int m = half * 64 + p0 + i;
-        const uint32_t off = blk * 16384 + sw128_off(m, s0 & 63);
-        st_shared_v2(sAhi + off, hi[i][0], hi[i][1]);
-        st_shared_v2(sAlo + off, lo[i][0], lo[i][1]);
-      }
-    } else if (cgp < 16) {  // missing second head: zero rows 64..127
-      const int p0 = (cgp & 7) * 8, blk = s0 >> 6;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t off = blk * 16384 + sw128_off(64 + p0 + i, s0 & 63);
-        st_shared_v2(sAhi + off, 0u, 0u);
-        st_shared_v2(sAlo + off, 0u, 0u);
-      }
-    } else if (cgp < 24) {
-      const int n0 = (cgp - 16) * 8;
-      float v[4][8];
-      const int64_t ch = pr.d_inner + (int64_t)g * kNS + n0;
-      conv8x4(a, bi, c0 + s0, ch, v);
-      if (pair == 0) store_u(a, bi, c0 + s0, ch, v);
-      const int blk = s0 >> 6;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float q[4], r[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          q[k] = __half2float(__float2half_rn(v[k][i]));
-          r[k] = v[k][i] - q[k];
-        }
-        const uint32_t off = blk * 8192 + sw128_off(n0 + i, s0 & 63);
-        st_shared_v2(sBhi + off, pack_half2(q[0], q[1]), pack_half2(q[2], q[3]));
-        st_shared_v2(sBlo + off, pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
-      }
-    } else {  // C channels (first pair of the group only): post-conv values to u
-      const int n0 = (cgp - 24) * 8;
-      float v[4][8];
-      const int64_t ch = pr.d_inner + (int64_t)(pr.G + g) * kNS + n0;
-      conv8x4(a, bi, c0 + s0, ch, v);
-      store_u(a, bi, c0 + s0, ch, v);
-    }
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  if (tid == 0) {
-    const uint32_t idesc = umma_idesc_f16(128, 64);
-    const uint32_t As[3] = {sAhi, sAhi, sAlo}, Bs[3] = {sBhi, sBlo, sBhi};
-    for (int prod = 0; prod < 3; ++prod)
-      for (int ks = 0; ks < 8; ++ks) {
-        const int blk = ks >> 2, kin = ks & 3;
-        umma_f16(tmem, umma_desc_sw128(As[prod] + blk * 16384 + kin * 32),
-                 umma_desc_sw128(Bs[prod] + blk * 8192 + kin * 32), idesc,
-                 (prod > 0 || ks > 0) ? 1u : 0u);
+  if (warp == kThreads / 32) {
+    // ---------------- producer: dt weights and raw tiles of the next items
+    int k = 0;
+    for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
+      const int st = k & 1;
+      if (k >= 2) {
+        bool got = lane == 0 ? mbar_wait_bounded(&empty[st], (uint32_t)(((k >> 1) - 1) & 1),
+                                                 &g_tc_errors)
+                             : true;
+        if (!__all_sync(0xffffffffu, got)) break;
       }
-    umma_commit(&mbar);
-  }
-  const bool ok = wait_all(&mbar, 0, true);
-  tc_fence_after();
-  if (ok) {
-    // rows m = 32*(warp%4) + lane; warps 0-3 columns 0-31, warps 4-7 columns 32-63
-    const int m = 32 * (warp & 3) + lane, half = m >> 6, p = m & 63, cb = 32 * (warp >> 2);
-    float v[32];
-    tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, v);
-    if (half == 0 || hasB) {
-      float4 *dst = reinterpret_cast<float4 *>(
-          a.S + (((bi * a.nch + c) * pr.H + hA + half) * kHP + p) * kNS + cb);
+      const K1Item w = k1_item(pr, a.nch, pairs, it);
+      const int64_t c0 = (int64_t)w.c * kQ;
+      const int hA = w.g * hpg + 2 * w.pair;
+      const bool hasB = 2 * w.pair + 1 < hpg;
+      if (!w.isC) {
+        for (int half = 0; half < 2; ++half) {
+          const bool hv = half == 0 || hasB;
+          const int h = hA + half;
+          float dt4[4], a4[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int q = 0; q < 4; ++q) {
+            const int64_t tt = c0 + 4 * lane + q;
+            dt4[q] = (hv && tt < pr.L)
+                         ? softplus_f(__bfloat162float(a.dt_raw[(w.bi * pr.L + tt) * a.ld_dt + h]) +
+                                      a.prm.dt_bias[h])
+                         : 0.0f;
+            a4[q] = hv ? dt4[q] * a.prm.A[h] : 0.0f;
+          }
+          const float tot = a4[0] + a4[1] + a4[2] + a4[3];
+          float run = warp_scan(tot, lane) - tot;
+          const float cum_end = __shfl_sync(0xffffffffu, run + tot, 31);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            run += a4[q];
+            ws[st][half][4 * lane + q] = expf(cum_end - run) * dt4[q];
+          }
+          if (lane == 0 && hv) a.cum_end[(w.bi * a.nch + w.c) * pr.H + h] = cum_end;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t stage = base + st * kK1Stage;
+        if (w.isC) {
+          mbar_arrive_expect_tx(&full[st], kRawBytes);
+          tma_load_3d(stage, &maps.xbc, (int)(pr.d_inner + (int64_t)(pr.G + w.g) * kNS),
+                      (int)c0 - 3, (int)w.bi, &full[st]);
+        } else {
+          mbar_arrive_expect_tx(&full[st], (hasB ? 3u : 2u) * kRawBytes);
+          tma_load_3d(stage, &maps.xbc, hA * kHP, (int)c0 - 3, (int)w.bi, &full[st]);
+          if (hasB)
+            tma_load_3d(stage + kRawBytes, &maps.xbc, (hA + 1) * kHP, (int)c0 - 3, (int)w.bi,
+                        &full[st]);
+          tma_load_3d(stage + 2 * kRawBytes, &maps.xbc, (int)(pr.d_inner + (int64_t)w.g * kNS),
+                      (int)c0 - 3, (int)w.bi, &full[st]);
+        }
+      }
+    }
+  } else {
+    // ---------------- compute warps
+    bool ok = true;
+    int k = 0, npair = 0;
+    for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++k) {
+      const int st = k & 1;
+      const uint32_t stage = base + st * kK1Stage;
+      ok = wait_compute(&full[st], (uint32_t)((k >> 1) & 1), ok);
+      if (!ok) break;
+      const K1Item w = k1_item(pr, a.nch, pairs, it);
+      const int64_t c0 = (int64_t)w.c * kQ;
+      const int hA = w.g * hpg + 2 * w.pair;
+      const bool hasB = 2 * w.pair + 1 < hpg;
+      // channel of slot s (C items use slot 0 for C)
+      auto slot_ch = [&](int sl) -> int64_t {
+        if (w.isC) return pr.d_inner + (int64_t)(pr.G + w.g) * kNS;
+        return sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS;
+      };
+      const int nslots = w.isC ? 1 : 3;
+      // first chunk: the 3 rows before token 0 come from the carried conv state
+      if (c0 == 0 && a.states_in) {
+        for (int idx = tid; idx < nslots * 3 * 64; idx += kThreads) {
+          const int sl = idx / 192, r = (idx / 64) % 3, chn = idx % 64;
+          if (sl == 1 && !hasB) continue;
+          const __nv_bfloat16 v = a.conv_in[(w.bi * pr.conv_dim + slot_ch(sl) + chn) * 4 + 1 + r];
+          const uint32_t addr = stage + sl * kRawBytes + r * 128 +
+                                ((((chn >> 3) ^ r) & 7) << 4) + ((chn & 7) << 1);
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(v))
+                       : "memory");
+        }
+        compute_sync();
+      }
+      // conv + SiLU over groups of 8 channels x 32 ranges of 4 tokens
+      const int ncg = w.isC ? 8 : 24;
+      for (int item = tid; item < ncg * 32; item += kThreads) {
+        const int cgp = item >> 5, tr = item & 31, s0 = tr * 4, cg = cgp & 7;
+        const int sl = w.isC ? 0 : cgp >> 3;
+        if (sl == 1 && !hasB) {  // missing second head: zero rows 64..127
+          const int blk = s0 >> 6;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t off = blk * 16384 + sw128_off(64 + cg * 8 + i, s0 & 63);
+            st_shared_v2(sAhi + off, 0u, 0u);
+            st_shared_v2(sAlo + off, 0u, 0u);
+          }
+          continue;
+        }
+        const int64_t ch = slot_ch(sl) + cg * 8;
+        float v[4][8];
+        conv8x4_smem(stage + sl * kRawBytes, s0, cg, a.prm.conv_w, a.prm.conv_b, ch, v);
+        if (w.isC || sl < 2 || w.pair == 0) store_u(a, w.bi, c0 + s0, ch, v);
+        if (w.isC) continue;
+        const int blk = s0 >> 6;
+        if (sl < 2) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float q[4], r[4];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const float x = v[kk][i] * ws[st][sl][s0 + kk];
+              q[kk] = __half2float(__float2half_rn(x));
+              r[kk] = x - q[kk];
+            }
+            const uint32_t off = blk * 16384 + sw128_off(sl * 64 + cg * 8 + i, s0 & 63);
+            st_shared_v2(sAhi + off, pack_half2(q[0], q[1]), pack_half2(q[2], q[3]));
+            st_shared_v2(sAlo + off, pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float q[4], r[4];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              q[kk] = __half2float(__float2half_rn(v[kk][i]));
+              r[kk] = v[kk][i] - q[kk];
+            }
+            const uint32_t off = blk * 8192 + sw128_off(cg * 8 + i, s0 & 63);
+            st_shared_v2(sBhi + off, pack_half2(q[0], q[1]), pack_half2(q[2], q[3]));
+            st_shared_v2(sBlo + off, pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      compute_sync();
+      if (tid == 0) mbar_arrive(&empty[st]);  // raw tiles of this stage consumed
+      if (w.isC) continue;
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t idesc = umma_idesc_f16(128, 64);
+        const uint32_t As[3] = {sAhi, sAhi, sAlo}, Bs[3] = {sBhi, sBlo, sBhi};
+        for (int prod = 0; prod < 3; ++prod)
+          for (int ks = 0; ks < 8; ++ks) {
+            const int blk = ks >> 2, kin = ks & 3;
+            umma_f16(tmem, umma_desc_sw128(As[prod] + blk * 16384 + kin * 32),
+                     umma_desc_sw128(Bs[prod] + blk * 8192 + kin * 32), idesc,
+                     (prod > 0 || ks > 0) ? 1u : 0u);
+          }
+        umma_commit(&mbar);
+      }
+      ok = wait_compute(&mbar, (uint32_t)(npair & 1), ok);
+      ++npair;
+      tc_fence_after();
+      if (ok) {
+        // rows m = 32*(warp%4) + lane; warp/4 selects 16 of the 64 columns
+        const int m = 32 * (warp & 3) + lane, half = m >> 6, p = m & 63, cb = 16 * (warp >> 2);
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, v);
+        if (half == 0 || hasB) {
+          float4 *dst = reinterpret_cast<float4 *>(
+              a.S + (((w.bi * a.nch + w.c) * pr.H + hA + half) * kHP + p) * kNS + cb);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      compute_sync();  // TMEM read and operand smem free before the next item
+    }
+    if (!ok && tid == 0) {
+      // a wait ran out: let copies already issued land before the CTA exits
+      for (int s2 = 0; s2 < 2; ++s2) mbar_wait_bounded(&full[s2], 0, &g_tc_errors);
     }
   }
   tc_fence_before();
@@ -393,23 +517,26 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a) {
 // warp.  Tiles arrive by TMA in 128-byte-swizzled layouts (1024-aligned):
 constexpr uint32_t kCt = 0;                      // C   [128 t][64 n] fp16     16 KB (u)
 constexpr uint32_t kBt = kCt + 16384;            // B   [128 s][64 n] fp16     16 KB (u)
-constexpr uint32_t kXt = kBt + 16384;            // x   2 x [128 s][64 p] fp16 2 x 16 KB (u)
-constexpr uint32_t kHt = kXt + 2 * 16384;        // H_c 2 x [64 p][64 n] fp16  2 x 8 KB
-constexpr uint32_t kZt = kHt + 2 * 8192;         // z   2 x [128 t][64 p] bf16 2 x 16 KB
-constexpr uint32_t kAt = kZt + 2 * 16384;        // A   [3][128 t][64 k] fp16  48 KB
-constexpr uint32_t kTcOutTiles = kAt + 3 * 16384;  // 160 KB
-constexpr int kOutThreads = kThreads + 32;       // + producer warp
-constexpr uint32_t kHeadBytes = 16384 + 8192 + 16384;  // x + H_c + z per head
+constexpr int kXhStages = 3, kZStages = 2;
+constexpr uint32_t kXhBytes = 16384 + 8192;      // per stage: x [128 s][64 p] + H_c [64 p][64 n]
+constexpr uint32_t kXh = kBt + 16384;            // x / H_c ring  3 x 24 KB (x at +0, H_c at +16 KB)
+constexpr uint32_t kZt = kXh + kXhStages * kXhBytes;  // z ring [128 t][64 p] bf16  2 x 16 KB
+constexpr uint32_t kAt = kZt + kZStages * 16384;      // A   [3][128 t][64 k] fp16  48 KB
+constexpr uint32_t kTcOutTiles = kAt + 3 * 16384;     // 184 KB
 
 struct OutShared {
   float cum2[kMaxHeadsPerCta][kQ];  // cumsum * log2(e)
   float dt[kMaxHeadsPerCta][kQ];
   float beta[kMaxHeadsPerCta][kQ];  // exp(cum_r - cum_s) dt_s, r = end of s's 32-token group
+  float betad[kMaxHeadsPerCta][kQ]; // exp(cum_s0 - cum_s) dt_s, s0 = start of s's group
+  int span_ok[kMaxHeadsPerCta][4];  // group's log2-decay span <= 60: factorise its diagonal
   float ecum[kMaxHeadsPerCta][kQ];  // exp(cumsum)
-  float ss[2][kQ];
+  float nw[kMaxHeadsPerCta][kHP];   // norm weight of the CTA's channels
+  float ss[4][kQ];
   float part[16][kQ];               // per-rank partial sums of squares (rank 0's is read)
   float inv[kQ];
-  uint64_t full_cb, full[2], empty[2], mbar_cb, mbar_mma;
+  uint64_t full_cb, full_xh[kXhStages], empty_xh[kXhStages], full_z[kZStages],
+      empty_z[kZStages], mbar_cb, mbar_mma;
   uint32_t tmem_holder;
   int ok_flag;
 };
@@ -419,53 +546,6 @@ struct OutMaps {
   CUtensorMap z;   // [b][L][d_inner] bf16 (row stride ld_z), box 64 x 128
   CUtensorMap hc;  // [rows][64] fp16, box 64 x 64
 };
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
-                                            int c2, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// barrier over the 256 compute threads only (the producer warp never joins)
-__device__ __forceinline__ void compute_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
-}
-__device__ __forceinline__ bool compute_all(bool v) {
-  int r;
-  asm volatile("{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.and.pred q, 1, 256, p;\n"
-               " selp.s32 %0, 1, 0, q;\n}"
-               : "=r"(r)
-               : "r"((int)v)
-               : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ bool wait_compute(uint64_t *bar, uint32_t parity, bool ok) {
-  const bool got = ok ? mbar_wait_bounded(bar, parity, &g_tc_errors) : false;
-  return compute_all(got);
-}
-// Smem descriptor for an MN-major SW128 operand: 8-row (K) atoms of 64
-// elements (N) x 128 B, K atoms 1024 B apart (SBO), N atoms `lbo` apart.
-__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)(1024u >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
 
 __global__ void __launch_bounds__(kOutThreads, 1)
     tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps) {
@@ -490,9 +570,13 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   if (warp == 0) tmem_alloc(&sh.tmem_holder, 512);
   if (tid == 0) {
     mbar_init(&sh.full_cb, 1);
-    for (int k = 0; k < 2; ++k) {
-      mbar_init(&sh.full[k], 1);
-      mbar_init(&sh.empty[k], 1);
+    for (int k = 0; k < kXhStages; ++k) {
+      mbar_init(&sh.full_xh[k], 1);
+      mbar_init(&sh.empty_xh[k], 1);
+    }
+    for (int k = 0; k < kZStages; ++k) {
+      mbar_init(&sh.full_z[k], 1);
+      mbar_init(&sh.empty_z[k], 1);
     }
     mbar_init(&sh.mbar_cb, 1);
     mbar_init(&sh.mbar_mma, 1);
@@ -511,17 +595,24 @@ __global__ void __launch_bounds__(kOutThreads, 1)
                   (int)bi, &sh.full_cb);
       tma_load_3d(base + kBt, &maps.u, (int)(pr.d_inner + (int64_t)g * kNS), (int)c0, (int)bi,
                   &sh.full_cb);
+      // x / H_c of head j go to stage j % 3, freed when MMA j has completed;
+      // z of head j to stage j % 2, freed after the epilogue of head j
       for (int j = 0; j < nh; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(&sh.empty[st], (uint32_t)(((j >> 1) - 1) & 1),
-                                         &g_tc_errors))
-          break;
         const int h = h0 + j;
-        mbar_arrive_expect_tx(&sh.full[st], kHeadBytes);
-        tma_load_3d(base + kXt + st * 16384, &maps.u, h * kHP, (int)c0, (int)bi, &sh.full[st]);
-        tma_load_2d(base + kHt + st * 8192, &maps.hc, 0,
-                    (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full[st]);
-        tma_load_3d(base + kZt + st * 16384, &maps.z, h * kHP, (int)c0, (int)bi, &sh.full[st]);
+        const int sx = j % kXhStages, sz = j % kZStages;
+        if (j >= kXhStages && !mbar_wait_bounded(&sh.empty_xh[sx],
+                                                 (uint32_t)((j / kXhStages - 1) & 1), &g_tc_errors))
+          break;
+        mbar_arrive_expect_tx(&sh.full_xh[sx], kXhBytes);
+        tma_load_3d(base + kXh + sx * kXhBytes, &maps.u, h * kHP, (int)c0, (int)bi,
+                    &sh.full_xh[sx]);
+        tma_load_2d(base + kXh + sx * kXhBytes + 16384, &maps.hc, 0,
+                    (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full_xh[sx]);
+        if (j >= kZStages && !mbar_wait_bounded(&sh.empty_z[sz],
+                                                (uint32_t)((j / kZStages - 1) & 1), &g_tc_errors))
+          break;
+        mbar_arrive_expect_tx(&sh.full_z[sz], 16384);
+        tma_load_3d(base + kZt + sz * 16384, &maps.z, h * kHP, (int)c0, (int)bi, &sh.full_z[sz]);
       }
     }
   } else {
@@ -551,9 +642,16 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         sh.ecum[j][4 * lane + k] = ex2_approx(c2[k]);
       }
       const float c2r = __shfl_sync(0xffffffffu, c2[3], (lane | 7));
+      const float c2s0 = __shfl_sync(0xffffffffu, c2[0], (lane & ~7));
 #pragma unroll
-      for (int k = 0; k < 4; ++k) sh.beta[j][4 * lane + k] = ex2_approx(c2r - c2[k]) * dt4[k];
+      for (int k = 0; k < 4; ++k) {
+        sh.beta[j][4 * lane + k] = ex2_approx(c2r - c2[k]) * dt4[k];
+        sh.betad[j][4 * lane + k] = ex2_approx(fminf(c2s0 - c2[k], 60.0f)) * dt4[k];
+      }
+      if ((lane & 7) == 7) sh.span_ok[j][lane >> 3] = (c2s0 - c2r) <= 60.0f;
     }
+    for (int i = tid; i < nh * kHP; i += kThreads)
+      sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
     bool ok = wait_compute(&sh.full_cb, 0, true);
     tc_fence_after();
     if (ok && tid == 0) {  // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
@@ -568,16 +666,17 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     float ss_acc = 0.0f;
 
-    // epilogue, part 1: gate with silu(z) (z tile in smem), sum of squares, g -> TMEM
+    // epilogue, part 1: gate with silu(z) (z tile in smem), sum of squares, g -> TMEM.
+    // Warp w handles rows 32*(w%4) .. +31 and columns 16*(w/4) .. +15 of a head.
     auto epilogue1 = [&](int j) {
-      float v[32];
-      const uint32_t col = 128 + 64 * j + 32 * hf;
-      tmem_ld32(tmem + lane_off + col, v);
+      float v[16];
+      const uint32_t col = 128 + 64 * j + 16 * hf;
+      tmem_ld16(tmem + lane_off + col, v);
       if (!pr.nbg) {
-        const uint32_t zt = base + kZt + (j & 1) * 16384;
+        const uint32_t zt = base + kZt + (j % kZStages) * 16384;
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const uint4 raw = ld_shared_v4(zt + sw128_chunk(t, 32 * hf + 8 * qq));
+        for (int qq = 0; qq < 2; ++qq) {
+          const uint4 raw = ld_shared_v4(zt + sw128_chunk(t, 16 * hf + 8 * qq));
           const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -588,31 +687,28 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         }
       }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ss_acc = fmaf(v[i], v[i], ss_acc);
-      if (!pr.nbg) tmem_st32(tmem + lane_off + col, v);
+      for (int i = 0; i < 16; ++i) ss_acc = fmaf(v[i], v[i], ss_acc);
+      if (!pr.nbg) tmem_st16(tmem + lane_off + col, v);
     };
 
     for (int j = 0; j < nh && ok; ++j) {
       const int h = h0 + j;
-      ok = wait_compute(&sh.full[j & 1], (uint32_t)((j >> 1) & 1), ok);
       ok = (j == 0) ? wait_compute(&sh.mbar_cb, 0, ok) : wait_compute(&sh.mbar_mma, (j - 1) & 1, ok);
       if (!ok) break;
       tc_fence_after();
+      if (j > 0 && tid == 0) mbar_arrive(&sh.empty_xh[(j - 1) % kXhStages]);  // MMA j-1 is done
       // A_j = [CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal | C o exp(cum_t)];
       // 32-column groups k above the row quarter q are zero, below it the decay
       // factorises as alpha_t beta_s (both <= 1), on it exponentials are direct.
       {
-        const uint32_t at = base + kAt + hf * 16384;
+        const int k = hf, s0 = 32 * k;  // this warp's 32-column group
+        const uint32_t at = base + kAt + (k >> 1) * 16384;
+        const int kc = 32 * (k & 1);       // column of the group inside its 64-wide block
         const float c2t = sh.cum2[j][t];
+        if (k > q) {
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const int k = 2 * hf + part, s0 = 32 * k;
-          if (k > q) {
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-              st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), 0u, 0u, 0u, 0u);
-            continue;
-          }
+          for (int qq = 0; qq < 4; ++qq) st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), 0u, 0u, 0u, 0u);
+        } else {
           float cb[32];
           tmem_ld32(tmem + lane_off + s0, cb);
           if (k < q) {
@@ -628,7 +724,32 @@ __global__ void __launch_bounds__(kOutThreads, 1)
                 const int sl = 8 * qq + 2 * e;
                 w4[e] = pack_half2(cb[sl] * alpha * bb[2 * e], cb[sl + 1] * alpha * bb[2 * e + 1]);
               }
-              st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+              st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+            }
+          } else if (sh.span_ok[j][k]) {
+            // diagonal group, decay span <= 2^60: alpha_t = exp(cum_t - cum_s0) and
+            // betad_s = exp(cum_s0 - cum_s) dt_s stay within [2^-60, 2^60]
+            const float Dh = a.prm.D[h];
+            const float alpha = ex2_approx(c2t - sh.cum2[j][s0]);
+            const float4 *b4 = reinterpret_cast<const float4 *>(&sh.betad[j][s0]);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const float4 bA = b4[2 * qq], bB = b4[2 * qq + 1];
+              const float bb[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+              uint32_t w4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float val[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
+                  float vv = cb[sl] * alpha * bb[2 * e + u];
+                  if (s == t) vv += Dh;
+                  val[u] = (s <= t) ? vv : 0.0f;
+                }
+                w4[e] = pack_half2(val[0], val[1]);
+              }
+              st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
             }
           } else {
             const float Dh = a.prm.D[h];
@@ -653,14 +774,15 @@ __global__ void __launch_bounds__(kOutThreads, 1)
                 }
                 w4[e] = pack_half2(val[0], val[1]);
               }
-              st_shared_v4(at + sw128_chunk(t, 32 * part + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+              st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
             }
           }
         }
+        // C scaled by exp(cum_t): this warp does n in [16 hf, 16 hf + 16)
         const float ec = sh.ecum[j][t];
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int n0 = 32 * hf + 8 * qq;
+        for (int qq = 0; qq < 2; ++qq) {
+          const int n0 = 16 * hf + 8 * qq;
           const uint4 cv = ld_shared_v4(base + kCt + sw128_chunk(t, n0));
           const uint32_t in[4] = {cv.x, cv.y, cv.z, cv.w};
           uint32_t o[4];
@@ -675,11 +797,14 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       compute_sync();
-      if (tid == 0) {
+      // only the issuing thread needs the x / H_c tiles of head j (the MMA reads them);
+      // if that wait runs out, no MMA is issued and the next wait fails for everyone
+      if (tid == 0 && mbar_wait_bounded(&sh.full_xh[j % kXhStages],
+                                        (uint32_t)((j / kXhStages) & 1), &g_tc_errors)) {
         tc_fence_after();
         const uint32_t idesc_k = umma_idesc_f16(128, 64);
         const uint32_t idesc_mn = idesc_k | (1u << 16);  // B operand MN-major (x tile)
-        const uint32_t xt = base + kXt + (j & 1) * 16384, ht = base + kHt + (j & 1) * 8192;
+        const uint32_t xt = base + kXh + (j % kXhStages) * kXhBytes, ht = xt + 16384;
         for (int ks = 0; ks < 12; ++ks) {
           const int blk = ks >> 2, kin = ks & 3;
           const uint64_t ad = umma_desc_sw128(base + kAt + blk * 16384 + kin * 32);
@@ -692,15 +817,17 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         umma_commit(&sh.mbar_mma);
       }
       if (j > 0) {
-        epilogue1(j - 1);  // overlaps the MMA of head j
+        ok = wait_compute(&sh.full_z[(j - 1) % kZStages], (uint32_t)(((j - 1) / kZStages) & 1), ok);
+        if (ok) epilogue1(j - 1);  // overlaps the MMA of head j
         compute_sync();
-        if (tid == 0) mbar_arrive(&sh.empty[(j - 1) & 1]);
+        if (tid == 0) mbar_arrive(&sh.empty_z[(j - 1) % kZStages]);
       }
       tc_fence_before();
       compute_sync();
     }
     if (ok && nh > 0) {
       ok = wait_compute(&sh.mbar_mma, (nh - 1) & 1, ok);
+      ok = wait_compute(&sh.full_z[(nh - 1) % kZStages], (uint32_t)(((nh - 1) / kZStages) & 1), ok);
       tc_fence_after();
       if (ok) epilogue1(nh - 1);
     }
@@ -708,7 +835,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       // a wait ran out: let issued MMAs and tile copies land before the CTA exits
       mbar_wait_bounded(&sh.mbar_cb, 0, &g_tc_errors);
       mbar_wait_bounded(&sh.full_cb, 0, &g_tc_errors);
-      for (int k = 0; k < 2; ++k) mbar_wait_bounded(&sh.full[k], 0, &g_tc_errors);
+      for (int k = 0; k < kXhStages; ++k) mbar_wait_bounded(&sh.full_xh[k], 0, &g_tc_errors);
+      for (int k = 0; k < kZStages; ++k) mbar_wait_bounded(&sh.full_z[k], 0, &g_tc_errors);
     }
     sh.ss[hf][t] = ss_acc;
     sh.ok_flag = ok;
@@ -717,7 +845,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
 
   // per-token sums of squares of this CTA -> rank 0's table; totals; scale
   float *part0 = cluster.map_shared_rank(&sh.part[0][0], 0);
-  if (tid < kQ) part0[rank * kQ + tid] = sh.ss[0][tid] + sh.ss[1][tid];
+  if (tid < kQ) part0[rank * kQ + tid] = (sh.ss[0][tid] + sh.ss[1][tid]) + (sh.ss[2][tid] + sh.ss[3][tid]);
   cluster.sync();
   if (tid < kQ) {
     float tot = 0.0f;
@@ -733,16 +861,16 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const float sc = sh.inv[t];
     for (int j = 0; j < nh; ++j) {
       const int h = h0 + j;
-      float v[32];
-      tmem_ld32(tmem + lane_off + 128 + 64 * j + 32 * hf, v);
+      float v[16];
+      tmem_ld16(tmem + lane_off + 128 + 64 * j + 16 * hf, v);
       if (!t_valid) continue;
-      const float *nw = a.prm.norm_w + (int64_t)h * kHP + 32 * hf;
+      const float4 *nw4 = reinterpret_cast<const float4 *>(&sh.nw[j][16 * hf]);
       const int64_t row = bi * pr.L + c0 + t;
       if (pr.nbg) {
         const uint4 *zp =
-            reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 32 * hf);
+            reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 16 * hf);
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
+        for (int qq = 0; qq < 2; ++qq) {
           const uint4 raw = __ldg(zp + qq);
           const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
@@ -753,15 +881,17 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           }
         }
       }
-      uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * pr.d_inner + (int64_t)h * kHP + 32 * hf);
+      uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * pr.d_inner + (int64_t)h * kHP + 16 * hf);
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
+      for (int qq = 0; qq < 2; ++qq) {
         uint32_t o[4];
+        const float4 wA = nw4[2 * qq], wB = nw4[2 * qq + 1];
+        const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = 8 * qq + 2 * e;
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i] * sc * __ldg(nw + i),
-                                                          v[i + 1] * sc * __ldg(nw + i + 1));
+          const __nv_bfloat162 b2 =
+              __floats2bfloat162_rn(v[i] * sc * ww[2 * e], v[i + 1] * sc * ww[2 * e + 1]);
           o[e] = *reinterpret_cast<const uint32_t *>(&b2);
         }
         dst[qq] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -824,6 +954,19 @@ TcWorkspace tc_carve(const Problem &pr, char *base) {
   return w;
 }
 
+// Number of SMs of the current device (cached per device).
+int sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 132;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 132;
+  }
+  return cache[dev];
+}
+
 // cuTensorMapEncodeTiled, fetched once through the runtime (no libcuda link-time dependency).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
@@ -857,7 +1000,7 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank
          CUDA_SUCCESS;
 }
 
-constexpr size_t kK1Smem = 2 * kK1A + 2 * kK1B + 1024;
+constexpr size_t kK1Smem = kK1Tiles + 1024;
 constexpr size_t kK3Smem = kTcOutTiles + sizeof(OutShared) + 1024;
 
 }  // namespace
@@ -926,8 +1069,17 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   if (e != cudaSuccess) return e;
 
   stage_mark(st, 0);
-  dim3 g1((unsigned)a.nch, (unsigned)(pr.G * ((hpg + 1) / 2)), (unsigned)pr.batch);
-  tc_chunk_state_kernel<<<g1, kThreads, kK1Smem, st>>>(a);
+  const int64_t n_items = pr.batch * a.nch * (int64_t)(pr.G * ((hpg + 1) / 2) + pr.G);
+  const unsigned g1 = (unsigned)std::min<int64_t>(n_items, sm_count());
+  {
+    K1Maps m1;
+    const uint64_t dx[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
+    const uint64_t sx[2] = {(uint64_t)pa.ld_xbc * 2, (uint64_t)pr.L * pa.ld_xbc * 2};
+    const uint32_t bx[3] = {64, kRawRows, 1};
+    if (!make_map(&m1.xbc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xBC, 3, dx, sx, bx))
+      return cudaErrorInvalidValue;
+    tc_chunk_state_kernel<<<g1, kOutThreads, kK1Smem, st>>>(a, m1, n_items);
+  }
   stage_mark(st, 1);
   dim3 g2((kHP * kNS) / 256, (unsigned)pr.H, (unsigned)pr.batch);
   tc_state_pass_kernel<<<g2, 256, 0, st>>>(a);
