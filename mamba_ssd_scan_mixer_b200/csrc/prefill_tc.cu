@@ -42,6 +42,7 @@ namespace {
 constexpr int kQ = 128;          // tokens per chunk = MMA M
 constexpr int kThreads = 512;    // 16 compute warps
 constexpr int kOutThreads = kThreads + 32;  // + one TMA producer warp
+constexpr int kK3Threads = kThreads + 64;   // + TMA producer warp + MMA issuer warp
 constexpr int kHP = 64;          // headdim
 constexpr int kNS = 64;          // d_state
 constexpr int kMaxHeadsPerCta = 6;  // TMEM: 128 (CB) + 6 x 64 (y) <= 512 columns
@@ -535,8 +536,9 @@ struct OutShared {
   float ss[4][kQ];
   float part[16][kQ];               // per-rank partial sums of squares (rank 0's is read)
   float inv[kQ];
+  float Dh[kMaxHeadsPerCta];
   uint64_t full_cb, full_xh[kXhStages], empty_xh[kXhStages], full_z[kZStages],
-      empty_z[kZStages], mbar_cb, mbar_mma;
+      empty_z[kZStages], a_ready, mbar_cb, mbar_mma;
   uint32_t tmem_holder;
   int ok_flag;
 };
@@ -547,7 +549,7 @@ struct OutMaps {
   CUtensorMap hc;  // [rows][64] fp16, box 64 x 64
 };
 
-__global__ void __launch_bounds__(kOutThreads, 1)
+__global__ void __launch_bounds__(kK3Threads, 1)
     tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -572,15 +574,17 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     mbar_init(&sh.full_cb, 1);
     for (int k = 0; k < kXhStages; ++k) {
       mbar_init(&sh.full_xh[k], 1);
-      mbar_init(&sh.empty_xh[k], 1);
+      mbar_init(&sh.empty_xh[k], 1);  // arrived by tcgen05.commit of the head's MMA
     }
     for (int k = 0; k < kZStages; ++k) {
       mbar_init(&sh.full_z[k], 1);
-      mbar_init(&sh.empty_z[k], 1);
+      mbar_init(&sh.empty_z[k], kThreads);  // every compute thread after its epilogue
     }
+    mbar_init(&sh.a_ready, kThreads);       // every compute thread after its A-build
     mbar_init(&sh.mbar_cb, 1);
     mbar_init(&sh.mbar_mma, 1);
     fence_mbar_init();
+    sh.ok_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
@@ -614,6 +618,41 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         mbar_arrive_expect_tx(&sh.full_z[sz], 16384);
         tma_load_3d(base + kZt + sz * 16384, &maps.z, h * kHP, (int)c0, (int)bi, &sh.full_z[sz]);
       }
+    }
+  } else if (warp == kThreads / 32 + 1) {
+    // ---------------- MMA issuer: CB once, then one K = 192 MMA per head
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(&sh.full_cb, 0, &g_tc_errors);
+      if (ok) {  // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
+        tc_fence_after();
+        const uint32_t idesc = umma_idesc_f16(128, 128);
+        for (int kin = 0; kin < 4; ++kin)
+          umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32),
+                   umma_desc_sw128(base + kBt + kin * 32), idesc, kin > 0 ? 1u : 0u);
+        umma_commit(&sh.mbar_cb);
+      }
+      const uint32_t idesc_k = umma_idesc_f16(128, 64);
+      const uint32_t idesc_mn = idesc_k | (1u << 16);  // B operand MN-major (x tile)
+      for (int j = 0; ok && j < nh; ++j) {
+        ok = mbar_wait_bounded(&sh.a_ready, (uint32_t)(j & 1), &g_tc_errors) &&
+             mbar_wait_bounded(&sh.full_xh[j % kXhStages], (uint32_t)((j / kXhStages) & 1),
+                               &g_tc_errors);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t xt = base + kXh + (j % kXhStages) * kXhBytes, ht = xt + 16384;
+        for (int ks = 0; ks < 12; ++ks) {
+          const int blk = ks >> 2, kin = ks & 3;
+          const uint64_t ad = umma_desc_sw128(base + kAt + blk * 16384 + kin * 32);
+          if (ks < 8)
+            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn,
+                     ks > 0 ? 1u : 0u);
+          else
+            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128(ht + kin * 32), idesc_k, 1u);
+        }
+        umma_commit(&sh.mbar_mma);
+        umma_commit(&sh.empty_xh[j % kXhStages]);  // its x / H_c stage is free once it completes
+      }
+      if (!ok) sh.ok_flag = 0;
     }
   } else {
     // ---------------- compute warps
@@ -652,19 +691,19 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     }
     for (int i = tid; i < nh * kHP; i += kThreads)
       sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
-    bool ok = wait_compute(&sh.full_cb, 0, true);
-    tc_fence_after();
-    if (ok && tid == 0) {  // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
-      const uint32_t idesc = umma_idesc_f16(128, 128);
-      for (int kin = 0; kin < 4; ++kin)
-        umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32),
-                 umma_desc_sw128(base + kBt + kin * 32), idesc, kin > 0 ? 1u : 0u);
-      umma_commit(&sh.mbar_cb);
-    }
+    for (int i = tid; i < nh * kHP; i += kThreads)
+      sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
+    if (tid < nh) sh.Dh[tid] = a.prm.D[h0 + tid];
+    compute_sync();  // cumsum, weights and D visible to every compute warp
 
     const int t = 32 * (warp & 3) + lane, hf = warp >> 2, q = warp & 3;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     float ss_acc = 0.0f;
+    bool ok = true;
+    auto wait_warp = [&](uint64_t *bar, uint32_t parity) {
+      const bool got = ok && mbar_wait_bounded(bar, parity, &g_tc_errors);
+      ok = __all_sync(0xffffffffu, got) != 0;
+    };
 
     // epilogue, part 1: gate with silu(z) (z tile in smem), sum of squares, g -> TMEM.
     // Warp w handles rows 32*(w%4) .. +31 and columns 16*(w/4) .. +15 of a head.
@@ -691,12 +730,16 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       if (!pr.nbg) tmem_st16(tmem + lane_off + col, v);
     };
 
-    for (int j = 0; j < nh && ok; ++j) {
-      const int h = h0 + j;
-      ok = (j == 0) ? wait_compute(&sh.mbar_cb, 0, ok) : wait_compute(&sh.mbar_mma, (j - 1) & 1, ok);
+    for (int j = 0; j < nh; ++j) {
+      // the A buffer is free (and Y_{j-1} complete) once the previous MMA is done
+      if (j == 0) {
+        wait_warp(&sh.full_cb, 0);  // the C tile (read below for the scaled-C block)
+        wait_warp(&sh.mbar_cb, 0);
+      } else {
+        wait_warp(&sh.mbar_mma, (uint32_t)((j - 1) & 1));
+      }
       if (!ok) break;
       tc_fence_after();
-      if (j > 0 && tid == 0) mbar_arrive(&sh.empty_xh[(j - 1) % kXhStages]);  // MMA j-1 is done
       // A_j = [CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal | C o exp(cum_t)];
       // 32-column groups k above the row quarter q are zero, below it the decay
       // factorises as alpha_t beta_s (both <= 1), on it exponentials are direct.
@@ -729,7 +772,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           } else if (sh.span_ok[j][k]) {
             // diagonal group, decay span <= 2^60: alpha_t = exp(cum_t - cum_s0) and
             // betad_s = exp(cum_s0 - cum_s) dt_s stay within [2^-60, 2^60]
-            const float Dh = a.prm.D[h];
+            const float Dh = sh.Dh[j];
             const float alpha = ex2_approx(c2t - sh.cum2[j][s0]);
             const float4 *b4 = reinterpret_cast<const float4 *>(&sh.betad[j][s0]);
 #pragma unroll
@@ -752,7 +795,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
               st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
             }
           } else {
-            const float Dh = a.prm.D[h];
+            const float Dh = sh.Dh[j];
             const float4 *c4 = reinterpret_cast<const float4 *>(&sh.cum2[j][s0]);
             const float4 *d4 = reinterpret_cast<const float4 *>(&sh.dt[j][s0]);
 #pragma unroll
@@ -796,50 +839,29 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      compute_sync();
-      // only the issuing thread needs the x / H_c tiles of head j (the MMA reads them);
-      // if that wait runs out, no MMA is issued and the next wait fails for everyone
-      if (tid == 0 && mbar_wait_bounded(&sh.full_xh[j % kXhStages],
-                                        (uint32_t)((j / kXhStages) & 1), &g_tc_errors)) {
-        tc_fence_after();
-        const uint32_t idesc_k = umma_idesc_f16(128, 64);
-        const uint32_t idesc_mn = idesc_k | (1u << 16);  // B operand MN-major (x tile)
-        const uint32_t xt = base + kXh + (j % kXhStages) * kXhBytes, ht = xt + 16384;
-        for (int ks = 0; ks < 12; ++ks) {
-          const int blk = ks >> 2, kin = ks & 3;
-          const uint64_t ad = umma_desc_sw128(base + kAt + blk * 16384 + kin * 32);
-          if (ks < 8)
-            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn,
-                     ks > 0 ? 1u : 0u);
-          else
-            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128(ht + kin * 32), idesc_k, 1u);
-        }
-        umma_commit(&sh.mbar_mma);
+      mbar_arrive(&sh.a_ready);
+      if (j > 0) {  // epilogue of the previous head overlaps this head's MMA
+        wait_warp(&sh.full_z[(j - 1) % kZStages], (uint32_t)(((j - 1) / kZStages) & 1));
+        if (!ok) break;
+        epilogue1(j - 1);
+        mbar_arrive(&sh.empty_z[(j - 1) % kZStages]);
       }
-      if (j > 0) {
-        ok = wait_compute(&sh.full_z[(j - 1) % kZStages], (uint32_t)(((j - 1) / kZStages) & 1), ok);
-        if (ok) epilogue1(j - 1);  // overlaps the MMA of head j
-        compute_sync();
-        if (tid == 0) mbar_arrive(&sh.empty_z[(j - 1) % kZStages]);
-      }
-      tc_fence_before();
-      compute_sync();
     }
     if (ok && nh > 0) {
-      ok = wait_compute(&sh.mbar_mma, (nh - 1) & 1, ok);
-      ok = wait_compute(&sh.full_z[(nh - 1) % kZStages], (uint32_t)(((nh - 1) / kZStages) & 1), ok);
+      wait_warp(&sh.mbar_mma, (uint32_t)((nh - 1) & 1));
+      wait_warp(&sh.full_z[(nh - 1) % kZStages], (uint32_t)(((nh - 1) / kZStages) & 1));
       tc_fence_after();
       if (ok) epilogue1(nh - 1);
     }
-    if (!ok && tid == 0) {
-      // a wait ran out: let issued MMAs and tile copies land before the CTA exits
-      mbar_wait_bounded(&sh.mbar_cb, 0, &g_tc_errors);
-      mbar_wait_bounded(&sh.full_cb, 0, &g_tc_errors);
-      for (int k = 0; k < kXhStages; ++k) mbar_wait_bounded(&sh.full_xh[k], 0, &g_tc_errors);
-      for (int k = 0; k < kZStages; ++k) mbar_wait_bounded(&sh.full_z[k], 0, &g_tc_errors);
+    if (!ok) {
+      sh.ok_flag = 0;
+      if (lane == 0) {
+        // a wait ran out: let issued MMAs and tile copies land before the CTA exits
+        mbar_wait_bounded(&sh.mbar_cb, 0, &g_tc_errors);
+        mbar_wait_bounded(&sh.full_cb, 0, &g_tc_errors);
+      }
     }
     sh.ss[hf][t] = ss_acc;
-    sh.ok_flag = ok;
   }
   __syncthreads();  // producer joins here
 
@@ -1087,7 +1109,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cs, (unsigned)a.nch, (unsigned)(pr.G * pr.batch));
-    cfg.blockDim = dim3(kOutThreads, 1, 1);
+    cfg.blockDim = dim3(kK3Threads, 1, 1);
     cfg.dynamicSmemBytes = kK3Smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
