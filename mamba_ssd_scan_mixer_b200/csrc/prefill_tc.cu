@@ -492,18 +492,20 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a) {
   const float *S = a.S + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
   __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
   const float *ce = a.cum_end + bi * a.nch * pr.H + h;
+  // loads run 8 chunks ahead of the (sequential) recurrence
+  constexpr int kAhead = 8;
   int c = 0;
-  for (; c + 4 <= a.nch; c += 4) {
-    float s[4], d[4];
+  for (; c + kAhead <= a.nch; c += kAhead) {
+    float sv[kAhead], d[kAhead];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      s[k] = S[(c + k) * stride];
+    for (int k = 0; k < kAhead; ++k) {
+      sv[k] = S[(c + k) * stride];
       d[k] = ce[(int64_t)(c + k) * pr.H];
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kAhead; ++k) {
       Hc[(c + k) * stride] = __float2half_rn(hc);
-      hc = expf(d[k]) * hc + s[k];
+      hc = expf(d[k]) * hc + sv[k];
     }
   }
   for (; c < a.nch; ++c) {
