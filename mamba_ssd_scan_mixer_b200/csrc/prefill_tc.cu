@@ -480,39 +480,75 @@ __global__ void __launch_bounds__(kOutThreads, 1)
 }
 
 // ============================================================== state passing
-// grid (P*N/256, H, b): one thread per state element, sequential over chunks.
-__global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a) {
+// grid (P*N/1024 + conv-state blocks, H, b): one thread per 4 consecutive state
+// elements (four independent recurrences, 16-byte loads), sequential over chunks.
+// Blocks with blockIdx.x >= P*N/1024 (only for h = 0) write the final conv
+// state instead: the last 4 raw inputs of [old state | new tokens], in place
+// (the chunk-state kernel, which reads the old state, has finished by now).
+constexpr int kPassBlocks = (kHP * kNS) / 1024;
+
+__global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloat16 *cs) {
   const Problem &pr = a.pr;
-  const int e = blockIdx.x * 256 + threadIdx.x;  // p * 64 + n
   const int h = blockIdx.y;
   const int64_t bi = blockIdx.z;
+  if ((int)blockIdx.x >= kPassBlocks) {
+    if (h != 0 || cs == nullptr) return;
+    const int64_t ch = (int64_t)(blockIdx.x - kPassBlocks) * 256 + threadIdx.x;
+    if (ch >= pr.conv_dim) return;
+    const int64_t i = bi * pr.conv_dim + ch;
+    __nv_bfloat16 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t tau = pr.L - 4 + k;
+      if (tau >= 0) v[k] = a.xBC[(bi * pr.L + tau) * a.ld_x + ch];
+      else v[k] = a.states_in ? cs[i * 4 + 4 + tau] : __float2bfloat16(0.0f);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) cs[i * 4 + k] = v[k];
+    return;
+  }
+  const int e = (blockIdx.x * 256 + threadIdx.x) * 4;  // p * 64 + n, 4 consecutive
   const int64_t hs = (bi * pr.H + h) * (int64_t)(kHP * kNS) + e;
-  float hc = a.states_in ? a.ssm_state[hs] : 0.0f;
+  float4 hc = a.states_in ? *reinterpret_cast<const float4 *>(a.ssm_state + hs)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
   const int64_t stride = (int64_t)pr.H * kHP * kNS;
   const float *S = a.S + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
   __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
   const float *ce = a.cum_end + bi * a.nch * pr.H + h;
+  auto put = [&](int64_t c) {
+    const __half2 lo = __floats2half2_rn(hc.x, hc.y), hi = __floats2half2_rn(hc.z, hc.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t *>(&lo);
+    o.y = *reinterpret_cast<const uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(Hc + c * stride) = o;
+  };
   // loads run 8 chunks ahead of the (sequential) recurrence
   constexpr int kAhead = 8;
   int c = 0;
   for (; c + kAhead <= a.nch; c += kAhead) {
-    float sv[kAhead], d[kAhead];
+    float4 sv[kAhead];
+    float d[kAhead];
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
-      sv[k] = S[(c + k) * stride];
+      sv[k] = *reinterpret_cast<const float4 *>(S + (c + k) * stride);
       d[k] = ce[(int64_t)(c + k) * pr.H];
     }
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
-      Hc[(c + k) * stride] = __float2half_rn(hc);
-      hc = expf(d[k]) * hc + sv[k];
+      put(c + k);
+      const float f = expf(d[k]);
+      hc = make_float4(fmaf(f, hc.x, sv[k].x), fmaf(f, hc.y, sv[k].y), fmaf(f, hc.z, sv[k].z),
+                       fmaf(f, hc.w, sv[k].w));
     }
   }
   for (; c < a.nch; ++c) {
-    Hc[c * stride] = __float2half_rn(hc);
-    hc = expf(ce[(int64_t)c * pr.H]) * hc + S[c * stride];
+    put(c);
+    const float4 sv = *reinterpret_cast<const float4 *>(S + c * stride);
+    const float f = expf(ce[(int64_t)c * pr.H]);
+    hc = make_float4(fmaf(f, hc.x, sv.x), fmaf(f, hc.y, sv.y), fmaf(f, hc.z, sv.z),
+                     fmaf(f, hc.w, sv.w));
   }
-  if (a.ssm_state != nullptr) a.ssm_state[hs] = hc;
+  if (a.ssm_state != nullptr) *reinterpret_cast<float4 *>(a.ssm_state + hs) = hc;
 }
 
 // ============================================================== chunk output
@@ -928,23 +964,6 @@ __global__ void __launch_bounds__(kK3Threads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// Final conv state = last 4 raw inputs of [old state | new tokens], in place.
-__global__ void tc_conv_state_kernel(TcArgs a, __nv_bfloat16 *cs) {
-  const Problem &pr = a.pr;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= pr.batch * pr.conv_dim) return;
-  const int64_t bi = i / pr.conv_dim, ch = i % pr.conv_dim;
-  __nv_bfloat16 v[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int64_t tau = pr.L - 4 + k;
-    if (tau >= 0) v[k] = a.xBC[(bi * pr.L + tau) * a.ld_x + ch];
-    else v[k] = a.states_in ? cs[i * 4 + 4 + tau] : __float2bfloat16(0.0f);
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) cs[i * 4 + k] = v[k];
-}
-
 // Heads per CTA and cluster size of tc_chunk_out for hpg heads per group.
 void out_split(int hpg, int *cs, int *hpc) {
   const int lo = (hpg + kMaxHeadsPerCta - 1) / kMaxHeadsPerCta;
@@ -1029,9 +1048,8 @@ constexpr size_t kK3Smem = kTcOutTiles + sizeof(OutShared) + 1024;
 
 }  // namespace
 
-const char *const kPrefillTcStages[] = {"tc_chunk_state", "tc_state_pass", "tc_chunk_out",
-                                        "tc_conv_state"};
-const int kPrefillTcStageCount = 4;
+const char *const kPrefillTcStages[] = {"tc_chunk_state", "tc_state_pass", "tc_chunk_out"};
+const int kPrefillTcStageCount = 3;
 
 bool prefill_tc_supported(const Problem &pr) {
   const int64_t nch = ceil_div(pr.L, kQ);
@@ -1105,8 +1123,9 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     tc_chunk_state_kernel<<<g1, kOutThreads, kK1Smem, st>>>(a, m1, n_items);
   }
   stage_mark(st, 1);
-  dim3 g2((kHP * kNS) / 256, (unsigned)pr.H, (unsigned)pr.batch);
-  tc_state_pass_kernel<<<g2, 256, 0, st>>>(a);
+  dim3 g2((unsigned)(kPassBlocks + ceil_div(pr.conv_dim, 256)), (unsigned)pr.H,
+          (unsigned)pr.batch);
+  tc_state_pass_kernel<<<g2, 256, 0, st>>>(a, static_cast<__nv_bfloat16 *>(pa.conv_state));
   stage_mark(st, 2);
   {
     cudaLaunchConfig_t cfg = {};
@@ -1140,12 +1159,6 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     if (e != cudaSuccess) return e;
   }
   stage_mark(st, 3);
-  if (pa.conv_state != nullptr) {
-    const int64_t n = pr.batch * pr.conv_dim;
-    tc_conv_state_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(
-        a, static_cast<__nv_bfloat16 *>(pa.conv_state));
-  }
-  stage_mark(st, 4);
   return cudaGetLastError();
 }
 

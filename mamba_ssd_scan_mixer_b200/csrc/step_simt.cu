@@ -34,6 +34,9 @@ constexpr int kMaxStages = 4;  // shared-memory ring of per-head state buffers
 
 static __device__ unsigned int g_step_errors = 0;
 
+// silu with the fast exponential and reciprocal (relative error ~1e-6)
+__device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
+
 template <typename T>
 __device__ __forceinline__ float conv4(const float *w, float b, T a0, T a1, T a2, T a3) {
   return b + w[0] * to_f(a0) + w[1] * to_f(a1) + w[2] * to_f(a2) + w[3] * to_f(a3);
@@ -109,12 +112,12 @@ __global__ void __launch_bounds__(kStepThreads)
       w4[1] = a1;
       w4[2] = a2;
       w4[3] = a3;
-      ux[i] = silu_f(conv4(prm.conv_w + c * 4, prm.conv_b[c], a0, a1, a2, a3));
+      ux[i] = silu_fast(conv4(prm.conv_w + c * 4, prm.conv_b[c], a0, a1, a2, a3));
     }
     for (int j = threadIdx.x; j < 2 * GN; j += blockDim.x) {
       const int64_t c = pr.d_inner + j;
       const T *w4 = csr + c * 4;
-      ubc[j] = silu_f(conv4(prm.conv_w + c * 4, prm.conv_b[c], w4[1], w4[2], w4[3], xr[c]));
+      ubc[j] = silu_fast(conv4(prm.conv_w + c * 4, prm.conv_b[c], w4[1], w4[2], w4[3], xr[c]));
     }
     for (int i = threadIdx.x; i < hpc; i += blockDim.x) {
       const int h = h0 + i;
@@ -173,7 +176,8 @@ __global__ void __launch_bounds__(kStepThreads)
       const int c0 = max(g * hpg, h0) * P - h0 * P, c1 = min((g + 1) * hpg, h0 + hpc) * P - h0 * P;
       float ss = 0.0f;
       for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
-        const float v = pr.nbg ? ys[c] : ys[c] * silu_f(to_f(zr[c]));
+        const float v = pr.nbg ? ys[c] : ys[c] * silu_fast(to_f(zr[c]));
+        if (!pr.nbg) ys[c] = v;  // keep the gated value for the scaling below
         ss += v * v;
       }
       ss = block_sum(ss, red);
@@ -191,8 +195,7 @@ __global__ void __launch_bounds__(kStepThreads)
     const float *nw = prm.norm_w + (int64_t)h0 * P;
     for (int c = threadIdx.x; c < hpc * P; c += blockDim.x) {
       const float sc = inv[(h0 + c / P) / hpg];
-      const float sz = silu_f(to_f(zr[c]));
-      const float o = pr.nbg ? ys[c] * sc * nw[c] * sz : ys[c] * sz * sc * nw[c];
+      const float o = pr.nbg ? ys[c] * sc * nw[c] * silu_fast(to_f(zr[c])) : ys[c] * sc * nw[c];
       yr[c] = from_f<T>(o);
     }
     // 4. shared B/C conv state, now that every CTA of the cluster has read it
@@ -232,6 +235,11 @@ cudaError_t run(const StepArgs &a) {
   cudaError_t e = cudaFuncSetAttribute(ssd_step_kernel<T, N>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  if (cs > 8) {
+    e = cudaFuncSetAttribute(ssd_step_kernel<T, N>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kStepThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
@@ -251,7 +259,11 @@ cudaError_t run(const StepArgs &a) {
     cudaGetLastError();  // clear a failed query; fall back to one cluster per row
     max_clusters = (int)std::min<int64_t>(pr.batch, 65535);
   }
-  const int nclusters = (int)std::max<int64_t>(1, std::min<int64_t>(pr.batch, max_clusters));
+  // the fewest clusters that keep the largest per-cluster row count: no cluster idles
+  // at the end while others still have a row left
+  const int64_t fit = std::max<int64_t>(1, std::min<int64_t>(pr.batch, max_clusters));
+  const int64_t rows_per = (pr.batch + fit - 1) / fit;
+  const int nclusters = (int)std::max<int64_t>(1, (pr.batch + rows_per - 1) / rows_per);
   cfg.gridDim = dim3((unsigned)cs, (unsigned)nclusters, 1);
   stage_mark(a.stream, 0);
   e = cudaLaunchKernelEx(&cfg, ssd_step_kernel<T, N>, pr, a.prm, static_cast<const T *>(a.xBC),
