@@ -182,14 +182,17 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t 
 }
 
 // ============================================================== chunk states
-// Persistent: grid = one CTA per SM, each looping over work items (chunk-major):
-//   pair items (b, chunk, group, head pair): conv + SiLU of x (2 heads) and B,
+// Persistent: grid = one CTA per SM; CTA k takes a contiguous range of work
+// items ordered (row, chunk, group, item), where the items of a (row, chunk,
+// group) are its head pairs followed by one C item:
+//   pair item: conv + SiLU of x (2 heads) and of B (only when the CTA's previous
+//     item had another (row, chunk, group): B's operands stay in shared memory),
 //     post-conv values to u, then S = (x o w)^T B on the tensor cores;
-//   C items (b, chunk, group): conv + SiLU of the group's C channels -> u.
-// 16 compute warps + 1 producer warp.  The producer computes dt / the chunk
-// weights of the next item and TMA-loads its raw bf16 tiles [136 tokens
-// c0-3 .. c0+132][64 ch] (128-byte swizzle) into a two-stage ring while the
-// compute warps work on the current item.
+//   C item: conv + SiLU of the group's C channels -> u.
+// 16 compute warps + 1 producer warp.  The producer computes the next item's
+// dt weights, stages its conv weights and TMA-loads its raw bf16 tiles
+// [136 tokens c0-3 .. c0+132][64 ch] (128-byte swizzle) into a two-stage ring
+// while the compute warps work on the current item.
 // Smem (1024-aligned): ring [2][x_A | x_B | B (a C item uses slot 0)], then the
 // operands A_hi, A_lo [2 k-blocks][128 rows][128 B] and B_hi, B_lo [2][64][128 B].
 constexpr uint32_t kRawRows = 136, kRawBytes = kRawRows * 128;  // 17 KB, 1024-multiple
@@ -203,18 +206,19 @@ struct K1Maps {
 };
 
 // conv1d + SiLU of the 8 channels in 16-byte column `cg` of a raw tile, for
-// output tokens at tile rows s0+3 .. s0+6 (inputs: rows s0 .. s0+6).
-__device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float *conv_w,
-                                             const float *conv_b, int64_t ch, float (&out)[4][8]) {
+// output tokens at tile rows s0+3 .. s0+6 (inputs: rows s0 .. s0+6); taps and
+// bias of the tile's 64 channels in shared memory (wt[64][4], bs[64]).
+__device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float *wt,
+                                             const float *bs, float (&out)[4][8]) {
   float w[8][4], bias[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float4 wv = __ldg(reinterpret_cast<const float4 *>(conv_w) + ch + i);
+    const float4 wv = reinterpret_cast<const float4 *>(wt)[cg * 8 + i];
     w[i][0] = wv.x;
     w[i][1] = wv.y;
     w[i][2] = wv.z;
     w[i][3] = wv.w;
-    bias[i] = __ldg(conv_b + ch + i);
+    bias[i] = bs[cg * 8 + i];
   }
   float rows[7][8];
 #pragma unroll
@@ -243,31 +247,36 @@ struct K1Item {
   int64_t bi;
   int c, g, pair;
   bool isC;
+  int64_t key;  // (row, chunk, group)
 };
 
 __device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs, int64_t it) {
-  const int per = pr.G * pairs + pr.G;  // items per (row, chunk)
-  const int64_t bc = it / per;
-  const int r = (int)(it % per);
+  const int64_t key = it / (pairs + 1);
+  const int r = (int)(it % (pairs + 1));
   K1Item w;
-  w.bi = bc / nch;
+  w.key = key;
+  w.g = (int)(key % pr.G);
+  const int64_t bc = key / pr.G;
   w.c = (int)(bc % nch);
-  if (r < pr.G * pairs) {
-    w.g = r / pairs;
-    w.pair = r % pairs;
-    w.isC = false;
-  } else {
-    w.g = r - pr.G * pairs;
-    w.pair = 0;
-    w.isC = true;
-  }
+  w.bi = bc / nch;
+  w.isC = r == pairs;
+  w.pair = w.isC ? 0 : r;
   return w;
+}
+
+// Whether item `it` (k-th of this CTA) must convolve B afresh.
+__device__ __forceinline__ bool k1_fresh_b(const Problem &pr, int nch, int pairs, int64_t it,
+                                           int k) {
+  if (k == 0) return true;
+  return k1_item(pr, nch, pairs, it).key != k1_item(pr, nch, pairs, it - 1).key;
 }
 
 __global__ void __launch_bounds__(kOutThreads, 1)
     tc_chunk_state_kernel(TcArgs a, const __grid_constant__ K1Maps maps, int64_t n_items) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ float ws[2][2][kQ];  // [stage][head of pair][token] chunk weights
+  __shared__ float ws[2][2][kQ];          // [stage][head of pair][token] chunk weights
+  __shared__ float4 wts[2][3][64];        // [stage][slot][channel] conv taps
+  __shared__ float bss[2][3][64];         // [stage][slot][channel] conv bias
   __shared__ uint64_t full[2], empty[2], mbar;
   __shared__ uint32_t tmem_holder;
   const Problem &pr = a.pr;
@@ -277,11 +286,12 @@ __global__ void __launch_bounds__(kOutThreads, 1)
                  sBlo = base + kK1Blo;
   const int hpg = pr.heads_per_group();
   const int pairs = (hpg + 1) / 2;
+  const int64_t it0 = n_items * blockIdx.x / gridDim.x, it1 = n_items * (blockIdx.x + 1) / gridDim.x;
 
   if (warp == 0) tmem_alloc(&tmem_holder, 64);
   if (tid == 0) {
     for (int k = 0; k < 2; ++k) {
-      mbar_init(&full[k], 1);
+      mbar_init(&full[k], 2);  // the tiles' transaction bytes + the producer's weights
       mbar_init(&empty[k], 1);
     }
     mbar_init(&mbar, 1);
@@ -293,9 +303,10 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   const uint32_t tmem = tmem_holder;
 
   if (warp == kThreads / 32) {
-    // ---------------- producer: dt weights and raw tiles of the next items
+    // ---------------- producer: raw tiles (issued first), then dt weights and conv
+    // taps of the next items
     int k = 0;
-    for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
+    for (int64_t it = it0; it < it1; ++it, ++k) {
       const int st = k & 1;
       if (k >= 2) {
         bool got = lane == 0 ? mbar_wait_bounded(&empty[st], (uint32_t)(((k >> 1) - 1) & 1),
@@ -304,22 +315,50 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         if (!__all_sync(0xffffffffu, got)) break;
       }
       const K1Item w = k1_item(pr, a.nch, pairs, it);
+      const bool freshB = !w.isC && k1_fresh_b(pr, a.nch, pairs, it, k);
       const int64_t c0 = (int64_t)w.c * kQ;
       const int hA = w.g * hpg + 2 * w.pair;
       const bool hasB = 2 * w.pair + 1 < hpg;
+      if (lane == 0) {
+        const uint32_t stage = base + st * kK1Stage;
+        if (w.isC) {
+          mbar_arrive_expect_tx(&full[st], kRawBytes);
+          tma_load_3d(stage, &maps.xbc, (int)(pr.d_inner + (int64_t)(pr.G + w.g) * kNS),
+                      (int)c0 - 3, (int)w.bi, &full[st]);
+        } else {
+          mbar_arrive_expect_tx(&full[st],
+                                (1u + (hasB ? 1u : 0u) + (freshB ? 1u : 0u)) * kRawBytes);
+          tma_load_3d(stage, &maps.xbc, hA * kHP, (int)c0 - 3, (int)w.bi, &full[st]);
+          if (hasB)
+            tma_load_3d(stage + kRawBytes, &maps.xbc, (hA + 1) * kHP, (int)c0 - 3, (int)w.bi,
+                        &full[st]);
+          if (freshB)
+            tma_load_3d(stage + 2 * kRawBytes, &maps.xbc, (int)(pr.d_inner + (int64_t)w.g * kNS),
+                        (int)c0 - 3, (int)w.bi, &full[st]);
+        }
+      }
       if (!w.isC) {
-        for (int half = 0; half < 2; ++half) {
-          const bool hv = half == 0 || hasB;
-          const int h = hA + half;
-          float dt4[4], a4[4];
+        // dt of both heads for this lane's 4 tokens: all loads first
+        float dtr[2][4];
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int64_t tt = c0 + 4 * lane + q;
-            dt4[q] = (hv && tt < pr.L)
-                         ? softplus_f(__bfloat162float(a.dt_raw[(w.bi * pr.L + tt) * a.ld_dt + h]) +
-                                      a.prm.dt_bias[h])
-                         : 0.0f;
-            a4[q] = hv ? dt4[q] * a.prm.A[h] : 0.0f;
+            dtr[half][q] = ((half == 0 || hasB) && tt < pr.L)
+                               ? __bfloat162float(a.dt_raw[(w.bi * pr.L + tt) * a.ld_dt + hA + half])
+                               : -INFINITY;
+          }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const bool hv = half == 0 || hasB;
+          const int h = hA + (hv ? half : 0);
+          const float dtb = a.prm.dt_bias[h], Ah = a.prm.A[h];
+          float dt4[4], a4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            dt4[q] = (hv && dtr[half][q] != -INFINITY) ? softplus_f(dtr[half][q] + dtb) : 0.0f;
+            a4[q] = dt4[q] * Ah;
           }
           const float tot = a4[0] + a4[1] + a4[2] + a4[3];
           float run = warp_scan(tot, lane) - tot;
@@ -329,37 +368,38 @@ __global__ void __launch_bounds__(kOutThreads, 1)
             run += a4[q];
             ws[st][half][4 * lane + q] = expf(cum_end - run) * dt4[q];
           }
-          if (lane == 0 && hv) a.cum_end[(w.bi * a.nch + w.c) * pr.H + h] = cum_end;
+          if (lane == 0 && hv) a.cum_end[(w.bi * a.nch + w.c) * pr.H + hA + half] = cum_end;
+        }
+      }
+      // conv taps and bias of the item's slots
+      for (int sl = 0; sl < 3; ++sl) {
+        int64_t ch0;
+        if (w.isC) {
+          if (sl > 0) break;
+          ch0 = pr.d_inner + (int64_t)(pr.G + w.g) * kNS;
+        } else {
+          if ((sl == 1 && !hasB) || (sl == 2 && !freshB)) continue;
+          ch0 = sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS;
+        }
+        for (int i = lane; i < 64; i += 32) {
+          wts[st][sl][i] = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + i);
+          bss[st][sl][i] = __ldg(a.prm.conv_b + ch0 + i);
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        const uint32_t stage = base + st * kK1Stage;
-        if (w.isC) {
-          mbar_arrive_expect_tx(&full[st], kRawBytes);
-          tma_load_3d(stage, &maps.xbc, (int)(pr.d_inner + (int64_t)(pr.G + w.g) * kNS),
-                      (int)c0 - 3, (int)w.bi, &full[st]);
-        } else {
-          mbar_arrive_expect_tx(&full[st], (hasB ? 3u : 2u) * kRawBytes);
-          tma_load_3d(stage, &maps.xbc, hA * kHP, (int)c0 - 3, (int)w.bi, &full[st]);
-          if (hasB)
-            tma_load_3d(stage + kRawBytes, &maps.xbc, (hA + 1) * kHP, (int)c0 - 3, (int)w.bi,
-                        &full[st]);
-          tma_load_3d(stage + 2 * kRawBytes, &maps.xbc, (int)(pr.d_inner + (int64_t)w.g * kNS),
-                      (int)c0 - 3, (int)w.bi, &full[st]);
-        }
-      }
+      if (lane == 0) mbar_arrive(&full[st]);  // weights of this stage written
     }
   } else {
     // ---------------- compute warps
     bool ok = true;
     int k = 0, npair = 0;
-    for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++k) {
+    for (int64_t it = it0; ok && it < it1; ++it, ++k) {
       const int st = k & 1;
       const uint32_t stage = base + st * kK1Stage;
       ok = wait_compute(&full[st], (uint32_t)((k >> 1) & 1), ok);
       if (!ok) break;
       const K1Item w = k1_item(pr, a.nch, pairs, it);
+      const bool freshB = !w.isC && k1_fresh_b(pr, a.nch, pairs, it, k);
       const int64_t c0 = (int64_t)w.c * kQ;
       const int hA = w.g * hpg + 2 * w.pair;
       const bool hasB = 2 * w.pair + 1 < hpg;
@@ -368,12 +408,15 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         if (w.isC) return pr.d_inner + (int64_t)(pr.G + w.g) * kNS;
         return sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS;
       };
+      auto slot_on = [&](int sl) -> bool {
+        return w.isC ? sl == 0 : (sl == 1 ? hasB : (sl == 2 ? freshB : true));
+      };
       const int nslots = w.isC ? 1 : 3;
       // first chunk: the 3 rows before token 0 come from the carried conv state
       if (c0 == 0 && a.states_in) {
         for (int idx = tid; idx < nslots * 3 * 64; idx += kThreads) {
           const int sl = idx / 192, r = (idx / 64) % 3, chn = idx % 64;
-          if (sl == 1 && !hasB) continue;
+          if (!slot_on(sl)) continue;
           const __nv_bfloat16 v = a.conv_in[(w.bi * pr.conv_dim + slot_ch(sl) + chn) * 4 + 1 + r];
           const uint32_t addr = stage + sl * kRawBytes + r * 128 +
                                 ((((chn >> 3) ^ r) & 7) << 4) + ((chn & 7) << 1);
@@ -382,8 +425,9 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         }
         compute_sync();
       }
-      // conv + SiLU over groups of 8 channels x 32 ranges of 4 tokens
-      const int ncg = w.isC ? 8 : 24;
+      // conv + SiLU over groups of 8 channels x 32 ranges of 4 tokens (one
+      // channel group per warp: the taps are broadcast from shared memory)
+      const int ncg = w.isC ? 8 : (freshB ? 24 : 16);
       for (int item = tid; item < ncg * 32; item += kThreads) {
         const int cgp = item >> 5, tr = item & 31, s0 = tr * 4, cg = cgp & 7;
         const int sl = w.isC ? 0 : cgp >> 3;
@@ -399,7 +443,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         }
         const int64_t ch = slot_ch(sl) + cg * 8;
         float v[4][8];
-        conv8x4_smem(stage + sl * kRawBytes, s0, cg, a.prm.conv_w, a.prm.conv_b, ch, v);
+        conv8x4_smem(stage + sl * kRawBytes, s0, cg, reinterpret_cast<const float *>(wts[st][sl]),
+                     bss[st][sl], v);
         if (w.isC || sl < 2 || w.pair == 0) store_u(a, w.bi, c0 + s0, ch, v);
         if (w.isC) continue;
         const int blk = s0 >> 6;
@@ -435,7 +480,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       compute_sync();
-      if (tid == 0) mbar_arrive(&empty[st]);  // raw tiles of this stage consumed
+      if (tid == 0) mbar_arrive(&empty[st]);  // raw tiles and taps of this stage consumed
       if (w.isC) continue;
       if (tid == 0) {
         tc_fence_after();
@@ -1111,7 +1156,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   if (e != cudaSuccess) return e;
 
   stage_mark(st, 0);
-  const int64_t n_items = pr.batch * a.nch * (int64_t)(pr.G * ((hpg + 1) / 2) + pr.G);
+  const int64_t n_items = pr.batch * a.nch * (int64_t)pr.G * ((hpg + 1) / 2 + 1);
   const unsigned g1 = (unsigned)std::min<int64_t>(n_items, sm_count());
   {
     K1Maps m1;
