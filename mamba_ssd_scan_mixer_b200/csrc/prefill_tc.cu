@@ -64,9 +64,11 @@ struct TcArgs {
   float *ssm_state;              // in (if states_in) / out (may be null)
   int states_in;
   int nch;                       // chunks of kQ tokens
-  float *S;                      // [b][nch][H][64][64] chunk states
+  float *S;                      // [b][nch][H][n/4 16][p 64][4] chunk states
   float *cum_end;                // [b][nch][H] chunk sum of dt*A
-  __half *Hc;                    // [b][nch][H][64][64] state entering each chunk
+  float *cum;                    // [b][nch][H][128] running sum of dt*A inside the chunk
+  float *dtv;                    // [b][nch][H][128] dt (0 past the end of the sequence)
+  __half *Hc;                    // [b][nch][H][n 64][p 64] state entering each chunk
   __half *u;                     // [b][L][conv_dim] post-conv x | B | C, fp16
   int hpc;                       // max heads per CTA in tc_chunk_out
 };
@@ -150,6 +152,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
+                                             int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+// Commit the issued bulk stores and wait until they have read shared memory.
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -207,18 +229,19 @@ struct K1Maps {
 
 // conv1d + SiLU of the 8 channels in 16-byte column `cg` of a raw tile, for
 // output tokens at tile rows s0+3 .. s0+6 (inputs: rows s0 .. s0+6); taps and
-// bias of the tile's 64 channels in shared memory (wt[64][4], bs[64]).
-__device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float *wt,
+// bias of the tile's 64 channels in shared memory, channel 8 g + i at [i][g]
+// (wt[8][8] float4, bs[8][8]) so that neighbouring groups read neighbouring words.
+__device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float4 *wt,
                                              const float *bs, float (&out)[4][8]) {
   float w[8][4], bias[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float4 wv = reinterpret_cast<const float4 *>(wt)[cg * 8 + i];
+    const float4 wv = wt[i * 8 + cg];
     w[i][0] = wv.x;
     w[i][1] = wv.y;
     w[i][2] = wv.z;
     w[i][3] = wv.w;
-    bias[i] = bs[cg * 8 + i];
+    bias[i] = bs[i * 8 + cg];
   }
   float rows[7][8];
 #pragma unroll
@@ -247,32 +270,28 @@ struct K1Item {
   int64_t bi;
   int c, g, pair;
   bool isC;
-  int64_t key;  // (row, chunk, group)
+  bool freshB;  // B must be convolved (the CTA's previous item had another key)
 };
 
-__device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs, int64_t it) {
-  const int64_t key = it / (pairs + 1);
-  const int r = (int)(it % (pairs + 1));
+// Item `it`, the k-th of its CTA.  Items are ordered (row, chunk, group, r) with
+// r = 0 .. pairs - 1 the head pairs and r = pairs the C item; every index fits
+// in 32 bits (the launch checks the item count).
+__device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs, int it, int k) {
+  const unsigned key = (unsigned)it / (unsigned)(pairs + 1);
+  const int r = it - (int)key * (pairs + 1);
+  const unsigned bc = key / (unsigned)pr.G;
   K1Item w;
-  w.key = key;
-  w.g = (int)(key % pr.G);
-  const int64_t bc = key / pr.G;
-  w.c = (int)(bc % nch);
-  w.bi = bc / nch;
+  w.g = (int)(key - bc * (unsigned)pr.G);
+  w.bi = (int64_t)(bc / (unsigned)nch);
+  w.c = (int)(bc - (unsigned)w.bi * (unsigned)nch);
   w.isC = r == pairs;
   w.pair = w.isC ? 0 : r;
+  w.freshB = !w.isC && (k == 0 || r == 0);
   return w;
 }
 
-// Whether item `it` (k-th of this CTA) must convolve B afresh.
-__device__ __forceinline__ bool k1_fresh_b(const Problem &pr, int nch, int pairs, int64_t it,
-                                           int k) {
-  if (k == 0) return true;
-  return k1_item(pr, nch, pairs, it).key != k1_item(pr, nch, pairs, it - 1).key;
-}
-
 __global__ void __launch_bounds__(kOutThreads, 1)
-    tc_chunk_state_kernel(TcArgs a, const __grid_constant__ K1Maps maps, int64_t n_items) {
+    tc_chunk_state_kernel(TcArgs a, const __grid_constant__ K1Maps maps, int n_items) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ float ws[2][2][kQ];          // [stage][head of pair][token] chunk weights
   __shared__ float4 wts[2][3][64];        // [stage][slot][channel] conv taps
@@ -286,7 +305,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
                  sBlo = base + kK1Blo;
   const int hpg = pr.heads_per_group();
   const int pairs = (hpg + 1) / 2;
-  const int64_t it0 = n_items * blockIdx.x / gridDim.x, it1 = n_items * (blockIdx.x + 1) / gridDim.x;
+  const int it0 = (int)((int64_t)n_items * blockIdx.x / gridDim.x),
+            it1 = (int)((int64_t)n_items * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == 0) tmem_alloc(&tmem_holder, 64);
   if (tid == 0) {
@@ -306,7 +326,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     // ---------------- producer: raw tiles (issued first), then dt weights and conv
     // taps of the next items
     int k = 0;
-    for (int64_t it = it0; it < it1; ++it, ++k) {
+    for (int it = it0; it < it1; ++it, ++k) {
       const int st = k & 1;
       if (k >= 2) {
         bool got = lane == 0 ? mbar_wait_bounded(&empty[st], (uint32_t)(((k >> 1) - 1) & 1),
@@ -314,8 +334,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
                              : true;
         if (!__all_sync(0xffffffffu, got)) break;
       }
-      const K1Item w = k1_item(pr, a.nch, pairs, it);
-      const bool freshB = !w.isC && k1_fresh_b(pr, a.nch, pairs, it, k);
+      const K1Item w = k1_item(pr, a.nch, pairs, it, k);
+      const bool freshB = w.freshB;
       const int64_t c0 = (int64_t)w.c * kQ;
       const int hA = w.g * hpg + 2 * w.pair;
       const bool hasB = 2 * w.pair + 1 < hpg;
@@ -363,12 +383,19 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           const float tot = a4[0] + a4[1] + a4[2] + a4[3];
           float run = warp_scan(tot, lane) - tot;
           const float cum_end = __shfl_sync(0xffffffffu, run + tot, 31);
+          float cq[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             run += a4[q];
+            cq[q] = run;
             ws[st][half][4 * lane + q] = expf(cum_end - run) * dt4[q];
           }
-          if (lane == 0 && hv) a.cum_end[(w.bi * a.nch + w.c) * pr.H + hA + half] = cum_end;
+          if (hv) {
+            const int64_t row = (w.bi * a.nch + w.c) * pr.H + hA + half;
+            reinterpret_cast<float4 *>(a.cum + row * kQ)[lane] = make_float4(cq[0], cq[1], cq[2], cq[3]);
+            reinterpret_cast<float4 *>(a.dtv + row * kQ)[lane] = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
+            if (lane == 0) a.cum_end[row] = cum_end;
+          }
         }
       }
       // conv taps and bias of the item's slots
@@ -382,8 +409,9 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           ch0 = sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS;
         }
         for (int i = lane; i < 64; i += 32) {
-          wts[st][sl][i] = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + i);
-          bss[st][sl][i] = __ldg(a.prm.conv_b + ch0 + i);
+          const int d = (i & 7) * 8 + (i >> 3);  // [channel in group][group]
+          wts[st][sl][d] = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + i);
+          bss[st][sl][d] = __ldg(a.prm.conv_b + ch0 + i);
         }
       }
       __syncwarp();
@@ -392,14 +420,38 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   } else {
     // ---------------- compute warps
     bool ok = true;
-    int k = 0, npair = 0;
-    for (int64_t it = it0; ok && it < it1; ++it, ++k) {
+    int k = 0, npair_done = 0;
+    // the pair item whose MMA is in flight: its chunk states are stored from TMEM
+    // (rows m = 32 (warp % 4) + lane, 16 columns per warp / 4; S is kept
+    // [n/4][p][4] per head so that a warp's float4 stores are contiguous)
+    struct Pending {
+      int64_t bi;
+      int c, hA;
+      bool hasB;
+    } pw{};
+    bool pending = false;
+    auto store_states = [&](const Pending &q) {
+      tc_fence_after();
+      const int m = 32 * (warp & 3) + lane, half = m >> 6, p = m & 63, cb = warp >> 2;
+      float sv[16];
+      tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 16 * cb, sv);
+      if (half == 0 || q.hasB) {
+        float4 *dst = reinterpret_cast<float4 *>(
+            a.S + ((q.bi * a.nch + q.c) * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[(4 * cb + i) * kHP + p] =
+              make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
+      }
+      tc_fence_before();  // TMEM read before the next MMA is issued
+    };
+    for (int it = it0; ok && it < it1; ++it, ++k) {
       const int st = k & 1;
       const uint32_t stage = base + st * kK1Stage;
       ok = wait_compute(&full[st], (uint32_t)((k >> 1) & 1), ok);
       if (!ok) break;
-      const K1Item w = k1_item(pr, a.nch, pairs, it);
-      const bool freshB = !w.isC && k1_fresh_b(pr, a.nch, pairs, it, k);
+      const K1Item w = k1_item(pr, a.nch, pairs, it, k);
+      const bool freshB = w.freshB;
       const int64_t c0 = (int64_t)w.c * kQ;
       const int hA = w.g * hpg + 2 * w.pair;
       const bool hasB = 2 * w.pair + 1 < hpg;
@@ -410,6 +462,46 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       };
       auto slot_on = [&](int sl) -> bool {
         return w.isC ? sl == 0 : (sl == 1 ? hasB : (sl == 2 ? freshB : true));
+      };
+      // missing second head: zero rows 64..127 of the x operands
+      auto zero_tile = [&](int cg, int s0) {
+        const int blk = s0 >> 6, kq = s0 & 63;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t off = blk * 16384 + sw128_off(64 + cg * 8 + i, kq);
+          st_shared_v2(sAhi + off, 0u, 0u);
+          st_shared_v2(sAlo + off, 0u, 0u);
+        }
+      };
+      // operands of one tile: x o w (slots 0, 1) or B (slot 2), split into fp16 hi + lo
+      auto put_operands = [&](int sl, int cg, int s0, const float (&v)[4][8]) {
+        const int blk = s0 >> 6, kq = s0 & 63;
+        float wk[4] = {1.0f, 1.0f, 1.0f, 1.0f};  // x is weighted per token, B is not
+        if (sl < 2) {
+          const float4 w4 = *reinterpret_cast<const float4 *>(&ws[st][sl][s0]);
+          wk[0] = w4.x;
+          wk[1] = w4.y;
+          wk[2] = w4.z;
+          wk[3] = w4.w;
+        }
+        const bool rot = (cg & 1) != 0;
+        const uint32_t hi_base = sl < 2 ? sAhi + blk * 16384 : sBhi + blk * 8192;
+        const uint32_t lo_base = sl < 2 ? sAlo + blk * 16384 : sBlo + blk * 8192;
+        const int row0 = (sl < 2 ? sl * 64 : 0) + cg * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float hq[4], lq[4];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const float x = (rot ? v[kk][i ^ 4] : v[kk][i]) * wk[kk];
+            // hi: x cut to 11 significant bits (an fp16 value), lo: the exact rest
+            hq[kk] = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+            lq[kk] = x - hq[kk];
+          }
+          const uint32_t off = sw128_off(row0 + (rot ? (i ^ 4) : i), kq);
+          st_shared_v2(hi_base + off, pack_half2(hq[0], hq[1]), pack_half2(hq[2], hq[3]));
+          st_shared_v2(lo_base + off, pack_half2(lq[0], lq[1]), pack_half2(lq[2], lq[3]));
+        }
       };
       const int nslots = w.isC ? 1 : 3;
       // first chunk: the 3 rows before token 0 come from the carried conv state
@@ -425,63 +517,62 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         }
         compute_sync();
       }
-      // conv + SiLU over groups of 8 channels x 32 ranges of 4 tokens (one
-      // channel group per warp: the taps are broadcast from shared memory)
-      const int ncg = w.isC ? 8 : (freshB ? 24 : 16);
-      for (int item = tid; item < ncg * 32; item += kThreads) {
-        const int cgp = item >> 5, tr = item & 31, s0 = tr * 4, cg = cgp & 7;
-        const int sl = w.isC ? 0 : cgp >> 3;
+      // conv + SiLU.  Warp tile: one slot x 4 groups of 8 channels x 8 quads of
+      // tokens (lane = group lane % 4, quad lane / 4).  This tile reads the
+      // swizzled raw rows, stores u (64 contiguous bytes per token) and, with the
+      // channel order of odd groups rotated by 4, stores the swizzled operands
+      // without shared-memory bank conflicts.
+      //
+      // A pair item whose B operand is already in shared memory has exactly one
+      // tile per warp: its values stay in registers until the previous item's MMA
+      // has completed, so that MMA runs under this item's convolution.  Other pair
+      // items first wait for that MMA, then write their operands tile by tile.
+      const bool overlap = !w.isC && !freshB;
+      if (!w.isC && !overlap && pending) {
+        ok = wait_compute(&mbar, (uint32_t)(npair_done & 1), ok);
+        if (ok) {
+          store_states(pw);
+          pending = false;
+          ++npair_done;
+        }
+      }
+      const int ntiles = 8 * (w.isC ? 1 : (freshB ? 3 : 2));
+      float v[4][8];
+      int keep_sl = 0, keep_cg = 0, keep_s0 = 0;
+      for (int wt = warp; wt < ntiles; wt += kThreads / 32) {
+        const int sl = wt >> 3;
+        const int cg = 4 * ((wt >> 2) & 1) + (lane & 3);
+        const int s0 = 4 * (8 * (wt & 3) + (lane >> 2));
+        keep_sl = sl;
+        keep_cg = cg;
+        keep_s0 = s0;
         if (sl == 1 && !hasB) {  // missing second head: zero rows 64..127
-          const int blk = s0 >> 6;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t off = blk * 16384 + sw128_off(64 + cg * 8 + i, s0 & 63);
-            st_shared_v2(sAhi + off, 0u, 0u);
-            st_shared_v2(sAlo + off, 0u, 0u);
-          }
+          if (!overlap) zero_tile(cg, s0);
           continue;
         }
-        const int64_t ch = slot_ch(sl) + cg * 8;
-        float v[4][8];
-        conv8x4_smem(stage + sl * kRawBytes, s0, cg, reinterpret_cast<const float *>(wts[st][sl]),
-                     bss[st][sl], v);
-        if (w.isC || sl < 2 || w.pair == 0) store_u(a, w.bi, c0 + s0, ch, v);
-        if (w.isC) continue;
-        const int blk = s0 >> 6;
-        if (sl < 2) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float q[4], r[4];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const float x = v[kk][i] * ws[st][sl][s0 + kk];
-              q[kk] = __half2float(__float2half_rn(x));
-              r[kk] = x - q[kk];
-            }
-            const uint32_t off = blk * 16384 + sw128_off(sl * 64 + cg * 8 + i, s0 & 63);
-            st_shared_v2(sAhi + off, pack_half2(q[0], q[1]), pack_half2(q[2], q[3]));
-            st_shared_v2(sAlo + off, pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
+        conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
+        if (w.isC || sl < 2 || w.pair == 0) store_u(a, w.bi, c0 + s0, slot_ch(sl) + cg * 8, v);
+        if (!w.isC && !overlap) put_operands(sl, cg, s0, v);
+      }
+      if (overlap) {
+        if (pending) {
+          ok = wait_compute(&mbar, (uint32_t)(npair_done & 1), ok);
+          if (ok) {
+            store_states(pw);
+            pending = false;
+            ++npair_done;
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float q[4], r[4];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              q[kk] = __half2float(__float2half_rn(v[kk][i]));
-              r[kk] = v[kk][i] - q[kk];
-            }
-            const uint32_t off = blk * 8192 + sw128_off(cg * 8 + i, s0 & 63);
-            st_shared_v2(sBhi + off, pack_half2(q[0], q[1]), pack_half2(q[2], q[3]));
-            st_shared_v2(sBlo + off, pack_half2(r[0], r[1]), pack_half2(r[2], r[3]));
-          }
+        }
+        if (ok) {
+          if (keep_sl == 1 && !hasB) zero_tile(keep_cg, keep_s0);
+          else put_operands(keep_sl, keep_cg, keep_s0, v);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       compute_sync();
       if (tid == 0) mbar_arrive(&empty[st]);  // raw tiles and taps of this stage consumed
-      if (w.isC) continue;
+      if (w.isC || !ok) continue;
       if (tid == 0) {
         tc_fence_after();
         const uint32_t idesc = umma_idesc_f16(128, 64);
@@ -495,27 +586,23 @@ __global__ void __launch_bounds__(kOutThreads, 1)
           }
         umma_commit(&mbar);
       }
-      ok = wait_compute(&mbar, (uint32_t)(npair & 1), ok);
-      ++npair;
-      tc_fence_after();
+      pending = true;
+      pw.bi = w.bi;
+      pw.c = w.c;
+      pw.hA = hA;
+      pw.hasB = hasB;
+    }
+    if (ok && pending) {
+      ok = wait_compute(&mbar, (uint32_t)(npair_done & 1), ok);
       if (ok) {
-        // rows m = 32*(warp%4) + lane; warp/4 selects 16 of the 64 columns
-        const int m = 32 * (warp & 3) + lane, half = m >> 6, p = m & 63, cb = 16 * (warp >> 2);
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + cb, v);
-        if (half == 0 || hasB) {
-          float4 *dst = reinterpret_cast<float4 *>(
-              a.S + (((w.bi * a.nch + w.c) * pr.H + hA + half) * kHP + p) * kNS + cb);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
+        store_states(pw);
+        pending = false;
       }
-      tc_fence_before();
-      compute_sync();  // TMEM read and operand smem free before the next item
     }
     if (!ok && tid == 0) {
-      // a wait ran out: let copies already issued land before the CTA exits
+      // a wait ran out: let the MMA and the copies already issued land before the
+      // CTA frees its tensor memory and exits
+      if (pending) mbar_wait_bounded(&mbar, (uint32_t)(npair_done & 1), &g_tc_errors);
       for (int s2 = 0; s2 < 2; ++s2) mbar_wait_bounded(&full[s2], 0, &g_tc_errors);
     }
   }
@@ -525,8 +612,9 @@ __global__ void __launch_bounds__(kOutThreads, 1)
 }
 
 // ============================================================== state passing
-// grid (P*N/1024 + conv-state blocks, H, b): one thread per 4 consecutive state
-// elements (four independent recurrences, 16-byte loads), sequential over chunks.
+// grid (P*N/1024 + conv-state blocks, H, b): one thread per 4 state elements of
+// one p and consecutive n (four independent recurrences, 16-byte loads of the
+// chunk states), sequential over chunks.
 // Blocks with blockIdx.x >= P*N/1024 (only for h = 0) write the final conv
 // state instead: the last 4 raw inputs of [old state | new tokens], in place
 // (the chunk-state kernel, which reads the old state, has finished by now).
@@ -552,20 +640,22 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
     for (int k = 0; k < 4; ++k) cs[i * 4 + k] = v[k];
     return;
   }
-  const int e = (blockIdx.x * 256 + threadIdx.x) * 4;  // p * 64 + n, 4 consecutive
-  const int64_t hs = (bi * pr.H + h) * (int64_t)(kHP * kNS) + e;
+  // float4 slot j of a head's 64 x 64 state: n = 4 (j / 64) .. +3, p = j % 64 (the
+  // chunk-state layout [n/4][p][4]); H_c is stored [n][p] (the MN-major MMA operand)
+  const int j = blockIdx.x * 256 + threadIdx.x, n4 = j >> 6, p = j & 63;
+  const int64_t hs = (bi * pr.H + h) * (int64_t)(kHP * kNS) + p * kNS + 4 * n4;
   float4 hc = a.states_in ? *reinterpret_cast<const float4 *>(a.ssm_state + hs)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
   const int64_t stride = (int64_t)pr.H * kHP * kNS;
-  const float *S = a.S + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
-  __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + e;
+  const float *S = a.S + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + 4 * j;
+  __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + (4 * n4) * kHP + p;
   const float *ce = a.cum_end + bi * a.nch * pr.H + h;
   auto put = [&](int64_t c) {
-    const __half2 lo = __floats2half2_rn(hc.x, hc.y), hi = __floats2half2_rn(hc.z, hc.w);
-    uint2 o;
-    o.x = *reinterpret_cast<const uint32_t *>(&lo);
-    o.y = *reinterpret_cast<const uint32_t *>(&hi);
-    *reinterpret_cast<uint2 *>(Hc + c * stride) = o;
+    __half *o = Hc + c * stride;
+    o[0] = __float2half_rn(hc.x);
+    o[kHP] = __float2half_rn(hc.y);
+    o[2 * kHP] = __float2half_rn(hc.z);
+    o[3 * kHP] = __float2half_rn(hc.w);
   };
   // loads run 8 chunks ahead of the (sequential) recurrence
   constexpr int kAhead = 8;
@@ -597,16 +687,24 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
 }
 
 // ============================================================== chunk output
-// grid (cs, nch, G * b), cluster (cs, 1, 1); 8 compute warps + 1 TMA producer
-// warp.  Tiles arrive by TMA in 128-byte-swizzled layouts (1024-aligned):
+// grid (cs, nch, G * b), cluster (cs, 1, 1); 16 compute warps + 1 TMA producer
+// warp + 1 MMA-issuer warp.  Tiles arrive by TMA in 128-byte-swizzled layouts
+// (1024-aligned).  The operand A is double-buffered so that the A-build of head
+// j + 1 overlaps the MMA of head j; buffer 1 reuses the B tile once CB is formed.
 constexpr uint32_t kCt = 0;                      // C   [128 t][64 n] fp16     16 KB (u)
 constexpr uint32_t kBt = kCt + 16384;            // B   [128 s][64 n] fp16     16 KB (u)
-constexpr int kXhStages = 3, kZStages = 2;
-constexpr uint32_t kXhBytes = 16384 + 8192;      // per stage: x [128 s][64 p] + H_c [64 p][64 n]
-constexpr uint32_t kXh = kBt + 16384;            // x / H_c ring  3 x 24 KB (x at +0, H_c at +16 KB)
+constexpr int kXhStages = 2, kZStages = 2;
+constexpr uint32_t kXhBytes = 16384 + 8192;      // per stage: x [128 s][64 p] + H_c [64 n][64 p]
+constexpr uint32_t kXh = kBt + 16384;            // x / H_c ring  2 x 24 KB (x at +0, H_c at +16 KB)
 constexpr uint32_t kZt = kXh + kXhStages * kXhBytes;  // z ring [128 t][64 p] bf16  2 x 16 KB
-constexpr uint32_t kAt = kZt + kZStages * 16384;      // A   [3][128 t][64 k] fp16  48 KB
-constexpr uint32_t kTcOutTiles = kAt + 3 * 16384;     // 184 KB
+constexpr uint32_t kA0 = kZt + kZStages * 16384;      // A buffer 0: [3][128 t][64 k] fp16  48 KB
+constexpr uint32_t kA1 = kA0 + 3 * 16384;             // A buffer 1, blocks 1 and 2 (block 0 at kBt)
+constexpr uint32_t kTcOutTiles = kA1 + 2 * 16384;     // 192 KB
+
+// Byte offset of k-block `blk` (0, 1: CB columns s; 2: scaled C) of A buffer `buf`.
+__device__ __forceinline__ uint32_t a_block(int buf, int blk) {
+  return buf == 0 ? kA0 + blk * 16384 : (blk == 0 ? kBt : kA1 + (blk - 1) * 16384);
+}
 
 struct OutShared {
   float cum2[kMaxHeadsPerCta][kQ];  // cumsum * log2(e)
@@ -617,11 +715,12 @@ struct OutShared {
   float ecum[kMaxHeadsPerCta][kQ];  // exp(cumsum)
   float nw[kMaxHeadsPerCta][kHP];   // norm weight of the CTA's channels
   float ss[4][kQ];
-  float part[16][kQ];               // per-rank partial sums of squares (rank 0's is read)
+  float part[16][kQ];               // partial sums of squares of every rank of the cluster
+  float mine[kQ];                   // this CTA's partial sums
   float inv[kQ];
   float Dh[kMaxHeadsPerCta];
   uint64_t full_cb, full_xh[kXhStages], empty_xh[kXhStages], full_z[kZStages],
-      empty_z[kZStages], a_ready, mbar_cb, mbar_mma;
+      empty_z[kZStages], a_ready[2], mbar_cb, mbar_mma[2];
   uint32_t tmem_holder;
   int ok_flag;
 };
@@ -630,6 +729,7 @@ struct OutMaps {
   CUtensorMap u;   // [b][L][conv_dim] fp16, box 64 ch x 128 tokens
   CUtensorMap z;   // [b][L][d_inner] bf16 (row stride ld_z), box 64 x 128
   CUtensorMap hc;  // [rows][64] fp16, box 64 x 64
+  CUtensorMap y;   // [b][L][d_inner] bf16, box 64 x 128 (stores)
 };
 
 __global__ void __launch_bounds__(kK3Threads, 1)
@@ -663,15 +763,18 @@ __global__ void __launch_bounds__(kK3Threads, 1)
       mbar_init(&sh.full_z[k], 1);
       mbar_init(&sh.empty_z[k], kThreads);  // every compute thread after its epilogue
     }
-    mbar_init(&sh.a_ready, kThreads);       // every compute thread after its A-build
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&sh.a_ready[k], kThreads);  // every compute thread after its A-build
+      mbar_init(&sh.mbar_mma[k], 1);        // MMA of a head that used A buffer k
+    }
     mbar_init(&sh.mbar_cb, 1);
-    mbar_init(&sh.mbar_mma, 1);
     fence_mbar_init();
     sh.ok_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  cluster_arrive_relaxed();  // waited for before the first remote store
   const uint32_t tmem = sh.tmem_holder;
 
   if (warp == kThreads / 32) {
@@ -714,10 +817,9 @@ __global__ void __launch_bounds__(kK3Threads, 1)
                    umma_desc_sw128(base + kBt + kin * 32), idesc, kin > 0 ? 1u : 0u);
         umma_commit(&sh.mbar_cb);
       }
-      const uint32_t idesc_k = umma_idesc_f16(128, 64);
-      const uint32_t idesc_mn = idesc_k | (1u << 16);  // B operand MN-major (x tile)
+      const uint32_t idesc_mn = umma_idesc_f16(128, 64) | (1u << 16);  // B operand MN-major
       for (int j = 0; ok && j < nh; ++j) {
-        ok = mbar_wait_bounded(&sh.a_ready, (uint32_t)(j & 1), &g_tc_errors) &&
+        ok = mbar_wait_bounded(&sh.a_ready[j & 1], (uint32_t)((j >> 1) & 1), &g_tc_errors) &&
              mbar_wait_bounded(&sh.full_xh[j % kXhStages], (uint32_t)((j / kXhStages) & 1),
                                &g_tc_errors);
         if (!ok) break;
@@ -725,40 +827,34 @@ __global__ void __launch_bounds__(kK3Threads, 1)
         const uint32_t xt = base + kXh + (j % kXhStages) * kXhBytes, ht = xt + 16384;
         for (int ks = 0; ks < 12; ++ks) {
           const int blk = ks >> 2, kin = ks & 3;
-          const uint64_t ad = umma_desc_sw128(base + kAt + blk * 16384 + kin * 32);
+          const uint64_t ad = umma_desc_sw128(base + a_block(j & 1, blk) + kin * 32);
+          // x [s][p] and H_c [n][p] are both MN-major (p contiguous)
           if (ks < 8)
             umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn,
                      ks > 0 ? 1u : 0u);
           else
-            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128(ht + kin * 32), idesc_k, 1u);
+            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(ht + (ks - 8) * 2048, 8192),
+                     idesc_mn, 1u);
         }
-        umma_commit(&sh.mbar_mma);
+        umma_commit(&sh.mbar_mma[j & 1]);
         umma_commit(&sh.empty_xh[j % kXhStages]);  // its x / H_c stage is free once it completes
       }
       if (!ok) sh.ok_flag = 0;
     }
   } else {
     // ---------------- compute warps
-    // dt / cumsum: one warp per head, 4 consecutive tokens per lane
+    // decay terms: one warp per head, 4 consecutive tokens per lane, from the
+    // per-chunk dt and cumsum rows the chunk-state kernel wrote
     if (warp < nh) {
       const int j = warp, h = h0 + j;
-      float dt4[4], a4[4];
-      const float dtb = a.prm.dt_bias[h], Ah = a.prm.A[h];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int64_t tt = c0 + 4 * lane + k;
-        dt4[k] = tt < pr.L ? softplus_f(__bfloat162float(a.dt_raw[(bi * pr.L + tt) * a.ld_dt + h]) +
-                                        dtb)
-                           : 0.0f;
-        a4[k] = dt4[k] * Ah;
-      }
-      const float tot = a4[0] + a4[1] + a4[2] + a4[3];
-      float run = warp_scan(tot, lane) - tot;
+      const int64_t row = (bi * a.nch + c) * pr.H + h;
+      const float4 cu = reinterpret_cast<const float4 *>(a.cum + row * kQ)[lane];
+      const float4 dv = reinterpret_cast<const float4 *>(a.dtv + row * kQ)[lane];
+      const float cum4[4] = {cu.x, cu.y, cu.z, cu.w}, dt4[4] = {dv.x, dv.y, dv.z, dv.w};
       float c2[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        run += a4[k];
-        c2[k] = run * kLog2e;
+        c2[k] = cum4[k] * kLog2e;
         sh.cum2[j][4 * lane + k] = c2[k];
         sh.dt[j][4 * lane + k] = dt4[k];
         sh.ecum[j][4 * lane + k] = ex2_approx(c2[k]);
@@ -772,8 +868,6 @@ __global__ void __launch_bounds__(kK3Threads, 1)
       }
       if ((lane & 7) == 7) sh.span_ok[j][lane >> 3] = (c2s0 - c2r) <= 60.0f;
     }
-    for (int i = tid; i < nh * kHP; i += kThreads)
-      sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
     for (int i = tid; i < nh * kHP; i += kThreads)
       sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
     if (tid < nh) sh.Dh[tid] = a.prm.D[h0 + tid];
@@ -814,21 +908,22 @@ __global__ void __launch_bounds__(kK3Threads, 1)
     };
 
     for (int j = 0; j < nh; ++j) {
-      // the A buffer is free (and Y_{j-1} complete) once the previous MMA is done
+      // A buffer j % 2 is free: the MMA of head j - 2 was waited for by the
+      // epilogue of that head in the previous iteration
       if (j == 0) {
         wait_warp(&sh.full_cb, 0);  // the C tile (read below for the scaled-C block)
-        wait_warp(&sh.mbar_cb, 0);
-      } else {
-        wait_warp(&sh.mbar_mma, (uint32_t)((j - 1) & 1));
+        wait_warp(&sh.mbar_cb, 0);  // CB in TMEM; the B tile is free (A buffer 1)
       }
       if (!ok) break;
       tc_fence_after();
+      const uint32_t abuf = base + a_block(j & 1, 0), abuf2 = base + a_block(j & 1, 2);
+      const uint32_t abuf1 = base + a_block(j & 1, 1);
       // A_j = [CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal | C o exp(cum_t)];
       // 32-column groups k above the row quarter q are zero, below it the decay
       // factorises as alpha_t beta_s (both <= 1), on it exponentials are direct.
       {
         const int k = hf, s0 = 32 * k;  // this warp's 32-column group
-        const uint32_t at = base + kAt + (k >> 1) * 16384;
+        const uint32_t at = (k >> 1) == 0 ? abuf : abuf1;
         const int kc = 32 * (k & 1);       // column of the group inside its 64-wide block
         const float c2t = sh.cum2[j][t];
         if (k > q) {
@@ -917,21 +1012,23 @@ __global__ void __launch_bounds__(kK3Threads, 1)
             const float2 f = unpack_half2(in[e]);
             o[e] = pack_half2(f.x * ec, f.y * ec);
           }
-          st_shared_v4(base + kAt + 2 * 16384 + sw128_chunk(t, n0), o[0], o[1], o[2], o[3]);
+          st_shared_v4(abuf2 + sw128_chunk(t, n0), o[0], o[1], o[2], o[3]);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&sh.a_ready);
+      mbar_arrive(&sh.a_ready[j & 1]);
       if (j > 0) {  // epilogue of the previous head overlaps this head's MMA
+        wait_warp(&sh.mbar_mma[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1));
         wait_warp(&sh.full_z[(j - 1) % kZStages], (uint32_t)(((j - 1) / kZStages) & 1));
         if (!ok) break;
+        tc_fence_after();
         epilogue1(j - 1);
         mbar_arrive(&sh.empty_z[(j - 1) % kZStages]);
       }
     }
     if (ok && nh > 0) {
-      wait_warp(&sh.mbar_mma, (uint32_t)((nh - 1) & 1));
+      wait_warp(&sh.mbar_mma[(nh - 1) & 1], (uint32_t)(((nh - 1) >> 1) & 1));
       wait_warp(&sh.full_z[(nh - 1) % kZStages], (uint32_t)(((nh - 1) / kZStages) & 1));
       tc_fence_after();
       if (ok) epilogue1(nh - 1);
@@ -948,17 +1045,30 @@ __global__ void __launch_bounds__(kK3Threads, 1)
   }
   __syncthreads();  // producer joins here
 
-  // per-token sums of squares of this CTA -> rank 0's table; totals; scale
-  float *part0 = cluster.map_shared_rank(&sh.part[0][0], 0);
-  if (tid < kQ) part0[rank * kQ + tid] = (sh.ss[0][tid] + sh.ss[1][tid]) + (sh.ss[2][tid] + sh.ss[3][tid]);
-  cluster.sync();
+  // per-token sums of squares of this CTA, pushed into every rank's table
+  // part[rank][t] (plain remote stores), then one cluster barrier; after it each
+  // CTA only reads its own shared memory, so none waits for the others to exit
+  if (tid < kQ) sh.mine[tid] = (sh.ss[0][tid] + sh.ss[1][tid]) + (sh.ss[2][tid] + sh.ss[3][tid]);
+  __syncthreads();
+  cluster_wait();  // (arrived at the start) every CTA of the cluster is running
+  for (int i = tid; i < cs * (kQ / 4); i += kK3Threads) {
+    const int r = i / (kQ / 4), f = i % (kQ / 4);
+    float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(&sh.part[rank][0], r));
+    dst[f] = reinterpret_cast<const float4 *>(sh.mine)[f];
+  }
+  cluster_arrive_release();
+  cluster_wait();
   if (tid < kQ) {
     float tot = 0.0f;
-    for (int r = 0; r < cs; ++r) tot += part0[r * kQ + tid];
+    for (int r = 0; r < cs; ++r) tot += sh.part[r][tid];
     sh.inv[tid] = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
   }
   __syncthreads();
   tc_fence_after();
+  // normalised bf16 output: each head's [128 t][64 p] tile is written into shared
+  // memory (128-byte swizzle; the tile buffers are all free now) and stored by TMA,
+  // which drops the rows past the end of the sequence
+  const uint32_t ybuf = base + kXh;
   if (sh.ok_flag && warp < kThreads / 32) {
     const int t = 32 * (warp & 3) + lane, hf = warp >> 2;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
@@ -968,10 +1078,9 @@ __global__ void __launch_bounds__(kK3Threads, 1)
       const int h = h0 + j;
       float v[16];
       tmem_ld16(tmem + lane_off + 128 + 64 * j + 16 * hf, v);
-      if (!t_valid) continue;
       const float4 *nw4 = reinterpret_cast<const float4 *>(&sh.nw[j][16 * hf]);
-      const int64_t row = bi * pr.L + c0 + t;
-      if (pr.nbg) {
+      if (pr.nbg && t_valid) {
+        const int64_t row = bi * pr.L + c0 + t;
         const uint4 *zp =
             reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 16 * hf);
 #pragma unroll
@@ -986,7 +1095,6 @@ __global__ void __launch_bounds__(kK3Threads, 1)
           }
         }
       }
-      uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * pr.d_inner + (int64_t)h * kHP + 16 * hf);
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         uint32_t o[4];
@@ -999,11 +1107,14 @@ __global__ void __launch_bounds__(kK3Threads, 1)
               __floats2bfloat162_rn(v[i] * sc * ww[2 * e], v[i + 1] * sc * ww[2 * e + 1]);
           o[e] = *reinterpret_cast<const uint32_t *>(&b2);
         }
-        dst[qq] = make_uint4(o[0], o[1], o[2], o[3]);
+        st_shared_v4(ybuf + j * 16384 + sw128_chunk(t, 16 * hf + 8 * qq), o[0], o[1], o[2], o[3]);
       }
+      fence_proxy_async_smem();
+      compute_sync();  // head j's tile is complete: store it while the next one is built
+      if (tid == 0) tma_store_3d(&maps.y, ybuf + j * 16384, (h0 + j) * kHP, (int)c0, (int)bi);
     }
+    if (tid == 0) bulk_commit_and_wait_read();
   }
-  cluster.sync();  // rank 0's table stays alive until every CTA has read it
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1023,7 +1134,7 @@ void out_split(int hpg, int *cs, int *hpc) {
 }
 
 struct TcWorkspace {
-  float *S, *cum_end;
+  float *S, *cum_end, *cum, *dtv;
   __half *Hc, *u;
 };
 
@@ -1036,6 +1147,10 @@ TcWorkspace tc_carve(const Problem &pr, char *base) {
   off += align_up(st * 4, 256);
   w.cum_end = reinterpret_cast<float *>(base + off);
   off += align_up((size_t)pr.batch * nch * pr.H * 4, 256);
+  w.cum = reinterpret_cast<float *>(base + off);
+  off += align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256);
+  w.dtv = reinterpret_cast<float *>(base + off);
+  off += align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256);
   w.Hc = reinterpret_cast<__half *>(base + off);
   off += align_up(st * 2, 256);
   w.u = reinterpret_cast<__half *>(base + off);
@@ -1107,7 +1222,8 @@ size_t prefill_tc_workspace(const Problem &pr) {
   const int64_t nch = ceil_div(pr.L, kQ);
   const size_t st = (size_t)pr.batch * nch * pr.H * kHP * kNS;
   return align_up(st * 4, 256) + align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
-         align_up(st * 2, 256) + align_up((size_t)pr.batch * pr.L * pr.conv_dim * 2, 256);
+         2 * align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256) + align_up(st * 2, 256) +
+         align_up((size_t)pr.batch * pr.L * pr.conv_dim * 2, 256);
 }
 
 cudaError_t take_prefill_tc_errors(unsigned int *out) {
@@ -1138,6 +1254,8 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   TcWorkspace w = tc_carve(pr, pa.ws);
   a.S = w.S;
   a.cum_end = w.cum_end;
+  a.cum = w.cum;
+  a.dtv = w.dtv;
   a.Hc = w.Hc;
   a.u = w.u;
   const int hpg = pr.heads_per_group();
@@ -1165,7 +1283,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     const uint32_t bx[3] = {64, kRawRows, 1};
     if (!make_map(&m1.xbc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xBC, 3, dx, sx, bx))
       return cudaErrorInvalidValue;
-    tc_chunk_state_kernel<<<g1, kOutThreads, kK1Smem, st>>>(a, m1, n_items);
+    tc_chunk_state_kernel<<<g1, kOutThreads, kK1Smem, st>>>(a, m1, (int)n_items);
   }
   stage_mark(st, 1);
   dim3 g2((unsigned)(kPassBlocks + ceil_div(pr.conv_dim, 256)), (unsigned)pr.H,
@@ -1195,9 +1313,12 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
       const uint64_t dh[2] = {(uint64_t)kNS, (uint64_t)pr.batch * a.nch * pr.H * kHP};
       const uint64_t shc[1] = {(uint64_t)kNS * 2};
       const uint32_t bh[2] = {64, 64};
+      const uint64_t dy[3] = {(uint64_t)pr.d_inner, (uint64_t)pr.L, (uint64_t)pr.batch};
+      const uint64_t sy[2] = {(uint64_t)pr.d_inner * 2, (uint64_t)pr.L * pr.d_inner * 2};
       if (!make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.u, 3, du, su, bu) ||
           !make_map(&maps.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.z, 3, dz, sz, bu) ||
-          !make_map(&maps.hc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Hc, 2, dh, shc, bh))
+          !make_map(&maps.hc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Hc, 2, dh, shc, bh) ||
+          !make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, 3, dy, sy, bu))
         return cudaErrorInvalidValue;
     }
     e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps);
