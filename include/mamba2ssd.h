@@ -86,7 +86,8 @@ typedef struct {
 
 /* fp32 parameters (device arrays, read only). */
 typedef struct {
-  const float *conv_w;  /* [conv_dim, d_conv]: tap k multiplies the input d_conv-1-k steps back */
+  const float *conv_w;  /* [conv_dim, d_conv], 16-byte aligned: tap k multiplies the input
+                          d_conv-1-k steps back */
   const float *conv_b;  /* [conv_dim] */
   const float *dt_bias; /* [nheads] */
   const float *A;       /* [nheads], A_h < 0 (callers holding A_log pass -exp(A_log)) */
@@ -152,7 +153,8 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
  *          16-byte aligned.
  *  dt_raw  [b, nheads] io_dtype, row stride >= nheads.
  *  y       [b, d_inner] io_dtype, contiguous, 16-byte aligned.  Output.
- *  conv_state  [b, conv_dim, d_conv] io_dtype, contiguous, updated in place.
+ *  conv_state  [b, conv_dim, d_conv] io_dtype, contiguous, 16-byte aligned,
+ *          updated in place.
  *  ssm_state   [b, nheads, headdim, dstate] fp32, contiguous, 16-byte
  *          aligned, updated in place.
  * Uses no workspace. */

@@ -56,7 +56,8 @@ size_t prefill_workspace(const Problem &pr) {
 }
 
 bool params_ok(const mamba2_params *p) {
-  return p != nullptr && p->conv_w && p->conv_b && p->dt_bias && p->A && p->D && p->norm_w;
+  return p != nullptr && p->conv_w && p->conv_b && p->dt_bias && p->A && p->D && p->norm_w &&
+         aligned(p->conv_w, 16);
 }
 
 // Disarms the stage events when a call returns, whatever the path taken.
@@ -205,7 +206,7 @@ MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *par
     return MAMBA2_ERR_INVALID_ARG;
   if (xBC_row_stride % 8 != 0 || z_row_stride % 8 != 0) return MAMBA2_ERR_INVALID_ARG;
   if (!aligned(xBC, 16) || !aligned(z, 16) || !aligned(y, 16) || !aligned(ssm_state, 16) ||
-      !aligned(conv_state, esz) || !aligned(dt_raw, esz))
+      !aligned(conv_state, 16) || !aligned(dt_raw, esz))
     return MAMBA2_ERR_INVALID_ARG;
   StepArgs a;
   a.pr = pr;

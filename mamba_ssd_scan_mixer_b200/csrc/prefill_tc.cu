@@ -41,8 +41,8 @@ namespace {
 
 constexpr int kQ = 128;          // tokens per chunk = MMA M
 constexpr int kThreads = 512;    // 16 compute warps
-constexpr int kOutThreads = kThreads + 32;  // + one TMA producer warp
-constexpr int kK3Threads = kThreads + 64;   // + TMA producer warp + MMA issuer warp
+constexpr int kWsThreads = kThreads + 64;   // + TMA producer warp + MMA issuer warp
+constexpr int kK1Threads = kThreads + 96;   // + 2 producer warps (even / odd items) + MMA warp
 constexpr int kHP = 64;          // headdim
 constexpr int kNS = 64;          // d_state
 constexpr int kMaxHeadsPerCta = 6;  // TMEM: 128 (CB) + 6 x 64 (y) <= 512 columns
@@ -172,9 +172,6 @@ __device__ __forceinline__ void cluster_arrive_release() {
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 // barrier over the 512 compute threads only (the producer warp never joins)
 __device__ __forceinline__ void compute_sync() {
   asm volatile("bar.sync 1, 512;" ::: "memory");
@@ -211,10 +208,14 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t 
 //     item had another (row, chunk, group): B's operands stay in shared memory),
 //     post-conv values to u, then S = (x o w)^T B on the tensor cores;
 //   C item: conv + SiLU of the group's C channels -> u.
-// 16 compute warps + 1 producer warp.  The producer computes the next item's
-// dt weights, stages its conv weights and TMA-loads its raw bf16 tiles
-// [136 tokens c0-3 .. c0+132][64 ch] (128-byte swizzle) into a two-stage ring
-// while the compute warps work on the current item.
+// 16 compute warps + 2 producer warps + 1 MMA-issuer warp.  The producer of an
+// item (one per ring stage, so they alternate) TMA-loads its raw bf16 tiles
+// [136 tokens c0-3 .. c0+132][64 ch] (128-byte swizzle) into its stage,
+// computes its dt weights (stored also as per-token dt and cumsum rows for the
+// output kernel) and stages its conv taps while the compute warps work on the
+// previous item; the MMA warp
+// issues a pair item's products once its operands are in shared memory, and
+// they run under the next item's convolution.
 // Smem (1024-aligned): ring [2][x_A | x_B | B (a C item uses slot 0)], then the
 // operands A_hi, A_lo [2 k-blocks][128 rows][128 B] and B_hi, B_lo [2][64][128 B].
 constexpr uint32_t kRawRows = 136, kRawBytes = kRawRows * 128;  // 17 KB, 1024-multiple
@@ -290,13 +291,13 @@ __device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs,
   return w;
 }
 
-__global__ void __launch_bounds__(kOutThreads, 1)
+__global__ void __launch_bounds__(kK1Threads, 1)
     tc_chunk_state_kernel(TcArgs a, const __grid_constant__ K1Maps maps, int n_items) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ float ws[2][2][kQ];          // [stage][head of pair][token] chunk weights
   __shared__ float4 wts[2][3][64];        // [stage][slot][channel] conv taps
   __shared__ float bss[2][3][64];         // [stage][slot][channel] conv bias
-  __shared__ uint64_t full[2], empty[2], mbar;
+  __shared__ uint64_t full[2], empty[2], ops_ready, mbar;
   __shared__ uint32_t tmem_holder;
   const Problem &pr = a.pr;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -314,7 +315,8 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       mbar_init(&full[k], 2);  // the tiles' transaction bytes + the producer's weights
       mbar_init(&empty[k], 1);
     }
-    mbar_init(&mbar, 1);
+    mbar_init(&ops_ready, 1);  // operands of a pair item written (compute thread 0)
+    mbar_init(&mbar, 1);       // its MMAs completed (tcgen05.commit)
     fence_mbar_init();
   }
   tc_fence_before();
@@ -322,23 +324,91 @@ __global__ void __launch_bounds__(kOutThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  if (warp == kThreads / 32) {
-    // ---------------- producer: raw tiles (issued first), then dt weights and conv
-    // taps of the next items
+  if (warp == kThreads / 32 || warp == kThreads / 32 + 2) {
+    // ---------------- producers: warp 16 takes the CTA's even items (ring stage
+    // 0), warp 18 the odd ones (stage 1).
+    const int mine = warp == kThreads / 32 ? 0 : 1;
     int k = 0;
     for (int it = it0; it < it1; ++it, ++k) {
       const int st = k & 1;
+      if (st != mine) continue;
+      const K1Item w = k1_item(pr, a.nch, pairs, it, k);
+      const bool freshB = w.freshB;
+      const int64_t c0 = (int64_t)w.c * kQ;
+      const int hA = w.g * hpg + 2 * w.pair;
+      const bool hasB = 2 * w.pair + 1 < hpg;
+      // everything that needs no shared memory first, while the stage may still be
+      // in use: the item's global loads (one round trip: dt of both heads for this
+      // lane's 4 tokens, their dt_bias and A, the conv taps of its slots), the dt
+      // weights, and the per-token dt and cumsum rows for the output kernel
+      float dtr[2][4], dtb[2] = {0.0f, 0.0f}, Ah[2] = {0.0f, 0.0f};
+      float4 tw[3][2];
+      float tb[3][2];
+      bool son[3];
+#pragma unroll
+      for (int sl = 0; sl < 3; ++sl) {
+        son[sl] = w.isC ? sl == 0 : (sl == 1 ? hasB : (sl == 2 ? freshB : true));
+        const int64_t ch0 = w.isC ? pr.d_inner + (int64_t)(pr.G + w.g) * kNS
+                                  : (sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (son[sl]) {
+            tw[sl][j] = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + lane + 32 * j);
+            tb[sl][j] = __ldg(a.prm.conv_b + ch0 + lane + 32 * j);
+          }
+        }
+      }
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const bool hv = !w.isC && (half == 0 || hasB);
+        if (hv) {
+          dtb[half] = __ldg(a.prm.dt_bias + hA + half);
+          Ah[half] = __ldg(a.prm.A + hA + half);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int64_t tt = c0 + 4 * lane + q;
+          dtr[half][q] = (hv && tt < pr.L)
+                             ? __bfloat162float(a.dt_raw[(w.bi * pr.L + tt) * a.ld_dt + hA + half])
+                             : -INFINITY;
+        }
+      }
+      float wsv[2][4];
+      if (!w.isC) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const bool hv = half == 0 || hasB;
+          float dt4[4], a4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            dt4[q] = dtr[half][q] != -INFINITY ? softplus_f(dtr[half][q] + dtb[half]) : 0.0f;
+            a4[q] = dt4[q] * Ah[half];
+          }
+          const float tot = a4[0] + a4[1] + a4[2] + a4[3];
+          float run = warp_scan(tot, lane) - tot;
+          const float cum_end = __shfl_sync(0xffffffffu, run + tot, 31);
+          float cq[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            run += a4[q];
+            cq[q] = run;
+            wsv[half][q] = expf(cum_end - run) * dt4[q];
+          }
+          if (hv) {
+            const int64_t row = (w.bi * a.nch + w.c) * pr.H + hA + half;
+            reinterpret_cast<float4 *>(a.cum + row * kQ)[lane] = make_float4(cq[0], cq[1], cq[2], cq[3]);
+            reinterpret_cast<float4 *>(a.dtv + row * kQ)[lane] = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
+            if (lane == 0) a.cum_end[row] = cum_end;
+          }
+        }
+      }
+      // the stage is free once the compute warps are done with item k - 2
       if (k >= 2) {
         bool got = lane == 0 ? mbar_wait_bounded(&empty[st], (uint32_t)(((k >> 1) - 1) & 1),
                                                  &g_tc_errors)
                              : true;
         if (!__all_sync(0xffffffffu, got)) break;
       }
-      const K1Item w = k1_item(pr, a.nch, pairs, it, k);
-      const bool freshB = w.freshB;
-      const int64_t c0 = (int64_t)w.c * kQ;
-      const int hA = w.g * hpg + 2 * w.pair;
-      const bool hasB = 2 * w.pair + 1 < hpg;
       if (lane == 0) {
         const uint32_t stage = base + st * kK1Stage;
         if (w.isC) {
@@ -358,64 +428,45 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         }
       }
       if (!w.isC) {
-        // dt of both heads for this lane's 4 tokens: all loads first
-        float dtr[2][4];
 #pragma unroll
         for (int half = 0; half < 2; ++half)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int64_t tt = c0 + 4 * lane + q;
-            dtr[half][q] = ((half == 0 || hasB) && tt < pr.L)
-                               ? __bfloat162float(a.dt_raw[(w.bi * pr.L + tt) * a.ld_dt + hA + half])
-                               : -INFINITY;
-          }
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const bool hv = half == 0 || hasB;
-          const int h = hA + (hv ? half : 0);
-          const float dtb = a.prm.dt_bias[h], Ah = a.prm.A[h];
-          float dt4[4], a4[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            dt4[q] = (hv && dtr[half][q] != -INFINITY) ? softplus_f(dtr[half][q] + dtb) : 0.0f;
-            a4[q] = dt4[q] * Ah;
-          }
-          const float tot = a4[0] + a4[1] + a4[2] + a4[3];
-          float run = warp_scan(tot, lane) - tot;
-          const float cum_end = __shfl_sync(0xffffffffu, run + tot, 31);
-          float cq[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            run += a4[q];
-            cq[q] = run;
-            ws[st][half][4 * lane + q] = expf(cum_end - run) * dt4[q];
-          }
-          if (hv) {
-            const int64_t row = (w.bi * a.nch + w.c) * pr.H + hA + half;
-            reinterpret_cast<float4 *>(a.cum + row * kQ)[lane] = make_float4(cq[0], cq[1], cq[2], cq[3]);
-            reinterpret_cast<float4 *>(a.dtv + row * kQ)[lane] = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
-            if (lane == 0) a.cum_end[row] = cum_end;
-          }
-        }
+          for (int q = 0; q < 4; ++q) ws[st][half][4 * lane + q] = wsv[half][q];
       }
-      // conv taps and bias of the item's slots
+      // conv taps and bias of the item's slots, channel 8 g + i at [i][g]
+#pragma unroll
       for (int sl = 0; sl < 3; ++sl) {
-        int64_t ch0;
-        if (w.isC) {
-          if (sl > 0) break;
-          ch0 = pr.d_inner + (int64_t)(pr.G + w.g) * kNS;
-        } else {
-          if ((sl == 1 && !hasB) || (sl == 2 && !freshB)) continue;
-          ch0 = sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS;
-        }
-        for (int i = lane; i < 64; i += 32) {
-          const int d = (i & 7) * 8 + (i >> 3);  // [channel in group][group]
-          wts[st][sl][d] = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + i);
-          bss[st][sl][d] = __ldg(a.prm.conv_b + ch0 + i);
+        if (!son[sl]) continue;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int i = lane + 32 * j, d = (i & 7) * 8 + (i >> 3);
+          wts[st][sl][d] = tw[sl][j];
+          bss[st][sl][d] = tb[sl][j];
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);  // weights of this stage written
+    }
+  } else if (warp == kThreads / 32 + 1) {
+    // ---------------- MMA issuer: S = x_hi B_hi + x_hi B_lo + x_lo B_hi per pair item
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_f16(128, 64);
+      const uint32_t As[3] = {sAhi, sAhi, sAlo}, Bs[3] = {sBhi, sBlo, sBhi};
+      int n = 0;
+      for (int it = it0; it < it1; ++it) {
+        if (k1_item(pr, a.nch, pairs, it, 1).isC) continue;
+        if (!mbar_wait_bounded(&ops_ready, (uint32_t)(n & 1), &g_tc_errors)) break;
+        ++n;
+        tc_fence_after();
+        for (int prod = 0; prod < 3; ++prod)
+          for (int ks = 0; ks < 8; ++ks) {
+            const int blk = ks >> 2, kin = ks & 3;
+            umma_f16(tmem, umma_desc_sw128(As[prod] + blk * 16384 + kin * 32),
+                     umma_desc_sw128(Bs[prod] + blk * 8192 + kin * 32), idesc,
+                     (prod > 0 || ks > 0) ? 1u : 0u);
+          }
+        umma_commit(&mbar);
+      }
     }
   } else {
     // ---------------- compute warps
@@ -573,19 +624,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
       compute_sync();
       if (tid == 0) mbar_arrive(&empty[st]);  // raw tiles and taps of this stage consumed
       if (w.isC || !ok) continue;
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t idesc = umma_idesc_f16(128, 64);
-        const uint32_t As[3] = {sAhi, sAhi, sAlo}, Bs[3] = {sBhi, sBlo, sBhi};
-        for (int prod = 0; prod < 3; ++prod)
-          for (int ks = 0; ks < 8; ++ks) {
-            const int blk = ks >> 2, kin = ks & 3;
-            umma_f16(tmem, umma_desc_sw128(As[prod] + blk * 16384 + kin * 32),
-                     umma_desc_sw128(Bs[prod] + blk * 8192 + kin * 32), idesc,
-                     (prod > 0 || ks > 0) ? 1u : 0u);
-          }
-        umma_commit(&mbar);
-      }
+      if (tid == 0) mbar_arrive(&ops_ready);  // the MMA warp issues S = (x o w)^T B
       pending = true;
       pw.bi = w.bi;
       pw.c = w.c;
@@ -732,7 +771,7 @@ struct OutMaps {
   CUtensorMap y;   // [b][L][d_inner] bf16, box 64 x 128 (stores)
 };
 
-__global__ void __launch_bounds__(kK3Threads, 1)
+__global__ void __launch_bounds__(kWsThreads, 1)
     tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -1051,7 +1090,7 @@ __global__ void __launch_bounds__(kK3Threads, 1)
   if (tid < kQ) sh.mine[tid] = (sh.ss[0][tid] + sh.ss[1][tid]) + (sh.ss[2][tid] + sh.ss[3][tid]);
   __syncthreads();
   cluster_wait();  // (arrived at the start) every CTA of the cluster is running
-  for (int i = tid; i < cs * (kQ / 4); i += kK3Threads) {
+  for (int i = tid; i < cs * (kQ / 4); i += kWsThreads) {
     const int r = i / (kQ / 4), f = i % (kQ / 4);
     float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(&sh.part[rank][0], r));
     dst[f] = reinterpret_cast<const float4 *>(sh.mine)[f];
@@ -1283,7 +1322,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     const uint32_t bx[3] = {64, kRawRows, 1};
     if (!make_map(&m1.xbc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xBC, 3, dx, sx, bx))
       return cudaErrorInvalidValue;
-    tc_chunk_state_kernel<<<g1, kOutThreads, kK1Smem, st>>>(a, m1, (int)n_items);
+    tc_chunk_state_kernel<<<g1, kK1Threads, kK1Smem, st>>>(a, m1, (int)n_items);
   }
   stage_mark(st, 1);
   dim3 g2((unsigned)(kPassBlocks + ceil_div(pr.conv_dim, 256)), (unsigned)pr.H,
@@ -1293,7 +1332,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cs, (unsigned)a.nch, (unsigned)(pr.G * pr.batch));
-    cfg.blockDim = dim3(kK3Threads, 1, 1);
+    cfg.blockDim = dim3(kWsThreads, 1, 1);
     cfg.dynamicSmemBytes = kK3Smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
