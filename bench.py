@@ -106,14 +106,16 @@ def stage_bytes(name, cfg) -> int | None:
         "ssd_step": decode_bytes(cfg),
     }
     # tensor-core path (128-token chunks; u = post-conv activations, fp16;
-    # S = chunk states fp32; Hc = carried states fp16)
+    # S = chunk states fp32; Hc = carried states fp16; per-token dt and cumsum
+    # rows fp32, written by the chunk-state kernel and read by the output kernel)
     nq = -(-cfg.seqlen // 128)
     pn = cfg.headdim * cfg.dstate
     S32 = cfg.batch * nq * H * pn * 4
+    rows = 2 * cfg.batch * nq * 128 * H * 4
     table.update({
-        "tc_chunk_state": bL * cd * (e + 2) + bL * H * e + S32 + cfg.batch * nq * H * 4,
+        "tc_chunk_state": bL * cd * (e + 2) + bL * H * e + S32 + cfg.batch * nq * H * 4 + rows,
         "tc_state_pass": S32 + S32 // 2 + cfg.batch * nq * H * 4 + 2 * cfg.batch * H * pn * 4,
-        "tc_chunk_out": bL * (cd * 2 + di * e + H * e + di * e) + S32 // 2,
+        "tc_chunk_out": bL * (cd * 2 + di * e + di * e) + rows + S32 // 2,
     })
     return table.get(name)
 

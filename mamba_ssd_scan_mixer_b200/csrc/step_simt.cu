@@ -22,8 +22,8 @@
 //   4. finish row r - 1: wait until every rank of the cluster has signalled
 //      it, scale and store its output, write this rank's share of its shifted
 //      B/C conv state (all ranks have read it by then);
-//   5. push row r's partial sums into every rank's table (distributed shared
-//      memory) and signal each rank's mbarrier.
+//   5. send row r's partial sums into every rank's table (distributed shared
+//      memory, asynchronous stores that complete bytes on that rank's mbarrier).
 // So the norm exchange of a row completes while the next row streams.  The
 // tables, mbarriers and per-row buffers alternate between rows; step 4 comes
 // before step 5 so that no rank can overwrite a table this CTA still reads.
@@ -68,11 +68,11 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, int r) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(r));
   return a;
 }
-__device__ __forceinline__ void st_cluster(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
+// asynchronous 4-byte store into another rank's shared memory that completes
+// 4 transaction bytes on that rank's mbarrier
+__device__ __forceinline__ void st_async_cluster(uint32_t addr, float v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr),
+               "r"(__float_as_uint(v)), "r"(bar)
                : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
@@ -209,7 +209,12 @@ __global__ void __launch_bounds__(kStepBlock, 2)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kStepThreads);
     }
-    for (int s = 0; s < 2; ++s) mbar_init(&sums_ready[s], cs);
+    // one local arrival (carrying the expected bytes: cs * G partial sums) and
+    // the ranks' asynchronous stores complete a phase; rows 0 and 1 armed here
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sums_ready[s], 1);
+      mbar_arrive_expect_tx(&sums_ready[s], (uint32_t)(cs * G * 4));
+    }
     fence_mbar_init();
   }
   // row-independent parameters of the CTA's channels and heads
@@ -297,6 +302,9 @@ __global__ void __launch_bounds__(kStepBlock, 2)
       inv[g] = rsqrtf(tot / gs + pr.eps);
     }
     step_bar();
+    // re-arm this parity for row rr + 2: no rank sends that row before this CTA
+    // has sent row rr + 1, which happens after this point
+    if (tid == 0 && rr + 2 < rows_mine) mbar_arrive_expect_tx(&sums_ready[par], (uint32_t)(cs * G * 4));
     T *yr = y + bi * pr.d_inner + (int64_t)h0 * P;
     const float *ysr = ys + par * C;
     for (int c = tid; c < C; c += kStepThreads) {
@@ -439,10 +447,11 @@ __global__ void __launch_bounds__(kStepBlock, 2)
     // 4. the previous row, whose partial sums have had a row's time to arrive
     if (rr > 0) finish(rr - 1);
     // 5. this row's partials into part[par][rank][*] of every rank; thread r
-    //    stores into rank r and release-arrives on its barrier
+    //    sends rank r's, completing bytes on its barrier
     if (tid < cs) {
-      for (int g = 0; g < G; ++g) st_cluster(cluster_addr(part + (par * cs + rank) * G + g, tid), mysum[g]);
-      mbar_arrive_cluster(cluster_addr(&sums_ready[par], tid));
+      const uint32_t bar = cluster_addr(&sums_ready[par], tid);
+      for (int g = 0; g < G; ++g)
+        st_async_cluster(cluster_addr(part + (par * cs + rank) * G + g, tid), mysum[g], bar);
     }
   }
   if (rows_mine > 0) finish(rows_mine - 1);
