@@ -26,7 +26,6 @@
 // tolerance on these workloads), accumulation is fp32.  The chunk-state
 // product uses a two-term fp16 split of both operands (hi*hi + hi*lo + lo*hi),
 // because the returned final state must hold 2e-2 of its RMS.
-#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -34,7 +33,6 @@
 
 #include "common.cuh"
 
-namespace cg = cooperative_groups;
 
 namespace m2 {
 namespace {
@@ -158,9 +156,20 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
                ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
 }
-// Commit the issued bulk stores and wait until they have read shared memory.
-__device__ __forceinline__ void bulk_commit_and_wait_read() {
+// Bulk-store groups: commit the stores issued so far; wait until at most one /
+// none of the committed groups still reads shared memory.
+__device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// (the group count of wait_group is an immediate: the cases used are spelled out)
+__device__ __forceinline__ void bulk_wait_read_le(int n) {
+  if (n >= 4) asm volatile("cp.async.bulk.wait_group.read 4;" ::: "memory");
+  else if (n == 3) asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
+  else if (n == 2) asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+  else if (n == 1) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+  else asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_arrive_relaxed() {
@@ -726,10 +735,14 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
 }
 
 // ============================================================== chunk output
-// grid (cs, nch, G * b), cluster (cs, 1, 1); 16 compute warps + 1 TMA producer
-// warp + 1 MMA-issuer warp.  Tiles arrive by TMA in 128-byte-swizzled layouts
-// (1024-aligned).  The operand A is double-buffered so that the A-build of head
-// j + 1 overlaps the MMA of head j; buffer 1 reuses the B tile once CB is formed.
+// Persistent clusters: grid (cs, ncl, 1), cluster (cs, 1, 1).  Cluster k takes
+// the units (row, chunk, group) k, k + ncl, ...; its cs CTAs split the group's
+// heads.  16 compute warps + 1 TMA producer warp + 1 MMA-issuer warp.  Tiles
+// arrive by TMA in 128-byte-swizzled layouts (1024-aligned).  The operand A is
+// double-buffered so that the A-build of head j + 1 overlaps the MMA of head j;
+// buffer 1 reuses the B tile once CB is formed.  The next unit's C and B tiles,
+// its CB product and its first x / H_c / z tiles arrive while the current
+// unit exchanges its norm sums and writes its output.
 constexpr uint32_t kCt = 0;                      // C   [128 t][64 n] fp16     16 KB (u)
 constexpr uint32_t kBt = kCt + 16384;            // B   [128 s][64 n] fp16     16 KB (u)
 constexpr int kXhStages = 2, kZStages = 2;
@@ -739,6 +752,9 @@ constexpr uint32_t kZt = kXh + kXhStages * kXhBytes;  // z ring [128 t][64 p] bf
 constexpr uint32_t kA0 = kZt + kZStages * 16384;      // A buffer 0: [3][128 t][64 k] fp16  48 KB
 constexpr uint32_t kA1 = kA0 + 3 * 16384;             // A buffer 1, blocks 1 and 2 (block 0 at kBt)
 constexpr uint32_t kTcOutTiles = kA1 + 2 * 16384;     // 192 KB
+// output staging: [128 t][64 p] bf16 tiles in the A buffers, idle while a unit
+// writes its output (A buffer 0 and blocks 1, 2 of buffer 1)
+constexpr int kYTiles = 5;
 
 // Byte offset of k-block `blk` (0, 1: CB columns s; 2: scaled C) of A buffer `buf`.
 __device__ __forceinline__ uint32_t a_block(int buf, int blk) {
@@ -751,15 +767,14 @@ struct OutShared {
   float beta[kMaxHeadsPerCta][kQ];  // exp(cum_r - cum_s) dt_s, r = end of s's 32-token group
   float betad[kMaxHeadsPerCta][kQ]; // exp(cum_s0 - cum_s) dt_s, s0 = start of s's group
   int span_ok[kMaxHeadsPerCta][4];  // group's log2-decay span <= 60: factorise its diagonal
-  float ecum[kMaxHeadsPerCta][kQ];  // exp(cumsum)
   float nw[kMaxHeadsPerCta][kHP];   // norm weight of the CTA's channels
   float ss[4][kQ];
-  float part[16][kQ];               // partial sums of squares of every rank of the cluster
+  float part[2][16][kQ];            // [unit parity][rank]: partial sums of squares per token
   float mine[kQ];                   // this CTA's partial sums
   float inv[kQ];
   float Dh[kMaxHeadsPerCta];
   uint64_t full_cb, full_xh[kXhStages], empty_xh[kXhStages], full_z[kZStages],
-      empty_z[kZStages], a_ready[2], mbar_cb, mbar_mma[2];
+      empty_z[kZStages], a_ready[2], mbar_cb, mbar_mma[2], tiles_free, sums_ready[2];
   uint32_t tmem_holder;
   int ok_flag;
 };
@@ -771,25 +786,70 @@ struct OutMaps {
   CUtensorMap y;   // [b][L][d_inner] bf16, box 64 x 128 (stores)
 };
 
+// 16-byte asynchronous store into another rank's shared memory that completes
+// 16 transaction bytes on that rank's mbarrier
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+      "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)), "r"(__float_as_uint(v.z)),
+      "r"(__float_as_uint(v.w)), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, int r) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(r));
+  return out;
+}
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity) {
+  auto probe = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (probe()) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!probe()) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_tc_errors, kErrWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Unit n of cluster `cid`: (row bi, chunk c, group g).
+__device__ __forceinline__ void out_unit(const Problem &pr, int nch, int ncl, int cid, int n,
+                                         int64_t &bi, int &c, int &g) {
+  const int64_t u = cid + (int64_t)n * ncl;
+  g = (int)(u % pr.G);
+  const int64_t bc = u / pr.G;
+  c = (int)(bc % nch);
+  bi = bc / nch;
+}
+
 __global__ void __launch_bounds__(kWsThreads, 1)
-    tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps) {
+    tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps, int ncl) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  cg::cluster_group cluster = cg::this_cluster();
-  const int cs = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
+  int cs, rank;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs));
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
   const Problem &pr = a.pr;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   OutShared &sh = *reinterpret_cast<OutShared *>(smem_raw + (base - smem_u32(smem_raw)) +
                                                  kTcOutTiles);
-  const int c = blockIdx.y;
-  const int g = (int)(blockIdx.z % pr.G);
-  const int64_t bi = blockIdx.z / pr.G;
+  const int cid = blockIdx.y;
   const int hpg = pr.heads_per_group();
   const int lh0 = rank * a.hpc;
-  const int nh = max(0, min(a.hpc, hpg - lh0));  // heads of this CTA
-  const int h0 = g * hpg + lh0;
-  const int64_t c0 = (int64_t)c * kQ;
+  const int nh = max(0, min(a.hpc, hpg - lh0));  // heads of this CTA in every unit
+  const int64_t n_all = pr.batch * (int64_t)a.nch * pr.G;
+  const int n_units = n_all > cid ? (int)((n_all - cid + ncl - 1) / ncl) : 0;
+  const uint32_t sum_bytes = (uint32_t)cs * kQ * 4;  // partial sums this CTA receives per unit
 
   if (warp == 0) tmem_alloc(&sh.tmem_holder, 512);
   if (tid == 0) {
@@ -805,8 +865,13 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     for (int k = 0; k < 2; ++k) {
       mbar_init(&sh.a_ready[k], kThreads);  // every compute thread after its A-build
       mbar_init(&sh.mbar_mma[k], 1);        // MMA of a head that used A buffer k
+      // the local arrival carries the bytes the ranks' partial sums complete;
+      // units 0 and 1 are armed here, unit n + 2 once unit n's sums are read
+      mbar_init(&sh.sums_ready[k], 1);
+      mbar_arrive_expect_tx(&sh.sums_ready[k], sum_bytes);
     }
     mbar_init(&sh.mbar_cb, 1);
+    mbar_init(&sh.tiles_free, 1);  // a unit's C / B tiles and CB columns no longer read
     fence_mbar_init();
     sh.ok_flag = 1;
   }
@@ -814,108 +879,105 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   __syncthreads();
   tc_fence_after();
   cluster_arrive_relaxed();  // waited for before the first remote store
+  bool started = false;
   const uint32_t tmem = sh.tmem_holder;
 
   if (warp == kThreads / 32) {
-    // ---------------- producer: C, B tiles, then x, H_c, z of each head
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&sh.full_cb, 2 * 16384);
-      tma_load_3d(base + kCt, &maps.u, (int)(pr.d_inner + (int64_t)(pr.G + g) * kNS), (int)c0,
-                  (int)bi, &sh.full_cb);
-      tma_load_3d(base + kBt, &maps.u, (int)(pr.d_inner + (int64_t)g * kNS), (int)c0, (int)bi,
-                  &sh.full_cb);
-      // x / H_c of head j go to stage j % 3, freed when MMA j has completed;
-      // z of head j to stage j % 2, freed after the epilogue of head j
-      for (int j = 0; j < nh; ++j) {
-        const int h = h0 + j;
-        const int sx = j % kXhStages, sz = j % kZStages;
-        if (j >= kXhStages && !mbar_wait_bounded(&sh.empty_xh[sx],
-                                                 (uint32_t)((j / kXhStages - 1) & 1), &g_tc_errors))
-          break;
-        mbar_arrive_expect_tx(&sh.full_xh[sx], kXhBytes);
-        tma_load_3d(base + kXh + sx * kXhBytes, &maps.u, h * kHP, (int)c0, (int)bi,
-                    &sh.full_xh[sx]);
-        tma_load_2d(base + kXh + sx * kXhBytes + 16384, &maps.hc, 0,
-                    (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full_xh[sx]);
-        if (j >= kZStages && !mbar_wait_bounded(&sh.empty_z[sz],
-                                                (uint32_t)((j / kZStages - 1) & 1), &g_tc_errors))
-          break;
-        mbar_arrive_expect_tx(&sh.full_z[sz], 16384);
-        tma_load_3d(base + kZt + sz * 16384, &maps.z, h * kHP, (int)c0, (int)bi, &sh.full_z[sz]);
+    // ---------------- producer: per unit, x / H_c / z of each head (rings released
+    // by the head's MMA and epilogue); after the first head's, the unit's C and B
+    // tiles, once the previous unit has finished reading them
+    if (lane == 0 && nh > 0) {
+      int J = 0;    // heads issued so far (ring position)
+      int ncb = 0;  // C / B loads issued
+      bool ok = true;
+      for (int n = 0; ok && n < n_units; ++n) {
+        int64_t bi;
+        int c, g;
+        out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+        const int h0 = g * hpg + lh0;
+        const int c0 = c * kQ;
+        for (int j = 0; ok && j < nh; ++j, ++J) {
+          const int h = h0 + j, sx = J % kXhStages, sz = J % kZStages;
+          ok = J < kXhStages ||
+               mbar_wait_bounded(&sh.empty_xh[sx], (uint32_t)((J / kXhStages - 1) & 1), &g_tc_errors);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh.full_xh[sx], kXhBytes);
+          tma_load_3d(base + kXh + sx * kXhBytes, &maps.u, h * kHP, c0, (int)bi, &sh.full_xh[sx]);
+          tma_load_2d(base + kXh + sx * kXhBytes + 16384, &maps.hc, 0,
+                      (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full_xh[sx]);
+          ok = J < kZStages ||
+               mbar_wait_bounded(&sh.empty_z[sz], (uint32_t)((J / kZStages - 1) & 1), &g_tc_errors);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&sh.full_z[sz], 16384);
+          tma_load_3d(base + kZt + sz * 16384, &maps.z, h * kHP, c0, (int)bi, &sh.full_z[sz]);
+          if (j == 0) {
+            ok = n == 0 || mbar_wait_bounded(&sh.tiles_free, (uint32_t)((n - 1) & 1), &g_tc_errors);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&sh.full_cb, 2 * 16384);
+            tma_load_3d(base + kCt, &maps.u, (int)(pr.d_inner + (int64_t)(pr.G + g) * kNS), c0,
+                        (int)bi, &sh.full_cb);
+            tma_load_3d(base + kBt, &maps.u, (int)(pr.d_inner + (int64_t)g * kNS), c0, (int)bi,
+                        &sh.full_cb);
+            ++ncb;
+          }
+        }
+      }
+      // no copy may be in flight when the CTA exits: the last copy into each buffer
+      if (ncb > 0) mbar_wait_bounded(&sh.full_cb, (uint32_t)((ncb - 1) & 1), &g_tc_errors);
+      for (int k = max(0, J - 2); k < J; ++k) {
+        mbar_wait_bounded(&sh.full_xh[k % kXhStages], (uint32_t)((k / kXhStages) & 1), &g_tc_errors);
+        mbar_wait_bounded(&sh.full_z[k % kZStages], (uint32_t)((k / kZStages) & 1), &g_tc_errors);
       }
     }
   } else if (warp == kThreads / 32 + 1) {
-    // ---------------- MMA issuer: CB once, then one K = 192 MMA per head
-    if (lane == 0) {
-      bool ok = mbar_wait_bounded(&sh.full_cb, 0, &g_tc_errors);
-      if (ok) {  // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
-        tc_fence_after();
-        const uint32_t idesc = umma_idesc_f16(128, 128);
-        for (int kin = 0; kin < 4; ++kin)
-          umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32),
-                   umma_desc_sw128(base + kBt + kin * 32), idesc, kin > 0 ? 1u : 0u);
-        umma_commit(&sh.mbar_cb);
-      }
+    // ---------------- MMA issuer: per unit CB once, then one K = 192 MMA per head
+    if (lane == 0 && nh > 0) {
+      const uint32_t idesc_cb = umma_idesc_f16(128, 128);
       const uint32_t idesc_mn = umma_idesc_f16(128, 64) | (1u << 16);  // B operand MN-major
-      for (int j = 0; ok && j < nh; ++j) {
-        ok = mbar_wait_bounded(&sh.a_ready[j & 1], (uint32_t)((j >> 1) & 1), &g_tc_errors) &&
-             mbar_wait_bounded(&sh.full_xh[j % kXhStages], (uint32_t)((j / kXhStages) & 1),
-                               &g_tc_errors);
+      int J = 0;
+      bool ok = true;
+      for (int n = 0; ok && n < n_units; ++n) {
+        // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
+        ok = mbar_wait_bounded(&sh.full_cb, (uint32_t)(n & 1), &g_tc_errors);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t xt = base + kXh + (j % kXhStages) * kXhBytes, ht = xt + 16384;
-        for (int ks = 0; ks < 12; ++ks) {
-          const int blk = ks >> 2, kin = ks & 3;
-          const uint64_t ad = umma_desc_sw128(base + a_block(j & 1, blk) + kin * 32);
-          // x [s][p] and H_c [n][p] are both MN-major (p contiguous)
-          if (ks < 8)
-            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn,
-                     ks > 0 ? 1u : 0u);
-          else
-            umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(ht + (ks - 8) * 2048, 8192),
-                     idesc_mn, 1u);
+        for (int kin = 0; kin < 4; ++kin)
+          umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32),
+                   umma_desc_sw128(base + kBt + kin * 32), idesc_cb, kin > 0 ? 1u : 0u);
+        umma_commit(&sh.mbar_cb);
+        for (int j = 0; j < nh; ++j, ++J) {
+          ok = mbar_wait_bounded(&sh.a_ready[J & 1], (uint32_t)((J >> 1) & 1), &g_tc_errors) &&
+               mbar_wait_bounded(&sh.full_xh[J % kXhStages], (uint32_t)((J / kXhStages) & 1),
+                                 &g_tc_errors);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t xt = base + kXh + (J % kXhStages) * kXhBytes, ht = xt + 16384;
+          for (int ks = 0; ks < 12; ++ks) {
+            const int blk = ks >> 2, kin = ks & 3;
+            const uint64_t ad = umma_desc_sw128(base + a_block(J & 1, blk) + kin * 32);
+            // x [s][p] and H_c [n][p] are both MN-major (p contiguous)
+            if (ks < 8)
+              umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(xt + ks * 2048, 16384),
+                       idesc_mn, ks > 0 ? 1u : 0u);
+            else
+              umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(ht + (ks - 8) * 2048, 8192),
+                       idesc_mn, 1u);
+          }
+          umma_commit(&sh.mbar_mma[J & 1]);
+          umma_commit(&sh.empty_xh[J % kXhStages]);  // its x / H_c stage is free once it completes
         }
-        umma_commit(&sh.mbar_mma[j & 1]);
-        umma_commit(&sh.empty_xh[j % kXhStages]);  // its x / H_c stage is free once it completes
       }
       if (!ok) sh.ok_flag = 0;
+      // no MMA may be in flight when the CTA frees its tensor memory
+      if (J > 0) mbar_wait_bounded(&sh.mbar_mma[(J - 1) & 1], (uint32_t)(((J - 1) >> 1) & 1), &g_tc_errors);
     }
   } else {
     // ---------------- compute warps
-    // decay terms: one warp per head, 4 consecutive tokens per lane, from the
-    // per-chunk dt and cumsum rows the chunk-state kernel wrote
-    if (warp < nh) {
-      const int j = warp, h = h0 + j;
-      const int64_t row = (bi * a.nch + c) * pr.H + h;
-      const float4 cu = reinterpret_cast<const float4 *>(a.cum + row * kQ)[lane];
-      const float4 dv = reinterpret_cast<const float4 *>(a.dtv + row * kQ)[lane];
-      const float cum4[4] = {cu.x, cu.y, cu.z, cu.w}, dt4[4] = {dv.x, dv.y, dv.z, dv.w};
-      float c2[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        c2[k] = cum4[k] * kLog2e;
-        sh.cum2[j][4 * lane + k] = c2[k];
-        sh.dt[j][4 * lane + k] = dt4[k];
-        sh.ecum[j][4 * lane + k] = ex2_approx(c2[k]);
-      }
-      const float c2r = __shfl_sync(0xffffffffu, c2[3], (lane | 7));
-      const float c2s0 = __shfl_sync(0xffffffffu, c2[0], (lane & ~7));
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        sh.beta[j][4 * lane + k] = ex2_approx(c2r - c2[k]) * dt4[k];
-        sh.betad[j][4 * lane + k] = ex2_approx(fminf(c2s0 - c2[k], 60.0f)) * dt4[k];
-      }
-      if ((lane & 7) == 7) sh.span_ok[j][lane >> 3] = (c2s0 - c2r) <= 60.0f;
-    }
-    for (int i = tid; i < nh * kHP; i += kThreads)
-      sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
-    if (tid < nh) sh.Dh[tid] = a.prm.D[h0 + tid];
-    compute_sync();  // cumsum, weights and D visible to every compute warp
-
     const int t = 32 * (warp & 3) + lane, hf = warp >> 2, q = warp & 3;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     float ss_acc = 0.0f;
     bool ok = true;
+    int J = 0;  // heads processed so far (ring and A-buffer position)
     auto wait_warp = [&](uint64_t *bar, uint32_t parity) {
       const bool got = ok && mbar_wait_bounded(bar, parity, &g_tc_errors);
       ok = __all_sync(0xffffffffu, got) != 0;
@@ -923,12 +985,12 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 
     // epilogue, part 1: gate with silu(z) (z tile in smem), sum of squares, g -> TMEM.
     // Warp w handles rows 32*(w%4) .. +31 and columns 16*(w/4) .. +15 of a head.
-    auto epilogue1 = [&](int j) {
+    auto epilogue1 = [&](int j, int zslot) {
       float v[16];
       const uint32_t col = 128 + 64 * j + 16 * hf;
       tmem_ld16(tmem + lane_off + col, v);
       if (!pr.nbg) {
-        const uint32_t zt = base + kZt + (j % kZStages) * 16384;
+        const uint32_t zt = base + kZt + zslot * 16384;
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
           const uint4 raw = ld_shared_v4(zt + sw128_chunk(t, 16 * hf + 8 * qq));
@@ -946,17 +1008,66 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       if (!pr.nbg) tmem_st16(tmem + lane_off + col, v);
     };
 
-    for (int j = 0; j < nh; ++j) {
-      // A buffer j % 2 is free: the MMA of head j - 2 was waited for by the
-      // epilogue of that head in the previous iteration
-      if (j == 0) {
-        wait_warp(&sh.full_cb, 0);  // the C tile (read below for the scaled-C block)
-        wait_warp(&sh.mbar_cb, 0);  // CB in TMEM; the B tile is free (A buffer 1)
+    // the per-chunk dt and cumsum rows (written by the chunk-state kernel) of a
+    // unit's heads: one warp per head, 4 consecutive tokens per lane; the next
+    // unit's are loaded before this unit's norm exchange and used after it
+    float4 cu = make_float4(0.f, 0.f, 0.f, 0.f), dv = cu;
+    auto load_rows = [&](int n) {
+      if (warp < nh && n < n_units) {
+        int64_t bi;
+        int c, g;
+        out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+        const int64_t row = (bi * a.nch + c) * pr.H + g * hpg + lh0 + warp;
+        cu = reinterpret_cast<const float4 *>(a.cum + row * kQ)[lane];
+        dv = reinterpret_cast<const float4 *>(a.dtv + row * kQ)[lane];
       }
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t abuf = base + a_block(j & 1, 0), abuf2 = base + a_block(j & 1, 2);
-      const uint32_t abuf1 = base + a_block(j & 1, 1);
+    };
+    load_rows(0);
+    for (int n = 0; ok && n < n_units; ++n) {
+      int64_t bi;
+      int c, g;
+      out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+      const int h0 = g * hpg + lh0;
+      const int64_t c0 = (int64_t)c * kQ;
+      const int par = n & 1;
+      // decay terms of the unit's heads
+      if (warp < nh) {
+        const int j = warp;
+        const float cum4[4] = {cu.x, cu.y, cu.z, cu.w}, dt4[4] = {dv.x, dv.y, dv.z, dv.w};
+        float c2[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          c2[k] = cum4[k] * kLog2e;
+          sh.cum2[j][4 * lane + k] = c2[k];
+          sh.dt[j][4 * lane + k] = dt4[k];
+        }
+        const float c2r = __shfl_sync(0xffffffffu, c2[3], (lane | 7));
+        const float c2s0 = __shfl_sync(0xffffffffu, c2[0], (lane & ~7));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          sh.beta[j][4 * lane + k] = ex2_approx(c2r - c2[k]) * dt4[k];
+          sh.betad[j][4 * lane + k] = ex2_approx(fminf(c2s0 - c2[k], 60.0f)) * dt4[k];
+        }
+        if ((lane & 7) == 7) sh.span_ok[j][lane >> 3] = (c2s0 - c2r) <= 60.0f;
+      }
+      for (int i = tid; i < nh * kHP; i += kThreads)
+        sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
+      if (tid < nh) sh.Dh[tid] = a.prm.D[h0 + tid];
+      if (n > 0 && tid == 0) bulk_wait_read_all();  // the previous unit's output staging
+      compute_sync();  // decay terms, weights and D visible; staging tiles free
+      ss_acc = 0.0f;
+
+      for (int j = 0; j < nh; ++j, ++J) {
+        // A buffer J % 2 is free: the MMA of head J - 2 was waited for by its
+        // epilogue in the previous iteration (or the previous unit)
+        if (j == 0) {
+          wait_warp(&sh.full_cb, (uint32_t)(n & 1));  // the C tile (read for the scaled-C block)
+          wait_warp(&sh.mbar_cb, (uint32_t)(n & 1));  // CB in TMEM; the B tile is free (A buffer 1)
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t abuf = base + a_block(J & 1, 0), abuf2 = base + a_block(J & 1, 2);
+        const uint32_t abuf1 = base + a_block(J & 1, 1);
       // A_j = [CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal | C o exp(cum_t)];
       // 32-column groups k above the row quarter q are zero, below it the decay
       // factorises as alpha_t beta_s (both <= 1), on it exponentials are direct.
@@ -1039,7 +1150,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           }
         }
         // C scaled by exp(cum_t): this warp does n in [16 hf, 16 hf + 16)
-        const float ec = sh.ecum[j][t];
+        const float ec = ex2_approx(c2t);
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
           const int n0 = 16 * hf + 8 * qq;
@@ -1054,122 +1165,168 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           st_shared_v4(abuf2 + sw128_chunk(t, n0), o[0], o[1], o[2], o[3]);
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&sh.a_ready[j & 1]);
-      if (j > 0) {  // epilogue of the previous head overlaps this head's MMA
-        wait_warp(&sh.mbar_mma[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1));
-        wait_warp(&sh.full_z[(j - 1) % kZStages], (uint32_t)(((j - 1) / kZStages) & 1));
-        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.a_ready[J & 1]);
+        if (j > 0) {  // epilogue of the previous head overlaps this head's MMA
+          const int P1 = J - 1;
+          wait_warp(&sh.mbar_mma[P1 & 1], (uint32_t)((P1 >> 1) & 1));
+          wait_warp(&sh.full_z[P1 % kZStages], (uint32_t)((P1 / kZStages) & 1));
+          if (!ok) break;
+          tc_fence_after();
+          epilogue1(j - 1, P1 % kZStages);
+          mbar_arrive(&sh.empty_z[P1 % kZStages]);
+        }
+      }
+      if (ok && nh > 0) {
+        const int P1 = J - 1;
+        wait_warp(&sh.mbar_mma[P1 & 1], (uint32_t)((P1 >> 1) & 1));
+        wait_warp(&sh.full_z[P1 % kZStages], (uint32_t)((P1 / kZStages) & 1));
         tc_fence_after();
-        epilogue1(j - 1);
-        mbar_arrive(&sh.empty_z[(j - 1) % kZStages]);
+        if (ok) {
+          epilogue1(nh - 1, P1 % kZStages);
+          mbar_arrive(&sh.empty_z[P1 % kZStages]);
+        }
       }
-    }
-    if (ok && nh > 0) {
-      wait_warp(&sh.mbar_mma[(nh - 1) & 1], (uint32_t)(((nh - 1) >> 1) & 1));
-      wait_warp(&sh.full_z[(nh - 1) % kZStages], (uint32_t)(((nh - 1) / kZStages) & 1));
-      tc_fence_after();
-      if (ok) epilogue1(nh - 1);
-    }
-    if (!ok) {
-      sh.ok_flag = 0;
-      if (lane == 0) {
-        // a wait ran out: let issued MMAs and tile copies land before the CTA exits
-        mbar_wait_bounded(&sh.mbar_cb, 0, &g_tc_errors);
-        mbar_wait_bounded(&sh.full_cb, 0, &g_tc_errors);
-      }
-    }
-    sh.ss[hf][t] = ss_acc;
-  }
-  __syncthreads();  // producer joins here
+      sh.ss[hf][t] = ss_acc;
+      load_rows(n + 1);
+      tc_fence_before();
+      compute_sync();
+      // the unit's C and B tiles and CB columns are no longer read; its last MMA is done
+      if (tid == 0) mbar_arrive(&sh.tiles_free);
 
-  // per-token sums of squares of this CTA, pushed into every rank's table
-  // part[rank][t] (plain remote stores), then one cluster barrier; after it each
-  // CTA only reads its own shared memory, so none waits for the others to exit
-  if (tid < kQ) sh.mine[tid] = (sh.ss[0][tid] + sh.ss[1][tid]) + (sh.ss[2][tid] + sh.ss[3][tid]);
-  __syncthreads();
-  cluster_wait();  // (arrived at the start) every CTA of the cluster is running
-  for (int i = tid; i < cs * (kQ / 4); i += kWsThreads) {
-    const int r = i / (kQ / 4), f = i % (kQ / 4);
-    float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(&sh.part[rank][0], r));
-    dst[f] = reinterpret_cast<const float4 *>(sh.mine)[f];
-  }
-  cluster_arrive_release();
-  cluster_wait();
-  if (tid < kQ) {
-    float tot = 0.0f;
-    for (int r = 0; r < cs; ++r) tot += sh.part[r][tid];
-    sh.inv[tid] = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
-  }
-  __syncthreads();
-  tc_fence_after();
-  // normalised bf16 output: each head's [128 t][64 p] tile is written into shared
-  // memory (128-byte swizzle; the tile buffers are all free now) and stored by TMA,
-  // which drops the rows past the end of the sequence
-  const uint32_t ybuf = base + kXh;
-  if (sh.ok_flag && warp < kThreads / 32) {
-    const int t = 32 * (warp & 3) + lane, hf = warp >> 2;
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const bool t_valid = c0 + t < pr.L;
-    const float sc = sh.inv[t];
-    for (int j = 0; j < nh; ++j) {
-      const int h = h0 + j;
-      float v[16];
-      tmem_ld16(tmem + lane_off + 128 + 64 * j + 16 * hf, v);
-      const float4 *nw4 = reinterpret_cast<const float4 *>(&sh.nw[j][16 * hf]);
-      if (pr.nbg && t_valid) {
-        const int64_t row = bi * pr.L + c0 + t;
-        const uint4 *zp =
-            reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 16 * hf);
+      // per-token partial sums of this CTA into part[par][rank][*] of every rank
+      // (asynchronous stores completing bytes on that rank's barrier)
+      if (tid < kQ) sh.mine[tid] = (sh.ss[0][tid] + sh.ss[1][tid]) + (sh.ss[2][tid] + sh.ss[3][tid]);
+      if (!started) {
+        cluster_wait();  // (arrived at the start) every CTA of the cluster is running
+        started = true;
+      }
+      compute_sync();
+      for (int i = tid; i < cs * (kQ / 4); i += kThreads) {
+        const int r = i / (kQ / 4), f = i % (kQ / 4);
+        st_async_v4(cluster_addr(&sh.part[par][rank][4 * f], r),
+                    reinterpret_cast<const float4 *>(sh.mine)[f], cluster_addr(&sh.sums_ready[par], r));
+      }
+      ok = __all_sync(0xffffffffu,
+                      ok && mbar_wait_cluster_bounded(&sh.sums_ready[par], (uint32_t)((n >> 1) & 1))) != 0;
+      if (tid < kQ) {
+        float tot = 0.0f;
+        for (int r = 0; r < cs; ++r) tot += sh.part[par][r][tid];
+        sh.inv[tid] = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
+      }
+      compute_sync();
+      // unit n + 2 uses this parity again; no rank sends it before this CTA has
+      // sent unit n + 1's sums, which happens after this point
+      if (tid == 0 && n + 2 < n_units) mbar_arrive_expect_tx(&sh.sums_ready[par], sum_bytes);
+      tc_fence_after();
+      // normalised bf16 output: each head's [128 t][64 p] tile is written into a
+      // staging tile (128-byte swizzle) and stored by TMA, which drops the rows past
+      // the end of the sequence.  The five staging tiles are the A buffers' blocks
+      // other than the B tile (the next unit's B may be arriving there); a sixth
+      // head reuses the first tile once its store has read it.
+      if (ok && sh.ok_flag) {
+        const bool t_valid = c0 + t < pr.L;
+        const float sc = sh.inv[t];
+        for (int j = 0; j < nh; ++j) {
+          const int h = h0 + j;
+          const int slot = j % kYTiles;
+          const uint32_t ybuf = base + (slot < 3 ? kA0 + slot * 16384 : kA1 + (slot - 3) * 16384);
+          if (j == kYTiles) {  // the store of head 0 has read its tile
+            if (tid == 0) bulk_wait_read_le(kYTiles - 1);
+            compute_sync();
+          }
+          float v[16];
+          tmem_ld16(tmem + lane_off + 128 + 64 * j + 16 * hf, v);
+          const float4 *nw4 = reinterpret_cast<const float4 *>(&sh.nw[j][16 * hf]);
+          if (pr.nbg && t_valid) {
+            const int64_t row = bi * pr.L + c0 + t;
+            const uint4 *zp =
+                reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 16 * hf);
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const uint4 raw = __ldg(zp + qq);
-          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+            for (int qq = 0; qq < 2; ++qq) {
+              const uint4 raw = __ldg(zp + qq);
+              const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(h2[i]);
-            v[8 * qq + 2 * i] *= silu_fast(f.x);
-            v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
+              for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h2[i]);
+                v[8 * qq + 2 * i] *= silu_fast(f.x);
+                v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
+              }
+            }
+          }
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            uint32_t o[4];
+            const float4 wA = nw4[2 * qq], wB = nw4[2 * qq + 1];
+            const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 8 * qq + 2 * e;
+              const __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(v[i] * sc * ww[2 * e], v[i + 1] * sc * ww[2 * e + 1]);
+              o[e] = *reinterpret_cast<const uint32_t *>(&b2);
+            }
+            st_shared_v4(ybuf + sw128_chunk(t, 16 * hf + 8 * qq), o[0], o[1], o[2], o[3]);
+          }
+          fence_proxy_async_smem();
+          compute_sync();  // head j's tile is complete: store it while the next one is built
+          if (tid == 0) {
+            tma_store_3d(&maps.y, ybuf, h * kHP, (int)c0, (int)bi);
+            bulk_commit();
           }
         }
       }
-#pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        uint32_t o[4];
-        const float4 wA = nw4[2 * qq], wB = nw4[2 * qq + 1];
-        const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 8 * qq + 2 * e;
-          const __nv_bfloat162 b2 =
-              __floats2bfloat162_rn(v[i] * sc * ww[2 * e], v[i + 1] * sc * ww[2 * e + 1]);
-          o[e] = *reinterpret_cast<const uint32_t *>(&b2);
-        }
-        st_shared_v4(ybuf + j * 16384 + sw128_chunk(t, 16 * hf + 8 * qq), o[0], o[1], o[2], o[3]);
-      }
-      fence_proxy_async_smem();
-      compute_sync();  // head j's tile is complete: store it while the next one is built
-      if (tid == 0) tma_store_3d(&maps.y, ybuf + j * 16384, (h0 + j) * kHP, (int)c0, (int)bi);
+      // the y columns of TMEM are read before the next unit's MMAs; its A-builds
+      // wait for the stores to have read the staging tiles
+      tc_fence_before();
+      compute_sync();
     }
-    if (tid == 0) bulk_commit_and_wait_read();
+    if (tid == 0) bulk_wait_read_all();  // the last unit's stores have read their tiles
+    if (!ok) sh.ok_flag = 0;
   }
+  // every thread: the cluster's start barrier (if not waited for yet), then one
+  // more: no CTA exits while another may still store into its shared memory
+  __syncwarp();
+  if (!started) cluster_wait();
+  cluster_arrive_release();
+  cluster_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+
 // Heads per CTA and cluster size of tc_chunk_out for hpg heads per group.
-void out_split(int hpg, int *cs, int *hpc) {
+// Most clusters of `cs` output-kernel CTAs resident at once on the current
+// device (cached per device; -1 if the query fails).
+int out_max_clusters(int cs);
+
+// Cluster size of the output kernel: every size from ceil(hpg / 6) to 16 whose
+// heads per CTA fit tensor memory is scored by the rounds of units its resident
+// clusters need times (heads per CTA + a per-unit cost of about 2.5 heads).
+void out_choose(int hpg, int64_t units, int *cs, int *hpc, int *ncl) {
   const int lo = (hpg + kMaxHeadsPerCta - 1) / kMaxHeadsPerCta;
-  for (int c = lo; c <= 16; ++c)
-    if (hpg % c == 0) {
+  int64_t best = -1;
+  for (int c = std::max(lo, 1); c <= 16; ++c) {
+    const int h = (hpg + c - 1) / c;
+    if (h > kMaxHeadsPerCta) continue;
+    const int m = out_max_clusters(c);
+    if (m <= 0) continue;
+    const int64_t rounds = (units + m - 1) / m;
+    const int64_t score = rounds * (2 * h + 5);
+    if (best < 0 || score < best) {
+      best = score;
       *cs = c;
-      *hpc = hpg / c;
-      return;
+      *hpc = h;
+      *ncl = (int)std::min<int64_t>(units, m);
     }
-  *cs = lo;
-  *hpc = (hpg + lo - 1) / lo;
+  }
+  if (best < 0) {  // no occupancy answer: the smallest cluster, one per unit
+    *cs = std::max(lo, 1);
+    *hpc = (hpg + *cs - 1) / *cs;
+    *ncl = (int)std::min<int64_t>(units, 65535);
+  }
 }
 
 struct TcWorkspace {
@@ -1244,6 +1401,34 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank
 
 constexpr size_t kK1Smem = kK1Tiles + 1024;
 constexpr size_t kK3Smem = kTcOutTiles + sizeof(OutShared) + 1024;
+static_assert(kK1Smem <= 227 * 1024 && kK3Smem <= 227 * 1024, "shared memory per CTA");
+
+int out_max_clusters(int cs) {
+  static int cache[64][17] = {};  // 0: not asked yet
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || cs < 1 || cs > 16) return -1;
+  int &m = cache[dev][cs];
+  if (m == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cs, 1, 1);
+    cfg.blockDim = dim3(kWsThreads, 1, 1);
+    cfg.dynamicSmemBytes = kK3Smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int v = 0;
+    if (cudaOccupancyMaxActiveClusters(&v, tc_chunk_out_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();  // clear the failed query
+      v = -1;
+    }
+    m = v > 0 ? v : -1;
+  }
+  return m;
+}
 
 }  // namespace
 
@@ -1298,10 +1483,6 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.Hc = w.Hc;
   a.u = w.u;
   const int hpg = pr.heads_per_group();
-  int cs = 1, hpc = 1;
-  out_split(hpg, &cs, &hpc);
-  a.hpc = hpc;
-
   cudaError_t e;
   e = cudaFuncSetAttribute(tc_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kK1Smem);
@@ -1311,6 +1492,9 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
+  int cs = 1, hpc = 1, ncl = 1;
+  out_choose(hpg, pr.batch * a.nch * (int64_t)pr.G, &cs, &hpc, &ncl);
+  a.hpc = hpc;
 
   stage_mark(st, 0);
   const int64_t n_items = pr.batch * a.nch * (int64_t)pr.G * ((hpg + 1) / 2 + 1);
@@ -1331,7 +1515,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   stage_mark(st, 2);
   {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)cs, (unsigned)a.nch, (unsigned)(pr.G * pr.batch));
+    cfg.gridDim = dim3((unsigned)cs, (unsigned)ncl, 1);
     cfg.blockDim = dim3(kWsThreads, 1, 1);
     cfg.dynamicSmemBytes = kK3Smem;
     cfg.stream = st;
@@ -1360,7 +1544,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
           !make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, 3, dy, sy, bu))
         return cudaErrorInvalidValue;
     }
-    e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps);
+    e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps, ncl);
     if (e != cudaSuccess) return e;
   }
   stage_mark(st, 3);
