@@ -5,8 +5,8 @@
 // It evaluates the chunked state-space-duality form of the scan (the Mamba-2
 // layer named on the state-spaces/mamba repository page, opendeer.net, "About
 // the project"; chunked prefill per "Zamba2 hybrid architecture in
-// Transformers", qwbw.cn, section 三 step 3) with 128-token chunks, one chunk
-// per CTA so that the token dimension is the MMA's M = 128:
+// Transformers", qwbw.cn, section 三 step 3) with 128-token chunks, so that
+// a chunk's tokens are the MMA's M = 128 rows:
 //
 //   tc_chunk_state  conv+SiLU of x (two heads) and B, dt/cumsum, then
 //                   S_c = (x o w)^T B with w_s = exp(cum_end - cum_s) dt_s:
@@ -14,8 +14,9 @@
 //   tc_state_pass   H_{c+1} = exp(cum_end) H_c + S_c over chunks in fp32; the
 //                   state entering each chunk is kept as the fp16 MMA operand,
 //                   the final state in fp32.
-//   tc_chunk_out    per chunk, a cluster of CTAs splits the heads of one B/C
-//                   group: CB = C B^T (M = N = 128, K = 64) once; per head the
+//   tc_chunk_out    persistent clusters; per (row, chunk, group) unit the
+//                   cluster's CTAs split the heads of the group:
+//                   CB = C B^T (M = N = 128, K = 64) once; per head the
 //                   operand [CB o exp(cum_t - cum_s) dt_s (causal) | C o exp(cum_t)]
 //                   times [x ; H_c] gives y_pre (K = 128 + 64) in TMEM; D x,
 //                   the silu(z) gate and sums of squares follow, the per-token
