@@ -1024,6 +1024,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       }
     };
     load_rows(0);
+    int nw_h0 = -1;  // heads whose norm weights are in shared memory
     for (int n = 0; ok && n < n_units; ++n) {
       int64_t bi;
       int c, g;
@@ -1051,9 +1052,12 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         }
         if ((lane & 7) == 7) sh.span_ok[j][lane >> 3] = (c2s0 - c2r) <= 60.0f;
       }
-      for (int i = tid; i < nh * kHP; i += kThreads)
-        sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
-      if (tid < nh) sh.Dh[tid] = a.prm.D[h0 + tid];
+      if (h0 != nw_h0) {  // norm weights and D of the CTA's heads (same in every unit if G = 1)
+        for (int i = tid; i < nh * kHP; i += kThreads)
+          sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
+        if (tid < nh) sh.Dh[tid] = a.prm.D[h0 + tid];
+        nw_h0 = h0;
+      }
       if (n > 0 && tid == 0) bulk_wait_read_all();  // the previous unit's output staging
       compute_sync();  // decay terms, weights and D visible; staging tiles free
       ss_acc = 0.0f;
