@@ -241,7 +241,8 @@ struct K1Maps {
 // conv1d + SiLU of the 8 channels in 16-byte column `cg` of a raw tile, for
 // output tokens at tile rows s0+3 .. s0+6 (inputs: rows s0 .. s0+6); taps and
 // bias of the tile's 64 channels in shared memory, channel 8 g + i at [i][g]
-// (wt[8][8] float4, bs[8][8]) so that neighbouring groups read neighbouring words.
+// (wt[8][8] float4, bs[8][8]) so that neighbouring groups read neighbouring words,
+// stored halved: the sum is then h = pre / 2 exactly, and silu(pre) = h + h tanh(h).
 __device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float4 *wt,
                                              const float *bs, float (&out)[4][8]) {
   float w[8][4], bias[8];
@@ -271,9 +272,9 @@ __device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, cons
   for (int k = 0; k < 4; ++k)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float pre = bias[i] + w[i][0] * rows[k][i] + w[i][1] * rows[k + 1][i] +
-                        w[i][2] * rows[k + 2][i] + w[i][3] * rows[k + 3][i];
-      out[k][i] = silu_fast(pre);
+      const float h = bias[i] + w[i][0] * rows[k][i] + w[i][1] * rows[k + 1][i] +
+                      w[i][2] * rows[k + 2][i] + w[i][3] * rows[k + 3][i];
+      out[k][i] = fmaf(h, tanh_approx(h), h);
     }
 }
 
@@ -450,8 +451,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int i = lane + 32 * j, d = (i & 7) * 8 + (i >> 3);
-          wts[st][sl][d] = tw[sl][j];
-          bss[st][sl][d] = tb[sl][j];
+          const float4 w4 = tw[sl][j];  // halved (exact), see conv8x4_smem
+          wts[st][sl][d] = make_float4(0.5f * w4.x, 0.5f * w4.y, 0.5f * w4.z, 0.5f * w4.w);
+          bss[st][sl][d] = 0.5f * tb[sl][j];
         }
       }
       __syncwarp();
