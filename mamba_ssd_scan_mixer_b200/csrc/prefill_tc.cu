@@ -44,7 +44,8 @@ constexpr int kWsThreads = kThreads + 64;   // + TMA producer warp + MMA issuer 
 constexpr int kK1Threads = kThreads + 96;   // + 2 producer warps (even / odd items) + MMA warp
 constexpr int kHP = 64;          // headdim
 constexpr int kNS = 64;          // d_state
-constexpr int kMaxHeadsPerCta = 6;  // TMEM: 128 (CB) + 6 x 64 (y) <= 512 columns
+constexpr int kMaxHeadsPerCta = 5;  // TMEM: 128 (CB) + 5 x 64 (y) + 64 (C H_c^T) = 512 columns
+constexpr uint32_t kTmemT = 128 + 64 * kMaxHeadsPerCta;  // column of the C H_c^T accumulator
 constexpr float kLog2e = 1.4426950408889634f;
 
 static __device__ unsigned int g_tc_errors = 0;
@@ -741,27 +742,35 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
 // Persistent clusters: grid (cs, ncl, 1), cluster (cs, 1, 1).  Cluster k takes
 // the units (row, chunk, group) k, k + ncl, ...; its cs CTAs split the group's
 // heads.  16 compute warps + 1 TMA producer warp + 1 MMA-issuer warp.  Tiles
-// arrive by TMA in 128-byte-swizzled layouts (1024-aligned).  The operand A is
-// double-buffered so that the A-build of head j + 1 overlaps the MMA of head j;
-// buffer 1 reuses the B tile once CB is formed.  The next unit's C and B tiles,
-// its CB product and its first x / H_c / z tiles arrive while the current
-// unit exchanges its norm sums and writes its output.
+// arrive by TMA in 128-byte-swizzled layouts (1024-aligned).  Per head the
+// intra-chunk part [CB o L o dt (+D)] x is one K = 128 MMA into the head's TMEM
+// columns, and the carried-state part C H_c^T a K = 64 MMA with the C tile
+// itself as operand into a shared TMEM accumulator, scaled by exp(cum_t) in
+// the epilogue.  The operand A is double-buffered so that the A-build of head
+// j + 1 overlaps the MMA of head j; buffer 1 reuses the B tile once CB is
+// formed.  The next unit's C and B tiles, its CB product and its first
+// x / H_c / z tiles arrive while the current unit exchanges its norm sums and
+// writes its output.
 constexpr uint32_t kCt = 0;                      // C   [128 t][64 n] fp16     16 KB (u)
 constexpr uint32_t kBt = kCt + 16384;            // B   [128 s][64 n] fp16     16 KB (u)
 constexpr int kXhStages = 2, kZStages = 2;
 constexpr uint32_t kXhBytes = 16384 + 8192;      // per stage: x [128 s][64 p] + H_c [64 n][64 p]
 constexpr uint32_t kXh = kBt + 16384;            // x / H_c ring  2 x 24 KB (x at +0, H_c at +16 KB)
 constexpr uint32_t kZt = kXh + kXhStages * kXhBytes;  // z ring [128 t][64 p] bf16  2 x 16 KB
-constexpr uint32_t kA0 = kZt + kZStages * 16384;      // A buffer 0: [3][128 t][64 k] fp16  48 KB
-constexpr uint32_t kA1 = kA0 + 3 * 16384;             // A buffer 1, blocks 1 and 2 (block 0 at kBt)
-constexpr uint32_t kTcOutTiles = kA1 + 2 * 16384;     // 192 KB
-// output staging: [128 t][64 p] bf16 tiles in the A buffers, idle while a unit
-// writes its output (A buffer 0 and blocks 1, 2 of buffer 1)
+constexpr uint32_t kA0 = kZt + kZStages * 16384;      // A buffer 0: [2][128 t][64 k] fp16  32 KB
+constexpr uint32_t kA1 = kA0 + 2 * 16384;             // A buffer 1, block 1 (block 0 at kBt)
+constexpr uint32_t kYst = kA1 + 16384;                // two output staging tiles  32 KB
+constexpr uint32_t kTcOutTiles = kYst + 2 * 16384;    // 192 KB
+// output staging: [128 t][64 p] bf16 tiles, idle while a unit writes its output:
+// A buffer 0, block 1 of buffer 1 and the two staging tiles
 constexpr int kYTiles = 5;
+__device__ __forceinline__ uint32_t y_tile(int slot) {
+  return slot < 2 ? kA0 + slot * 16384 : (slot == 2 ? kA1 : kYst + (slot - 3) * 16384);
+}
 
-// Byte offset of k-block `blk` (0, 1: CB columns s; 2: scaled C) of A buffer `buf`.
+// Byte offset of k-block `blk` (CB columns s 0..63, 64..127) of A buffer `buf`.
 __device__ __forceinline__ uint32_t a_block(int buf, int blk) {
-  return buf == 0 ? kA0 + blk * 16384 : (blk == 0 ? kBt : kA1 + (blk - 1) * 16384);
+  return buf == 0 ? kA0 + blk * 16384 : (blk == 0 ? kBt : kA1);
 }
 
 struct OutShared {
@@ -777,7 +786,7 @@ struct OutShared {
   float inv[kQ];
   float Dh[kMaxHeadsPerCta];
   uint64_t full_cb, full_xh[kXhStages], empty_xh[kXhStages], full_z[kZStages],
-      empty_z[kZStages], a_ready[2], mbar_cb, mbar_mma[2], tiles_free, sums_ready[2];
+      empty_z[kZStages], a_ready[2], mbar_cb, mbar_mma[2], tiles_free, sums_ready[2], t_free;
   uint32_t tmem_holder;
   int ok_flag;
 };
@@ -875,6 +884,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     }
     mbar_init(&sh.mbar_cb, 1);
     mbar_init(&sh.tiles_free, 1);  // a unit's C / B tiles and CB columns no longer read
+    mbar_init(&sh.t_free, kThreads);  // every compute thread has read the C H_c^T columns
     fence_mbar_init();
     sh.ok_flag = 1;
   }
@@ -955,17 +965,20 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t xt = base + kXh + (J % kXhStages) * kXhBytes, ht = xt + 16384;
-          for (int ks = 0; ks < 12; ++ks) {
-            const int blk = ks >> 2, kin = ks & 3;
-            const uint64_t ad = umma_desc_sw128(base + a_block(J & 1, blk) + kin * 32);
-            // x [s][p] and H_c [n][p] are both MN-major (p contiguous)
-            if (ks < 8)
-              umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(xt + ks * 2048, 16384),
-                       idesc_mn, ks > 0 ? 1u : 0u);
-            else
-              umma_f16(tmem + 128 + 64 * j, ad, umma_desc_sw128_mn(ht + (ks - 8) * 2048, 8192),
-                       idesc_mn, 1u);
+          // y_j = [CB o L o dt (+D)] x : K = 128 (x [s][p] MN-major)
+          for (int ks = 0; ks < 8; ++ks)
+            umma_f16(tmem + 128 + 64 * j, umma_desc_sw128(base + a_block(J & 1, ks >> 2) + (ks & 3) * 32),
+                     umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn, ks > 0 ? 1u : 0u);
+          // T = C H_c^T : K = 64, the C tile as operand (H_c [n][p] MN-major), once the
+          // previous head's epilogue has read T
+          if (J > 0 && !mbar_wait_bounded(&sh.t_free, (uint32_t)((J - 1) & 1), &g_tc_errors)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          for (int kin = 0; kin < 4; ++kin)
+            umma_f16(tmem + kTmemT, umma_desc_sw128(base + kCt + kin * 32),
+                     umma_desc_sw128_mn(ht + kin * 2048, 8192), idesc_mn, kin > 0 ? 1u : 0u);
           umma_commit(&sh.mbar_mma[J & 1]);
           umma_commit(&sh.empty_xh[J % kXhStages]);  // its x / H_c stage is free once it completes
         }
@@ -989,9 +1002,15 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     // epilogue, part 1: gate with silu(z) (z tile in smem), sum of squares, g -> TMEM.
     // Warp w handles rows 32*(w%4) .. +31 and columns 16*(w/4) .. +15 of a head.
     auto epilogue1 = [&](int j, int zslot) {
-      float v[16];
+      float v[16], w[16];
       const uint32_t col = 128 + 64 * j + 16 * hf;
       tmem_ld16(tmem + lane_off + col, v);
+      tmem_ld16(tmem + lane_off + kTmemT + 16 * hf, w);
+      tc_fence_before();
+      mbar_arrive(&sh.t_free);  // the C H_c^T columns may take the next head's product
+      const float ec = ex2_approx(sh.cum2[j][t]);  // exp(cum_t)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = fmaf(ec, w[i], v[i]);
       if (!pr.nbg) {
         const uint32_t zt = base + kZt + zslot * 16384;
 #pragma unroll
@@ -1008,7 +1027,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) ss_acc = fmaf(v[i], v[i], ss_acc);
-      if (!pr.nbg) tmem_st16(tmem + lane_off + col, v);
+      tmem_st16(tmem + lane_off + col, v);
     };
 
     // the per-chunk dt and cumsum rows (written by the chunk-state kernel) of a
@@ -1073,9 +1092,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         }
         if (!ok) break;
         tc_fence_after();
-        const uint32_t abuf = base + a_block(J & 1, 0), abuf2 = base + a_block(J & 1, 2);
-        const uint32_t abuf1 = base + a_block(J & 1, 1);
-      // A_j = [CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal | C o exp(cum_t)];
+        const uint32_t abuf = base + a_block(J & 1, 0), abuf1 = base + a_block(J & 1, 1);
+      // A_j = CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal;
       // 32-column groups k above the row quarter q are zero, below it the decay
       // factorises as alpha_t beta_s (both <= 1), on it exponentials are direct.
       {
@@ -1156,21 +1174,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             }
           }
         }
-        // C scaled by exp(cum_t): this warp does n in [16 hf, 16 hf + 16)
-        const float ec = ex2_approx(c2t);
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int n0 = 16 * hf + 8 * qq;
-          const uint4 cv = ld_shared_v4(base + kCt + sw128_chunk(t, n0));
-          const uint32_t in[4] = {cv.x, cv.y, cv.z, cv.w};
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_half2(in[e]);
-            o[e] = pack_half2(f.x * ec, f.y * ec);
-          }
-          st_shared_v4(abuf2 + sw128_chunk(t, n0), o[0], o[1], o[2], o[3]);
-        }
       }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1230,15 +1233,15 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       // normalised bf16 output: each head's [128 t][64 p] tile is written into a
       // staging tile (128-byte swizzle) and stored by TMA, which drops the rows past
       // the end of the sequence.  The five staging tiles are the A buffers' blocks
-      // other than the B tile (the next unit's B may be arriving there); a sixth
-      // head reuses the first tile once its store has read it.
+      // other than the B tile (the next unit's B may be arriving there) and two
+      // tiles of their own.
       if (ok && sh.ok_flag) {
         const bool t_valid = c0 + t < pr.L;
         const float sc = sh.inv[t];
         for (int j = 0; j < nh; ++j) {
           const int h = h0 + j;
           const int slot = j % kYTiles;
-          const uint32_t ybuf = base + (slot < 3 ? kA0 + slot * 16384 : kA1 + (slot - 3) * 16384);
+          const uint32_t ybuf = base + y_tile(slot);
           if (j == kYTiles) {  // the store of head 0 has read its tile
             if (tid == 0) bulk_wait_read_le(kYTiles - 1);
             compute_sync();
