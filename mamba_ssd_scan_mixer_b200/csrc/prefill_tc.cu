@@ -17,8 +17,9 @@
 //   tc_chunk_out    persistent clusters; per (row, chunk, group) unit the
 //                   cluster's CTAs split the heads of the group:
 //                   CB = C B^T (M = N = 128, K = 64) once; per head the
-//                   operand [CB o exp(cum_t - cum_s) dt_s (causal) | C o exp(cum_t)]
-//                   times [x ; H_c] gives y_pre (K = 128 + 64) in TMEM; D x,
+//                   operand CB o exp(cum_t - cum_s) dt_s (causal, D on the
+//                   diagonal) times x (K = 128) and C times H_c^T (K = 64, a
+//                   second accumulator scaled by exp(cum_t)) give y_pre in TMEM;
 //                   the silu(z) gate and sums of squares follow, the per-token
 //                   sums are exchanged through distributed shared memory, and
 //                   the normalised output is written in bf16.
