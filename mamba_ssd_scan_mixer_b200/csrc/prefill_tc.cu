@@ -944,7 +944,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       }
     }
   } else if (warp == kThreads / 32 + 1) {
-    // ---------------- MMA issuer: per unit CB once, then one K = 192 MMA per head
+    // ---------------- MMA issuer: per unit CB once, then per head the K = 128 and K = 64 MMAs
     if (lane == 0 && nh > 0) {
       const uint32_t idesc_cb = umma_idesc_f16(128, 128);
       const uint32_t idesc_mn = umma_idesc_f16(128, 64) | (1u << 16);  // B operand MN-major

@@ -38,11 +38,14 @@ def test_tiny_f32_config():
     case("zamba2_2p7b_prefill", batch=3, seqlen=129, nheads=6, ngroups=3, chunk_size=128),
     case("zamba2_2p7b_prefill", batch=2, seqlen=300, nheads=4, norm_before_gate=True),
     # head splits of the tensor-core output kernel: odd heads per group (a lone head in
-    # the last pair), a cluster of 13 CTAs, an uneven 6/6/5 split, four CTAs of 4 heads
+    # the last pair of the chunk-state kernel), 13 and 17 heads (uneven splits with a
+    # short last CTA), two groups of 16 heads, and 20 heads over 24 (row, chunk)
+    # units, more units than resident clusters
     case("zamba2_2p7b_prefill", batch=1, seqlen=300, nheads=6, ngroups=2),
     case("zamba2_2p7b_prefill", batch=1, seqlen=260, nheads=13),
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=17),
     case("zamba2_2p7b_prefill", batch=2, seqlen=256, nheads=32, ngroups=2),
+    case("zamba2_2p7b_prefill", batch=3, seqlen=1000, nheads=20),
     case("zamba2_2p7b_prefill", batch=1, seqlen=257, nheads=4, headdim=32, dstate=128),
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=4, headdim=16, dstate=32),
     case("tiny_f32", batch=2, seqlen=517, nheads=6, ngroups=2, headdim=64, dstate=64,
@@ -172,6 +175,8 @@ def test_prefill_then_decode_steps_equals_prefill(io):
     case("zamba2_2p7b_decode", batch=3, nheads=6, ngroups=2),
     case("zamba2_2p7b_decode", batch=2, nheads=4, headdim=16, dstate=128, io_dtype="f32"),
     case("zamba2_2p7b_decode", batch=2, nheads=4, norm_before_gate=True),
+    # a prime batch: clusters with one and with two rows (the deferred row finish)
+    case("zamba2_2p7b_decode", batch=37, nheads=8),
 ], ids=lambda c: c.name)
 def test_decode_small(cfg):
     params = W.make_params(cfg, 8)
