@@ -7,10 +7,16 @@ with % of roofline, one JSON line on rank 0.
 A step is one prefill call of the whole mixer core (conv1d+SiLU, dt softplus,
 chunked SSD scan, D skip, gated RMSNorm, final conv/SSM states) over the
 Zamba2-2.7B-shaped workload (batch 1, 4096 tokens, 80 heads x 64, d_state 64,
-chunk 256, bf16 I/O, fp32 state), on synthetic seeded inputs already resident in
-HBM.  Four input/output/workspace sets rotate so that no step finds its data in
-the 126 MB L2.  The decode workload (batch 256, 1024 consecutive single-token
-steps) is reported in the `decode` object of the same line.
+bf16 I/O, fp32 state), on synthetic seeded inputs already resident in HBM.
+Input/output/workspace sets rotate so that no step finds its data in the
+126 MB L2.  The decode workload (batch 256, 1024 consecutive single-token
+steps) is reported in the `decode` object of the same line, and the other
+prefill workloads (1.2B-shaped b8 x 2048, 7B-shaped 32768-token long prefill,
+the tiny fp32 case) in `workloads`, each timed the same way.
+
+`roofline.achieved` is the path's algorithmic bytes (every input read once, y
+and the final states written once) over the dominant kernel's average launch
+time; `roofline.stage_bytes` is that kernel's own compulsory traffic.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
 sequence (seed = rank); there is no data-path collective (weak scaling).  The
@@ -35,6 +41,7 @@ sys.path.insert(0, ROOT)
 
 PREFILL = "zamba2_2p7b_prefill"
 DECODE = "zamba2_2p7b_decode"
+OTHER_PREFILL = ("zamba2_1p2b_prefill", "zamba2_7b_long_prefill", "tiny_f32")
 METRIC = "SSD mixer prefill tokens/s and decode steps/s at 1 B200; % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROTATE = 4
@@ -51,6 +58,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only the headline prefill workload and decode")
     return ap.parse_args()
 
 
@@ -234,17 +243,26 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
-def run_ours(args, rank, world, local_rank):
+def kernel_chunk(cfg, stage_names) -> int:
+    """Chunk length the kernels of this call really use: the tensor-core path
+    (its stages are named tc_*) always runs 128-token chunks, the CUDA-core path
+    honours the configured chunk_size."""
+    return 128 if any(n.startswith("tc_") for n in stage_names) else cfg.chunk_size
+
+
+def measure_prefill(name, args, dev, stream, seed, world, peaks, peak_src, m2, W, lib,
+                    steps=None, warmup=None, flush_l2=False):
+    """Device-timed prefill steps of workload `name` (inputs resident in HBM).
+
+    Input/output/workspace sets rotate so that a step never finds its data in
+    L2 (the rotation's total exceeds the 126 MB L2); with flush_l2 (for
+    workloads too small for that) a 256 MB buffer is written between steps and
+    each step is timed on its own.  Every stage is bracketed once per warm-up
+    step; the dominant one is then bracketed by its own events in every timed
+    step."""
     import torch
     import torch.distributed as dist
-    import mamba_ssd_scan_mixer_b200 as m2
-    from mamba_ssd_scan_mixer_b200 import workloads as W
-
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    cfg = W.CONFIGS[PREFILL]
-    seed = rank_seed(rank)
-    lib = m2.lib()
+    cfg = W.CONFIGS[name]
     dims = m2.dims_from_config(cfg)
     params = {k: v.to(dev) for k, v in W.make_params(cfg, seed).items()}
     pp = m2.make_params(params["conv_w"], params["conv_b"], params["dt_bias"], params["A"],
@@ -252,8 +270,10 @@ def run_ours(args, rank, world, local_rank):
     host_in = W.make_prefill_inputs(cfg, seed)["zxbcdt"]
     di, cd = cfg.d_inner, cfg.conv_dim
     ws_bytes = m2.mamba2_prefill_workspace_size(dims)
+    in_bytes = host_in.numel() * host_in.element_size()
+    rotate = 1 if flush_l2 else max(2, min(ROTATE, -(-4 * 126_000_000 // max(1, in_bytes))))
     sets = []
-    for r in range(ROTATE):
+    for r in range(rotate):
         packed = host_in.to(dev)
         v = W.split_packed(cfg, packed)
         sets.append(dict(
@@ -261,14 +281,14 @@ def run_ours(args, rank, world, local_rank):
             y=torch.empty(cfg.batch, cfg.seqlen, di, dtype=cfg.torch_dtype, device=dev),
             cs=torch.zeros(cfg.batch, cd, cfg.d_conv, dtype=cfg.torch_dtype, device=dev),
             hs=torch.zeros(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, device=dev),
-            ws=torch.empty(ws_bytes, dtype=torch.uint8, device=dev)))
+            ws=torch.empty(max(1, ws_bytes), dtype=torch.uint8, device=dev)))
     rot_bytes = sum(sum(t.numel() * t.element_size() for k, t in s.items()
                         if k in ("packed", "y", "cs", "hs", "ws")) for s in sets)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if flush_l2 else None
 
     names_arr = (ctypes.c_char_p * 16)()
     nst = lib.mamba2_stage_names(0, ctypes.byref(dims), names_arr, 16)
     stage_names = [names_arr[i].decode() for i in range(nst)]
-    stream = torch.cuda.current_stream(dev)
 
     def call(s, events=None):
         if events is not None:
@@ -282,68 +302,73 @@ def run_ours(args, rank, world, local_rank):
         e.record(stream)
         return e
 
-    # warm-up, with every stage bracketed once to find the dominant kernel
-    W_ = max(3, args.warmup)
+    W_ = max(3, args.warmup if warmup is None else warmup)
     stage_ms = [0.0] * nst
     for i in range(W_):
+        if flush is not None:
+            flush.fill_(i & 255)
         evs = [new_event() for _ in range(nst + 1)]
-        call(sets[i % ROTATE], [e.cuda_event for e in evs])
+        call(sets[i % rotate], [e.cuda_event for e in evs])
         torch.cuda.synchronize(dev)
         for j in range(nst):
             stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
     dom = max(range(nst), key=lambda j: stage_ms[j])
 
-    # timed region: exactly K steps; the dominant stage bracketed by its own events
-    K = args.steps
+    K = args.steps if steps is None else steps
     dom_evs = [(new_event(), new_event()) for _ in range(K)]
+    step_evs = [(new_event(), new_event()) for _ in range(K)] if flush is not None else None
     torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local_rank) if rank == 0 else None
-    if sampler:
-        sampler.start()
-        time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for k in range(K):
+        if flush is not None:
+            flush.fill_(k & 255)
+            step_evs[k][0].record(stream)
         a, b = dom_evs[k]
-        evs = [None] * dom + [a.cuda_event, b.cuda_event]
-        call(sets[k % ROTATE], evs)
+        call(sets[k % rotate], [None] * dom + [a.cuda_event, b.cuda_event])
+        if flush is not None:
+            step_evs[k][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    elapsed = t0.elapsed_time(t1)
+    elapsed = (sum(a.elapsed_time(b) for a, b in step_evs) if flush is not None
+               else t0.elapsed_time(t1))
     dom_ms = sum(a.elapsed_time(b) for a, b in dom_evs) / K
-    clocks = sampler.stop() if sampler else None
     elapsed = max_over_ranks(elapsed, world, dev)
-
-    peaks, peak_src = load_peaks()
     ms = elapsed / K
     tokens = cfg.batch * cfg.seqlen
-    value = job_rate(tokens, K, elapsed, world)
     path_bytes = prefill_bytes(cfg)
     path_flops = prefill_flops(cfg)
-    t_roof = max(path_bytes / (peaks["hbm_gbs"] * 1e9), path_flops / (peaks["bf16_tflops"] * 1e12))
+    t_roof = max(path_bytes / (peaks["hbm_gbs"] * 1e9),
+                 path_flops / (peaks["bf16_tflops"] * 1e12))
     dom_name = stage_names[dom]
-    dbytes = stage_bytes(dom_name, cfg)
-    achieved = dbytes / (dom_ms * 1e-3) / 1e9 if dbytes else None
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": W_, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": PREFILL, "batch": cfg.batch, "seqlen": cfg.seqlen,
+    achieved = path_bytes / (dom_ms * 1e-3) / 1e9
+    sbytes = stage_bytes(dom_name, cfg)
+    out = {
+        "value": job_rate(tokens, K, elapsed, world), "unit": "tokens/s", "steps": K,
+        "warmup": W_, "ms_per_step": ms,
+        "config": {"workload": name, "batch": cfg.batch, "seqlen": cfg.seqlen,
                    "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
-                   "ngroups": cfg.ngroups, "chunk": cfg.chunk_size, "state_dtype": "f32",
-                   "parallelism": f"dp{world} (independent sequences)",
-                   "l2": f"{ROTATE} rotating input/output/workspace sets, "
-                         f"{rot_bytes / 1e9:.2f} GB > 126 MB L2"},
+                   "ngroups": cfg.ngroups, "io_dtype": cfg.io_dtype,
+                   "chunk": kernel_chunk(cfg, stage_names),
+                   "chunk_size_setting": cfg.chunk_size, "state_dtype": "f32",
+                   "l2": (f"L2 flushed (256 MB write) before every step, steps timed one by one"
+                          if flush is not None else
+                          f"{rotate} rotating input/output/workspace sets, "
+                          f"{rot_bytes / 1e9:.2f} GB > 126 MB L2")},
+        # achieved = the path's algorithmic bytes (every input read once, y and the
+        # final states written once) over the dominant kernel's average launch time
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"] if achieved else None,
-                     "traffic": traffic_for(dom_name, PREFILL),
-                     "algorithmic_bytes": dbytes, "avg_launch_ms": dom_ms,
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic_for(dom_name, name),
+                     "algorithmic_bytes": path_bytes, "avg_launch_ms": dom_ms,
+                     "stage_bytes": sbytes,
+                     "stage_gbs": sbytes / (dom_ms * 1e-3) / 1e9 if sbytes else None,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_src == "measured" else "fallback 6650 GB/s"},
         "path_roofline": {"bytes": path_bytes, "flops": path_flops,
@@ -352,16 +377,70 @@ def run_ours(args, rank, world, local_rank):
                           "frac": t_roof * 1e3 / ms, "peak_source": peak_src},
         "stages_ms_warmup_avg": {n: stage_ms[j] / W_ for j, n in enumerate(stage_names)},
         "gpu_launches": K * nst,
-        "clocks": clocks,
+    }
+    del sets, flush
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import mamba_ssd_scan_mixer_b200 as m2
+    from mamba_ssd_scan_mixer_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = W.CONFIGS[PREFILL]
+    seed = rank_seed(rank)
+    lib = m2.lib()
+    dims = m2.dims_from_config(cfg)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    head = measure_prefill(PREFILL, args, dev, stream, seed, world, peaks, peak_src, m2, W, lib)
+    clocks = sampler.stop() if sampler else None
+
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": head["steps"], "warmup": head["warmup"], "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(head["config"], parallelism=f"dp{world} (independent sequences)"),
+        "roofline": head["roofline"], "path_roofline": head["path_roofline"],
+        "stages_ms_warmup_avg": head["stages_ms_warmup_avg"],
+        "gpu_launches": head["gpu_launches"], "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_e2e:
-        line["e2e"] = run_e2e(args, cfg, dims, pp, host_in, dev, stream, m2)
+        line["e2e"] = run_e2e(args, cfg, dims, head_params(cfg, seed, dev, m2, W),
+                              W.make_prefill_inputs(cfg, seed)["zxbcdt"], dev, stream, m2)
     if not args.no_decode:
         line["decode"] = run_decode(args, dev, stream, rank, world, peaks, peak_src, m2, W)
         line["gpu_launches"] += line["decode"]["gpu_launches"]
+    if not args.no_workloads:
+        # the other prefill workloads: parity-tested shapes, timed the same way
+        other = {}
+        for name in OTHER_PREFILL:
+            small = W.CONFIGS[name].batch * W.CONFIGS[name].seqlen < 65536
+            o = measure_prefill(name, args, dev, stream, seed, world, peaks, peak_src, m2, W,
+                                lib, steps=min(args.steps, 20), warmup=3, flush_l2=small)
+            line["gpu_launches"] += o.pop("gpu_launches")
+            other[name] = o
+        line["workloads"] = other
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, seconds=10.0)
     return line
+
+
+def head_params(cfg, seed, dev, m2, W):
+    params = {k: v.to(dev) for k, v in W.make_params(cfg, seed).items()}
+    pp = m2.make_params(params["conv_w"], params["conv_b"], params["dt_bias"], params["A"],
+                        params["D"], params["norm_w"])
+    pp._keep = params  # the tensors must outlive the pointers
+    return pp
 
 
 def run_e2e(args, cfg, dims, pp, host_in, dev, stream, m2):

@@ -173,6 +173,17 @@ MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *par
  * NULL) or MAMBA2_ERR_CUDA. */
 MAMBA2_API int mamba2_device_errors(unsigned int *flags);
 
+/* Test aid (no counterpart on the pages): makes the time limit of a kernel's
+ * wait run out on purpose, without a fault.  While enabled (1) on the current
+ * device, every kernel that waits for asynchronous work starts with a wait on
+ * a barrier that nothing completes, limited to 20 ms; when it runs out the
+ * kernel raises the flag that mamba2_device_errors reports (bit 0) and
+ * returns before it has issued any copy, so the call's outputs are left
+ * unwritten and the context stays usable.  0 restores normal operation.
+ * Synchronises the device.  Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG or
+ * MAMBA2_ERR_CUDA. */
+MAMBA2_API int mamba2_debug_stall_waits(int enable);
+
 /* Size of the fixed device scratch array used by
  * mamba2_conv_ssd_prefill_noalloc (64 MiB). */
 #define MAMBA2_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
@@ -190,8 +201,12 @@ MAMBA2_API int mamba2_device_errors(unsigned int *flags);
  *  - Problems whose mamba2_prefill_workspace_size exceeds
  *    MAMBA2_STATIC_SCRATCH_BYTES are rejected with MAMBA2_ERR_WORKSPACE and
  *    nothing is enqueued.
- *  - The first call on a device looks up the array's device address (with
- *    that device current); make that first call before any stream capture.
+ *  - The first call in a device's context looks up the array's device
+ *    address (with that device current), and so does the first call after
+ *    that context was destroyed and re-created (cudaDeviceReset); make such a
+ *    call before any stream capture.
+ *  - Invalid dims return MAMBA2_ERR_INVALID_ARG / MAMBA2_ERR_UNSUPPORTED as
+ *    for mamba2_conv_ssd_prefill, before the size check.
  *  - All calls share the one array: calls that may overlap on the GPU (other
  *    streams, other host threads using the same device) race on it and must
  *    be serialised by the caller.  No part of the array needs to start at
@@ -206,9 +221,10 @@ MAMBA2_API int mamba2_conv_ssd_prefill_noalloc(const mamba2_dims *dims,
                                                void *stream);
 
 /* Profiling aid (no counterpart on the pages).  Arms the calling host thread
- * so that its NEXT call of mamba2_conv_ssd_prefill or mamba2_ssd_step records
- * events[i] (cudaEvent_t passed as void*, created by the caller) on the
- * call's stream just before the call's kernel stage i, and events[S] after
+ * so that its NEXT call of mamba2_conv_ssd_prefill,
+ * mamba2_conv_ssd_prefill_noalloc or mamba2_ssd_step records events[i]
+ * (cudaEvent_t passed as void*, created by the caller) on the call's stream
+ * just before the call's kernel stage i, and events[S] after
  * its last stage, S being the stage count that mamba2_stage_names reports.
  * Entries beyond n_events, and NULL entries, are not recorded, so a caller
  * can bracket a single stage.  The call disarms the thread when it returns,

@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
                                                       vp, i32, vp]
         L.mamba2_device_errors.restype = ctypes.c_int
         L.mamba2_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        L.mamba2_debug_stall_waits.restype = ctypes.c_int
+        L.mamba2_debug_stall_waits.argtypes = [ctypes.c_int]
         L.mamba2_ssd_step.restype = ctypes.c_int
         L.mamba2_ssd_step.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp, vp]
         _lib = L
@@ -92,6 +94,15 @@ def device_errors() -> int:
     if st != 0:
         raise Mamba2Error(st, "mamba2_device_errors")
     return int(f.value)
+
+
+def debug_stall_waits(enable: bool) -> None:
+    """Test aid: while enabled, every waiting kernel's first wait runs out (20 ms)
+    and the kernel returns without doing its work, raising the flag that
+    device_errors() reports (bit 0).  Synchronises the current device."""
+    st = lib().mamba2_debug_stall_waits(int(bool(enable)))
+    if st != 0:
+        raise Mamba2Error(st, "mamba2_debug_stall_waits")
 
 
 def status_string(status: int) -> str:

@@ -1,7 +1,10 @@
 // C ABI of libmamba2ssd.so: argument validation and launch.  See
 // include/mamba2ssd.h for the contract of every entry point.
+#include <cuda.h>
+
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -69,6 +72,53 @@ struct DisarmOnExit {
 
 thread_local StageEvents g_stage_events = {{}, 0};
 
+// Driver entry points fetched through the runtime, so that the library has no
+// load-time dependency on libcuda (it loads, and its host logic is testable,
+// on a machine without a driver).
+template <typename F>
+F driver_fn(const char *name) {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return reinterpret_cast<F>(p);
+}
+
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext *);
+  using GetId = CUresult (*)(CUcontext, unsigned long long *);
+  static const GetCurrent get_current = driver_fn<GetCurrent>("cuCtxGetCurrent");
+  static const GetId get_id = driver_fn<GetId>("cuCtxGetId");
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+bool first_use_in_context(int slot) {
+  static std::mutex mu;
+  static unsigned long long seen[64][16] = {};
+  int dev = 0;
+  if (slot < 0 || slot >= 16 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return true;
+  const unsigned long long id = current_context_id();
+  if (id == 0) return true;
+  std::lock_guard<std::mutex> lock(mu);
+  if (seen[dev][slot] == id) return false;
+  seen[dev][slot] = id;
+  return true;
+}
+
+int validate_prefill_dims(const mamba2_dims *dims) {
+  Problem pr;
+  return make_problem(dims, true, &pr);
+}
+
 }  // namespace m2
 
 using namespace m2;
@@ -105,6 +155,15 @@ MAMBA2_API int mamba2_device_errors(unsigned int *flags) {
   *flags |= f;
   if (take_prefill_tc_errors(&f) != cudaSuccess) return MAMBA2_ERR_CUDA;
   *flags |= f;
+  return MAMBA2_OK;
+}
+
+MAMBA2_API int mamba2_debug_stall_waits(int enable) {
+  if (enable != 0 && enable != 1) return MAMBA2_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MAMBA2_ERR_CUDA;
+  if (set_step_stall((unsigned)enable) != cudaSuccess ||
+      set_prefill_tc_stall((unsigned)enable) != cudaSuccess)
+    return MAMBA2_ERR_CUDA;
   return MAMBA2_OK;
 }
 

@@ -116,6 +116,10 @@ extern const char *const kStepSimtStages[];
 extern const int kStepSimtStageCount;
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// MAMBA2_OK if `dims` describe a valid prefill problem, else the status the
+// prefill entry point would return for them.
+int validate_prefill_dims(const mamba2_dims *dims);
+
 // Launchers (one per translation unit).
 cudaError_t prefill_simt(const PrefillArgs &a);
 size_t prefill_simt_workspace(const Problem &pr);
@@ -194,9 +198,53 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   return true;
 }
 
+// Waits for phase `parity` of `bar` for at most `limit_ns`; returns false (and
+// raises the device error flag) if it never completed.
+__device__ __forceinline__ bool mbar_wait_bounded_ns(uint64_t *bar, uint32_t parity,
+                                                     unsigned int *err,
+                                                     unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(err, kErrWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Test aid behind mamba2_debug_stall_waits: when the translation unit's stall
+// word is set, thread 0 of every CTA waits on a barrier that nothing completes
+// until the (short) limit runs out, which raises kErrWaitTimeout exactly as a
+// timed-out wait in the kernel's main loop does; the caller then returns before
+// it has issued any asynchronous copy, MMA or cluster access, so nothing is in
+// flight.  Every CTA of a launch reads the same word, so a cluster's CTAs all
+// return together.
+constexpr unsigned long long kTestStallNs = 20000000ull;  // 20 ms
+__device__ __forceinline__ bool test_stall(const unsigned int *stall, unsigned int *err) {
+  if (*reinterpret_cast<const volatile unsigned int *>(stall) == 0u) return false;
+  __shared__ uint64_t dead;
+  if (threadIdx.x == 0) {
+    mbar_init(&dead, 1);
+    mbar_wait_bounded_ns(&dead, 0, err, kTestStallNs);
+  }
+  return true;
+}
+
 // Host: read and clear the error words of the kernels that wait (one per
 // translation unit).  Synchronous.
 cudaError_t take_step_errors(unsigned int *out);
+// Host: set the stall word of every translation unit whose kernels wait.
+cudaError_t set_step_stall(unsigned int v);
+cudaError_t set_prefill_tc_stall(unsigned int v);
+
+// Host: true exactly once per CUDA context for each `slot` (0 .. 15): launch
+// attributes (cudaFuncSetAttribute) belong to a context and are set again
+// when the context is re-created.
+bool first_use_in_context(int slot);
+// Host: unique id of the calling thread's current CUDA context (0 if none).
+unsigned long long current_context_id();
 
 }  // namespace m2
 

@@ -10,12 +10,14 @@
 //
 // The array is MAMBA2_STATIC_SCRATCH_BYTES large and lives in every GPU that
 // loads this library until the process exits.  Host code cannot use the
-// array's name as a device address, so its address is looked up once per
-// device (with that device current) and cached.  Every call shares the array:
-// calls that overlap on the GPU (different streams, or different host threads
-// on the same device) race on it.  The prefill writes each part of its
-// scratch before reading it, so stale contents from an earlier call do no
-// harm and nothing needs clearing.
+// array's name as a device address, so its address is looked up with the
+// device current and cached per CUDA context: a context that is destroyed and
+// re-created (cudaDeviceReset, or the primary context released and retained
+// again) reloads this module, the array may move, and the new context's id
+// forces a fresh lookup.  Every call shares the array: calls that overlap on
+// the GPU (different streams, or different host threads on the same device)
+// race on it.  The prefill writes each part of its scratch before reading it,
+// so stale contents from an earlier call do no harm and nothing needs clearing.
 #include <mutex>
 
 #include "common.cuh"
@@ -26,23 +28,30 @@ namespace {
 static __device__ __align__(256) unsigned char g_static_scratch[MAMBA2_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
+struct ScratchEntry {
+  unsigned long long ctx_id;  // 0: not looked up
+  void *addr;
+};
 std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device (set up on first use).
+// Device address of g_static_scratch in the current device's context.
 cudaError_t static_scratch_address(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  const unsigned long long id = current_context_id();
+  ScratchEntry &c = g_scratch[dev];
+  if (id == 0 || c.ctx_id != id || c.addr == nullptr) {
     void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    e = cudaGetSymbolAddress(&p, g_static_scratch);  // makes the primary context current
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    c.addr = p;
+    c.ctx_id = current_context_id();
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return cudaSuccess;
 }
 
@@ -54,8 +63,11 @@ extern "C" MAMBA2_API int mamba2_conv_ssd_prefill_noalloc(
     int64_t xBC_row_stride, const void *z, int64_t z_row_stride, const void *dt_raw,
     int64_t dt_row_stride, void *y, void *conv_state, float *ssm_state, int32_t states_in,
     void *stream) {
-  // Sizes are validated by the ordinary entry point below; only the scratch
-  // limit is checked here.
+  struct Disarm {  // stage events are disarmed on every return, as for the other entries
+    ~Disarm() { m2::g_stage_events.n = 0; }
+  } disarm;
+  const int st = m2::validate_prefill_dims(dims);
+  if (st != MAMBA2_OK) return st;
   if (mamba2_prefill_workspace_size(dims) > (size_t)MAMBA2_STATIC_SCRATCH_BYTES)
     return MAMBA2_ERR_WORKSPACE;
   void *scratch = nullptr;

@@ -50,6 +50,7 @@ constexpr uint32_t kTmemT = 128 + 64 * kMaxHeadsPerCta;  // column of the C H_c^
 constexpr float kLog2e = 1.4426950408889634f;
 
 static __device__ unsigned int g_tc_errors = 0;
+static __device__ unsigned int g_tc_stall = 0;  // mamba2_debug_stall_waits
 
 struct TcArgs {
   Problem pr;
@@ -306,6 +307,7 @@ __device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs,
 
 __global__ void __launch_bounds__(kK1Threads, 1)
     tc_chunk_state_kernel(TcArgs a, const __grid_constant__ K1Maps maps, int n_items) {
+  if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA alike (test aid)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ float ws[2][2][kQ];          // [stage][head of pair][token] chunk weights
   __shared__ float4 wts[2][3][64];        // [stage][slot][channel] conv taps
@@ -847,6 +849,7 @@ __device__ __forceinline__ void out_unit(const Problem &pr, int nch, int ncl, in
 
 __global__ void __launch_bounds__(kWsThreads, 1)
     tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps, int ncl) {
+  if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA of every cluster alike
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   int cs, rank;
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs));
@@ -1461,6 +1464,10 @@ size_t prefill_tc_workspace(const Problem &pr) {
          align_up((size_t)pr.batch * pr.L * pr.conv_dim * 2, 256);
 }
 
+cudaError_t set_prefill_tc_stall(unsigned int v) {
+  return cudaMemcpyToSymbol(g_tc_stall, &v, sizeof(v));
+}
+
 cudaError_t take_prefill_tc_errors(unsigned int *out) {
   unsigned int v = 0, zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(&v, g_tc_errors, sizeof(v));
@@ -1495,14 +1502,17 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.u = w.u;
   const int hpg = pr.heads_per_group();
   cudaError_t e;
-  e = cudaFuncSetAttribute(tc_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kK1Smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kK3Smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e != cudaSuccess) return e;
+  if (first_use_in_context(0)) {  // attributes belong to the context: set them once in each
+    e = cudaFuncSetAttribute(tc_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kK1Smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kK3Smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1);
+    if (e != cudaSuccess) return e;
+  }
   int cs = 1, hpc = 1, ncl = 1;
   out_choose(hpg, pr.batch * a.nch * (int64_t)pr.G, &cs, &hpc, &ncl);
   a.hpc = hpc;

@@ -29,6 +29,8 @@
 // before step 5 so that no rank can overwrite a table this CTA still reads.
 #include <algorithm>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace m2 {
@@ -40,6 +42,7 @@ constexpr int kMaxStages = 4;  // shared-memory ring of per-head state buffers (
 constexpr uint32_t kStepSmemPerCta = 112 * 1024;  // two CTAs per SM
 
 static __device__ unsigned int g_step_errors = 0;
+static __device__ unsigned int g_step_stall = 0;  // mamba2_debug_stall_waits
 
 // silu with the fast exponential and reciprocal (relative error ~1e-6)
 __device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
@@ -163,6 +166,7 @@ __global__ void __launch_bounds__(kStepBlock, 2)
                     const T *__restrict__ z, int64_t ld_z, const T *__restrict__ dt_raw,
                     int64_t ld_dt, T *__restrict__ y, T *__restrict__ conv_state,
                     float *__restrict__ ssm, int hpc, int stages, int nclusters) {
+  if (test_stall(&g_step_stall, &g_step_errors)) return;  // every CTA alike (test aid)
   int cs, rank;
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs));
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
@@ -478,13 +482,36 @@ cudaError_t run(const StepArgs &a) {
   if ((size_t)stages * head_bytes > 65536) stages = 2;
   const size_t smem = step_layout<T>(stages, hpc, pr.P, pr.G, pr.N, cs).total;
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(ssd_step_kernel<T, N>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // The shared-memory attribute (per context) and the occupancy answer (per
+  // device, shared-memory size and cluster size) are kept from the previous
+  // call with the same key, so a decode loop pays for neither on every step.
+  struct LaunchCache {
+    unsigned long long ctx;
+    size_t smem;
+    int cs, max_clusters;
+  };
+  static std::mutex mu;
+  static LaunchCache cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (cs > 8) {
-    e = cudaFuncSetAttribute(ssd_step_kernel<T, N>, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                             1);
+  const unsigned long long ctx = current_context_id();
+  LaunchCache hit = {};
+  const bool cacheable = dev >= 0 && dev < 64 && ctx != 0;
+  if (cacheable) {
+    std::lock_guard<std::mutex> lock(mu);
+    hit = cache[dev];
+  }
+  const bool fresh = !(cacheable && hit.ctx == ctx && hit.smem == smem && hit.cs == cs);
+  if (fresh) {
+    e = cudaFuncSetAttribute(ssd_step_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
     if (e != cudaSuccess) return e;
+    if (cs > 8) {
+      e = cudaFuncSetAttribute(ssd_step_kernel<T, N>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kStepBlock, 1, 1);
@@ -499,12 +526,19 @@ cudaError_t run(const StepArgs &a) {
   cfg.numAttrs = 1;
   // as many clusters as fit on the device at once, each looping over rows
   cfg.gridDim = dim3((unsigned)cs, 1, 1);
-  int max_clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&max_clusters, ssd_step_kernel<T, N>, &cfg) != cudaSuccess ||
-      max_clusters <= 0) {
-    cudaGetLastError();  // clear a failed query; fall back to one cluster per row
-    max_clusters = (int)std::min<int64_t>(pr.batch, 65535);
+  int max_clusters = fresh ? 0 : hit.max_clusters;
+  if (fresh) {
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, ssd_step_kernel<T, N>, &cfg) !=
+            cudaSuccess ||
+        max_clusters <= 0) {
+      cudaGetLastError();  // clear a failed query; fall back to one cluster per row
+      max_clusters = 0;
+    } else if (cacheable) {
+      std::lock_guard<std::mutex> lock(mu);
+      cache[dev] = LaunchCache{ctx, smem, cs, max_clusters};
+    }
   }
+  if (max_clusters <= 0) max_clusters = (int)std::min<int64_t>(pr.batch, 65535);
   // the fewest clusters that keep the largest per-cluster row count: no cluster idles
   // at the end while others still have a row left
   const int64_t fit = std::max<int64_t>(1, std::min<int64_t>(pr.batch, max_clusters));
@@ -532,6 +566,10 @@ cudaError_t take_step_errors(unsigned int *out) {
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_step_errors, &zero, sizeof(zero));
   *out = v;
   return e;
+}
+
+cudaError_t set_step_stall(unsigned int v) {
+  return cudaMemcpyToSymbol(g_step_stall, &v, sizeof(v));
 }
 
 template <typename T>

@@ -158,3 +158,20 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(m2, "library_path", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         m2.lib()
+
+
+def test_debug_stall_rejects_bad_values():
+    # validated before any CUDA call, so this runs without a GPU
+    assert m2.lib().mamba2_debug_stall_waits(2) == INVALID
+    assert m2.lib().mamba2_debug_stall_waits(-1) == INVALID
+
+
+def test_noalloc_rejects_bad_dims_before_touching_the_device():
+    lib = m2.lib()
+    p = _fake_params()
+    for kw, expect in [(dict(nheads=6, ngroups=4), INVALID), (dict(d_conv=2), UNSUPPORTED),
+                       (dict(seqlen=-1), INVALID)]:
+        d = _dims(**kw)
+        st = lib.mamba2_conv_ssd_prefill_noalloc(ctypes.byref(d), ctypes.byref(p), A0, 5248,
+                                                 A0, 5120, A0, 80, A0, None, None, 0, None)
+        assert st == expect, kw

@@ -37,6 +37,53 @@ def test_full_size_prefill(name):
     print(name, rep, f"oracle {time.time() - t:.1f}s")
 
 
+@pytest.mark.parametrize("L1", [2048, 1000])
+def test_full_size_chunked_prefill_continuation(L1):
+    # the 2.7B workload split into two prefills (the second continuing from the
+    # first's conv and SSM states) equals the whole prefill (the cache test of
+    # chunked prefill); compared with the oracle's whole-sequence result
+    cfg = W.CONFIGS["zamba2_2p7b_prefill"]
+    params = W.make_params(cfg, 1)
+    inp = W.make_prefill_inputs(cfg, 1)
+    st = W.make_states(cfg, 1)
+    ref = oracle_prefill(cfg, inp, params, states=st)
+    a = gpu_prefill(cfg.with_(seqlen=L1), {"zxbcdt": inp["zxbcdt"][:, :L1].contiguous()},
+                    params, states={k: v.clone() for k, v in st.items()}, states_in=True)
+    b = gpu_prefill(cfg.with_(seqlen=cfg.seqlen - L1),
+                    {"zxbcdt": inp["zxbcdt"][:, L1:].contiguous()}, params,
+                    states={"conv_state": a["conv_state"], "ssm_state": a["ssm_state"]},
+                    states_in=True)
+    got = {"y": torch.cat([a["y"], b["y"]], dim=1), "conv_state": b["conv_state"],
+           "ssm_state": b["ssm_state"]}
+    print(L1, compare_prefill(cfg, got, ref))
+    assert m2.device_errors() == 0
+
+
+def test_full_size_prefill_then_decode_steps():
+    # prefill of the first 4096 - 8 tokens, then 8 single-token decode steps, equals
+    # the whole prefill (the cached-decode test)
+    cfg = W.CONFIGS["zamba2_2p7b_prefill"]
+    k = 8
+    params = W.make_params(cfg, 2)
+    inp = W.make_prefill_inputs(cfg, 2)
+    ref = oracle_prefill(cfg, inp, params)
+    a = gpu_prefill(cfg.with_(seqlen=cfg.seqlen - k),
+                    {"zxbcdt": inp["zxbcdt"][:, :-k].contiguous()}, params)
+    dims = m2.dims_from_config(cfg)
+    pt, pp = dev_params(params)
+    cs = a["conv_state"].cuda().contiguous()
+    hs = a["ssm_state"].cuda().contiguous()
+    ys = []
+    for t in range(cfg.seqlen - k, cfg.seqlen):
+        v = W.split_packed(cfg, inp["zxbcdt"][:, t].contiguous().cuda())
+        ys.append(m2.step(dims, pp, v["xBC"], v["z"], v["dt_raw"], cs, hs).cpu())
+    torch.cuda.synchronize()
+    got = {"y": torch.cat([a["y"], torch.stack(ys, dim=1)], dim=1), "conv_state": cs.cpu(),
+           "ssm_state": hs.cpu()}
+    print(compare_prefill(cfg, got, ref))
+    assert m2.device_errors() == 0
+
+
 def test_full_size_decode_1024_steps():
     cfg = W.CONFIGS["zamba2_2p7b_decode"]
     seed = 0

@@ -15,7 +15,7 @@ import torch
 import mamba_ssd_scan_mixer_b200 as m2
 from mamba_ssd_scan_mixer_b200 import workloads as W
 
-from harness import case, check_bf16_out, check_f32, check_rms, dev_params
+from harness import case, dev_params
 
 pytestmark = pytest.mark.gpu
 
@@ -49,16 +49,17 @@ def _outputs(cfg, seed, noalloc):
 ], ids=lambda c: c.name)
 def test_noalloc_prefill_matches_workspace_prefill_twice(cfg):
     assert m2.mamba2_prefill_workspace_size(m2.dims_from_config(cfg)) <= 64 * 1024 * 1024
+    # a larger call of another shape first, so that the scratch holds differently
+    # laid-out leftovers when the checked calls run
+    other = cfg.with_(batch=3, seqlen=1500, nheads=cfg.nheads * 2, ngroups=1)
+    assert m2.mamba2_prefill_workspace_size(m2.dims_from_config(other)) <= 64 * 1024 * 1024
+    _outputs(other, 10, noalloc=True)
     for seed in (11, 12):  # two calls in a row, different inputs
         ref = _outputs(cfg, seed, noalloc=False)
         got = _outputs(cfg, seed, noalloc=True)
-        if cfg.io_dtype == "f32":
-            check_f32(got["y"], ref["y"], "y")
-            check_f32(got["ssm_state"], ref["ssm_state"], "ssm_state")
-        else:
-            check_bf16_out(got["y"], ref["y"].double().numpy(), "y")
-            check_rms(got["ssm_state"], ref["ssm_state"], "ssm_state")
-        assert torch.equal(got["conv_state"], ref["conv_state"])
+        # same kernels, same launch configuration, no atomics: bitwise identical
+        for k in ("y", "conv_state", "ssm_state"):
+            assert torch.equal(got[k], ref[k]), k
 
 
 def test_noalloc_prefill_rejects_problems_beyond_the_static_scratch():
