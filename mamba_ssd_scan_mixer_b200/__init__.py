@@ -26,7 +26,9 @@ __all__ = [
 
 MAMBA2_F32, MAMBA2_BF16 = 0, 1
 _PKG = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_PKG, "libmamba2ssd.so")
+# MAMBA2SSD_LIBRARY selects another build of the library, e.g. the bounds-checked
+# libmamba2ssd_checked.so (see build.py)
+library_path = os.environ.get("MAMBA2SSD_LIBRARY") or os.path.join(_PKG, "libmamba2ssd.so")
 
 
 class Mamba2Dims(ctypes.Structure):

@@ -232,6 +232,40 @@ __device__ __forceinline__ bool test_stall(const unsigned int *stall, unsigned i
   return true;
 }
 
+// ---------------------------------------------------------------- checked build
+// Built with -DMAMBA2_BOUNDS_CHECK (libmamba2ssd_checked.so, a debugging aid in
+// place of a memory checker), every plain global load and store of the
+// tensor-core prefill kernels and of the decode kernel is checked against the
+// byte range of the buffer it addresses and against the alignment of its
+// access size; an access that fails is skipped and raises kErrBounds in the
+// kernel's error word (mamba2_device_errors bit 1).  Tensor-memory copies
+// (TMA) are bounded by their tensor maps and need no check.  In the ordinary
+// build the checks compile to nothing.
+constexpr unsigned int kErrBounds = 2u;
+struct Span {  // [lo, hi) byte addresses of one device buffer (lo == hi: none)
+  unsigned long long lo, hi;
+};
+inline Span span_of(const void *p, size_t bytes) {
+  const unsigned long long a = reinterpret_cast<unsigned long long>(p);
+  return Span{a, p == nullptr ? a : a + bytes};
+}
+#ifdef MAMBA2_BOUNDS_CHECK
+__device__ __forceinline__ bool span_ok(const void *p, unsigned int bytes, unsigned int align,
+                                        const Span &s, unsigned int *err) {
+  const unsigned long long a = reinterpret_cast<unsigned long long>(p);
+  if (a >= s.lo && a + bytes <= s.hi && (a & (unsigned long long)(align - 1)) == 0) return true;
+  atomicOr(err, kErrBounds);
+  return false;
+}
+// an access of `bytes` (1, 2, 4, 8 or 16) at p, aligned to its size
+#define M2_OK(p, bytes, span, err) ::m2::span_ok((p), (bytes), (bytes), (span), (err))
+// a bulk copy of `bytes` at p (16-byte aligned)
+#define M2_OK_BULK(p, bytes, span, err) ::m2::span_ok((p), (bytes), 16u, (span), (err))
+#else
+#define M2_OK(p, bytes, span, err) true
+#define M2_OK_BULK(p, bytes, span, err) true
+#endif
+
 // Host: read and clear the error words of the kernels that wait (one per
 // translation unit).  Synchronous.
 cudaError_t take_step_errors(unsigned int *out);

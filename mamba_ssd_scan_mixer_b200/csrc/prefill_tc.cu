@@ -32,6 +32,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstddef>
 
 #include "common.cuh"
 
@@ -70,9 +71,17 @@ struct TcArgs {
   float *cum_end;                // [b][nch][H] chunk sum of dt*A
   float *cum;                    // [b][nch][H][128] running sum of dt*A inside the chunk
   float *dtv;                    // [b][nch][H][128] dt (0 past the end of the sequence)
-  __half *Hc;                    // [b][nch][H][n 64][p 64] state entering each chunk
+  __half *Hc;                    // [b][nch][H][p 64][n 64] state entering each chunk, scaled
+  float *hsc;                    // [b][nch][H][32] 2^s: H_c rows p = 2i, 2i + 1 hold H / 2^s
+  float *cbd;                    // [b][G][nch * 128] C_t . B_t in fp32 (the decay operand's diagonal)
+  // byte ranges of every buffer, for the checked build (see M2_OK)
+  struct Spans {
+    Span xbc, z, dt, y, conv, ssm, S, cum_end, cum, dtv, Hc, hsc, cbd, u, conv_w, conv_b, dt_bias,
+        A, D, norm_w;
+  } sp;
   __half *u;                     // [b][L][conv_dim] post-conv x | B | C, fp16
   int hpc;                       // max heads per CTA in tc_chunk_out
+  int y32;                       // y is 32-byte aligned: rows are written in whole 32-byte sectors
 };
 
 // silu(v) = v * sigmoid(v) with sigmoid(v) = (1 + tanh(v / 2)) / 2, using the
@@ -115,7 +124,8 @@ __device__ __forceinline__ void store_u(const TcArgs &a, int64_t bi, int64_t t0,
       o.y = pack_half2(v[k][2], v[k][3]);
       o.z = pack_half2(v[k][4], v[k][5]);
       o.w = pack_half2(v[k][6], v[k][7]);
-      *reinterpret_cast<uint4 *>(a.u + (bi * a.pr.L + t) * a.pr.conv_dim + ch) = o;
+      uint4 *dst = reinterpret_cast<uint4 *>(a.u + (bi * a.pr.L + t) * a.pr.conv_dim + ch);
+      if (M2_OK(dst, 16, a.sp.u, &g_tc_errors)) *dst = o;
     }
   }
 }
@@ -154,27 +164,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int c0, int c1,
-                                             int c2) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream drains;
+// grid_dependency_wait blocks until that kernel has completed and its memory
+// operations are visible.  launch_dependents lets the next kernel's CTAs be
+// scheduled once every CTA of this one has called it (or exited).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
-// Bulk-store groups: commit the stores issued so far; wait until at most one /
-// none of the committed groups still reads shared memory.
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// (the group count of wait_group is an immediate: the cases used are spelled out)
-__device__ __forceinline__ void bulk_wait_read_le(int n) {
-  if (n >= 4) asm volatile("cp.async.bulk.wait_group.read 4;" ::: "memory");
-  else if (n == 3) asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
-  else if (n == 2) asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
-  else if (n == 1) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-  else asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -184,23 +183,6 @@ __device__ __forceinline__ void cluster_arrive_release() {
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// barrier over the 512 compute threads only (the producer warp never joins)
-__device__ __forceinline__ void compute_sync() {
-  asm volatile("bar.sync 1, 512;" ::: "memory");
-}
-__device__ __forceinline__ bool compute_all(bool v) {
-  int r;
-  asm volatile("{\n .reg .pred p, q;\n setp.ne.s32 p, %1, 0;\n bar.red.and.pred q, 1, 512, p;\n"
-               " selp.s32 %0, 1, 0, q;\n}"
-               : "=r"(r)
-               : "r"((int)v)
-               : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ bool wait_compute(uint64_t *bar, uint32_t parity, bool ok) {
-  const bool got = ok ? mbar_wait_bounded(bar, parity, &g_tc_errors) : false;
-  return compute_all(got);
 }
 // Smem descriptor for an MN-major SW128 operand: 8-row (K) atoms of 64
 // elements (N) x 128 B, K atoms 1024 B apart (SBO), N atoms `lbo` apart.
@@ -216,25 +198,32 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t 
 // ============================================================== chunk states
 // Persistent: grid = one CTA per SM; CTA k takes a contiguous range of work
 // items ordered (row, chunk, group, item), where the items of a (row, chunk,
-// group) are its head pairs followed by one C item:
-//   pair item: conv + SiLU of x (2 heads) and of B (only when the CTA's previous
-//     item had another (row, chunk, group): B's operands stay in shared memory),
-//     post-conv values to u, then S = (x o w)^T B on the tensor cores;
-//   C item: conv + SiLU of the group's C channels -> u.
+// group) key are its head pairs followed by one C item:
+//   pair item: conv + SiLU of x (2 heads) and, for the first pair item of a key
+//     in the CTA ("fresh"), of B; post-conv values to u (fp16); then
+//     S = (x o w)^T B on the tensor cores (w_s = exp(cum_end - cum_s) dt_s);
+//   C item: conv + SiLU of the key's C channels -> u.
 // 16 compute warps + 2 producer warps + 1 MMA-issuer warp.  The producer of an
-// item (one per ring stage, so they alternate) TMA-loads its raw bf16 tiles
-// [136 tokens c0-3 .. c0+132][64 ch] (128-byte swizzle) into its stage,
-// computes its dt weights (stored also as per-token dt and cumsum rows for the
-// output kernel) and stages its conv taps while the compute warps work on the
-// previous item; the MMA warp
-// issues a pair item's products once its operands are in shared memory, and
-// they run under the next item's convolution.
-// Smem (1024-aligned): ring [2][x_A | x_B | B (a C item uses slot 0)], then the
-// operands A_hi, A_lo [2 k-blocks][128 rows][128 B] and B_hi, B_lo [2][64][128 B].
+// item (one per x-ring stage; they alternate) computes its dt weights (and the
+// per-token dt and cumsum rows the output kernel reads), stages its conv taps
+// and TMA-loads its raw bf16 tiles [136 tokens c0-3 .. c0+132][64 ch] (128-byte
+// swizzle, rows before the sequence read as zeros): the x tiles into the
+// item's ring stage, the B or C tile into the key's B/C buffer (two, by key
+// parity, so the next key's B arrives while this key is being worked on).
+// The compute warps keep a pair item's convolved tile in registers until the
+// previous pair item's MMA (the reader of the single operand buffer) has
+// completed, write the fp16 hi/lo operands, release them to the MMA warp, and
+// then store the previous item's chunk states from its TMEM accumulator (two
+// accumulators alternate) while the current item multiplies.  No CTA-wide
+// barrier is taken per item: every hand-over is an mbarrier.
+// Smem (1024-aligned): x ring [2 stages][2 slots] raw tiles, B/C raw [2], then
+// the operands A_hi, A_lo [2 k-blocks][128 rows][128 B] and B_hi, B_lo
+// [2][64][128 B].
 constexpr uint32_t kRawRows = 136, kRawBytes = kRawRows * 128;  // 17 KB, 1024-multiple
-constexpr uint32_t kK1Stage = 3 * kRawBytes;
+constexpr uint32_t kK1Stage = 2 * kRawBytes;
+constexpr uint32_t kK1BC = 2 * kK1Stage;                      // B/C raw buffers [2]
 constexpr uint32_t kK1A = 2 * 128 * 128, kK1B = 2 * 64 * 128;
-constexpr uint32_t kK1Ahi = 2 * kK1Stage, kK1Alo = kK1Ahi + kK1A, kK1Bhi = kK1Alo + kK1A,
+constexpr uint32_t kK1Ahi = kK1BC + 2 * kRawBytes, kK1Alo = kK1Ahi + kK1A, kK1Bhi = kK1Alo + kK1A,
                    kK1Blo = kK1Bhi + kK1B, kK1Tiles = kK1Blo + kK1B;
 
 struct K1Maps {
@@ -281,9 +270,44 @@ __device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, cons
     }
 }
 
+// As conv8x4_smem for the same 8 channels x 4 tokens, but each output is folded
+// at once into d4[k] += out[k][i] * v[k][i] (the dot product over the 8 channels
+// of token k) and the taps and rows are read per token, so that only `v` stays
+// live across the call.
+__device__ __forceinline__ void conv8x4_dot(uint32_t tile, int s0, int cg, const float4 *wt,
+                                            const float *bs, const float (&v)[4][8],
+                                            float (&d4)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float rows[4][8];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int R = s0 + k + r;
+      const uint4 raw = ld_shared_v4(tile + R * 128 + (((cg ^ R) & 7) << 4));
+      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h2[i]);
+        rows[r][2 * i] = f.x;
+        rows[r][2 * i + 1] = f.y;
+      }
+    }
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 wv = wt[i * 8 + cg];
+      const float h = bs[i * 8 + cg] + wv.x * rows[0][i] + wv.y * rows[1][i] + wv.z * rows[2][i] +
+                      wv.w * rows[3][i];
+      acc = fmaf(v[k][i], fmaf(h, tanh_approx(h), h), acc);
+    }
+    d4[k] = acc;
+  }
+}
+
 struct K1Item {
   int64_t bi;
   int c, g, pair;
+  unsigned key;  // (row, chunk, group) index
   bool isC;
   bool freshB;  // B must be convolved (the CTA's previous item had another key)
 };
@@ -296,6 +320,7 @@ __device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs,
   const int r = it - (int)key * (pairs + 1);
   const unsigned bc = key / (unsigned)pr.G;
   K1Item w;
+  w.key = key;
   w.g = (int)(key - bc * (unsigned)pr.G);
   w.bi = (int64_t)(bc / (unsigned)nch);
   w.c = (int)(bc - (unsigned)w.bi * (unsigned)nch);
@@ -309,10 +334,12 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     tc_chunk_state_kernel(TcArgs a, const __grid_constant__ K1Maps maps, int n_items) {
   if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA alike (test aid)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ float ws[2][2][kQ];          // [stage][head of pair][token] chunk weights
-  __shared__ float4 wts[2][3][64];        // [stage][slot][channel] conv taps
-  __shared__ float bss[2][3][64];         // [stage][slot][channel] conv bias
-  __shared__ uint64_t full[2], empty[2], ops_ready, mbar;
+  __shared__ __align__(16) float ws[2][2][kQ];    // [stage][head of pair][token] chunk weights (read as float4)
+  __shared__ float4 wts[2][3][64];                // [stage][slot x_A, x_B, B/C][channel] conv taps
+  __shared__ __align__(16) float bss[2][3][64];   // [stage][slot][channel] conv bias
+  __shared__ uint64_t full[2], empty[2], bc_empty[2], ops_ready, mma_done[2], tmem_free[2],
+      mma_final, halo_bar[2], cbd_bar;
+  __shared__ __align__(16) float cbd_s[2][kQ];  // C-item parity: per-token partials of channel groups 4-7
   __shared__ uint32_t tmem_holder;
   const Problem &pr = a.pr;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -324,14 +351,19 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   const int it0 = (int)((int64_t)n_items * blockIdx.x / gridDim.x),
             it1 = (int)((int64_t)n_items * (blockIdx.x + 1) / gridDim.x);
 
-  if (warp == 0) tmem_alloc(&tmem_holder, 64);
+  if (warp == 0) tmem_alloc(&tmem_holder, 128);
   if (tid == 0) {
     for (int k = 0; k < 2; ++k) {
-      mbar_init(&full[k], 2);  // the tiles' transaction bytes + the producer's weights
-      mbar_init(&empty[k], 1);
+      mbar_init(&full[k], 2);          // the tiles' transaction bytes + the producer's weights
+      mbar_init(&empty[k], kThreads);  // every compute thread has read the stage's x tiles
+      mbar_init(&bc_empty[k], 256);    // warps 0-7 have read the B/C tile
+      mbar_init(&mma_done[k], 1);      // tcgen05.commit of a pair item's MMAs
+      mbar_init(&tmem_free[k], kThreads);  // its chunk states read out of TMEM
     }
-    mbar_init(&ops_ready, 1);  // operands of a pair item written (compute thread 0)
-    mbar_init(&mbar, 1);       // its MMAs completed (tcgen05.commit)
+    mbar_init(&ops_ready, kThreads);  // operands of a pair item written
+    mbar_init(&mma_final, 1);
+    for (int k = 0; k < 2; ++k) mbar_init(&halo_bar[k], 1);  // a halo item's tiles landed
+    mbar_init(&cbd_bar, 128);  // warps 4-7 have written a C item's diagonal partials
     fence_mbar_init();
   }
   tc_fence_before();
@@ -341,14 +373,19 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 
   if (warp == kThreads / 32 || warp == kThreads / 32 + 2) {
     // ---------------- producers: warp 16 takes the CTA's even items (ring stage
-    // 0), warp 18 the odd ones (stage 1).
+    // 0), warp 18 the odd ones (stage 1).  Both walk every item to count the
+    // uses of the two B/C buffers.
     const int mine = warp == kThreads / 32 ? 0 : 1;
     int k = 0;
-    for (int it = it0; it < it1; ++it, ++k) {
+    int bc_use0 = 0, bc_use1 = 0, halo_use0 = 0, halo_use1 = 0;  // (scalars: no local memory)
+    bool ok = true;
+    for (int it = it0; ok && it < it1; ++it, ++k) {
       const int st = k & 1;
-      if (st != mine) continue;
       const K1Item w = k1_item(pr, a.nch, pairs, it, k);
-      const bool freshB = w.freshB;
+      const bool useBC = w.isC || w.freshB;
+      const int bcb = (int)(w.key & 1u);
+      const int bc_use = !useBC ? 0 : (bcb ? bc_use1++ : bc_use0++);
+      if (st != mine) continue;
       const int64_t c0 = (int64_t)w.c * kQ;
       const int hA = w.g * hpg + 2 * w.pair;
       const bool hasB = 2 * w.pair + 1 < hpg;
@@ -362,29 +399,36 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       bool son[3];
 #pragma unroll
       for (int sl = 0; sl < 3; ++sl) {
-        son[sl] = w.isC ? sl == 0 : (sl == 1 ? hasB : (sl == 2 ? freshB : true));
-        const int64_t ch0 = w.isC ? pr.d_inner + (int64_t)(pr.G + w.g) * kNS
-                                  : (sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS);
+        // a C item convolves the key's C channels (B/C buffer) and its B channels (x slot
+        // 0) to form the fp32 diagonal C_t . B_t
+        son[sl] = w.isC ? sl != 1 : (sl == 1 ? hasB : (sl == 2 ? w.freshB : true));
+        const int64_t ch0 = (w.isC && sl == 0) ? pr.d_inner + (int64_t)w.g * kNS
+                            : sl < 2 ? (int64_t)(hA + sl) * kHP
+                                     : pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           if (son[sl]) {
-            tw[sl][j] = __ldg(reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + lane + 32 * j);
-            tb[sl][j] = __ldg(a.prm.conv_b + ch0 + lane + 32 * j);
+            const float4 *wp = reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + lane + 32 * j;
+            const float *bp = a.prm.conv_b + ch0 + lane + 32 * j;
+            tw[sl][j] = M2_OK(wp, 16, a.sp.conv_w, &g_tc_errors) ? __ldg(wp) : make_float4(0.f, 0.f, 0.f, 0.f);
+            tb[sl][j] = M2_OK(bp, 4, a.sp.conv_b, &g_tc_errors) ? __ldg(bp) : 0.0f;
           }
         }
       }
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const bool hv = !w.isC && (half == 0 || hasB);
-        if (hv) {
+        if (hv && M2_OK(a.prm.dt_bias + hA + half, 4, a.sp.dt_bias, &g_tc_errors) &&
+            M2_OK(a.prm.A + hA + half, 4, a.sp.A, &g_tc_errors)) {
           dtb[half] = __ldg(a.prm.dt_bias + hA + half);
           Ah[half] = __ldg(a.prm.A + hA + half);
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int64_t tt = c0 + 4 * lane + q;
-          dtr[half][q] = (hv && tt < pr.L)
-                             ? __bfloat162float(a.dt_raw[(w.bi * pr.L + tt) * a.ld_dt + hA + half])
+          const __nv_bfloat16 *dp = a.dt_raw + (w.bi * pr.L + tt) * a.ld_dt + hA + half;
+          dtr[half][q] = (hv && tt < pr.L && M2_OK(dp, 2, a.sp.dt, &g_tc_errors))
+                             ? __bfloat162float(*dp)
                              : -INFINITY;
         }
       }
@@ -402,45 +446,89 @@ __global__ void __launch_bounds__(kK1Threads, 1)
           const float tot = a4[0] + a4[1] + a4[2] + a4[3];
           float run = warp_scan(tot, lane) - tot;
           const float cum_end = __shfl_sync(0xffffffffu, run + tot, 31);
+          // decay from token s to the chunk end, sum_{r > s} dt_r A, summed directly
+          // (exclusive suffix sums) rather than as cum_end - cum_s: with strong decays
+          // |cum| is large and that difference would lose the small exponents that matter
+          const float r3 = a4[3], r2 = a4[2] + r3, r1 = a4[1] + r2, r0 = a4[0] + r1;
+          float e = __shfl_down_sync(0xffffffffu, r0, 1);
+          if (lane == 31) e = 0.0f;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float nx = __shfl_down_sync(0xffffffffu, e, o);
+            if (lane + o < 32) e += nx;
+          }
+          const float sfx[4] = {e + r1, e + r2, e + r3, e};
           float cq[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             run += a4[q];
             cq[q] = run;
-            wsv[half][q] = expf(cum_end - run) * dt4[q];
+            wsv[half][q] = expf(sfx[q]) * dt4[q];
           }
           if (hv) {
             const int64_t row = (w.bi * a.nch + w.c) * pr.H + hA + half;
-            reinterpret_cast<float4 *>(a.cum + row * kQ)[lane] = make_float4(cq[0], cq[1], cq[2], cq[3]);
-            reinterpret_cast<float4 *>(a.dtv + row * kQ)[lane] = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
-            if (lane == 0) a.cum_end[row] = cum_end;
+            float4 *cp = reinterpret_cast<float4 *>(a.cum + row * kQ) + lane;
+            float4 *dp = reinterpret_cast<float4 *>(a.dtv + row * kQ) + lane;
+            if (M2_OK(cp, 16, a.sp.cum, &g_tc_errors)) *cp = make_float4(cq[0], cq[1], cq[2], cq[3]);
+            if (M2_OK(dp, 16, a.sp.dtv, &g_tc_errors)) *dp = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
+            if (lane == 0 && M2_OK(a.cum_end + row, 4, a.sp.cum_end, &g_tc_errors))
+              a.cum_end[row] = cum_end;
           }
         }
       }
-      // the stage is free once the compute warps are done with item k - 2
-      if (k >= 2) {
-        bool got = lane == 0 ? mbar_wait_bounded(&empty[st], (uint32_t)(((k >> 1) - 1) & 1),
-                                                 &g_tc_errors)
-                             : true;
-        if (!__all_sync(0xffffffffu, got)) break;
-      }
+      // the stage is free once the compute warps are done with item k - 2, the B/C
+      // buffer once warps 0-7 are done with its previous use
+      bool got = true;
       if (lane == 0) {
-        const uint32_t stage = base + st * kK1Stage;
-        if (w.isC) {
-          mbar_arrive_expect_tx(&full[st], kRawBytes);
-          tma_load_3d(stage, &maps.xbc, (int)(pr.d_inner + (int64_t)(pr.G + w.g) * kNS),
-                      (int)c0 - 3, (int)w.bi, &full[st]);
-        } else {
-          mbar_arrive_expect_tx(&full[st],
-                                (1u + (hasB ? 1u : 0u) + (freshB ? 1u : 0u)) * kRawBytes);
-          tma_load_3d(stage, &maps.xbc, hA * kHP, (int)c0 - 3, (int)w.bi, &full[st]);
+        if (k >= 2) got = mbar_wait_bounded(&empty[st], (uint32_t)(((k >> 1) - 1) & 1), &g_tc_errors);
+        if (got && useBC && bc_use >= 1)
+          got = mbar_wait_bounded(&bc_empty[bcb], (uint32_t)((bc_use - 1) & 1), &g_tc_errors);
+      }
+      ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      // the first chunk of a sequence that continues from a carried conv state: its
+      // tiles land on a side barrier, then rows 0..2 (tokens -3 .. -1, read as zeros)
+      // are overwritten with that state before the stage is released
+      const bool halo = c0 == 0 && a.states_in;
+      const uint32_t stage = base + st * kK1Stage;
+      const uint32_t bcbuf = base + kK1BC + bcb * kRawBytes;
+      const int64_t bc_ch = pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
+      if (lane == 0) {
+        uint64_t *bar = halo ? &halo_bar[st] : &full[st];
+        const uint32_t nbytes =
+            (w.isC ? 1u : (1u + (hasB ? 1u : 0u))) * kRawBytes + (useBC ? kRawBytes : 0u);
+        mbar_arrive_expect_tx(bar, nbytes);
+        if (w.isC)
+          tma_load_3d(stage, &maps.xbc, (int)(pr.d_inner + (int64_t)w.g * kNS), (int)c0 - 3,
+                      (int)w.bi, bar);
+        if (!w.isC) {
+          tma_load_3d(stage, &maps.xbc, hA * kHP, (int)c0 - 3, (int)w.bi, bar);
           if (hasB)
-            tma_load_3d(stage + kRawBytes, &maps.xbc, (hA + 1) * kHP, (int)c0 - 3, (int)w.bi,
-                        &full[st]);
-          if (freshB)
-            tma_load_3d(stage + 2 * kRawBytes, &maps.xbc, (int)(pr.d_inner + (int64_t)w.g * kNS),
-                        (int)c0 - 3, (int)w.bi, &full[st]);
+            tma_load_3d(stage + kRawBytes, &maps.xbc, (hA + 1) * kHP, (int)c0 - 3, (int)w.bi, bar);
         }
+        if (useBC) tma_load_3d(bcbuf, &maps.xbc, (int)bc_ch, (int)c0 - 3, (int)w.bi, bar);
+      }
+      if (halo) {
+        const int nh_used = st ? halo_use1++ : halo_use0++;
+        bool landed = lane == 0 ? mbar_wait_bounded(&halo_bar[st], (uint32_t)(nh_used & 1), &g_tc_errors)
+                                : true;
+        ok = __shfl_sync(0xffffffffu, landed ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        // slot x_A, x_B (if any) and the B/C tile: 3 rows x 64 channels each
+        for (int idx = lane; idx < 3 * 3 * 64; idx += 32) {
+          const int sl = idx / 192, r = (idx / 64) % 3, chn = idx % 64;
+          if (!son[sl]) continue;
+          const int64_t ch = ((w.isC && sl == 0) ? pr.d_inner + (int64_t)w.g * kNS
+                              : sl < 2 ? (int64_t)(hA + sl) * kHP : bc_ch) + chn;
+          const __nv_bfloat16 *hp = a.conv_in + (w.bi * pr.conv_dim + ch) * 4 + 1 + r;
+          const __nv_bfloat16 v =
+              M2_OK(hp, 2, a.sp.conv, &g_tc_errors) ? *hp : __float2bfloat16(0.0f);
+          const uint32_t tile = sl < 2 ? stage + sl * kRawBytes : bcbuf;
+          const uint32_t addr = tile + r * 128 + ((((chn >> 3) ^ r) & 7) << 4) + ((chn & 7) << 1);
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(v))
+                       : "memory");
+        }
+        if (lane == 0) mbar_arrive(&full[st]);  // stands for the tiles' transaction bytes
       }
       if (!w.isC) {
 #pragma unroll
@@ -463,94 +551,103 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);  // weights of this stage written
     }
+    // no copy may be in flight when the CTA exits: the last stage loads issued
+    if (lane == 0) {
+      for (int kk = max(0, k - 2); kk < k; ++kk)
+        if ((kk & 1) == mine) mbar_wait_bounded(&full[kk & 1], (uint32_t)((kk >> 1) & 1), &g_tc_errors);
+    }
   } else if (warp == kThreads / 32 + 1) {
-    // ---------------- MMA issuer: S = x_hi B_hi + x_hi B_lo + x_lo B_hi per pair item
+    // ---------------- MMA issuer: S = x_hi B_hi + x_hi B_lo + x_lo B_hi per pair item,
+    // into TMEM accumulator np % 2
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(128, 64);
       const uint32_t As[3] = {sAhi, sAhi, sAlo}, Bs[3] = {sBhi, sBlo, sBhi};
-      int n = 0;
+      int np = 0;
       for (int it = it0; it < it1; ++it) {
         if (k1_item(pr, a.nch, pairs, it, 1).isC) continue;
-        if (!mbar_wait_bounded(&ops_ready, (uint32_t)(n & 1), &g_tc_errors)) break;
-        ++n;
+        if (!mbar_wait_bounded(&ops_ready, (uint32_t)(np & 1), &g_tc_errors)) break;
+        if (np >= 2 &&
+            !mbar_wait_bounded(&tmem_free[np & 1], (uint32_t)(((np - 2) >> 1) & 1), &g_tc_errors))
+          break;
         tc_fence_after();
+        const uint32_t acc = tmem + 64 * (np & 1);
         for (int prod = 0; prod < 3; ++prod)
           for (int ks = 0; ks < 8; ++ks) {
             const int blk = ks >> 2, kin = ks & 3;
-            umma_f16(tmem, umma_desc_sw128(As[prod] + blk * 16384 + kin * 32),
+            umma_f16(acc, umma_desc_sw128(As[prod] + blk * 16384 + kin * 32),
                      umma_desc_sw128(Bs[prod] + blk * 8192 + kin * 32), idesc,
                      (prod > 0 || ks > 0) ? 1u : 0u);
           }
-        umma_commit(&mbar);
+        umma_commit(&mma_done[np & 1]);
+        ++np;
       }
+      // no MMA may be in flight when the CTA frees its tensor memory
+      umma_commit(&mma_final);
+      mbar_wait_bounded(&mma_final, 0, &g_tc_errors);
     }
   } else {
     // ---------------- compute warps
     bool ok = true;
-    int k = 0, npair_done = 0;
-    // the pair item whose MMA is in flight: its chunk states are stored from TMEM
-    // (rows m = 32 (warp % 4) + lane, 16 columns per warp / 4; S is kept
-    // [n/4][p][4] per head so that a warp's float4 stores are contiguous)
+    int k = 0, np = 0, nc = 0;  // items, pair items and C items so far
+    // chunk states of pair item q out of TMEM accumulator q % 2: rows m = 32 (warp % 4)
+    // + lane (head half m / 64, lane p = m % 64), 16 columns per warp / 4; S is kept
+    // [n/4][p][4] per head so that a warp's float4 stores are contiguous
     struct Pending {
       int64_t bi;
       int c, hA;
       bool hasB;
     } pw{};
-    bool pending = false;
-    auto store_states = [&](const Pending &q) {
-      tc_fence_after();
+    auto store_states = [&](const Pending &q, int acc) {
       const int m = 32 * (warp & 3) + lane, half = m >> 6, p = m & 63, cb = warp >> 2;
       float sv[16];
-      tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 16 * cb, sv);
+      tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * acc + 16 * cb, sv);
+      tc_fence_before();  // TMEM read before the accumulator takes the next item
+      mbar_arrive(&tmem_free[acc]);
       if (half == 0 || q.hasB) {
         float4 *dst = reinterpret_cast<float4 *>(
             a.S + ((q.bi * a.nch + q.c) * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          dst[(4 * cb + i) * kHP + p] =
-              make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
+          if (M2_OK(dst + (4 * cb + i) * kHP + p, 16, a.sp.S, &g_tc_errors))
+            dst[(4 * cb + i) * kHP + p] =
+                make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
       }
-      tc_fence_before();  // TMEM read before the next MMA is issued
+    };
+    auto wait_mma = [&](int q) {  // pair item q's MMAs completed (operands free, S in TMEM)
+      const bool got = ok && mbar_wait_bounded(&mma_done[q & 1], (uint32_t)((q >> 1) & 1), &g_tc_errors);
+      ok = __all_sync(0xffffffffu, got) != 0;
     };
     for (int it = it0; ok && it < it1; ++it, ++k) {
       const int st = k & 1;
       const uint32_t stage = base + st * kK1Stage;
-      ok = wait_compute(&full[st], (uint32_t)((k >> 1) & 1), ok);
-      if (!ok) break;
       const K1Item w = k1_item(pr, a.nch, pairs, it, k);
-      const bool freshB = w.freshB;
+      const int bcb = (int)(w.key & 1u);
+      {
+        const bool got = mbar_wait_bounded(&full[st], (uint32_t)((k >> 1) & 1), &g_tc_errors);
+        ok = __all_sync(0xffffffffu, got) != 0;
+      }
+      if (!ok) break;
       const int64_t c0 = (int64_t)w.c * kQ;
       const int hA = w.g * hpg + 2 * w.pair;
       const bool hasB = 2 * w.pair + 1 < hpg;
-      // channel of slot s (C items use slot 0 for C)
-      auto slot_ch = [&](int sl) -> int64_t {
-        if (w.isC) return pr.d_inner + (int64_t)(pr.G + w.g) * kNS;
-        return sl < 2 ? (int64_t)(hA + sl) * kHP : pr.d_inner + (int64_t)w.g * kNS;
-      };
-      auto slot_on = [&](int sl) -> bool {
-        return w.isC ? sl == 0 : (sl == 1 ? hasB : (sl == 2 ? freshB : true));
-      };
-      // missing second head: zero rows 64..127 of the x operands
-      auto zero_tile = [&](int cg, int s0) {
-        const int blk = s0 >> 6, kq = s0 & 63;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t off = blk * 16384 + sw128_off(64 + cg * 8 + i, kq);
-          st_shared_v2(sAhi + off, 0u, 0u);
-          st_shared_v2(sAlo + off, 0u, 0u);
-        }
+      const uint32_t bcbuf = base + kK1BC + bcb * kRawBytes;
+      const int64_t bc_ch = pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
+      // warp tile: 4 groups of 8 channels x 8 quads of tokens (lane = group lane % 4,
+      // quad lane / 4); it reads the swizzled raw rows, stores u (64 contiguous bytes
+      // per token) and, with the channel order of odd groups rotated by 4, stores the
+      // swizzled operands without shared-memory bank conflicts
+      const int cg = 4 * ((warp >> 2) & 1) + (lane & 3);
+      const int s0 = 4 * (8 * (warp & 3) + (lane >> 2));
+      // the tile's 4 token weights (x slots; B is not weighted).  Read before the
+      // stage is released: the producer of item k + 2 overwrites ws[st] after that
+      auto tile_weights = [&](int sl) -> float4 {
+        return sl < 2 ? *reinterpret_cast<const float4 *>(&ws[st][sl][s0])
+                      : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
       };
       // operands of one tile: x o w (slots 0, 1) or B (slot 2), split into fp16 hi + lo
-      auto put_operands = [&](int sl, int cg, int s0, const float (&v)[4][8]) {
+      auto put_operands = [&](int sl, const float (&v)[4][8], float4 w4) {
         const int blk = s0 >> 6, kq = s0 & 63;
-        float wk[4] = {1.0f, 1.0f, 1.0f, 1.0f};  // x is weighted per token, B is not
-        if (sl < 2) {
-          const float4 w4 = *reinterpret_cast<const float4 *>(&ws[st][sl][s0]);
-          wk[0] = w4.x;
-          wk[1] = w4.y;
-          wk[2] = w4.z;
-          wk[3] = w4.w;
-        }
+        const float wk[4] = {w4.x, w4.y, w4.z, w4.w};
         const bool rot = (cg & 1) != 0;
         const uint32_t hi_base = sl < 2 ? sAhi + blk * 16384 : sBhi + blk * 8192;
         const uint32_t lo_base = sl < 2 ? sAlo + blk * 16384 : sBlo + blk * 8192;
@@ -570,112 +667,141 @@ __global__ void __launch_bounds__(kK1Threads, 1)
           st_shared_v2(lo_base + off, pack_half2(lq[0], lq[1]), pack_half2(lq[2], lq[3]));
         }
       };
-      const int nslots = w.isC ? 1 : 3;
-      // first chunk: the 3 rows before token 0 come from the carried conv state
-      if (c0 == 0 && a.states_in) {
-        for (int idx = tid; idx < nslots * 3 * 64; idx += kThreads) {
-          const int sl = idx / 192, r = (idx / 64) % 3, chn = idx % 64;
-          if (!slot_on(sl)) continue;
-          const __nv_bfloat16 v = a.conv_in[(w.bi * pr.conv_dim + slot_ch(sl) + chn) * 4 + 1 + r];
-          const uint32_t addr = stage + sl * kRawBytes + r * 128 +
-                                ((((chn >> 3) ^ r) & 7) << 4) + ((chn & 7) << 1);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(v))
-                       : "memory");
+      // missing second head: zero rows 64..127 of the x operands
+      auto zero_tile = [&]() {
+        const int blk = s0 >> 6, kq = s0 & 63;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t off = blk * 16384 + sw128_off(64 + cg * 8 + i, kq);
+          st_shared_v2(sAhi + off, 0u, 0u);
+          st_shared_v2(sAlo + off, 0u, 0u);
         }
-        compute_sync();
-      }
-      // conv + SiLU.  Warp tile: one slot x 4 groups of 8 channels x 8 quads of
-      // tokens (lane = group lane % 4, quad lane / 4).  This tile reads the
-      // swizzled raw rows, stores u (64 contiguous bytes per token) and, with the
-      // channel order of odd groups rotated by 4, stores the swizzled operands
-      // without shared-memory bank conflicts.
-      //
-      // A pair item whose B operand is already in shared memory has exactly one
-      // tile per warp: its values stay in registers until the previous item's MMA
-      // has completed, so that MMA runs under this item's convolution.  Other pair
-      // items first wait for that MMA, then write their operands tile by tile.
-      const bool overlap = !w.isC && !freshB;
-      if (!w.isC && !overlap && pending) {
-        ok = wait_compute(&mbar, (uint32_t)(npair_done & 1), ok);
-        if (ok) {
-          store_states(pw);
-          pending = false;
-          ++npair_done;
-        }
-      }
-      const int ntiles = 8 * (w.isC ? 1 : (freshB ? 3 : 2));
+      };
       float v[4][8];
-      int keep_sl = 0, keep_cg = 0, keep_s0 = 0;
-      for (int wt = warp; wt < ntiles; wt += kThreads / 32) {
-        const int sl = wt >> 3;
-        const int cg = 4 * ((wt >> 2) & 1) + (lane & 3);
-        const int s0 = 4 * (8 * (wt & 3) + (lane >> 2));
-        keep_sl = sl;
-        keep_cg = cg;
-        keep_s0 = s0;
-        if (sl == 1 && !hasB) {  // missing second head: zero rows 64..127
-          if (!overlap) zero_tile(cg, s0);
-          continue;
-        }
-        conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
-        if (w.isC || sl < 2 || w.pair == 0) store_u(a, w.bi, c0 + s0, slot_ch(sl) + cg * 8, v);
-        if (!w.isC && !overlap) put_operands(sl, cg, s0, v);
-      }
-      if (overlap) {
-        if (pending) {
-          ok = wait_compute(&mbar, (uint32_t)(npair_done & 1), ok);
-          if (ok) {
-            store_states(pw);
-            pending = false;
-            ++npair_done;
+      if (w.isC) {
+        // C item: warps 0-7 convolve the C channels (B/C buffer) into u, then the B
+        // channels (x slot 0) for C_t . B_t in fp32: each thread's 8 channels x 4
+        // tokens, summed over the 4 lanes of a token quad, then warps 4-7 (channel
+        // groups 4-7) hand their sums to warps 0-3 through shared memory
+        if (warp < 8) {
+          conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v);
+          store_u(a, w.bi, c0 + s0, bc_ch + cg * 8, v);
+          mbar_arrive(&bc_empty[bcb]);
+          float d4[4];
+          conv8x4_dot(stage, s0, cg, wts[st][0], bss[st][0], v, d4);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            d4[kk] += __shfl_xor_sync(0xffffffffu, d4[kk], 1);
+            d4[kk] += __shfl_xor_sync(0xffffffffu, d4[kk], 2);
+          }
+          const int cpar = nc & 1;
+          if (warp >= 4) {
+            if ((lane & 3) == 0)
+              *reinterpret_cast<float4 *>(&cbd_s[cpar][s0]) = make_float4(d4[0], d4[1], d4[2], d4[3]);
+            mbar_arrive(&cbd_bar);
+          } else {
+            const bool got = mbar_wait_bounded(&cbd_bar, (uint32_t)(nc & 1), &g_tc_errors);
+            ok = __all_sync(0xffffffffu, got) != 0;
+            if (ok && (lane & 3) == 0) {
+              const float4 o = *reinterpret_cast<const float4 *>(&cbd_s[cpar][s0]);
+              float4 *dp = reinterpret_cast<float4 *>(a.cbd + ((w.bi * pr.G + w.g) * a.nch + w.c) * kQ + s0);
+              if (M2_OK(dp, 16, a.sp.cbd, &g_tc_errors))
+                *dp = make_float4(d4[0] + o.x, d4[1] + o.y, d4[2] + o.z, d4[3] + o.w);
+            }
           }
         }
-        if (ok) {
-          if (keep_sl == 1 && !hasB) zero_tile(keep_cg, keep_s0);
-          else put_operands(keep_sl, keep_cg, keep_s0, v);
-        }
+        ++nc;
+        mbar_arrive(&empty[st]);
+        continue;
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      compute_sync();
-      if (tid == 0) mbar_arrive(&empty[st]);  // raw tiles and taps of this stage consumed
-      if (w.isC || !ok) continue;
-      if (tid == 0) mbar_arrive(&ops_ready);  // the MMA warp issues S = (x o w)^T B
-      pending = true;
+      const int sl = warp >> 3;  // x slot of this warp: head A (warps 0-7) or B
+      const int64_t xch = (int64_t)(hA + sl) * kHP;
+      if (w.freshB) {
+        // B changes: the previous pair item's MMAs must have read the old operands
+        if (np >= 1) wait_mma(np - 1);
+        if (!ok) break;
+        if (warp < 8) {
+          conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v);
+          if (w.pair == 0) store_u(a, w.bi, c0 + s0, bc_ch + cg * 8, v);
+          put_operands(2, v, tile_weights(2));
+          mbar_arrive(&bc_empty[bcb]);
+        }
+        if (sl == 1 && !hasB) zero_tile();
+        else {
+          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
+          store_u(a, w.bi, c0 + s0, xch + cg * 8, v);
+          put_operands(sl, v, tile_weights(sl));
+        }
+        mbar_arrive(&empty[st]);
+      } else {
+        // the tile stays in registers while the previous pair item's MMAs run; its u
+        // stores follow the operand hand-off, so the MMA does not wait behind them
+        float4 wk4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        const bool has_tile = !(sl == 1 && !hasB);
+        if (has_tile) {
+          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
+          wk4 = tile_weights(sl);
+        }
+        mbar_arrive(&empty[st]);  // nothing of the stage is read after this
+        if (np >= 1) wait_mma(np - 1);
+        if (!ok) break;
+        if (!has_tile) zero_tile();
+        else put_operands(sl, v, wk4);
+        fence_proxy_async_smem();
+        mbar_arrive(&ops_ready);  // the MMA warp issues S = (x o w)^T B into accumulator np % 2
+        if (has_tile) store_u(a, w.bi, c0 + s0, xch + cg * 8, v);
+      }
+      if (w.freshB) {
+        fence_proxy_async_smem();
+        mbar_arrive(&ops_ready);
+      }
+      // meanwhile: the previous pair item's chunk states out of its accumulator
+      if (np >= 1) store_states(pw, (np - 1) & 1);
       pw.bi = w.bi;
       pw.c = w.c;
       pw.hA = hA;
       pw.hasB = hasB;
+      ++np;
     }
-    if (ok && pending) {
-      ok = wait_compute(&mbar, (uint32_t)(npair_done & 1), ok);
-      if (ok) {
-        store_states(pw);
-        pending = false;
-      }
-    }
-    if (!ok && tid == 0) {
-      // a wait ran out: let the MMA and the copies already issued land before the
-      // CTA frees its tensor memory and exits
-      if (pending) mbar_wait_bounded(&mbar, (uint32_t)(npair_done & 1), &g_tc_errors);
-      for (int s2 = 0; s2 < 2; ++s2) mbar_wait_bounded(&full[s2], 0, &g_tc_errors);
+    if (ok && np >= 1) {
+      wait_mma(np - 1);
+      if (ok) store_states(pw, (np - 1) & 1);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 64);
+  launch_dependents();
+  if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
 // ============================================================== state passing
-// grid (P*N/1024 + conv-state blocks, H, b): one thread per 4 state elements of
-// one p and consecutive n (four independent recurrences, 16-byte loads of the
-// chunk states), sequential over chunks.
-// Blocks with blockIdx.x >= P*N/1024 (only for h = 0) write the final conv
-// state instead: the last 4 raw inputs of [old state | new tokens], in place
-// (the chunk-state kernel, which reads the old state, has finished by now).
-constexpr int kPassBlocks = (kHP * kNS) / 1024;
+// grid (4 + conv-state blocks, H, b).  Block q < 4 runs the recurrence
+// H_{c+1} = exp(cum_end_c) H_c + S_c in fp32 for the rows p in [16q, 16q + 16)
+// of one head, sequential over chunks: warp w owns the rows p = 16q + 2w and
+// 16q + 2w + 1, lane l the row 16q + 2w + l / 16 and the columns
+// n = 4 (l % 16) .. +3 (one 16-byte load of the chunk states per chunk; loads run
+// 8 chunks ahead).  The state entering each chunk is stored as the fp16 operand
+// of the output kernel's C H_c^T product, [p][n] (n contiguous: each lane writes
+// 8 bytes, each warp two whole 128-byte rows), divided by a power of two 2^s
+// chosen per (chunk, head, pair of rows) from the warp's max |H_c| so that every
+// stored value is below 2^14: fp16 cannot overflow whatever the state's size.
+// The output kernel multiplies those columns of C H_c^T by 2^s (exact).  No
+// barrier is needed: each warp's scale is its own.
+// Blocks with blockIdx.x >= 4 (only for h = 0) write the final conv state
+// instead: the last 4 raw inputs of [old state | new tokens], in place (the
+// chunk-state kernel, which reads the old state, has finished by now).
+constexpr int kPassBlocks = 4;
+
+// 2^s with s = max(0, floor(log2 m) - 13), so that m / 2^s < 2^14.
+__device__ __forceinline__ float state_scale(float m) {
+  const int e = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;  // floor(log2 m) for normal m
+  const int s = min(max(e - 13, 0), 100);
+  return __uint_as_float((uint32_t)(127 + s) << 23);
+}
 
 __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloat16 *cs) {
+  grid_dependency_wait();  // the chunk-state kernel's results (launched early, see prefill_tc)
+  launch_dependents();
   const Problem &pr = a.pr;
   const int h = blockIdx.y;
   const int64_t bi = blockIdx.z;
@@ -688,117 +814,147 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int64_t tau = pr.L - 4 + k;
-      if (tau >= 0) v[k] = a.xBC[(bi * pr.L + tau) * a.ld_x + ch];
-      else v[k] = a.states_in ? cs[i * 4 + 4 + tau] : __float2bfloat16(0.0f);
+      const __nv_bfloat16 *xp = a.xBC + (bi * pr.L + tau) * a.ld_x + ch;
+      v[k] = __float2bfloat16(0.0f);
+      if (tau >= 0) {
+        if (M2_OK(xp, 2, a.sp.xbc, &g_tc_errors)) v[k] = *xp;
+      } else if (a.states_in && M2_OK(cs + i * 4 + 4 + tau, 2, a.sp.conv, &g_tc_errors)) {
+        v[k] = cs[i * 4 + 4 + tau];
+      }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) cs[i * 4 + k] = v[k];
+    for (int k = 0; k < 4; ++k)
+      if (M2_OK(cs + i * 4 + k, 2, a.sp.conv, &g_tc_errors)) cs[i * 4 + k] = v[k];
     return;
   }
-  // float4 slot j of a head's 64 x 64 state: n = 4 (j / 64) .. +3, p = j % 64 (the
-  // chunk-state layout [n/4][p][4]); H_c is stored [n][p] (the MN-major MMA operand)
-  const int j = blockIdx.x * 256 + threadIdx.x, n4 = j >> 6, p = j & 63;
+  const int q = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = 16 * q + 2 * warp + (lane >> 4), n4 = lane & 15;
+  const int j = n4 * kHP + p;  // float4 slot in the chunk-state layout [n/4][p][4]
   const int64_t hs = (bi * pr.H + h) * (int64_t)(kHP * kNS) + p * kNS + 4 * n4;
-  float4 hc = a.states_in ? *reinterpret_cast<const float4 *>(a.ssm_state + hs)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 hc = (a.states_in && M2_OK(a.ssm_state + hs, 16, a.sp.ssm, &g_tc_errors))
+                  ? *reinterpret_cast<const float4 *>(a.ssm_state + hs)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
   const int64_t stride = (int64_t)pr.H * kHP * kNS;
   const float *S = a.S + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + 4 * j;
-  __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + (4 * n4) * kHP + p;
+  __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + p * kNS + 4 * n4;
+  float *hsc = a.hsc + (bi * a.nch * pr.H + h) * 32 + 8 * q + warp;
   const float *ce = a.cum_end + bi * a.nch * pr.H + h;
+  // H_c / 2^s into the operand, 2^s into the scale table (a warp-wide max per chunk)
   auto put = [&](int64_t c) {
+    float m = fmaxf(fmaxf(fabsf(hc.x), fabsf(hc.y)), fmaxf(fabsf(hc.z), fabsf(hc.w)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float sc = state_scale(m), inv = 1.0f / sc;  // powers of two: exact
+    if (lane == 0 && M2_OK(hsc + c * pr.H * 32, 4, a.sp.hsc, &g_tc_errors)) hsc[c * pr.H * 32] = sc;
     __half *o = Hc + c * stride;
-    o[0] = __float2half_rn(hc.x);
-    o[kHP] = __float2half_rn(hc.y);
-    o[2 * kHP] = __float2half_rn(hc.z);
-    o[3 * kHP] = __float2half_rn(hc.w);
+    const __half2 lo = __floats2half2_rn(hc.x * inv, hc.y * inv);
+    const __half2 hi = __floats2half2_rn(hc.z * inv, hc.w * inv);
+    uint2 u2;
+    u2.x = *reinterpret_cast<const uint32_t *>(&lo);
+    u2.y = *reinterpret_cast<const uint32_t *>(&hi);
+    if (M2_OK(o, 8, a.sp.Hc, &g_tc_errors)) *reinterpret_cast<uint2 *>(o) = u2;
   };
-  // loads run 8 chunks ahead of the (sequential) recurrence
+  // a rolling window of 8 chunks in flight: chunk c + 8 is requested as soon as
+  // chunk c has been used, so the memory latency is paid once, not once per 8 chunks
   constexpr int kAhead = 8;
-  int c = 0;
-  for (; c + kAhead <= a.nch; c += kAhead) {
-    float4 sv[kAhead];
-    float d[kAhead];
+  float4 sv[kAhead];
+  float d[kAhead];
+  auto fetch = [&](int cc, float4 &svk, float &dk) {
+    if (cc < a.nch) {
+      const float *sp = S + cc * stride;
+      const float *cp = ce + (int64_t)cc * pr.H;
+      svk = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      dk = M2_OK(cp, 4, a.sp.cum_end, &g_tc_errors) ? *cp : 0.0f;
+    }
+  };
+#pragma unroll
+  for (int k = 0; k < kAhead; ++k) fetch(k, sv[k], d[k]);
+  for (int c0 = 0; c0 < a.nch; c0 += kAhead) {
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
-      sv[k] = *reinterpret_cast<const float4 *>(S + (c + k) * stride);
-      d[k] = ce[(int64_t)(c + k) * pr.H];
-    }
-#pragma unroll
-    for (int k = 0; k < kAhead; ++k) {
-      put(c + k);
-      const float f = expf(d[k]);
-      hc = make_float4(fmaf(f, hc.x, sv[k].x), fmaf(f, hc.y, sv[k].y), fmaf(f, hc.z, sv[k].z),
-                       fmaf(f, hc.w, sv[k].w));
+      const int c = c0 + k;
+      if (c < a.nch) {
+        put(c);
+        const float f = expf(d[k]);
+        hc = make_float4(fmaf(f, hc.x, sv[k].x), fmaf(f, hc.y, sv[k].y), fmaf(f, hc.z, sv[k].z),
+                         fmaf(f, hc.w, sv[k].w));
+        fetch(c + kAhead, sv[k], d[k]);
+      }
     }
   }
-  for (; c < a.nch; ++c) {
-    put(c);
-    const float4 sv = *reinterpret_cast<const float4 *>(S + c * stride);
-    const float f = expf(ce[(int64_t)c * pr.H]);
-    hc = make_float4(fmaf(f, hc.x, sv.x), fmaf(f, hc.y, sv.y), fmaf(f, hc.z, sv.z),
-                     fmaf(f, hc.w, sv.w));
-  }
-  if (a.ssm_state != nullptr) *reinterpret_cast<float4 *>(a.ssm_state + hs) = hc;
+  if (a.ssm_state != nullptr && M2_OK(a.ssm_state + hs, 16, a.sp.ssm, &g_tc_errors))
+    *reinterpret_cast<float4 *>(a.ssm_state + hs) = hc;
 }
 
 // ============================================================== chunk output
 // Persistent clusters: grid (cs, ncl, 1), cluster (cs, 1, 1).  Cluster k takes
 // the units (row, chunk, group) k, k + ncl, ...; its cs CTAs split the group's
-// heads.  16 compute warps + 1 TMA producer warp + 1 MMA-issuer warp.  Tiles
-// arrive by TMA in 128-byte-swizzled layouts (1024-aligned).  Per head the
-// intra-chunk part [CB o L o dt (+D)] x is one K = 128 MMA into the head's TMEM
-// columns, and the carried-state part C H_c^T a K = 64 MMA with the C tile
-// itself as operand into a shared TMEM accumulator, scaled by exp(cum_t) in
-// the epilogue.  The operand A is double-buffered so that the A-build of head
-// j + 1 overlaps the MMA of head j; buffer 1 reuses the B tile once CB is
-// formed.  The next unit's C and B tiles, its CB product and its first
-// x / H_c / z tiles arrive while the current unit exchanges its norm sums and
-// writes its output.
-constexpr uint32_t kCt = 0;                      // C   [128 t][64 n] fp16     16 KB (u)
-constexpr uint32_t kBt = kCt + 16384;            // B   [128 s][64 n] fp16     16 KB (u)
-constexpr int kXhStages = 2, kZStages = 2;
-constexpr uint32_t kXhBytes = 16384 + 8192;      // per stage: x [128 s][64 p] + H_c [64 n][64 p]
-constexpr uint32_t kXh = kBt + 16384;            // x / H_c ring  2 x 24 KB (x at +0, H_c at +16 KB)
-constexpr uint32_t kZt = kXh + kXhStages * kXhBytes;  // z ring [128 t][64 p] bf16  2 x 16 KB
-constexpr uint32_t kA0 = kZt + kZStages * 16384;      // A buffer 0: [2][128 t][64 k] fp16  32 KB
-constexpr uint32_t kA1 = kA0 + 2 * 16384;             // A buffer 1, block 1 (block 0 at kBt)
-constexpr uint32_t kYst = kA1 + 16384;                // two output staging tiles  32 KB
-constexpr uint32_t kTcOutTiles = kYst + 2 * 16384;    // 192 KB
-// output staging: [128 t][64 p] bf16 tiles, idle while a unit writes its output:
-// A buffer 0, block 1 of buffer 1 and the two staging tiles
-constexpr int kYTiles = 5;
-__device__ __forceinline__ uint32_t y_tile(int slot) {
-  return slot < 2 ? kA0 + slot * 16384 : (slot == 2 ? kA1 : kYst + (slot - 3) * 16384);
-}
+// heads (the same nh <= 5 heads of the group in every unit).  Per CTA:
+//   warp 16      TMA producer: per unit the C and B tiles of u (C double-
+//                buffered, so the next unit's arrive during this one), per head
+//                the x and H_c tiles (ring of 2) and the z tile (ring of 2);
+//   warp 17      MMA issuer: CB = C B^T once per unit (M = N = 128, K = 64), per
+//                head y_j = A_j x_j (K = 128, into the head's 64 TMEM columns)
+//                and T = C H_c^T (K = 64, one shared 64-column accumulator);
+//   warps 0-7    decay operand: A_j = CB o exp(cum_t - cum_s) dt_s (s <= t, D_h
+//                on the diagonal) in fp16, double-buffered, up to two heads
+//                ahead of the epilogue; warp w builds rows 32 (w % 4) .. +31
+//                (its TMEM lane quarter) and columns 64 (w / 4) .. +63.  The
+//                same warps write the previous unit's output: after building
+//                head j's operand of unit n they scale head j of unit n - 1 by
+//                the per-token norm and the norm weight and store it to y
+//                (32-byte stores), which hands head j's TMEM columns back to
+//                the MMA warp for unit n;
+//   warps 8-15   epilogue: y_j + exp(cum_t) 2^s T, gate by silu(z), per-token
+//                sums of squares, the gated value back into TMEM; after the
+//                unit's last head the per-token sums go to every CTA of the
+//                cluster (asynchronous DSMEM stores completing on the receiver's
+//                mbarrier) and the per-token norm scales to the operand warps.
+// All waits are bounded (they raise the error flag and the CTA leaves its loop).
+constexpr uint32_t kCt0 = 0;                       // C [2][128 t][64 n] fp16 (u), 2 x 16 KB
+constexpr uint32_t kBt = 2 * 16384;                // B [128 s][64 n] fp16 (u), 16 KB
+constexpr uint32_t kXhBytes = 16384 + 8192;        // per stage: x [128 s][64 p] + H_c [64 n][64 p]
+constexpr uint32_t kXh = kBt + 16384;              // x / H_c ring, 2 x 24 KB
+constexpr uint32_t kZt = kXh + 2 * kXhBytes;       // z ring [128 t][64 p] bf16, 2 x 16 KB
+constexpr uint32_t kAbuf = kZt + 2 * 16384;        // A [2][2 k-blocks][128 t][64 s] fp16, 2 x 32 KB
+constexpr uint32_t kTcOutTiles = kAbuf + 2 * 32768;  // 176 KB
+constexpr int kGroupThreads = 256;                 // threads of the operand / epilogue groups
 
-// Byte offset of k-block `blk` (CB columns s 0..63, 64..127) of A buffer `buf`.
-__device__ __forceinline__ uint32_t a_block(int buf, int blk) {
-  return buf == 0 ? kA0 + blk * 16384 : (blk == 0 ? kBt : kA1);
-}
-
+// Every array read or written with 16-byte accesses (float4 loads, st.async.v4
+// into other ranks) is 16-byte aligned; the static_asserts below check it.
 struct OutShared {
-  float cum2[kMaxHeadsPerCta][kQ];  // cumsum * log2(e)
-  float dt[kMaxHeadsPerCta][kQ];
-  float beta[kMaxHeadsPerCta][kQ];  // exp(cum_r - cum_s) dt_s, r = end of s's 32-token group
-  float betad[kMaxHeadsPerCta][kQ]; // exp(cum_s0 - cum_s) dt_s, s0 = start of s's group
-  int span_ok[kMaxHeadsPerCta][4];  // group's log2-decay span <= 60: factorise its diagonal
-  float nw[kMaxHeadsPerCta][kHP];   // norm weight of the CTA's channels
-  float ss[4][kQ];
-  float part[2][16][kQ];            // [unit parity][rank]: partial sums of squares per token
-  float mine[kQ];                   // this CTA's partial sums
-  float inv[kQ];
+  // decay terms of the unit's heads (operand group)
+  alignas(16) float cum2[kMaxHeadsPerCta][kQ];   // cumsum * log2(e)
+  alignas(16) float dt[kMaxHeadsPerCta][kQ];
+  alignas(16) float beta[kMaxHeadsPerCta][kQ];   // exp(cum_r - cum_s) dt_s, r = end of s's 32-token group
+  alignas(16) float betad[kMaxHeadsPerCta][kQ];  // exp(cum_s0 - cum_s) dt_s, s0 = start of s's group
+  // epilogue group
+  alignas(16) float inv[2][kQ];                  // [unit parity] per-token norm scales, for the output
+  alignas(16) float half_ss[2][kQ];              // per-token sums of squares of the two column halves
+  alignas(16) float mine[kQ];                    // this CTA's per-token partial sums
+  alignas(16) float part[2][16][kQ];             // [unit parity][rank] partial sums received
+  alignas(16) float cbd[kQ];                     // C_t . B_t (fp32) of the unit's chunk and group
+  int span_ok[kMaxHeadsPerCta][4];   // group's log2-decay span <= 60: factorise its diagonal
   float Dh[kMaxHeadsPerCta];
-  uint64_t full_cb, full_xh[kXhStages], empty_xh[kXhStages], full_z[kZStages],
-      empty_z[kZStages], a_ready[2], mbar_cb, mbar_mma[2], tiles_free, sums_ready[2], t_free;
+  uint64_t full_cb[2], b_free, c_free[2], full_xh[2], empty_xh[2], full_z[2], empty_z[2],
+      a_ready[2], mma_done[2], mbar_cb, cb_free, t_free, y_free[kMaxHeadsPerCta], sums_ready[2],
+      mma_final, inv_ready;
   uint32_t tmem_holder;
-  int ok_flag;
 };
+
+static_assert(offsetof(OutShared, cum2) % 16 == 0 && offsetof(OutShared, dt) % 16 == 0 &&
+                  offsetof(OutShared, beta) % 16 == 0 && offsetof(OutShared, betad) % 16 == 0 &&
+                  offsetof(OutShared, inv) % 16 == 0 && offsetof(OutShared, mine) % 16 == 0 &&
+                  offsetof(OutShared, part) % 16 == 0 && offsetof(OutShared, cbd) % 16 == 0 &&
+                  offsetof(OutShared, full_cb) % 8 == 0,
+              "16-byte accessed shared arrays must be 16-byte aligned");
+static_assert(kTcOutTiles % 1024 == 0, "OutShared starts 16-byte aligned");
 
 struct OutMaps {
   CUtensorMap u;   // [b][L][conv_dim] fp16, box 64 ch x 128 tokens
   CUtensorMap z;   // [b][L][d_inner] bf16 (row stride ld_z), box 64 x 128
   CUtensorMap hc;  // [rows][64] fp16, box 64 x 64
-  CUtensorMap y;   // [b][L][d_inner] bf16, box 64 x 128 (stores)
 };
 
 // 16-byte asynchronous store into another rank's shared memory that completes
@@ -836,6 +992,31 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_
   }
   return true;
 }
+// Barriers over one 256-thread group (id 1: operand group, id 2: epilogue group);
+// the _and form also returns whether every thread of the group passed `v`.
+__device__ __forceinline__ void group_sync(int id) {
+  asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool group_all(int id, bool v) {
+  int r;
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.s32 p, %2, 0;\n bar.red.and.pred q, %1, 256, p;\n"
+               " selp.s32 %0, 1, 0, q;\n}"
+               : "=r"(r)
+               : "r"(id), "r"((int)v)
+               : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void st_global_v4(void *p, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+// 32-byte store (one whole L2 sector), 32-byte aligned address
+__device__ __forceinline__ void st_global_v8(void *p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
 
 // Unit n of cluster `cid`: (row bi, chunk c, group g).
 __device__ __forceinline__ void out_unit(const Problem &pr, int nch, int ncl, int cid, int n,
@@ -847,6 +1028,92 @@ __device__ __forceinline__ void out_unit(const Problem &pr, int nch, int ncl, in
   bi = bc / nch;
 }
 
+// One 32-column group k of row t of the decay operand A_j (j = head), written as
+// four 16-byte chunks at column kc (0 or 32) of the 64-wide k-block at `at`:
+// zero above the diagonal group, factorised alpha_t beta_s below it, and on it
+// either factorised (decay span within 2^60) or with direct exponentials.
+__device__ __forceinline__ void build_a_group(const OutShared &sh, int j, int k, int q, int t,
+                                              uint32_t at, int kc, uint32_t tmem_cb) {
+  const int s0 = 32 * k;
+  if (k > q) {
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), 0u, 0u, 0u, 0u);
+    return;
+  }
+  float cb[32];
+  tmem_ld32(tmem_cb + s0, cb);
+  const float c2t = sh.cum2[j][t];
+  if (k < q) {
+    const float alpha = ex2_approx(c2t - sh.cum2[j][s0 + 31]);
+    const float4 *b4 = reinterpret_cast<const float4 *>(&sh.beta[j][s0]);
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      const float4 bA = b4[2 * qq], bB = b4[2 * qq + 1];
+      const float bb[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int sl = 8 * qq + 2 * e;
+        w4[e] = pack_half2(cb[sl] * alpha * bb[2 * e], cb[sl + 1] * alpha * bb[2 * e + 1]);
+      }
+      st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+    }
+    return;
+  }
+  const float Dh = sh.Dh[j];
+  if (sh.span_ok[j][k]) {
+    // diagonal group, decay span <= 2^60: alpha_t = exp(cum_t - cum_s0) and
+    // betad_s = exp(cum_s0 - cum_s) dt_s stay within [2^-60, 2^60]
+    const float alpha = ex2_approx(c2t - sh.cum2[j][s0]);
+    const float4 *b4 = reinterpret_cast<const float4 *>(&sh.betad[j][s0]);
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      const float4 bA = b4[2 * qq], bB = b4[2 * qq + 1];
+      const float bb[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float val[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
+          float vv = cb[sl] * alpha * bb[2 * e + u];
+          if (s == t) vv = fmaf(sh.cbd[t], sh.dt[j][t], Dh);  // exp(0) = 1; fp32 C_t . B_t
+          val[u] = (s <= t) ? vv : 0.0f;
+        }
+        w4[e] = pack_half2(val[0], val[1]);
+      }
+      st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+    }
+  } else {
+    const float4 *c4 = reinterpret_cast<const float4 *>(&sh.cum2[j][s0]);
+    const float4 *d4 = reinterpret_cast<const float4 *>(&sh.dt[j][s0]);
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      const float4 cA = c4[2 * qq], cB = c4[2 * qq + 1];
+      const float4 dA = d4[2 * qq], dB = d4[2 * qq + 1];
+      const float cc[8] = {cA.x, cA.y, cA.z, cA.w, cB.x, cB.y, cB.z, cB.w};
+      const float dd[8] = {dA.x, dA.y, dA.z, dA.w, dB.x, dB.y, dB.z, dB.w};
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float val[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
+          float vv = cb[sl] * ex2_approx(fminf(c2t - cc[2 * e + u], 0.0f)) * dd[2 * e + u];
+          if (s == t) vv = fmaf(sh.cbd[t], sh.dt[j][t], Dh);
+          val[u] = (s <= t) ? vv : 0.0f;
+        }
+        w4[e] = pack_half2(val[0], val[1]);
+      }
+      st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+}
+
+// (18 warps: one SM sub-partition holds 5 of them, and 5 x 32 x 96 registers is what
+// its quarter of the register file allows)
 __global__ void __launch_bounds__(kWsThreads, 1)
     tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps, int ncl) {
   if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA of every cluster alike
@@ -869,197 +1136,234 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 
   if (warp == 0) tmem_alloc(&sh.tmem_holder, 512);
   if (tid == 0) {
-    mbar_init(&sh.full_cb, 1);
-    for (int k = 0; k < kXhStages; ++k) {
-      mbar_init(&sh.full_xh[k], 1);
-      mbar_init(&sh.empty_xh[k], 1);  // arrived by tcgen05.commit of the head's MMA
-    }
-    for (int k = 0; k < kZStages; ++k) {
-      mbar_init(&sh.full_z[k], 1);
-      mbar_init(&sh.empty_z[k], kThreads);  // every compute thread after its epilogue
-    }
     for (int k = 0; k < 2; ++k) {
-      mbar_init(&sh.a_ready[k], kThreads);  // every compute thread after its A-build
-      mbar_init(&sh.mbar_mma[k], 1);        // MMA of a head that used A buffer k
+      mbar_init(&sh.full_cb[k], 1);
+      mbar_init(&sh.c_free[k], 1);
+      mbar_init(&sh.full_xh[k], 1);
+      mbar_init(&sh.empty_xh[k], 1);  // tcgen05.commit after the head's MMAs
+      mbar_init(&sh.full_z[k], 1);
+      mbar_init(&sh.empty_z[k], kGroupThreads);
+      mbar_init(&sh.a_ready[k], kGroupThreads);
+      mbar_init(&sh.mma_done[k], 1);
       // the local arrival carries the bytes the ranks' partial sums complete;
       // units 0 and 1 are armed here, unit n + 2 once unit n's sums are read
       mbar_init(&sh.sums_ready[k], 1);
       mbar_arrive_expect_tx(&sh.sums_ready[k], sum_bytes);
     }
+    mbar_init(&sh.b_free, 1);
     mbar_init(&sh.mbar_cb, 1);
-    mbar_init(&sh.tiles_free, 1);  // a unit's C / B tiles and CB columns no longer read
-    mbar_init(&sh.t_free, kThreads);  // every compute thread has read the C H_c^T columns
+    mbar_init(&sh.mma_final, 1);
+    mbar_init(&sh.cb_free, kGroupThreads);
+    mbar_init(&sh.t_free, kGroupThreads);
+    mbar_init(&sh.inv_ready, kGroupThreads);  // the epilogue group wrote a unit's norm scales
+    for (int j = 0; j < kMaxHeadsPerCta; ++j) mbar_init(&sh.y_free[j], kGroupThreads);
     fence_mbar_init();
-    sh.ok_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   cluster_arrive_relaxed();  // waited for before the first remote store
+  grid_dependency_wait();    // u, H_c, the scales and the dt rows are complete from here on
   bool started = false;
   const uint32_t tmem = sh.tmem_holder;
+  constexpr uint32_t kTmemY = 128;                     // y_j at columns 128 + 64 j
 
-  if (warp == kThreads / 32) {
-    // ---------------- producer: per unit, x / H_c / z of each head (rings released
-    // by the head's MMA and epilogue); after the first head's, the unit's C and B
-    // tiles, once the previous unit has finished reading them
+  if (warp == 16) {
+    // ---------------- producer
     if (lane == 0 && nh > 0) {
-      int J = 0;    // heads issued so far (ring position)
-      int ncb = 0;  // C / B loads issued
       bool ok = true;
+      int J = 0, ncb = 0, nxh = 0, nz = 0;  // copies issued into each ring
+      auto load_cb = [&](int n) {  // C and B tiles of unit n
+        int64_t bi;
+        int c, g;
+        out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+        const int cbuf = n & 1;
+        if (n >= 2) ok = ok && mbar_wait_bounded(&sh.c_free[cbuf], (uint32_t)(((n - 2) >> 1) & 1), &g_tc_errors);
+        if (n >= 1) ok = ok && mbar_wait_bounded(&sh.b_free, (uint32_t)((n - 1) & 1), &g_tc_errors);
+        if (!ok) return;
+        mbar_arrive_expect_tx(&sh.full_cb[cbuf], 2 * 16384);
+        tma_load_3d(base + kCt0 + cbuf * 16384, &maps.u,
+                    (int)(pr.d_inner + (int64_t)(pr.G + g) * kNS), c * kQ, (int)bi, &sh.full_cb[cbuf]);
+        tma_load_3d(base + kBt, &maps.u, (int)(pr.d_inner + (int64_t)g * kNS), c * kQ, (int)bi,
+                    &sh.full_cb[cbuf]);
+        ++ncb;
+      };
+      load_cb(0);
       for (int n = 0; ok && n < n_units; ++n) {
         int64_t bi;
         int c, g;
         out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
         const int h0 = g * hpg + lh0;
-        const int c0 = c * kQ;
         for (int j = 0; ok && j < nh; ++j, ++J) {
-          const int h = h0 + j, sx = J % kXhStages, sz = J % kZStages;
-          ok = J < kXhStages ||
-               mbar_wait_bounded(&sh.empty_xh[sx], (uint32_t)((J / kXhStages - 1) & 1), &g_tc_errors);
+          const int h = h0 + j, sl = J & 1;
+          if (J >= 2) ok = mbar_wait_bounded(&sh.empty_xh[sl], (uint32_t)(((J - 2) >> 1) & 1), &g_tc_errors);
           if (!ok) break;
-          mbar_arrive_expect_tx(&sh.full_xh[sx], kXhBytes);
-          tma_load_3d(base + kXh + sx * kXhBytes, &maps.u, h * kHP, c0, (int)bi, &sh.full_xh[sx]);
-          tma_load_2d(base + kXh + sx * kXhBytes + 16384, &maps.hc, 0,
-                      (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full_xh[sx]);
-          ok = J < kZStages ||
-               mbar_wait_bounded(&sh.empty_z[sz], (uint32_t)((J / kZStages - 1) & 1), &g_tc_errors);
+          mbar_arrive_expect_tx(&sh.full_xh[sl], kXhBytes);
+          tma_load_3d(base + kXh + sl * kXhBytes, &maps.u, h * kHP, c * kQ, (int)bi, &sh.full_xh[sl]);
+          tma_load_2d(base + kXh + sl * kXhBytes + 16384, &maps.hc, 0,
+                      (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full_xh[sl]);
+          ++nxh;
+          if (J >= 2) ok = mbar_wait_bounded(&sh.empty_z[sl], (uint32_t)(((J - 2) >> 1) & 1), &g_tc_errors);
           if (!ok) break;
-          mbar_arrive_expect_tx(&sh.full_z[sz], 16384);
-          tma_load_3d(base + kZt + sz * 16384, &maps.z, h * kHP, c0, (int)bi, &sh.full_z[sz]);
-          if (j == 0) {
-            ok = n == 0 || mbar_wait_bounded(&sh.tiles_free, (uint32_t)((n - 1) & 1), &g_tc_errors);
-            if (!ok) break;
-            mbar_arrive_expect_tx(&sh.full_cb, 2 * 16384);
-            tma_load_3d(base + kCt, &maps.u, (int)(pr.d_inner + (int64_t)(pr.G + g) * kNS), c0,
-                        (int)bi, &sh.full_cb);
-            tma_load_3d(base + kBt, &maps.u, (int)(pr.d_inner + (int64_t)g * kNS), c0, (int)bi,
-                        &sh.full_cb);
-            ++ncb;
-          }
+          mbar_arrive_expect_tx(&sh.full_z[sl], 16384);
+          tma_load_3d(base + kZt + sl * 16384, &maps.z, h * kHP, c * kQ, (int)bi, &sh.full_z[sl]);
+          ++nz;
+          if (j == min(1, nh - 1) && n + 1 < n_units) load_cb(n + 1);
         }
       }
-      // no copy may be in flight when the CTA exits: the last copy into each buffer
-      if (ncb > 0) mbar_wait_bounded(&sh.full_cb, (uint32_t)((ncb - 1) & 1), &g_tc_errors);
-      for (int k = max(0, J - 2); k < J; ++k) {
-        mbar_wait_bounded(&sh.full_xh[k % kXhStages], (uint32_t)((k / kXhStages) & 1), &g_tc_errors);
-        mbar_wait_bounded(&sh.full_z[k % kZStages], (uint32_t)((k / kZStages) & 1), &g_tc_errors);
-      }
+      // no copy may be in flight when the CTA exits: the last copies into each ring
+      for (int k = max(0, ncb - 2); k < ncb; ++k)
+        mbar_wait_bounded(&sh.full_cb[k & 1], (uint32_t)((k >> 1) & 1), &g_tc_errors);
+      for (int k = max(0, nxh - 2); k < nxh; ++k)
+        mbar_wait_bounded(&sh.full_xh[k & 1], (uint32_t)((k >> 1) & 1), &g_tc_errors);
+      for (int k = max(0, nz - 2); k < nz; ++k)
+        mbar_wait_bounded(&sh.full_z[k & 1], (uint32_t)((k >> 1) & 1), &g_tc_errors);
     }
-  } else if (warp == kThreads / 32 + 1) {
-    // ---------------- MMA issuer: per unit CB once, then per head the K = 128 and K = 64 MMAs
+  } else if (warp == 17) {
+    // ---------------- MMA issuer
     if (lane == 0 && nh > 0) {
       const uint32_t idesc_cb = umma_idesc_f16(128, 128);
       const uint32_t idesc_mn = umma_idesc_f16(128, 64) | (1u << 16);  // B operand MN-major
+      const uint32_t idesc_t = umma_idesc_f16(128, 64);                 // both K-major
       int J = 0;
       bool ok = true;
       for (int n = 0; ok && n < n_units; ++n) {
-        // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
-        ok = mbar_wait_bounded(&sh.full_cb, (uint32_t)(n & 1), &g_tc_errors);
+        const int cbuf = n & 1;
+        const uint32_t ct = base + kCt0 + cbuf * 16384;
+        ok = mbar_wait_bounded(&sh.full_cb[cbuf], (uint32_t)((n >> 1) & 1), &g_tc_errors) &&
+             (n == 0 || mbar_wait_bounded(&sh.cb_free, (uint32_t)((n - 1) & 1), &g_tc_errors));
         if (!ok) break;
         tc_fence_after();
+        // CB = C B^T : M = 128 (t), N = 128 (s), K = 64 (n)
         for (int kin = 0; kin < 4; ++kin)
-          umma_f16(tmem, umma_desc_sw128(base + kCt + kin * 32),
-                   umma_desc_sw128(base + kBt + kin * 32), idesc_cb, kin > 0 ? 1u : 0u);
+          umma_f16(tmem, umma_desc_sw128(ct + kin * 32), umma_desc_sw128(base + kBt + kin * 32),
+                   idesc_cb, kin > 0 ? 1u : 0u);
         umma_commit(&sh.mbar_cb);
+        umma_commit(&sh.b_free);
         for (int j = 0; j < nh; ++j, ++J) {
-          ok = mbar_wait_bounded(&sh.a_ready[J & 1], (uint32_t)((J >> 1) & 1), &g_tc_errors) &&
-               mbar_wait_bounded(&sh.full_xh[J % kXhStages], (uint32_t)((J / kXhStages) & 1),
-                                 &g_tc_errors);
+          const int sl = J & 1;
+          ok = mbar_wait_bounded(&sh.a_ready[sl], (uint32_t)((J >> 1) & 1), &g_tc_errors) &&
+               mbar_wait_bounded(&sh.full_xh[sl], (uint32_t)((J >> 1) & 1), &g_tc_errors) &&
+               (n == 0 || mbar_wait_bounded(&sh.y_free[j], (uint32_t)((n - 1) & 1), &g_tc_errors));
           if (!ok) break;
           tc_fence_after();
-          const uint32_t xt = base + kXh + (J % kXhStages) * kXhBytes, ht = xt + 16384;
+          const uint32_t xt = base + kXh + sl * kXhBytes, ht = xt + 16384;
+          const uint32_t ab = base + kAbuf + sl * 32768;
           // y_j = [CB o L o dt (+D)] x : K = 128 (x [s][p] MN-major)
           for (int ks = 0; ks < 8; ++ks)
-            umma_f16(tmem + 128 + 64 * j, umma_desc_sw128(base + a_block(J & 1, ks >> 2) + (ks & 3) * 32),
+            umma_f16(tmem + kTmemY + 64 * j, umma_desc_sw128(ab + (ks >> 2) * 16384 + (ks & 3) * 32),
                      umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn, ks > 0 ? 1u : 0u);
-          // T = C H_c^T : K = 64, the C tile as operand (H_c [n][p] MN-major), once the
-          // previous head's epilogue has read T
+          // T = C H_c^T : K = 64 (n), H_c [p][n] K-major; once the epilogue has read the
+          // previous head's T
           if (J > 0 && !mbar_wait_bounded(&sh.t_free, (uint32_t)((J - 1) & 1), &g_tc_errors)) {
             ok = false;
             break;
           }
           tc_fence_after();
           for (int kin = 0; kin < 4; ++kin)
-            umma_f16(tmem + kTmemT, umma_desc_sw128(base + kCt + kin * 32),
-                     umma_desc_sw128_mn(ht + kin * 2048, 8192), idesc_mn, kin > 0 ? 1u : 0u);
-          umma_commit(&sh.mbar_mma[J & 1]);
-          umma_commit(&sh.empty_xh[J % kXhStages]);  // its x / H_c stage is free once it completes
+            umma_f16(tmem + kTmemT, umma_desc_sw128(ct + kin * 32), umma_desc_sw128(ht + kin * 32),
+                     idesc_t, kin > 0 ? 1u : 0u);
+          umma_commit(&sh.mma_done[sl]);
+          umma_commit(&sh.empty_xh[sl]);  // its x / H_c stage is free once they complete
         }
+        if (ok) umma_commit(&sh.c_free[cbuf]);
       }
-      if (!ok) sh.ok_flag = 0;
-      // no MMA may be in flight when the CTA frees its tensor memory
-      if (J > 0) mbar_wait_bounded(&sh.mbar_mma[(J - 1) & 1], (uint32_t)(((J - 1) >> 1) & 1), &g_tc_errors);
+      // no MMA may be in flight when the CTA frees its tensor memory: one more commit
+      // tracks every MMA this thread issued, whichever way the loop ended
+      umma_commit(&sh.mma_final);
+      mbar_wait_bounded(&sh.mma_final, 0, &g_tc_errors);
     }
-  } else {
-    // ---------------- compute warps
-    const int t = 32 * (warp & 3) + lane, hf = warp >> 2, q = warp & 3;
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    float ss_acc = 0.0f;
+  } else if (warp < 8) {
+    // ---------------- decay operands, and the previous unit's output
+    const int q = warp & 3, blk = warp >> 2, t = 32 * q + lane;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     bool ok = true;
-    int J = 0;  // heads processed so far (ring and A-buffer position)
-    auto wait_warp = [&](uint64_t *bar, uint32_t parity) {
-      const bool got = ok && mbar_wait_bounded(bar, parity, &g_tc_errors);
-      ok = __all_sync(0xffffffffu, got) != 0;
-    };
-
-    // epilogue, part 1: gate with silu(z) (z tile in smem), sum of squares, g -> TMEM.
-    // Warp w handles rows 32*(w%4) .. +31 and columns 16*(w/4) .. +15 of a head.
-    auto epilogue1 = [&](int j, int zslot) {
-      float v[16], w[16];
-      const uint32_t col = 128 + 64 * j + 16 * hf;
-      tmem_ld16(tmem + lane_off + col, v);
-      tmem_ld16(tmem + lane_off + kTmemT + 16 * hf, w);
-      tc_fence_before();
-      mbar_arrive(&sh.t_free);  // the C H_c^T columns may take the next head's product
-      const float ec = ex2_approx(sh.cum2[j][t]);  // exp(cum_t)
+    int J = 0;
+    // normalised bf16 output of head j of unit `un` (columns 32 blk .. +31 of row t);
+    // the head's TMEM columns go back to the MMA warp as soon as they are read
+    auto output_head = [&](int un, int j) {
+      int64_t obi;
+      int oc, og;
+      out_unit(pr, a.nch, ncl, cid, un, obi, oc, og);
+      const int h = og * hpg + lh0 + j;
+      const int64_t tok = (int64_t)oc * kQ + t;
+      const bool t_valid = tok < pr.L;
+      const float inv = sh.inv[un & 1][t];
+      __nv_bfloat16 *yrow = a.y + (obi * pr.L + tok) * pr.d_inner + (int64_t)h * kHP + 32 * blk;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = fmaf(ec, w[i], v[i]);
-      if (!pr.nbg) {
-        const uint32_t zt = base + kZt + zslot * 16384;
+      for (int hh = 0; hh < 2; ++hh) {
+        float v[16];
+        tmem_ld16(tmem + lane_off + kTmemY + 64 * j + 32 * blk + 16 * hh, v);
+        if (hh == 1) {
+          tc_fence_before();
+          mbar_arrive(&sh.y_free[j]);
+        }
+        if (!t_valid) continue;
+        if (pr.nbg) {
+          const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (obi * pr.L + tok) * a.ld_z +
+                                                            (int64_t)h * kHP + 32 * blk + 16 * hh);
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const uint4 raw = ld_shared_v4(zt + sw128_chunk(t, 16 * hf + 8 * qq));
-          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+          for (int qq = 0; qq < 2; ++qq) {
+            const uint4 raw = M2_OK(zp + qq, 16, a.sp.z, &g_tc_errors) ? __ldg(zp + qq)
+                                                                        : make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(h2[i]);
-            v[8 * qq + 2 * i] *= silu_fast(f.x);
-            v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(h2[i]);
+              v[8 * qq + 2 * i] *= silu_fast(f.x);
+              v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
+            }
           }
         }
-      }
+        const float4 *nw4 =
+            reinterpret_cast<const float4 *>(a.prm.norm_w + (int64_t)h * kHP + 32 * blk + 16 * hh);
+        uint32_t o[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) ss_acc = fmaf(v[i], v[i], ss_acc);
-      tmem_st16(tmem + lane_off + col, v);
-    };
-
-    // the per-chunk dt and cumsum rows (written by the chunk-state kernel) of a
-    // unit's heads: one warp per head, 4 consecutive tokens per lane; the next
-    // unit's are loaded before this unit's norm exchange and used after it
-    float4 cu = make_float4(0.f, 0.f, 0.f, 0.f), dv = cu;
-    auto load_rows = [&](int n) {
-      if (warp < nh && n < n_units) {
-        int64_t bi;
-        int c, g;
-        out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
-        const int64_t row = (bi * a.nch + c) * pr.H + g * hpg + lh0 + warp;
-        cu = reinterpret_cast<const float4 *>(a.cum + row * kQ)[lane];
-        dv = reinterpret_cast<const float4 *>(a.dtv + row * kQ)[lane];
+        for (int qq = 0; qq < 2; ++qq) {
+          const bool wok = M2_OK(nw4 + 2 * qq, 16, a.sp.norm_w, &g_tc_errors) &&
+                           M2_OK(nw4 + 2 * qq + 1, 16, a.sp.norm_w, &g_tc_errors);
+          const float4 wA = wok ? __ldg(nw4 + 2 * qq) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 wB = wok ? __ldg(nw4 + 2 * qq + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 8 * qq + 2 * e;
+            const __nv_bfloat162 b2 =
+                __floats2bfloat162_rn(v[i] * inv * ww[2 * e], v[i + 1] * inv * ww[2 * e + 1]);
+            o[4 * qq + e] = *reinterpret_cast<const uint32_t *>(&b2);
+          }
+        }
+        __nv_bfloat16 *yp = yrow + 16 * hh;  // 16 columns = 32 bytes
+        if (a.y32) {
+          if (M2_OK(yp, 16, a.sp.y, &g_tc_errors) && M2_OK(yp + 8, 16, a.sp.y, &g_tc_errors))
+            st_global_v8(yp, o);
+        } else {
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq)
+            if (M2_OK(yp + 8 * qq, 16, a.sp.y, &g_tc_errors))
+              st_global_v4(yp + 8 * qq, o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]);
+        }
       }
     };
-    load_rows(0);
-    int nw_h0 = -1;  // heads whose norm weights are in shared memory
-    for (int n = 0; ok && n < n_units; ++n) {
+    // wait until the epilogue warps have written unit un's norm scales
+    auto wait_inv = [&](int un) {
+      const bool got = ok && mbar_wait_bounded(&sh.inv_ready, (uint32_t)(un & 1), &g_tc_errors);
+      ok = __all_sync(0xffffffffu, got) != 0;
+    };
+    for (int n = 0; ok && n < n_units && nh > 0; ++n) {
       int64_t bi;
       int c, g;
       out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
       const int h0 = g * hpg + lh0;
-      const int64_t c0 = (int64_t)c * kQ;
-      const int par = n & 1;
-      // decay terms of the unit's heads
+      // decay terms of head j = warp (from the per-chunk dt and cumsum rows)
       if (warp < nh) {
         const int j = warp;
+        const int64_t row = (bi * a.nch + c) * pr.H + h0 + j;
+        const float4 *cup = reinterpret_cast<const float4 *>(a.cum + row * kQ) + lane;
+        const float4 *dvp = reinterpret_cast<const float4 *>(a.dtv + row * kQ) + lane;
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 cu = M2_OK(cup, 16, a.sp.cum, &g_tc_errors) ? *cup : z4;
+        const float4 dv = M2_OK(dvp, 16, a.sp.dtv, &g_tc_errors) ? *dvp : z4;
         const float cum4[4] = {cu.x, cu.y, cu.z, cu.w}, dt4[4] = {dv.x, dv.y, dv.z, dv.w};
         float c2[4];
 #pragma unroll
@@ -1076,190 +1380,102 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           sh.betad[j][4 * lane + k] = ex2_approx(fminf(c2s0 - c2[k], 60.0f)) * dt4[k];
         }
         if ((lane & 7) == 7) sh.span_ok[j][lane >> 3] = (c2s0 - c2r) <= 60.0f;
+        if (lane == 0)
+          sh.Dh[j] = M2_OK(a.prm.D + h0 + j, 4, a.sp.D, &g_tc_errors) ? a.prm.D[h0 + j] : 0.0f;
       }
-      if (h0 != nw_h0) {  // norm weights and D of the CTA's heads (same in every unit if G = 1)
-        for (int i = tid; i < nh * kHP; i += kThreads)
-          sh.nw[i / kHP][i % kHP] = a.prm.norm_w[(int64_t)h0 * kHP + i];
-        if (tid < nh) sh.Dh[tid] = a.prm.D[h0 + tid];
-        nw_h0 = h0;
+      if (warp == 7) {  // the unit's fp32 diagonal C_t . B_t
+        const float4 *src = reinterpret_cast<const float4 *>(a.cbd + ((bi * pr.G + g) * a.nch + c) * kQ) + lane;
+        reinterpret_cast<float4 *>(sh.cbd)[lane] =
+            M2_OK(src, 16, a.sp.cbd, &g_tc_errors) ? *src : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      if (n > 0 && tid == 0) bulk_wait_read_all();  // the previous unit's output staging
-      compute_sync();  // decay terms, weights and D visible; staging tiles free
-      ss_acc = 0.0f;
-
+      group_sync(1);
       for (int j = 0; j < nh; ++j, ++J) {
-        // A buffer J % 2 is free: the MMA of head J - 2 was waited for by its
-        // epilogue in the previous iteration (or the previous unit)
-        if (j == 0) {
-          wait_warp(&sh.full_cb, (uint32_t)(n & 1));  // the C tile (read for the scaled-C block)
-          wait_warp(&sh.mbar_cb, (uint32_t)(n & 1));  // CB in TMEM; the B tile is free (A buffer 1)
-        }
+        const int sl = J & 1;
+        if (j == 0) ok = mbar_wait_bounded(&sh.mbar_cb, (uint32_t)(n & 1), &g_tc_errors);
+        // A buffer sl is free once the MMAs of head J - 2 (which read it) completed
+        if (ok && J >= 2) ok = mbar_wait_bounded(&sh.mma_done[sl], (uint32_t)(((J - 2) >> 1) & 1), &g_tc_errors);
+        ok = __all_sync(0xffffffffu, ok) != 0;
         if (!ok) break;
         tc_fence_after();
-        const uint32_t abuf = base + a_block(J & 1, 0), abuf1 = base + a_block(J & 1, 1);
-      // A_j = CB o exp(cum_t - cum_s) dt_s (s <= t), D on the diagonal;
-      // 32-column groups k above the row quarter q are zero, below it the decay
-      // factorises as alpha_t beta_s (both <= 1), on it exponentials are direct.
-      {
-        const int k = hf, s0 = 32 * k;  // this warp's 32-column group
-        const uint32_t at = (k >> 1) == 0 ? abuf : abuf1;
-        const int kc = 32 * (k & 1);       // column of the group inside its 64-wide block
-        const float c2t = sh.cum2[j][t];
-        if (k > q) {
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), 0u, 0u, 0u, 0u);
-        } else {
-          float cb[32];
-          tmem_ld32(tmem + lane_off + s0, cb);
-          if (k < q) {
-            const float alpha = ex2_approx(c2t - sh.cum2[j][s0 + 31]);
-            const float4 *b4 = reinterpret_cast<const float4 *>(&sh.beta[j][s0]);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const float4 bA = b4[2 * qq], bB = b4[2 * qq + 1];
-              const float bb[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
-              uint32_t w4[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int sl = 8 * qq + 2 * e;
-                w4[e] = pack_half2(cb[sl] * alpha * bb[2 * e], cb[sl + 1] * alpha * bb[2 * e + 1]);
-              }
-              st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
-            }
-          } else if (sh.span_ok[j][k]) {
-            // diagonal group, decay span <= 2^60: alpha_t = exp(cum_t - cum_s0) and
-            // betad_s = exp(cum_s0 - cum_s) dt_s stay within [2^-60, 2^60]
-            const float Dh = sh.Dh[j];
-            const float alpha = ex2_approx(c2t - sh.cum2[j][s0]);
-            const float4 *b4 = reinterpret_cast<const float4 *>(&sh.betad[j][s0]);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const float4 bA = b4[2 * qq], bB = b4[2 * qq + 1];
-              const float bb[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
-              uint32_t w4[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float val[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
-                  float vv = cb[sl] * alpha * bb[2 * e + u];
-                  if (s == t) vv += Dh;
-                  val[u] = (s <= t) ? vv : 0.0f;
-                }
-                w4[e] = pack_half2(val[0], val[1]);
-              }
-              st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
-            }
-          } else {
-            const float Dh = sh.Dh[j];
-            const float4 *c4 = reinterpret_cast<const float4 *>(&sh.cum2[j][s0]);
-            const float4 *d4 = reinterpret_cast<const float4 *>(&sh.dt[j][s0]);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const float4 cA = c4[2 * qq], cB = c4[2 * qq + 1];
-              const float4 dA = d4[2 * qq], dB = d4[2 * qq + 1];
-              const float cc[8] = {cA.x, cA.y, cA.z, cA.w, cB.x, cB.y, cB.z, cB.w};
-              const float dd[8] = {dA.x, dA.y, dA.z, dA.w, dB.x, dB.y, dB.z, dB.w};
-              uint32_t w4[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float val[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  const int sl = 8 * qq + 2 * e + u, s = s0 + sl;
-                  float vv = cb[sl] * ex2_approx(fminf(c2t - cc[2 * e + u], 0.0f)) * dd[2 * e + u];
-                  if (s == t) vv += Dh;
-                  val[u] = (s <= t) ? vv : 0.0f;
-                }
-                w4[e] = pack_half2(val[0], val[1]);
-              }
-              st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
-            }
-          }
-        }
-      }
+        const uint32_t at = base + kAbuf + sl * 32768 + blk * 16384;
+        build_a_group(sh, j, 2 * blk, q, t, at, 0, tmem + lane_off);
+        build_a_group(sh, j, 2 * blk + 1, q, t, at, 32, tmem + lane_off);
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&sh.a_ready[J & 1]);
-        if (j > 0) {  // epilogue of the previous head overlaps this head's MMA
-          const int P1 = J - 1;
-          wait_warp(&sh.mbar_mma[P1 & 1], (uint32_t)((P1 >> 1) & 1));
-          wait_warp(&sh.full_z[P1 % kZStages], (uint32_t)((P1 / kZStages) & 1));
+        mbar_arrive(&sh.a_ready[sl]);
+        if (n >= 1) {  // head j of the previous unit, whose columns this head's MMA takes
+          if (j == 0) wait_inv(n - 1);
           if (!ok) break;
-          tc_fence_after();
-          epilogue1(j - 1, P1 % kZStages);
-          mbar_arrive(&sh.empty_z[P1 % kZStages]);
+          output_head(n - 1, j);
         }
       }
-      if (ok && nh > 0) {
-        const int P1 = J - 1;
-        wait_warp(&sh.mbar_mma[P1 & 1], (uint32_t)((P1 >> 1) & 1));
-        wait_warp(&sh.full_z[P1 % kZStages], (uint32_t)((P1 / kZStages) & 1));
-        tc_fence_after();
-        if (ok) {
-          epilogue1(nh - 1, P1 % kZStages);
-          mbar_arrive(&sh.empty_z[P1 % kZStages]);
-        }
-      }
-      sh.ss[hf][t] = ss_acc;
-      load_rows(n + 1);
+      // this unit's CB columns and decay terms are no longer read
       tc_fence_before();
-      compute_sync();
-      // the unit's C and B tiles and CB columns are no longer read; its last MMA is done
-      if (tid == 0) mbar_arrive(&sh.tiles_free);
-
-      // per-token partial sums of this CTA into part[par][rank][*] of every rank
-      // (asynchronous stores completing bytes on that rank's barrier)
-      if (tid < kQ) sh.mine[tid] = (sh.ss[0][tid] + sh.ss[1][tid]) + (sh.ss[2][tid] + sh.ss[3][tid]);
-      if (!started) {
-        cluster_wait();  // (arrived at the start) every CTA of the cluster is running
-        started = true;
-      }
-      compute_sync();
-      for (int i = tid; i < cs * (kQ / 4); i += kThreads) {
-        const int r = i / (kQ / 4), f = i % (kQ / 4);
-        st_async_v4(cluster_addr(&sh.part[par][rank][4 * f], r),
-                    reinterpret_cast<const float4 *>(sh.mine)[f], cluster_addr(&sh.sums_ready[par], r));
-      }
-      ok = __all_sync(0xffffffffu,
-                      ok && mbar_wait_cluster_bounded(&sh.sums_ready[par], (uint32_t)((n >> 1) & 1))) != 0;
-      if (tid < kQ) {
-        float tot = 0.0f;
-        for (int r = 0; r < cs; ++r) tot += sh.part[par][r][tid];
-        sh.inv[tid] = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
-      }
-      compute_sync();
-      // unit n + 2 uses this parity again; no rank sends it before this CTA has
-      // sent unit n + 1's sums, which happens after this point
-      if (tid == 0 && n + 2 < n_units) mbar_arrive_expect_tx(&sh.sums_ready[par], sum_bytes);
-      tc_fence_after();
-      // normalised bf16 output: each head's [128 t][64 p] tile is written into a
-      // staging tile (128-byte swizzle) and stored by TMA, which drops the rows past
-      // the end of the sequence.  The five staging tiles are the A buffers' blocks
-      // other than the B tile (the next unit's B may be arriving there) and two
-      // tiles of their own.
-      if (ok && sh.ok_flag) {
-        const bool t_valid = c0 + t < pr.L;
-        const float sc = sh.inv[t];
-        for (int j = 0; j < nh; ++j) {
-          const int h = h0 + j;
-          const int slot = j % kYTiles;
-          const uint32_t ybuf = base + y_tile(slot);
-          if (j == kYTiles) {  // the store of head 0 has read its tile
-            if (tid == 0) bulk_wait_read_le(kYTiles - 1);
-            compute_sync();
+      if (ok) mbar_arrive(&sh.cb_free);
+      ok = group_all(1, ok);
+    }
+    if (ok && nh > 0 && n_units > 0) {  // the last unit's output
+      wait_inv(n_units - 1);
+      for (int j = 0; ok && j < nh; ++j) output_head(n_units - 1, j);
+    }
+  } else {
+    // ---------------- epilogue
+    const int q = warp & 3, eh = (warp - 8) >> 2, t = 32 * q + lane, gt = tid - 256;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    bool ok = true;
+    int J = 0;
+    for (int n = 0; ok && n < n_units; ++n) {
+      int64_t bi;
+      int c, g;
+      out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+      const int h0 = g * hpg + lh0;
+      const int par = n & 1;
+      float ss = 0.0f;
+      // cum_t of head j for this thread's token (the next head's is loaded while this
+      // one is worked on)
+      auto head_cum = [&](int j) -> float {
+        const int64_t row = (bi * a.nch + c) * pr.H + h0 + j;
+        const float *cp = a.cum + row * kQ + t;
+        return M2_OK(cp, 4, a.sp.cum, &g_tc_errors) ? *cp : 0.0f;
+      };
+      float cum_n = nh > 0 ? head_cum(0) : 0.0f;
+      for (int j = 0; j < nh; ++j, ++J) {
+        const int sl = J & 1;
+        const float ec = ex2_approx(cum_n * kLog2e);  // exp(cum_t)
+        if (j + 1 < nh) cum_n = head_cum(j + 1);
+        // the scales 2^s of H_c's rows p (pairs) that this thread's 32 columns use
+        const float4 *sp4 = reinterpret_cast<const float4 *>(
+            a.hsc + ((bi * a.nch + c) * pr.H + h0 + j) * 32 + 16 * eh);
+        float4 sc4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          sc4[i] = M2_OK(sp4 + i, 16, a.sp.hsc, &g_tc_errors) ? sp4[i]
+                                                            : make_float4(1.f, 1.f, 1.f, 1.f);
+        ok = ok && mbar_wait_bounded(&sh.mma_done[sl], (uint32_t)((J >> 1) & 1), &g_tc_errors) &&
+             mbar_wait_bounded(&sh.full_z[sl], (uint32_t)((J >> 1) & 1), &g_tc_errors);
+        ok = __all_sync(0xffffffffu, ok) != 0;
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t ycol = tmem + lane_off + kTmemY + 64 * j + 32 * eh;
+        const uint32_t zt = base + kZt + sl * 16384;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v[16], w[16];
+          tmem_ld16(ycol + 16 * hh, v);
+          tmem_ld16(tmem + lane_off + kTmemT + 32 * eh + 16 * hh, w);
+          if (hh == 1) {
+            tc_fence_before();
+            mbar_arrive(&sh.t_free);  // the C H_c^T columns may take the next head's product
           }
-          float v[16];
-          tmem_ld16(tmem + lane_off + 128 + 64 * j + 16 * hf, v);
-          const float4 *nw4 = reinterpret_cast<const float4 *>(&sh.nw[j][16 * hf]);
-          if (pr.nbg && t_valid) {
-            const int64_t row = bi * pr.L + c0 + t;
-            const uint4 *zp =
-                reinterpret_cast<const uint4 *>(a.z + row * a.ld_z + (int64_t)h * kHP + 16 * hf);
+          const float scp[8] = {sc4[2 * hh].x, sc4[2 * hh].y, sc4[2 * hh].z, sc4[2 * hh].w,
+                                sc4[2 * hh + 1].x, sc4[2 * hh + 1].y, sc4[2 * hh + 1].z,
+                                sc4[2 * hh + 1].w};
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = fmaf(ec * scp[i >> 1], w[i], v[i]);
+          if (!pr.nbg) {
 #pragma unroll
             for (int qq = 0; qq < 2; ++qq) {
-              const uint4 raw = __ldg(zp + qq);
+              const uint4 raw = ld_shared_v4(zt + sw128_chunk(t, 32 * eh + 16 * hh + 8 * qq));
               const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
@@ -1270,34 +1486,39 @@ __global__ void __launch_bounds__(kWsThreads, 1)
             }
           }
 #pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            uint32_t o[4];
-            const float4 wA = nw4[2 * qq], wB = nw4[2 * qq + 1];
-            const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = 8 * qq + 2 * e;
-              const __nv_bfloat162 b2 =
-                  __floats2bfloat162_rn(v[i] * sc * ww[2 * e], v[i + 1] * sc * ww[2 * e + 1]);
-              o[e] = *reinterpret_cast<const uint32_t *>(&b2);
-            }
-            st_shared_v4(ybuf + sw128_chunk(t, 16 * hf + 8 * qq), o[0], o[1], o[2], o[3]);
-          }
-          fence_proxy_async_smem();
-          compute_sync();  // head j's tile is complete: store it while the next one is built
-          if (tid == 0) {
-            tma_store_3d(&maps.y, ybuf, h * kHP, (int)c0, (int)bi);
-            bulk_commit();
-          }
+          for (int i = 0; i < 16; ++i) ss = fmaf(v[i], v[i], ss);
+          tmem_st16(ycol + 16 * hh, v);
         }
+        mbar_arrive(&sh.empty_z[sl]);
       }
-      // the y columns of TMEM are read before the next unit's MMAs; its A-builds
-      // wait for the stores to have read the staging tiles
-      tc_fence_before();
-      compute_sync();
+      // per-token sums of this CTA into part[par][rank][*] of every rank
+      sh.half_ss[eh][t] = ss;
+      ok = group_all(2, ok);
+      if (!ok) break;
+      if (gt < kQ) sh.mine[gt] = sh.half_ss[0][gt] + sh.half_ss[1][gt];
+      if (!started) {
+        cluster_wait();  // (arrived at the start) every CTA of the cluster is running
+        started = true;
+      }
+      group_sync(2);
+      for (int i = gt; i < cs * (kQ / 4); i += kGroupThreads) {
+        const int r = i / (kQ / 4), f = i % (kQ / 4);
+        st_async_v4(cluster_addr(&sh.part[par][rank][4 * f], r),
+                    reinterpret_cast<const float4 *>(sh.mine)[f], cluster_addr(&sh.sums_ready[par], r));
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster_bounded(&sh.sums_ready[par], (uint32_t)((n >> 1) & 1))) != 0;
+      float tot = 0.0f;
+      for (int r = 0; r < cs; ++r) tot += sh.part[par][r][t];
+      const float inv = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
+      ok = group_all(2, ok);
+      // unit n + 2 uses this parity again; no rank sends it before this CTA has
+      // sent unit n + 1's sums, which happens after this point
+      if (gt == 0 && n + 2 < n_units) mbar_arrive_expect_tx(&sh.sums_ready[par], sum_bytes);
+      if (!ok) break;
+      // the per-token norm scales to the operand warps, which write the output
+      if (eh == 0) sh.inv[par][t] = inv;
+      mbar_arrive(&sh.inv_ready);
     }
-    if (tid == 0) bulk_wait_read_all();  // the last unit's stores have read their tiles
-    if (!ok) sh.ok_flag = 0;
   }
   // every thread: the cluster's start barrier (if not waited for yet), then one
   // more: no CTA exits while another may still store into its shared memory
@@ -1344,7 +1565,7 @@ void out_choose(int hpg, int64_t units, int *cs, int *hpc, int *ncl) {
 }
 
 struct TcWorkspace {
-  float *S, *cum_end, *cum, *dtv;
+  float *S, *cum_end, *cum, *dtv, *hsc, *cbd;
   __half *Hc, *u;
 };
 
@@ -1363,6 +1584,10 @@ TcWorkspace tc_carve(const Problem &pr, char *base) {
   off += align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256);
   w.Hc = reinterpret_cast<__half *>(base + off);
   off += align_up(st * 2, 256);
+  w.hsc = reinterpret_cast<float *>(base + off);
+  off += align_up((size_t)pr.batch * nch * pr.H * 32 * 4, 256);
+  w.cbd = reinterpret_cast<float *>(base + off);
+  off += align_up((size_t)pr.batch * pr.G * nch * kQ * 4, 256);
   w.u = reinterpret_cast<__half *>(base + off);
   return w;
 }
@@ -1461,6 +1686,8 @@ size_t prefill_tc_workspace(const Problem &pr) {
   const size_t st = (size_t)pr.batch * nch * pr.H * kHP * kNS;
   return align_up(st * 4, 256) + align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
          2 * align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256) + align_up(st * 2, 256) +
+         align_up((size_t)pr.batch * nch * pr.H * 32 * 4, 256) +
+         align_up((size_t)pr.batch * pr.G * nch * kQ * 4, 256) +
          align_up((size_t)pr.batch * pr.L * pr.conv_dim * 2, 256);
 }
 
@@ -1489,6 +1716,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.dt_raw = static_cast<const __nv_bfloat16 *>(pa.dt_raw);
   a.ld_dt = pa.ld_dt;
   a.y = static_cast<__nv_bfloat16 *>(pa.y);
+  a.y32 = (reinterpret_cast<uintptr_t>(pa.y) % 32) == 0;
   a.conv_in = static_cast<const __nv_bfloat16 *>(pa.conv_state);
   a.ssm_state = pa.ssm_state;
   a.states_in = pa.states_in;
@@ -1499,7 +1727,33 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.cum = w.cum;
   a.dtv = w.dtv;
   a.Hc = w.Hc;
+  a.hsc = w.hsc;
+  a.cbd = w.cbd;
   a.u = w.u;
+  {
+    const int64_t bl = pr.batch * pr.L, nq = a.nch;
+    const size_t st1 = (size_t)pr.batch * nq * pr.H * kHP * kNS;
+    a.sp.xbc = span_of(a.xBC, (size_t)((bl - 1) * pa.ld_xbc + pr.conv_dim) * 2);
+    a.sp.z = span_of(a.z, (size_t)((bl - 1) * pa.ld_z + pr.d_inner) * 2);
+    a.sp.dt = span_of(a.dt_raw, (size_t)((bl - 1) * pa.ld_dt + pr.H) * 2);
+    a.sp.y = span_of(a.y, (size_t)bl * pr.d_inner * 2);
+    a.sp.conv = span_of(pa.conv_state, (size_t)pr.batch * pr.conv_dim * 4 * 2);
+    a.sp.ssm = span_of(a.ssm_state, (size_t)pr.batch * pr.H * kHP * kNS * 4);
+    a.sp.S = span_of(a.S, st1 * 4);
+    a.sp.cum_end = span_of(a.cum_end, (size_t)pr.batch * nq * pr.H * 4);
+    a.sp.cum = span_of(a.cum, (size_t)pr.batch * nq * pr.H * kQ * 4);
+    a.sp.dtv = span_of(a.dtv, (size_t)pr.batch * nq * pr.H * kQ * 4);
+    a.sp.Hc = span_of(a.Hc, st1 * 2);
+    a.sp.hsc = span_of(a.hsc, (size_t)pr.batch * nq * pr.H * 32 * 4);
+    a.sp.cbd = span_of(a.cbd, (size_t)pr.batch * pr.G * nq * kQ * 4);
+    a.sp.u = span_of(a.u, (size_t)bl * pr.conv_dim * 2);
+    a.sp.conv_w = span_of(a.prm.conv_w, (size_t)pr.conv_dim * 4 * 4);
+    a.sp.conv_b = span_of(a.prm.conv_b, (size_t)pr.conv_dim * 4);
+    a.sp.dt_bias = span_of(a.prm.dt_bias, (size_t)pr.H * 4);
+    a.sp.A = span_of(a.prm.A, (size_t)pr.H * 4);
+    a.sp.D = span_of(a.prm.D, (size_t)pr.H * 4);
+    a.sp.norm_w = span_of(a.prm.norm_w, (size_t)pr.d_inner * 4);
+  }
   const int hpg = pr.heads_per_group();
   cudaError_t e;
   if (first_use_in_context(0)) {  // attributes belong to the context: set them once in each
@@ -1532,7 +1786,22 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   stage_mark(st, 1);
   dim3 g2((unsigned)(kPassBlocks + ceil_div(pr.conv_dim, 256)), (unsigned)pr.H,
           (unsigned)pr.batch);
-  tc_state_pass_kernel<<<g2, 256, 0, st>>>(a, static_cast<__nv_bfloat16 *>(pa.conv_state));
+  {
+    // programmatic dependent launches: the state pass and the output kernel are
+    // scheduled while their predecessor drains and wait for it on the device
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = g2;
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, tc_state_pass_kernel, a,
+                           static_cast<__nv_bfloat16 *>(pa.conv_state));
+    if (e != cudaSuccess) return e;
+  }
   stage_mark(st, 2);
   {
     cudaLaunchConfig_t cfg = {};
@@ -1540,13 +1809,15 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     cfg.blockDim = dim3(kWsThreads, 1, 1);
     cfg.dynamicSmemBytes = kK3Smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     OutMaps maps;
     {
       const uint64_t du[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
@@ -1557,12 +1828,9 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
       const uint64_t dh[2] = {(uint64_t)kNS, (uint64_t)pr.batch * a.nch * pr.H * kHP};
       const uint64_t shc[1] = {(uint64_t)kNS * 2};
       const uint32_t bh[2] = {64, 64};
-      const uint64_t dy[3] = {(uint64_t)pr.d_inner, (uint64_t)pr.L, (uint64_t)pr.batch};
-      const uint64_t sy[2] = {(uint64_t)pr.d_inner * 2, (uint64_t)pr.L * pr.d_inner * 2};
       if (!make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.u, 3, du, su, bu) ||
           !make_map(&maps.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.z, 3, dz, sz, bu) ||
-          !make_map(&maps.hc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Hc, 2, dh, shc, bh) ||
-          !make_map(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, 3, dy, sy, bu))
+          !make_map(&maps.hc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Hc, 2, dh, shc, bh))
         return cudaErrorInvalidValue;
     }
     e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps, ncl);

@@ -160,12 +160,18 @@ __host__ __device__ inline StepLayout step_layout(int stages, int hpc, int P, in
   return L;
 }
 
+// Byte ranges of the decode step's buffers (checked build, see M2_OK).
+struct StepSpans {
+  Span xbc, z, dt, y, conv, ssm, conv_w, conv_b, norm_w, dt_bias, A, D;
+};
+
 template <typename T, int N>
 __global__ void __launch_bounds__(kStepBlock, 2)
     ssd_step_kernel(Problem pr, mamba2_params prm, const T *__restrict__ xBC, int64_t ld_x,
                     const T *__restrict__ z, int64_t ld_z, const T *__restrict__ dt_raw,
                     int64_t ld_dt, T *__restrict__ y, T *__restrict__ conv_state,
-                    float *__restrict__ ssm, int hpc, int stages, int nclusters) {
+                    float *__restrict__ ssm, int hpc, int stages, int nclusters,
+                    const StepSpans sp) {
   if (test_stall(&g_step_stall, &g_step_errors)) return;  // every CTA alike (test aid)
   int cs, rank;
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs));
@@ -224,15 +230,22 @@ __global__ void __launch_bounds__(kStepBlock, 2)
   // row-independent parameters of the CTA's channels and heads
   for (int i = threadIdx.x; i < C + BC; i += blockDim.x) {
     const int64_t ch = i < C ? (int64_t)h0 * P + i : pr.d_inner + (i - C);
+    const float4 *wp = reinterpret_cast<const float4 *>(prm.conv_w) + ch;
     reinterpret_cast<float4 *>(smem_raw + Lo.cw)[i] =
-        __ldg(reinterpret_cast<const float4 *>(prm.conv_w) + ch);
-    reinterpret_cast<float *>(smem_raw + Lo.cb)[i] = __ldg(prm.conv_b + ch);
-    if (i < C) reinterpret_cast<float *>(smem_raw + Lo.nw)[i] = __ldg(prm.norm_w + ch);
+        M2_OK(wp, 16, sp.conv_w, &g_step_errors) ? __ldg(wp) : make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float *>(smem_raw + Lo.cb)[i] =
+        M2_OK(prm.conv_b + ch, 4, sp.conv_b, &g_step_errors) ? __ldg(prm.conv_b + ch) : 0.0f;
+    if (i < C)
+      reinterpret_cast<float *>(smem_raw + Lo.nw)[i] =
+          M2_OK(prm.norm_w + ch, 4, sp.norm_w, &g_step_errors) ? __ldg(prm.norm_w + ch) : 0.0f;
   }
   for (int i = threadIdx.x; i < hpc; i += blockDim.x) {
-    reinterpret_cast<float *>(smem_raw + Lo.dtb)[i] = prm.dt_bias[h0 + i];
-    reinterpret_cast<float *>(smem_raw + Lo.Ah)[i] = prm.A[h0 + i];
-    reinterpret_cast<float *>(smem_raw + Lo.Dh)[i] = prm.D[h0 + i];
+    reinterpret_cast<float *>(smem_raw + Lo.dtb)[i] =
+        M2_OK(prm.dt_bias + h0 + i, 4, sp.dt_bias, &g_step_errors) ? prm.dt_bias[h0 + i] : 0.0f;
+    reinterpret_cast<float *>(smem_raw + Lo.Ah)[i] =
+        M2_OK(prm.A + h0 + i, 4, sp.A, &g_step_errors) ? prm.A[h0 + i] : 0.0f;
+    reinterpret_cast<float *>(smem_raw + Lo.Dh)[i] =
+        M2_OK(prm.D + h0 + i, 4, sp.D, &g_step_errors) ? prm.D[h0 + i] : 0.0f;
   }
   __syncthreads();
   // every CTA of the cluster runs (and has initialised its barriers) before any
@@ -249,9 +262,13 @@ __global__ void __launch_bounds__(kStepBlock, 2)
             !mbar_wait_bounded(&empty[s], (uint32_t)((np / stages - 1) & 1), &g_step_errors))
           break;
         const int64_t r = cid + (np / hpc) * nclusters;
-        mbar_arrive_expect_tx(&full[s], head_bytes);
-        bulk_g2s(sbuf + s * head_floats, ssm + (r * H + h0 + (int)(np % hpc)) * (int64_t)head_floats,
-                 head_bytes, &full[s]);
+        const float *src = ssm + (r * H + h0 + (int)(np % hpc)) * (int64_t)head_floats;
+        if (M2_OK_BULK(src, head_bytes, sp.ssm, &g_step_errors)) {
+          mbar_arrive_expect_tx(&full[s], head_bytes);
+          bulk_g2s(sbuf + s * head_floats, src, head_bytes, &full[s]);
+        } else {
+          mbar_arrive(&full[s]);  // nothing copied: the stage completes without bytes
+        }
       }
       // no copy may be in flight when the CTA exits (each stage's last copy)
       for (int64_t kk = std::max<int64_t>(0, np - stages); kk < np; ++kk)
@@ -288,7 +305,8 @@ __global__ void __launch_bounds__(kStepBlock, 2)
       else if (i < n2) src = reinterpret_cast<const char *>(xBC + bi * ld_x + (int64_t)h0 * P) + 16 * (i - n1);
       else if (i < n3) src = reinterpret_cast<const char *>(xBC + bi * ld_x + pr.d_inner) + 16 * (i - n2);
       else src = reinterpret_cast<const char *>(z + bi * ld_z + (int64_t)h0 * P) + 16 * (i - n3);
-      cp_async16(pb + 16 * i, src);
+      const Span &spn = i < n1 ? sp.conv : (i < n3 ? sp.xbc : sp.z);
+      if (M2_OK(src, 16, spn, &g_step_errors)) cp_async16(pb + 16 * i, src);
     }
     cp_async_commit();
   };
@@ -314,17 +332,23 @@ __global__ void __launch_bounds__(kStepBlock, 2)
     for (int c = tid; c < C; c += kStepThreads) {
       float o = ysr[c] * inv[(h0 + c / P) / hpg] * nw[c];
       if (pr.nbg) o *= silu_fast(to_f(zk[par * C + c]));
-      yr[c] = from_f<T>(o);
+      if (M2_OK(yr + c, (unsigned)sizeof(T), sp.y, &g_step_errors)) yr[c] = from_f<T>(o);
     }
     T *csr = conv_state + bi * pr.conv_dim * 4;
     const T *bn = bcn + par * 4 * BC;
     for (int jb = rank + cs * tid; jb < BC; jb += cs * kStepThreads)
-      store4(csr + (pr.d_inner + jb) * 4, bn[jb * 4], bn[jb * 4 + 1], bn[jb * 4 + 2], bn[jb * 4 + 3]);
+      if (M2_OK(csr + (pr.d_inner + jb) * 4, 4 * (unsigned)sizeof(T), sp.conv, &g_step_errors))
+        store4(csr + (pr.d_inner + jb) * 4, bn[jb * 4], bn[jb * 4 + 1], bn[jb * 4 + 2],
+               bn[jb * 4 + 3]);
   };
 
   if (rows_mine > 0) {
     prefetch(0);
-    if (tid < hpc) dtr[tid] = to_f(dt_raw[(int64_t)cid * ld_dt + h0 + tid]);
+    if (tid < hpc)
+      dtr[tid] = M2_OK(dt_raw + (int64_t)cid * ld_dt + h0 + tid, (unsigned)sizeof(T), sp.dt,
+                       &g_step_errors)
+                     ? to_f(dt_raw[(int64_t)cid * ld_dt + h0 + tid])
+                     : 0.0f;
   }
   for (int64_t rr = 0; rr < rows_mine; ++rr) {
     const int64_t bi = cid + rr * nclusters;
@@ -340,7 +364,8 @@ __global__ void __launch_bounds__(kStepBlock, 2)
       const float w[4] = {w4.x, w4.y, w4.z, w4.w};
       if (i < C) {
         const T a0 = pcx[i * 4 + 1], a1 = pcx[i * 4 + 2], a2 = pcx[i * 4 + 3], a3 = px[i];
-        store4(csr + ((int64_t)h0 * P + i) * 4, a0, a1, a2, a3);
+        if (M2_OK(csr + ((int64_t)h0 * P + i) * 4, 4 * (unsigned)sizeof(T), sp.conv, &g_step_errors))
+          store4(csr + ((int64_t)h0 * P + i) * 4, a0, a1, a2, a3);
         ux[i] = silu_fast(conv4(w, cb[i], a0, a1, a2, a3));
         if (pr.nbg) zk[par * C + i] = pz[i];
       } else {
@@ -366,7 +391,11 @@ __global__ void __launch_bounds__(kStepBlock, 2)
     float dtn = 0.0f;
     if (rr + 1 < rows_mine) {
       prefetch(rr + 1);
-      if (tid < hpc) dtn = to_f(dt_raw[(bi + nclusters) * ld_dt + h0 + tid]);
+      if (tid < hpc)
+        dtn = M2_OK(dt_raw + (bi + nclusters) * ld_dt + h0 + tid, (unsigned)sizeof(T), sp.dt,
+                    &g_step_errors)
+                  ? to_f(dt_raw[(bi + nclusters) * ld_dt + h0 + tid])
+                  : 0.0f;
     }
     float *st_row = ssm + (bi * H + h0) * (int64_t)head_floats;
     float *ysr = ys + par * C;
@@ -397,7 +426,7 @@ __global__ void __launch_bounds__(kStepBlock, 2)
             v.y = fmaf(dA, v.y, xdt * b.y);
             v.z = fmaf(dA, v.z, xdt * b.z);
             v.w = fmaf(dA, v.w, xdt * b.w);
-            dst[idx] = v;
+            if (M2_OK(dst + idx, 16, sp.ssm, &g_step_errors)) dst[idx] = v;
             pt[i] = fmaf(v.x, cc.x, fmaf(v.y, cc.y, fmaf(v.z, cc.z, v.w * cc.w)));
             xs[i] = xv;
           }
@@ -418,7 +447,7 @@ __global__ void __launch_bounds__(kStepBlock, 2)
           v.y = fmaf(dA, v.y, xdt * b.y);
           v.z = fmaf(dA, v.z, xdt * b.z);
           v.w = fmaf(dA, v.w, xdt * b.w);
-          dst[idx] = v;
+          if (M2_OK(dst + idx, 16, sp.ssm, &g_step_errors)) dst[idx] = v;
           float t = fmaf(v.x, cc.x, fmaf(v.y, cc.y, fmaf(v.z, cc.z, v.w * cc.w)));
 #pragma unroll
           for (int o = NQ / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
@@ -546,10 +575,26 @@ cudaError_t run(const StepArgs &a) {
   const int nclusters = (int)std::max<int64_t>(1, (pr.batch + rows_per - 1) / rows_per);
   cfg.gridDim = dim3((unsigned)cs, (unsigned)nclusters, 1);
   stage_mark(a.stream, 0);
+  StepSpans sp;
+  {
+    const size_t ts = sizeof(T), b = (size_t)pr.batch;
+    sp.xbc = span_of(a.xBC, ((b - 1) * a.ld_xbc + pr.conv_dim) * ts);
+    sp.z = span_of(a.z, ((b - 1) * a.ld_z + pr.d_inner) * ts);
+    sp.dt = span_of(a.dt_raw, ((b - 1) * a.ld_dt + pr.H) * ts);
+    sp.y = span_of(a.y, b * pr.d_inner * ts);
+    sp.conv = span_of(a.conv_state, b * pr.conv_dim * 4 * ts);
+    sp.ssm = span_of(a.ssm_state, b * pr.H * pr.P * pr.N * 4);
+    sp.conv_w = span_of(a.prm.conv_w, (size_t)pr.conv_dim * 16);
+    sp.conv_b = span_of(a.prm.conv_b, (size_t)pr.conv_dim * 4);
+    sp.norm_w = span_of(a.prm.norm_w, (size_t)pr.d_inner * 4);
+    sp.dt_bias = span_of(a.prm.dt_bias, (size_t)pr.H * 4);
+    sp.A = span_of(a.prm.A, (size_t)pr.H * 4);
+    sp.D = span_of(a.prm.D, (size_t)pr.H * 4);
+  }
   e = cudaLaunchKernelEx(&cfg, ssd_step_kernel<T, N>, pr, a.prm, static_cast<const T *>(a.xBC),
                          a.ld_xbc, static_cast<const T *>(a.z), a.ld_z,
                          static_cast<const T *>(a.dt_raw), a.ld_dt, static_cast<T *>(a.y),
-                         static_cast<T *>(a.conv_state), a.ssm_state, hpc, stages, nclusters);
+                         static_cast<T *>(a.conv_state), a.ssm_state, hpc, stages, nclusters, sp);
   stage_mark(a.stream, 1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

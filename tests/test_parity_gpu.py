@@ -46,6 +46,10 @@ def test_tiny_f32_config():
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=17),
     case("zamba2_2p7b_prefill", batch=2, seqlen=256, nheads=32, ngroups=2),
     case("zamba2_2p7b_prefill", batch=3, seqlen=1000, nheads=20),
+    # 80 heads (16-CTA output clusters, several (chunk, group) units per cluster;
+    # several chunk-state items per CTA, crossing (row, chunk) keys)
+    case("zamba2_2p7b_prefill", batch=1, seqlen=1100, nheads=80),
+    case("zamba2_2p7b_prefill", batch=2, seqlen=640, nheads=64),
     case("zamba2_2p7b_prefill", batch=1, seqlen=257, nheads=4, headdim=32, dstate=128),
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=4, headdim=16, dstate=32),
     case("tiny_f32", batch=2, seqlen=517, nheads=6, ngroups=2, headdim=64, dstate=64,
@@ -139,6 +143,20 @@ def test_tc_large_dt(bias):
                       states_in=True)
     ref = oracle_prefill(cfg, inp, params, states=st)
     compare_prefill(cfg, got, ref)
+
+
+@pytest.mark.parametrize("mag", [1e5, 3e7])
+def test_tc_large_carried_state(mag):
+    # a carried SSM state far beyond the fp16 range: the output kernel's operand
+    # holds each (chunk, head, 16-column) block of the state divided by a power
+    # of two, so y and the final state still match the oracle
+    cfg, params, inp, st = _tc_case(24)
+    st = dict(st, ssm_state=st["ssm_state"] * (mag / 0.1))
+    got = gpu_prefill(cfg, inp, params, states={k: v.clone() for k, v in st.items()},
+                      states_in=True)
+    ref = oracle_prefill(cfg, inp, params, states=st)
+    compare_prefill(cfg, got, ref)
+    assert m2.device_errors() == 0
 
 
 def test_without_state_buffers():
