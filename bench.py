@@ -304,14 +304,17 @@ def measure_prefill(name, args, dev, stream, seed, world, peaks, peak_src, m2, W
 
     W_ = max(3, args.warmup if warmup is None else warmup)
     stage_ms = [0.0] * nst
+    n_stage = 0
     for i in range(W_):
         if flush is not None:
             flush.fill_(i & 255)
         evs = [new_event() for _ in range(nst + 1)]
         call(sets[i % rotate], [e.cuda_event for e in evs])
         torch.cuda.synchronize(dev)
-        for j in range(nst):
-            stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
+        if i >= min(2, W_ - 1):  # the first calls pay one-time costs: not counted
+            n_stage += 1
+            for j in range(nst):
+                stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
     dom = max(range(nst), key=lambda j: stage_ms[j])
 
     K = args.steps if steps is None else steps
@@ -375,7 +378,7 @@ def measure_prefill(name, args, dev, stream, seed, world, peaks, peak_src, m2, W
                           "roofline_ms": t_roof * 1e3,
                           "achieved_gbs": path_bytes / (ms * 1e-3) / 1e9,
                           "frac": t_roof * 1e3 / ms, "peak_source": peak_src},
-        "stages_ms_warmup_avg": {n: stage_ms[j] / W_ for j, n in enumerate(stage_names)},
+        "stages_ms_warmup_avg": {n: stage_ms[j] / n_stage for j, n in enumerate(stage_names)},
         "gpu_launches": K * nst,
     }
     del sets, flush

@@ -191,6 +191,7 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
                                        int64_t dt_row_stride, void *y, void *conv_state,
                                        float *ssm_state, int32_t states_in, void *workspace,
                                        size_t workspace_bytes, void *stream) {
+  NvtxRange range("mamba2_conv_ssd_prefill");
   DisarmOnExit disarm;
   Problem pr;
   int st = make_problem(dims, true, &pr);
@@ -251,6 +252,7 @@ MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *par
                                const void *xBC, int64_t xBC_row_stride, const void *z,
                                int64_t z_row_stride, const void *dt_raw, int64_t dt_row_stride,
                                void *y, void *conv_state, float *ssm_state, void *stream) {
+  NvtxRange range("mamba2_ssd_step");
   DisarmOnExit disarm;
   Problem pr;
   int st = make_problem(dims, false, &pr);

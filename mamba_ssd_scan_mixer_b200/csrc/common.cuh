@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "mamba2ssd.h"
@@ -108,6 +109,16 @@ inline void stage_mark(cudaStream_t s, int i) {
   if (i < g_stage_events.n && g_stage_events.ev[i] != nullptr)
     cudaEventRecord(g_stage_events.ev[i], s);
 }
+
+// NVTX range for the lifetime of the object (header-only NVTX 3: without a
+// profiler attached the calls return at once).  Each entry point and each
+// kernel stage it enqueues is named, so a timeline shows the call structure.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Names of the kernel stages each path enqueues, in order.
 extern const char *const kPrefillSimtStages[];

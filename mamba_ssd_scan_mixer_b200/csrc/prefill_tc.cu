@@ -148,6 +148,20 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 
+// Asynchronous global -> shared copies of 16 and 4 bytes (no registers held),
+// and an arrival on an mbarrier once all of this thread's earlier copies have
+// landed (.noinc: the barrier's expected count includes these arrivals).
+__device__ __forceinline__ void cp_async_ca16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_ca4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
                                             int c2, uint64_t *bar) {
   asm volatile(
@@ -233,79 +247,41 @@ struct K1Maps {
 // conv1d + SiLU of the 8 channels in 16-byte column `cg` of a raw tile, for
 // output tokens at tile rows s0+3 .. s0+6 (inputs: rows s0 .. s0+6); taps and
 // bias of the tile's 64 channels in shared memory, channel 8 g + i at [i][g]
-// (wt[8][8] float4, bs[8][8]) so that neighbouring groups read neighbouring words,
-// stored halved: the sum is then h = pre / 2 exactly, and silu(pre) = h + h tanh(h).
+// (wt[8][8] float4, bs[8][8]) so that neighbouring groups read neighbouring words.
+// With h = pre / 2 (exact), silu(pre) = h + h tanh(h).
+// The 7 rows stay packed (2 bf16 per register) and are widened one channel at a
+// time, so that only 28 registers of inputs and one channel's taps are live.
 __device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float4 *wt,
                                              const float *bs, float (&out)[4][8]) {
-  float w[8][4], bias[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 wv = wt[i * 8 + cg];
-    w[i][0] = wv.x;
-    w[i][1] = wv.y;
-    w[i][2] = wv.z;
-    w[i][3] = wv.w;
-    bias[i] = bs[i * 8 + cg];
-  }
-  float rows[7][8];
+  uint32_t raw[7][4];
 #pragma unroll
   for (int r = 0; r < 7; ++r) {
     const int R = s0 + r;
-    const uint4 raw = ld_shared_v4(tile + R * 128 + (((cg ^ R) & 7) << 4));
-    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h2[i]);
-      rows[r][2 * i] = f.x;
-      rows[r][2 * i + 1] = f.y;
-    }
+    const uint4 q = ld_shared_v4(tile + R * 128 + (((cg ^ R) & 7) << 4));
+    raw[r][0] = q.x;
+    raw[r][1] = q.y;
+    raw[r][2] = q.z;
+    raw[r][3] = q.w;
   }
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
+  for (int i = 0; i < 8; ++i) {
+    const float4 wv = wt[i * 8 + cg];
+    const float bias = bs[i * 8 + cg];
+    float col[7];  // channel i of the rows: bf16 -> fp32 is a 16-bit shift
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float h = bias[i] + w[i][0] * rows[k][i] + w[i][1] * rows[k + 1][i] +
-                      w[i][2] * rows[k + 2][i] + w[i][3] * rows[k + 3][i];
+    for (int r = 0; r < 7; ++r)
+      col[r] = __uint_as_float((i & 1) ? (raw[r][i >> 1] & 0xFFFF0000u) : (raw[r][i >> 1] << 16));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float h = 0.5f * (bias + wv.x * col[k] + wv.y * col[k + 1] + wv.z * col[k + 2] +
+                              wv.w * col[k + 3]);
       out[k][i] = fmaf(h, tanh_approx(h), h);
     }
-}
-
-// As conv8x4_smem for the same 8 channels x 4 tokens, but each output is folded
-// at once into d4[k] += out[k][i] * v[k][i] (the dot product over the 8 channels
-// of token k) and the taps and rows are read per token, so that only `v` stays
-// live across the call.
-__device__ __forceinline__ void conv8x4_dot(uint32_t tile, int s0, int cg, const float4 *wt,
-                                            const float *bs, const float (&v)[4][8],
-                                            float (&d4)[4]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float rows[4][8];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int R = s0 + k + r;
-      const uint4 raw = ld_shared_v4(tile + R * 128 + (((cg ^ R) & 7) << 4));
-      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(h2[i]);
-        rows[r][2 * i] = f.x;
-        rows[r][2 * i + 1] = f.y;
-      }
-    }
-    float acc = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 wv = wt[i * 8 + cg];
-      const float h = bs[i * 8 + cg] + wv.x * rows[0][i] + wv.y * rows[1][i] + wv.z * rows[2][i] +
-                      wv.w * rows[3][i];
-      acc = fmaf(v[k][i], fmaf(h, tanh_approx(h), h), acc);
-    }
-    d4[k] = acc;
   }
 }
 
 struct K1Item {
-  int64_t bi;
+  int bi;  // row (every index of the item fits in 32 bits)
   int c, g, pair;
   unsigned key;  // (row, chunk, group) index
   bool isC;
@@ -322,7 +298,7 @@ __device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs,
   K1Item w;
   w.key = key;
   w.g = (int)(key - bc * (unsigned)pr.G);
-  w.bi = (int64_t)(bc / (unsigned)nch);
+  w.bi = (int)(bc / (unsigned)nch);
   w.c = (int)(bc - (unsigned)w.bi * (unsigned)nch);
   w.isC = r == pairs;
   w.pair = w.isC ? 0 : r;
@@ -338,7 +314,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   __shared__ float4 wts[2][3][64];                // [stage][slot x_A, x_B, B/C][channel] conv taps
   __shared__ __align__(16) float bss[2][3][64];   // [stage][slot][channel] conv bias
   __shared__ uint64_t full[2], empty[2], bc_empty[2], ops_ready, mma_done[2], tmem_free[2],
-      mma_final, halo_bar[2], cbd_bar;
+      mma_final, halo_bar[2], cbd_bar, park_bar;
   __shared__ __align__(16) float cbd_s[2][kQ];  // C-item parity: per-token partials of channel groups 4-7
   __shared__ uint32_t tmem_holder;
   const Problem &pr = a.pr;
@@ -354,7 +330,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   if (warp == 0) tmem_alloc(&tmem_holder, 128);
   if (tid == 0) {
     for (int k = 0; k < 2; ++k) {
-      mbar_init(&full[k], 2);          // the tiles' transaction bytes + the producer's weights
+      // the tiles' transaction bytes + the producer's weights + each producer lane's tap copies
+      mbar_init(&full[k], 2 + 32);
       mbar_init(&empty[k], kThreads);  // every compute thread has read the stage's x tiles
       mbar_init(&bc_empty[k], 256);    // warps 0-7 have read the B/C tile
       mbar_init(&mma_done[k], 1);      // tcgen05.commit of a pair item's MMAs
@@ -363,7 +340,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     mbar_init(&ops_ready, kThreads);  // operands of a pair item written
     mbar_init(&mma_final, 1);
     for (int k = 0; k < 2; ++k) mbar_init(&halo_bar[k], 1);  // a halo item's tiles landed
-    mbar_init(&cbd_bar, 128);  // warps 4-7 have written a C item's diagonal partials
+    mbar_init(&cbd_bar, 128);   // warps 12-15 have written a C item's diagonal partials
+    mbar_init(&park_bar, 256);  // warps 0-7 have parked a C item's convolved C values
     fence_mbar_init();
   }
   tc_fence_before();
@@ -391,30 +369,20 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       const bool hasB = 2 * w.pair + 1 < hpg;
       // everything that needs no shared memory first, while the stage may still be
       // in use: the item's global loads (one round trip: dt of both heads for this
-      // lane's 4 tokens, their dt_bias and A, the conv taps of its slots), the dt
-      // weights, and the per-token dt and cumsum rows for the output kernel
+      // lane's 4 tokens, their dt_bias and A), the dt weights, and the per-token dt
+      // and cumsum rows for the output kernel.  The conv taps are read after the
+      // stage's tiles are requested (not held in registers across the wait)
       float dtr[2][4], dtb[2] = {0.0f, 0.0f}, Ah[2] = {0.0f, 0.0f};
-      float4 tw[3][2];
-      float tb[3][2];
-      bool son[3];
-#pragma unroll
-      for (int sl = 0; sl < 3; ++sl) {
-        // a C item convolves the key's C channels (B/C buffer) and its B channels (x slot
-        // 0) to form the fp32 diagonal C_t . B_t
-        son[sl] = w.isC ? sl != 1 : (sl == 1 ? hasB : (sl == 2 ? w.freshB : true));
-        const int64_t ch0 = (w.isC && sl == 0) ? pr.d_inner + (int64_t)w.g * kNS
-                            : sl < 2 ? (int64_t)(hA + sl) * kHP
-                                     : pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (son[sl]) {
-            const float4 *wp = reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + lane + 32 * j;
-            const float *bp = a.prm.conv_b + ch0 + lane + 32 * j;
-            tw[sl][j] = M2_OK(wp, 16, a.sp.conv_w, &g_tc_errors) ? __ldg(wp) : make_float4(0.f, 0.f, 0.f, 0.f);
-            tb[sl][j] = M2_OK(bp, 4, a.sp.conv_b, &g_tc_errors) ? __ldg(bp) : 0.0f;
-          }
-        }
-      }
+      // slots in use (a C item convolves the key's C channels (B/C buffer) and its B
+      // channels (x slot 0) to form the fp32 diagonal C_t . B_t) and their first channel
+      auto slot_on = [&](int sl) -> bool {
+        return w.isC ? sl != 1 : (sl == 1 ? hasB : (sl == 2 ? w.freshB : true));
+      };
+      auto slot_ch = [&](int sl) -> int64_t {
+        return (w.isC && sl == 0) ? pr.d_inner + (int64_t)w.g * kNS
+               : sl < 2           ? (int64_t)(hA + sl) * kHP
+                                  : pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
+      };
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const bool hv = !w.isC && (half == 0 || hasB);
@@ -466,7 +434,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             wsv[half][q] = expf(sfx[q]) * dt4[q];
           }
           if (hv) {
-            const int64_t row = (w.bi * a.nch + w.c) * pr.H + hA + half;
+            const int64_t row = ((int64_t)w.bi * a.nch + w.c) * pr.H + hA + half;
             float4 *cp = reinterpret_cast<float4 *>(a.cum + row * kQ) + lane;
             float4 *dp = reinterpret_cast<float4 *>(a.dtv + row * kQ) + lane;
             if (M2_OK(cp, 16, a.sp.cum, &g_tc_errors)) *cp = make_float4(cq[0], cq[1], cq[2], cq[3]);
@@ -517,9 +485,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         // slot x_A, x_B (if any) and the B/C tile: 3 rows x 64 channels each
         for (int idx = lane; idx < 3 * 3 * 64; idx += 32) {
           const int sl = idx / 192, r = (idx / 64) % 3, chn = idx % 64;
-          if (!son[sl]) continue;
-          const int64_t ch = ((w.isC && sl == 0) ? pr.d_inner + (int64_t)w.g * kNS
-                              : sl < 2 ? (int64_t)(hA + sl) * kHP : bc_ch) + chn;
+          if (!slot_on(sl)) continue;
+          const int64_t ch = slot_ch(sl) + chn;
           const __nv_bfloat16 *hp = a.conv_in + (w.bi * pr.conv_dim + ch) * 4 + 1 + r;
           const __nv_bfloat16 v =
               M2_OK(hp, 2, a.sp.conv, &g_tc_errors) ? *hp : __float2bfloat16(0.0f);
@@ -536,18 +503,24 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) ws[st][half][4 * lane + q] = wsv[half][q];
       }
-      // conv taps and bias of the item's slots, channel 8 g + i at [i][g]
-#pragma unroll
+      // conv taps and bias of the item's slots, channel 8 g + i at [i][g], copied
+      // asynchronously; each lane's copies complete on the stage's barrier
+#pragma unroll 1
       for (int sl = 0; sl < 3; ++sl) {
-        if (!son[sl]) continue;
+        if (!slot_on(sl)) continue;
+        const int64_t ch0 = slot_ch(sl);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int i = lane + 32 * j, d = (i & 7) * 8 + (i >> 3);
-          const float4 w4 = tw[sl][j];  // halved (exact), see conv8x4_smem
-          wts[st][sl][d] = make_float4(0.5f * w4.x, 0.5f * w4.y, 0.5f * w4.z, 0.5f * w4.w);
-          bss[st][sl][d] = 0.5f * tb[sl][j];
+          const float4 *wp = reinterpret_cast<const float4 *>(a.prm.conv_w) + ch0 + i;
+          const float *bp = a.prm.conv_b + ch0 + i;
+          if (M2_OK(wp, 16, a.sp.conv_w, &g_tc_errors)) cp_async_ca16(smem_u32(&wts[st][sl][d]), wp);
+          else wts[st][sl][d] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (M2_OK(bp, 4, a.sp.conv_b, &g_tc_errors)) cp_async_ca4(smem_u32(&bss[st][sl][d]), bp);
+          else bss[st][sl][d] = 0.0f;
         }
       }
+      cp_async_mbar_arrive_noinc(&full[st]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);  // weights of this stage written
     }
@@ -593,7 +566,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     // + lane (head half m / 64, lane p = m % 64), 16 columns per warp / 4; S is kept
     // [n/4][p][4] per head so that a warp's float4 stores are contiguous
     struct Pending {
-      int64_t bi;
+      int bi;
       int c, hA;
       bool hasB;
     } pw{};
@@ -605,7 +578,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       mbar_arrive(&tmem_free[acc]);
       if (half == 0 || q.hasB) {
         float4 *dst = reinterpret_cast<float4 *>(
-            a.S + ((q.bi * a.nch + q.c) * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
+            a.S + (((int64_t)q.bi * a.nch + q.c) * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           if (M2_OK(dst + (4 * cb + i) * kHP + p, 16, a.sp.S, &g_tc_errors))
@@ -679,23 +652,54 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       };
       float v[4][8];
       if (w.isC) {
-        // C item: warps 0-7 convolve the C channels (B/C buffer) into u, then the B
-        // channels (x slot 0) for C_t . B_t in fp32: each thread's 8 channels x 4
-        // tokens, summed over the 4 lanes of a token quad, then warps 4-7 (channel
-        // groups 4-7) hand their sums to warps 0-3 through shared memory
+        // C item: warps 0-7 convolve the C channels (B/C buffer) into u and park the
+        // values, fp32, in the B operand buffers (free once the last pair item's MMAs
+        // are done); warps 8-15, whose lanes hold the same 8 channels x 4 tokens,
+        // convolve the B channels (x slot 0) and form C_t . B_t in fp32: summed over
+        // the 4 lanes of a token quad, then warps 12-15 (channel groups 4-7) hand
+        // their sums to warps 8-11 through shared memory
+        if (np >= 1) wait_mma(np - 1);
+        if (!ok) break;
+        const uint32_t park = sBhi + (uint32_t)(((warp & 7) * 32 + lane) * 16);  // [8][256] float4
         if (warp < 8) {
           conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v);
-          store_u(a, w.bi, c0 + s0, bc_ch + cg * 8, v);
           mbar_arrive(&bc_empty[bcb]);
+          store_u(a, w.bi, c0 + s0, bc_ch + cg * 8, v);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              st_shared_v4(park + (2 * kk + h) * 4096, __float_as_uint(v[kk][4 * h]),
+                           __float_as_uint(v[kk][4 * h + 1]), __float_as_uint(v[kk][4 * h + 2]),
+                           __float_as_uint(v[kk][4 * h + 3]));
+          mbar_arrive(&empty[st]);
+          mbar_arrive(&park_bar);
+        } else {
+          conv8x4_smem(stage, s0, cg, wts[st][0], bss[st][0], v);
+          mbar_arrive(&empty[st]);
+          {
+            const bool got = mbar_wait_bounded(&park_bar, (uint32_t)(nc & 1), &g_tc_errors);
+            ok = __all_sync(0xffffffffu, got) != 0;
+          }
+          if (!ok) break;
           float d4[4];
-          conv8x4_dot(stage, s0, cg, wts[st][0], bss[st][0], v, d4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            d4[kk] += __shfl_xor_sync(0xffffffffu, d4[kk], 1);
-            d4[kk] += __shfl_xor_sync(0xffffffffu, d4[kk], 2);
+            float acc = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint4 q = ld_shared_v4(park + (2 * kk + h) * 4096);
+              acc = fmaf(__uint_as_float(q.x), v[kk][4 * h], acc);
+              acc = fmaf(__uint_as_float(q.y), v[kk][4 * h + 1], acc);
+              acc = fmaf(__uint_as_float(q.z), v[kk][4 * h + 2], acc);
+              acc = fmaf(__uint_as_float(q.w), v[kk][4 * h + 3], acc);
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            d4[kk] = acc;
           }
           const int cpar = nc & 1;
-          if (warp >= 4) {
+          if (warp >= 12) {
             if ((lane & 3) == 0)
               *reinterpret_cast<float4 *>(&cbd_s[cpar][s0]) = make_float4(d4[0], d4[1], d4[2], d4[3]);
             mbar_arrive(&cbd_bar);
@@ -704,14 +708,13 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             ok = __all_sync(0xffffffffu, got) != 0;
             if (ok && (lane & 3) == 0) {
               const float4 o = *reinterpret_cast<const float4 *>(&cbd_s[cpar][s0]);
-              float4 *dp = reinterpret_cast<float4 *>(a.cbd + ((w.bi * pr.G + w.g) * a.nch + w.c) * kQ + s0);
+              float4 *dp = reinterpret_cast<float4 *>(a.cbd + (((int64_t)w.bi * pr.G + w.g) * a.nch + w.c) * kQ + s0);
               if (M2_OK(dp, 16, a.sp.cbd, &g_tc_errors))
                 *dp = make_float4(d4[0] + o.x, d4[1] + o.y, d4[2] + o.z, d4[3] + o.w);
             }
           }
         }
         ++nc;
-        mbar_arrive(&empty[st]);
         continue;
       }
       const int sl = warp >> 3;  // x slot of this warp: head A (warps 0-7) or B
@@ -734,19 +737,22 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         }
         mbar_arrive(&empty[st]);
       } else {
-        // the tile stays in registers while the previous pair item's MMAs run; its u
-        // stores follow the operand hand-off, so the MMA does not wait behind them
-        float4 wk4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        // the previous pair item's MMAs (the readers of the single operand buffer) are
+        // normally done by now; waiting first keeps the tile out of registers across
+        // the wait.  The u stores follow the operand hand-off, so the MMA does not wait
+        // behind them
         const bool has_tile = !(sl == 1 && !hasB);
-        if (has_tile) {
-          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
-          wk4 = tile_weights(sl);
-        }
-        mbar_arrive(&empty[st]);  // nothing of the stage is read after this
         if (np >= 1) wait_mma(np - 1);
         if (!ok) break;
-        if (!has_tile) zero_tile();
-        else put_operands(sl, v, wk4);
+        if (has_tile) {
+          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
+          const float4 wk4 = tile_weights(sl);
+          mbar_arrive(&empty[st]);  // nothing of the stage is read after this
+          put_operands(sl, v, wk4);
+        } else {
+          mbar_arrive(&empty[st]);
+          zero_tile();
+        }
         fence_proxy_async_smem();
         mbar_arrive(&ops_ready);  // the MMA warp issues S = (x o w)^T B into accumulator np % 2
         if (has_tile) store_u(a, w.bi, c0 + s0, xch + cg * 8, v);
@@ -779,8 +785,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 // H_{c+1} = exp(cum_end_c) H_c + S_c in fp32 for the rows p in [16q, 16q + 16)
 // of one head, sequential over chunks: warp w owns the rows p = 16q + 2w and
 // 16q + 2w + 1, lane l the row 16q + 2w + l / 16 and the columns
-// n = 4 (l % 16) .. +3 (one 16-byte load of the chunk states per chunk; loads run
-// 8 chunks ahead).  The state entering each chunk is stored as the fp16 operand
+// n = 4 (l % 16) .. +3 (one 16-byte load of the chunk states per chunk; loads are
+// issued 8 chunks at a time).  The state entering each chunk is stored as the fp16 operand
 // of the output kernel's C H_c^T product, [p][n] (n contiguous: each lane writes
 // 8 bytes, each warp two whole 128-byte rows), divided by a power of two 2^s
 // chosen per (chunk, head, pair of rows) from the warp's max |H_c| so that every
@@ -854,34 +860,37 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
     u2.y = *reinterpret_cast<const uint32_t *>(&hi);
     if (M2_OK(o, 8, a.sp.Hc, &g_tc_errors)) *reinterpret_cast<uint2 *>(o) = u2;
   };
-  // a rolling window of 8 chunks in flight: chunk c + 8 is requested as soon as
-  // chunk c has been used, so the memory latency is paid once, not once per 8 chunks
+  // loads run 8 chunks ahead of the (sequential) recurrence
   constexpr int kAhead = 8;
-  float4 sv[kAhead];
-  float d[kAhead];
-  auto fetch = [&](int cc, float4 &svk, float &dk) {
-    if (cc < a.nch) {
-      const float *sp = S + cc * stride;
-      const float *cp = ce + (int64_t)cc * pr.H;
-      svk = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-      dk = M2_OK(cp, 4, a.sp.cum_end, &g_tc_errors) ? *cp : 0.0f;
-    }
-  };
-#pragma unroll
-  for (int k = 0; k < kAhead; ++k) fetch(k, sv[k], d[k]);
-  for (int c0 = 0; c0 < a.nch; c0 += kAhead) {
+  int c = 0;
+  for (; c + kAhead <= a.nch; c += kAhead) {
+    float4 sv[kAhead];
+    float d[kAhead];
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
-      const int c = c0 + k;
-      if (c < a.nch) {
-        put(c);
-        const float f = expf(d[k]);
-        hc = make_float4(fmaf(f, hc.x, sv[k].x), fmaf(f, hc.y, sv[k].y), fmaf(f, hc.z, sv[k].z),
-                         fmaf(f, hc.w, sv[k].w));
-        fetch(c + kAhead, sv[k], d[k]);
-      }
+      const float *sp = S + (c + k) * stride;
+      const float *cp = ce + (int64_t)(c + k) * pr.H;
+      sv[k] = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      d[k] = M2_OK(cp, 4, a.sp.cum_end, &g_tc_errors) ? *cp : 0.0f;
     }
+#pragma unroll
+    for (int k = 0; k < kAhead; ++k) {
+      put(c + k);
+      const float f = expf(d[k]);
+      hc = make_float4(fmaf(f, hc.x, sv[k].x), fmaf(f, hc.y, sv[k].y), fmaf(f, hc.z, sv[k].z),
+                       fmaf(f, hc.w, sv[k].w));
+    }
+  }
+  for (; c < a.nch; ++c) {
+    put(c);
+    const float *sp = S + c * stride;
+    const float *cp = ce + (int64_t)c * pr.H;
+    const float4 sv = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
+                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float f = expf(M2_OK(cp, 4, a.sp.cum_end, &g_tc_errors) ? *cp : 0.0f);
+    hc = make_float4(fmaf(f, hc.x, sv.x), fmaf(f, hc.y, sv.y), fmaf(f, hc.z, sv.z),
+                     fmaf(f, hc.w, sv.w));
   }
   if (a.ssm_state != nullptr && M2_OK(a.ssm_state + hs, 16, a.sp.ssm, &g_tc_errors))
     *reinterpret_cast<float4 *>(a.ssm_state + hs) = hc;
@@ -900,17 +909,15 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
 //   warps 0-7    decay operand: A_j = CB o exp(cum_t - cum_s) dt_s (s <= t, D_h
 //                on the diagonal) in fp16, double-buffered, up to two heads
 //                ahead of the epilogue; warp w builds rows 32 (w % 4) .. +31
-//                (its TMEM lane quarter) and columns 64 (w / 4) .. +63.  The
-//                same warps write the previous unit's output: after building
-//                head j's operand of unit n they scale head j of unit n - 1 by
-//                the per-token norm and the norm weight and store it to y
-//                (32-byte stores), which hands head j's TMEM columns back to
-//                the MMA warp for unit n;
+//                (its TMEM lane quarter) and columns 64 (w / 4) .. +63;
 //   warps 8-15   epilogue: y_j + exp(cum_t) 2^s T, gate by silu(z), per-token
 //                sums of squares, the gated value back into TMEM; after the
 //                unit's last head the per-token sums go to every CTA of the
 //                cluster (asynchronous DSMEM stores completing on the receiver's
-//                mbarrier) and the per-token norm scales to the operand warps.
+//                mbarrier), and each head is scaled by the norm and the norm
+//                weight and written to y (32-byte stores).  That output phase
+//                overlaps the next unit's operand builds and MMAs: a head's TMEM
+//                columns are handed back to the MMA warp one by one.
 // All waits are bounded (they raise the error flag and the CTA leaves its loop).
 constexpr uint32_t kCt0 = 0;                       // C [2][128 t][64 n] fp16 (u), 2 x 16 KB
 constexpr uint32_t kBt = 2 * 16384;                // B [128 s][64 n] fp16 (u), 16 KB
@@ -930,7 +937,6 @@ struct OutShared {
   alignas(16) float beta[kMaxHeadsPerCta][kQ];   // exp(cum_r - cum_s) dt_s, r = end of s's 32-token group
   alignas(16) float betad[kMaxHeadsPerCta][kQ];  // exp(cum_s0 - cum_s) dt_s, s0 = start of s's group
   // epilogue group
-  alignas(16) float inv[2][kQ];                  // [unit parity] per-token norm scales, for the output
   alignas(16) float half_ss[2][kQ];              // per-token sums of squares of the two column halves
   alignas(16) float mine[kQ];                    // this CTA's per-token partial sums
   alignas(16) float part[2][16][kQ];             // [unit parity][rank] partial sums received
@@ -939,13 +945,13 @@ struct OutShared {
   float Dh[kMaxHeadsPerCta];
   uint64_t full_cb[2], b_free, c_free[2], full_xh[2], empty_xh[2], full_z[2], empty_z[2],
       a_ready[2], mma_done[2], mbar_cb, cb_free, t_free, y_free[kMaxHeadsPerCta], sums_ready[2],
-      mma_final, inv_ready;
+      mma_final;
   uint32_t tmem_holder;
 };
 
 static_assert(offsetof(OutShared, cum2) % 16 == 0 && offsetof(OutShared, dt) % 16 == 0 &&
                   offsetof(OutShared, beta) % 16 == 0 && offsetof(OutShared, betad) % 16 == 0 &&
-                  offsetof(OutShared, inv) % 16 == 0 && offsetof(OutShared, mine) % 16 == 0 &&
+                  offsetof(OutShared, mine) % 16 == 0 &&
                   offsetof(OutShared, part) % 16 == 0 && offsetof(OutShared, cbd) % 16 == 0 &&
                   offsetof(OutShared, full_cb) % 8 == 0,
               "16-byte accessed shared arrays must be 16-byte aligned");
@@ -1155,7 +1161,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     mbar_init(&sh.mma_final, 1);
     mbar_init(&sh.cb_free, kGroupThreads);
     mbar_init(&sh.t_free, kGroupThreads);
-    mbar_init(&sh.inv_ready, kGroupThreads);  // the epilogue group wrote a unit's norm scales
     for (int j = 0; j < kMaxHeadsPerCta; ++j) mbar_init(&sh.y_free[j], kGroupThreads);
     fence_mbar_init();
   }
@@ -1274,82 +1279,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       mbar_wait_bounded(&sh.mma_final, 0, &g_tc_errors);
     }
   } else if (warp < 8) {
-    // ---------------- decay operands, and the previous unit's output
+    // ---------------- decay operands
     const int q = warp & 3, blk = warp >> 2, t = 32 * q + lane;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     bool ok = true;
     int J = 0;
-    // normalised bf16 output of head j of unit `un` (columns 32 blk .. +31 of row t);
-    // the head's TMEM columns go back to the MMA warp as soon as they are read
-    auto output_head = [&](int un, int j) {
-      int64_t obi;
-      int oc, og;
-      out_unit(pr, a.nch, ncl, cid, un, obi, oc, og);
-      const int h = og * hpg + lh0 + j;
-      const int64_t tok = (int64_t)oc * kQ + t;
-      const bool t_valid = tok < pr.L;
-      const float inv = sh.inv[un & 1][t];
-      __nv_bfloat16 *yrow = a.y + (obi * pr.L + tok) * pr.d_inner + (int64_t)h * kHP + 32 * blk;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float v[16];
-        tmem_ld16(tmem + lane_off + kTmemY + 64 * j + 32 * blk + 16 * hh, v);
-        if (hh == 1) {
-          tc_fence_before();
-          mbar_arrive(&sh.y_free[j]);
-        }
-        if (!t_valid) continue;
-        if (pr.nbg) {
-          const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (obi * pr.L + tok) * a.ld_z +
-                                                            (int64_t)h * kHP + 32 * blk + 16 * hh);
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const uint4 raw = M2_OK(zp + qq, 16, a.sp.z, &g_tc_errors) ? __ldg(zp + qq)
-                                                                        : make_uint4(0, 0, 0, 0);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = __bfloat1622float2(h2[i]);
-              v[8 * qq + 2 * i] *= silu_fast(f.x);
-              v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
-            }
-          }
-        }
-        const float4 *nw4 =
-            reinterpret_cast<const float4 *>(a.prm.norm_w + (int64_t)h * kHP + 32 * blk + 16 * hh);
-        uint32_t o[8];
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const bool wok = M2_OK(nw4 + 2 * qq, 16, a.sp.norm_w, &g_tc_errors) &&
-                           M2_OK(nw4 + 2 * qq + 1, 16, a.sp.norm_w, &g_tc_errors);
-          const float4 wA = wok ? __ldg(nw4 + 2 * qq) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 wB = wok ? __ldg(nw4 + 2 * qq + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 8 * qq + 2 * e;
-            const __nv_bfloat162 b2 =
-                __floats2bfloat162_rn(v[i] * inv * ww[2 * e], v[i + 1] * inv * ww[2 * e + 1]);
-            o[4 * qq + e] = *reinterpret_cast<const uint32_t *>(&b2);
-          }
-        }
-        __nv_bfloat16 *yp = yrow + 16 * hh;  // 16 columns = 32 bytes
-        if (a.y32) {
-          if (M2_OK(yp, 16, a.sp.y, &g_tc_errors) && M2_OK(yp + 8, 16, a.sp.y, &g_tc_errors))
-            st_global_v8(yp, o);
-        } else {
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq)
-            if (M2_OK(yp + 8 * qq, 16, a.sp.y, &g_tc_errors))
-              st_global_v4(yp + 8 * qq, o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]);
-        }
-      }
-    };
-    // wait until the epilogue warps have written unit un's norm scales
-    auto wait_inv = [&](int un) {
-      const bool got = ok && mbar_wait_bounded(&sh.inv_ready, (uint32_t)(un & 1), &g_tc_errors);
-      ok = __all_sync(0xffffffffu, got) != 0;
-    };
     for (int n = 0; ok && n < n_units && nh > 0; ++n) {
       int64_t bi;
       int c, g;
@@ -1403,27 +1337,84 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sh.a_ready[sl]);
-        if (n >= 1) {  // head j of the previous unit, whose columns this head's MMA takes
-          if (j == 0) wait_inv(n - 1);
-          if (!ok) break;
-          output_head(n - 1, j);
-        }
       }
       // this unit's CB columns and decay terms are no longer read
       tc_fence_before();
       if (ok) mbar_arrive(&sh.cb_free);
       ok = group_all(1, ok);
     }
-    if (ok && nh > 0 && n_units > 0) {  // the last unit's output
-      wait_inv(n_units - 1);
-      for (int j = 0; ok && j < nh; ++j) output_head(n_units - 1, j);
-    }
+
   } else {
     // ---------------- epilogue
     const int q = warp & 3, eh = (warp - 8) >> 2, t = 32 * q + lane, gt = tid - 256;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     bool ok = true;
     int J = 0;
+    // normalised bf16 output of head j of unit `un` (columns 32 blk .. +31 of row t);
+    // the head's TMEM columns go back to the MMA warp as soon as they are read
+    auto output_head = [&](int un, int j, float inv) {
+      int64_t obi;
+      int oc, og;
+      out_unit(pr, a.nch, ncl, cid, un, obi, oc, og);
+      const int h = og * hpg + lh0 + j;
+      const int64_t tok = (int64_t)oc * kQ + t;
+      const bool t_valid = tok < pr.L;
+      __nv_bfloat16 *yrow = a.y + (obi * pr.L + tok) * pr.d_inner + (int64_t)h * kHP + 32 * eh;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float v[16];
+        tmem_ld16(tmem + lane_off + kTmemY + 64 * j + 32 * eh + 16 * hh, v);
+        if (hh == 1) {
+          tc_fence_before();
+          mbar_arrive(&sh.y_free[j]);
+        }
+        if (!t_valid) continue;
+        if (pr.nbg) {
+          const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (obi * pr.L + tok) * a.ld_z +
+                                                            (int64_t)h * kHP + 32 * eh + 16 * hh);
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const uint4 raw = M2_OK(zp + qq, 16, a.sp.z, &g_tc_errors) ? __ldg(zp + qq)
+                                                                        : make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(h2[i]);
+              v[8 * qq + 2 * i] *= silu_fast(f.x);
+              v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
+            }
+          }
+        }
+        const float4 *nw4 =
+            reinterpret_cast<const float4 *>(a.prm.norm_w + (int64_t)h * kHP + 32 * eh + 16 * hh);
+        uint32_t o[8];
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const bool wok = M2_OK(nw4 + 2 * qq, 16, a.sp.norm_w, &g_tc_errors) &&
+                           M2_OK(nw4 + 2 * qq + 1, 16, a.sp.norm_w, &g_tc_errors);
+          const float4 wA = wok ? __ldg(nw4 + 2 * qq) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 wB = wok ? __ldg(nw4 + 2 * qq + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 8 * qq + 2 * e;
+            const __nv_bfloat162 b2 =
+                __floats2bfloat162_rn(v[i] * inv * ww[2 * e], v[i + 1] * inv * ww[2 * e + 1]);
+            o[4 * qq + e] = *reinterpret_cast<const uint32_t *>(&b2);
+          }
+        }
+        __nv_bfloat16 *yp = yrow + 16 * hh;  // 16 columns = 32 bytes
+        if (a.y32) {
+          if (M2_OK(yp, 16, a.sp.y, &g_tc_errors) && M2_OK(yp + 8, 16, a.sp.y, &g_tc_errors))
+            st_global_v8(yp, o);
+        } else {
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq)
+            if (M2_OK(yp + 8 * qq, 16, a.sp.y, &g_tc_errors))
+              st_global_v4(yp + 8 * qq, o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]);
+        }
+      }
+    };
     for (int n = 0; ok && n < n_units; ++n) {
       int64_t bi;
       int c, g;
@@ -1515,9 +1506,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       // sent unit n + 1's sums, which happens after this point
       if (gt == 0 && n + 2 < n_units) mbar_arrive_expect_tx(&sh.sums_ready[par], sum_bytes);
       if (!ok) break;
-      // the per-token norm scales to the operand warps, which write the output
-      if (eh == 0) sh.inv[par][t] = inv;
-      mbar_arrive(&sh.inv_ready);
+      // normalised bf16 output, head by head; each head's TMEM columns go back to the
+      // MMA warp (for the next unit) as soon as they are read
+      for (int j = 0; j < nh; ++j) output_head(n, j, inv);
     }
   }
   // every thread: the cluster's start barrier (if not waited for yet), then one
@@ -1775,6 +1766,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   const int64_t n_items = pr.batch * a.nch * (int64_t)pr.G * ((hpg + 1) / 2 + 1);
   const unsigned g1 = (unsigned)std::min<int64_t>(n_items, sm_count());
   {
+    NvtxRange r1("tc_chunk_state");
     K1Maps m1;
     const uint64_t dx[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
     const uint64_t sx[2] = {(uint64_t)pa.ld_xbc * 2, (uint64_t)pr.L * pa.ld_xbc * 2};
@@ -1784,6 +1776,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     tc_chunk_state_kernel<<<g1, kK1Threads, kK1Smem, st>>>(a, m1, (int)n_items);
   }
   stage_mark(st, 1);
+  NvtxRange r2("tc_state_pass + tc_chunk_out");
   dim3 g2((unsigned)(kPassBlocks + ceil_div(pr.conv_dim, 256)), (unsigned)pr.H,
           (unsigned)pr.batch);
   {
