@@ -71,13 +71,14 @@ struct TcArgs {
   float *cum_end;                // [b][nch][H] chunk sum of dt*A
   float *cum;                    // [b][nch][H][128] running sum of dt*A inside the chunk
   float *dtv;                    // [b][nch][H][128] dt (0 past the end of the sequence)
-  __half *Hc;                    // [b][nch][H][p 64][n 64] state entering each chunk, scaled
+  __half *Hc;                    // [b][nch][H][n 64][p 64] state entering each chunk, scaled
   float *hsc;                    // [b][nch][H][32] 2^s: H_c rows p = 2i, 2i + 1 hold H / 2^s
+  float *smax;                   // [b][nch][H] max |S_c| of each chunk's states (bounds |H_c|)
   float *cbd;                    // [b][G][nch * 128] C_t . B_t in fp32 (the decay operand's diagonal)
   // byte ranges of every buffer, for the checked build (see M2_OK)
   struct Spans {
-    Span xbc, z, dt, y, conv, ssm, S, cum_end, cum, dtv, Hc, hsc, cbd, u, conv_w, conv_b, dt_bias,
-        A, D, norm_w;
+    Span xbc, z, dt, y, conv, ssm, S, cum_end, cum, dtv, Hc, hsc, smax, cbd, u, conv_w, conv_b,
+        dt_bias, A, D, norm_w;
   } sp;
   __half *u;                     // [b][L][conv_dim] post-conv x | B | C, fp16
   int hpc;                       // max heads per CTA in tc_chunk_out
@@ -441,6 +442,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             if (M2_OK(dp, 16, a.sp.dtv, &g_tc_errors)) *dp = make_float4(dt4[0], dt4[1], dt4[2], dt4[3]);
             if (lane == 0 && M2_OK(a.cum_end + row, 4, a.sp.cum_end, &g_tc_errors))
               a.cum_end[row] = cum_end;
+            // max |S_c| of this head: raised by the compute warps' atomics after the MMA
+            if (lane == 0 && M2_OK(a.smax + row, 4, a.sp.smax, &g_tc_errors)) a.smax[row] = 0.0f;
           }
         }
       }
@@ -576,7 +579,17 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 64 * acc + 16 * cb, sv);
       tc_fence_before();  // TMEM read before the accumulator takes the next item
       mbar_arrive(&tmem_free[acc]);
+      // max |S| over the warp's 32 rows x 16 columns (all of one head) into the head's
+      // bound (non-negative floats order as their bit patterns)
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(sv[i]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (half == 0 || q.hasB) {
+        float *mp = a.smax + ((int64_t)q.bi * a.nch + q.c) * pr.H + q.hA + half;
+        if (lane == 0 && M2_OK(mp, 4, a.sp.smax, &g_tc_errors))
+          atomicMax(reinterpret_cast<int *>(mp), __float_as_int(mx));
         float4 *dst = reinterpret_cast<float4 *>(
             a.S + (((int64_t)q.bi * a.nch + q.c) * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
 #pragma unroll
@@ -781,22 +794,27 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 }
 
 // ============================================================== state passing
-// grid (4 + conv-state blocks, H, b).  Block q < 4 runs the recurrence
-// H_{c+1} = exp(cum_end_c) H_c + S_c in fp32 for the rows p in [16q, 16q + 16)
-// of one head, sequential over chunks: warp w owns the rows p = 16q + 2w and
-// 16q + 2w + 1, lane l the row 16q + 2w + l / 16 and the columns
-// n = 4 (l % 16) .. +3 (one 16-byte load of the chunk states per chunk; loads are
-// issued 8 chunks at a time).  The state entering each chunk is stored as the fp16 operand
-// of the output kernel's C H_c^T product, [p][n] (n contiguous: each lane writes
-// 8 bytes, each warp two whole 128-byte rows), divided by a power of two 2^s
-// chosen per (chunk, head, pair of rows) from the warp's max |H_c| so that every
-// stored value is below 2^14: fp16 cannot overflow whatever the state's size.
-// The output kernel multiplies those columns of C H_c^T by 2^s (exact).  No
-// barrier is needed: each warp's scale is its own.
-// Blocks with blockIdx.x >= 4 (only for h = 0) write the final conv state
-// instead: the last 4 raw inputs of [old state | new tokens], in place (the
-// chunk-state kernel, which reads the old state, has finished by now).
-constexpr int kPassBlocks = 4;
+// grid (H * 4 + conv-state blocks, b) of 256-thread blocks.  Block 4 h + q runs
+// the recurrence H_{c+1} = exp(cum_end_c) H_c + S_c in fp32 for the float4 slots
+// j = 256 q + thread of head h's chunk states ([n/4][p][4]: columns n = 4 (j / 64)
+// .. +3 of row p = j % 64), sequential over chunks, with loads issued 8 chunks at
+// a time: a warp reads 512 contiguous bytes per chunk and writes the fp16 state
+// entering each chunk as H_c [n][p] (the output kernel's MN-major operand), four
+// coalesced 64-byte rows.
+// H_c is stored divided by 2^s, one power of two per (chunk, head), so that fp16
+// cannot overflow whatever the state's size: s comes from a bound on max |H_c|
+// that every thread of the head computes alike, B_0 = max |initial state| and
+// B_{c+1} = exp(cum_end_c) B_c + max |S_c| (the chunk-state kernel supplies the
+// last term), with s = max(0, floor(log2 B_c) - 13) so that |H_c| / 2^s < 2^14.
+// Overestimating B only moves small values towards fp16's subnormals, whose
+// absolute spacing 2^-24 2^s stays below 2^-37 B.  The output kernel multiplies
+// C H_c^T by 2^s (exact); the scale table keeps one entry per row pair, here all
+// equal.
+// Blocks 4 H and up write the final conv state instead: the last 4 raw inputs of
+// [old state | new tokens], in place (the chunk-state kernel, which reads the old
+// state, has finished by now).
+constexpr int kPassBlocks = 4;     // blocks per head
+constexpr int kPassThreads = 256;  // 1024 float4 slots of a head's 64 x 64 state
 
 // 2^s with s = max(0, floor(log2 m) - 13), so that m / 2^s < 2^14.
 __device__ __forceinline__ float state_scale(float m) {
@@ -805,15 +823,16 @@ __device__ __forceinline__ float state_scale(float m) {
   return __uint_as_float((uint32_t)(127 + s) << 23);
 }
 
-__global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloat16 *cs) {
+__global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, __nv_bfloat16 *cs) {
+  __shared__ float red[kPassThreads / 32];
   grid_dependency_wait();  // the chunk-state kernel's results (launched early, see prefill_tc)
   launch_dependents();
   const Problem &pr = a.pr;
-  const int h = blockIdx.y;
-  const int64_t bi = blockIdx.z;
-  if ((int)blockIdx.x >= kPassBlocks) {
-    if (h != 0 || cs == nullptr) return;
-    const int64_t ch = (int64_t)(blockIdx.x - kPassBlocks) * 256 + threadIdx.x;
+  const int64_t bi = blockIdx.y;
+  const int nrb = pr.H * kPassBlocks;
+  if ((int)blockIdx.x >= nrb) {
+    if (cs == nullptr) return;
+    const int64_t ch = (int64_t)(blockIdx.x - nrb) * kPassThreads + threadIdx.x;
     if (ch >= pr.conv_dim) return;
     const int64_t i = bi * pr.conv_dim + ch;
     __nv_bfloat16 v[4];
@@ -833,64 +852,86 @@ __global__ void __launch_bounds__(256) tc_state_pass_kernel(TcArgs a, __nv_bfloa
       if (M2_OK(cs + i * 4 + k, 2, a.sp.conv, &g_tc_errors)) cs[i * 4 + k] = v[k];
     return;
   }
-  const int q = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p = 16 * q + 2 * warp + (lane >> 4), n4 = lane & 15;
-  const int j = n4 * kHP + p;  // float4 slot in the chunk-state layout [n/4][p][4]
-  const int64_t hs = (bi * pr.H + h) * (int64_t)(kHP * kNS) + p * kNS + 4 * n4;
+  const int h = blockIdx.x / kPassBlocks, q = blockIdx.x % kPassBlocks;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = q * kPassThreads + tid, n4 = j >> 6, p = j & 63;
+  const int64_t head = bi * pr.H + h;
+  const int64_t hs = head * (int64_t)(kHP * kNS) + p * kNS + 4 * n4;
   float4 hc = (a.states_in && M2_OK(a.ssm_state + hs, 16, a.sp.ssm, &g_tc_errors))
                   ? *reinterpret_cast<const float4 *>(a.ssm_state + hs)
                   : make_float4(0.f, 0.f, 0.f, 0.f);
-  const int64_t stride = (int64_t)pr.H * kHP * kNS;
-  const float *S = a.S + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + 4 * j;
-  __half *Hc = a.Hc + (bi * a.nch * pr.H + h) * (int64_t)(kHP * kNS) + p * kNS + 4 * n4;
-  float *hsc = a.hsc + (bi * a.nch * pr.H + h) * 32 + 8 * q + warp;
-  const float *ce = a.cum_end + bi * a.nch * pr.H + h;
-  // H_c / 2^s into the operand, 2^s into the scale table (a warp-wide max per chunk)
-  auto put = [&](int64_t c) {
-    float m = fmaxf(fmaxf(fabsf(hc.x), fabsf(hc.y)), fmaxf(fabsf(hc.z), fabsf(hc.w)));
+  // B_0: max |initial state| over the whole head (each block of the head alike)
+  float bnd = 0.0f;
+  if (a.states_in) {
+    const float4 *h0 = reinterpret_cast<const float4 *>(a.ssm_state + head * (int64_t)(kHP * kNS));
+    float m = 0.0f;
+    for (int i = tid; i < kHP * kNS / 4; i += kPassThreads) {
+      if (!M2_OK(h0 + i, 16, a.sp.ssm, &g_tc_errors)) continue;
+      const float4 v = h0[i];
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float sc = state_scale(m), inv = 1.0f / sc;  // powers of two: exact
-    if (lane == 0 && M2_OK(hsc + c * pr.H * 32, 4, a.sp.hsc, &g_tc_errors)) hsc[c * pr.H * 32] = sc;
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kPassThreads / 32; ++w) bnd = fmaxf(bnd, red[w]);
+  }
+  const int64_t stride = (int64_t)pr.H * kHP * kNS;  // one chunk further
+  const int64_t c0h = bi * a.nch * pr.H + h;           // (row, chunk 0, head)
+  const float *S = a.S + c0h * (int64_t)(kHP * kNS) + 4 * j;
+  __half *Hc = a.Hc + c0h * (int64_t)(kHP * kNS) + (4 * n4) * kHP + p;
+  const float *ce = a.cum_end + c0h;
+  const float *sm = a.smax + c0h;
+  const bool scale_writer = q == 0 && warp == 0;  // the head's 32 scale entries per chunk
+  // H_c / 2^s into the operand (4 coalesced 2-byte stores), 2^s into the scale table
+  auto put = [&](int64_t c) {
+    const float sc = state_scale(bnd), inv = 1.0f / sc;  // powers of two: exact
     __half *o = Hc + c * stride;
-    const __half2 lo = __floats2half2_rn(hc.x * inv, hc.y * inv);
-    const __half2 hi = __floats2half2_rn(hc.z * inv, hc.w * inv);
-    uint2 u2;
-    u2.x = *reinterpret_cast<const uint32_t *>(&lo);
-    u2.y = *reinterpret_cast<const uint32_t *>(&hi);
-    if (M2_OK(o, 8, a.sp.Hc, &g_tc_errors)) *reinterpret_cast<uint2 *>(o) = u2;
+    if (M2_OK(o, 2, a.sp.Hc, &g_tc_errors) && M2_OK(o + 3 * kHP, 2, a.sp.Hc, &g_tc_errors)) {
+      o[0] = __float2half_rn(hc.x * inv);
+      o[kHP] = __float2half_rn(hc.y * inv);
+      o[2 * kHP] = __float2half_rn(hc.z * inv);
+      o[3 * kHP] = __float2half_rn(hc.w * inv);
+    }
+    float *hp = a.hsc + (c0h + c * pr.H) * 32 + lane;
+    if (scale_writer && M2_OK(hp, 4, a.sp.hsc, &g_tc_errors)) *hp = sc;
+  };
+  auto step = [&](float4 sv, float d, float msv) {
+    const float f = expf(d);
+    hc = make_float4(fmaf(f, hc.x, sv.x), fmaf(f, hc.y, sv.y), fmaf(f, hc.z, sv.z),
+                     fmaf(f, hc.w, sv.w));
+    bnd = fmaf(f, bnd, msv);
   };
   // loads run 8 chunks ahead of the (sequential) recurrence
   constexpr int kAhead = 8;
   int c = 0;
   for (; c + kAhead <= a.nch; c += kAhead) {
     float4 sv[kAhead];
-    float d[kAhead];
+    float d[kAhead], msv[kAhead];
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
       const float *sp = S + (c + k) * stride;
-      const float *cp = ce + (int64_t)(c + k) * pr.H;
+      const int64_t r = (int64_t)(c + k) * pr.H;
       sv[k] = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-      d[k] = M2_OK(cp, 4, a.sp.cum_end, &g_tc_errors) ? *cp : 0.0f;
+      d[k] = M2_OK(ce + r, 4, a.sp.cum_end, &g_tc_errors) ? ce[r] : 0.0f;
+      msv[k] = M2_OK(sm + r, 4, a.sp.smax, &g_tc_errors) ? sm[r] : 0.0f;
     }
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
       put(c + k);
-      const float f = expf(d[k]);
-      hc = make_float4(fmaf(f, hc.x, sv[k].x), fmaf(f, hc.y, sv[k].y), fmaf(f, hc.z, sv[k].z),
-                       fmaf(f, hc.w, sv[k].w));
+      step(sv[k], d[k], msv[k]);
     }
   }
   for (; c < a.nch; ++c) {
     put(c);
     const float *sp = S + c * stride;
-    const float *cp = ce + (int64_t)c * pr.H;
-    const float4 sv = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
-                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float f = expf(M2_OK(cp, 4, a.sp.cum_end, &g_tc_errors) ? *cp : 0.0f);
-    hc = make_float4(fmaf(f, hc.x, sv.x), fmaf(f, hc.y, sv.y), fmaf(f, hc.z, sv.z),
-                     fmaf(f, hc.w, sv.w));
+    const int64_t r = (int64_t)c * pr.H;
+    step(M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f),
+         M2_OK(ce + r, 4, a.sp.cum_end, &g_tc_errors) ? ce[r] : 0.0f,
+         M2_OK(sm + r, 4, a.sp.smax, &g_tc_errors) ? sm[r] : 0.0f);
   }
   if (a.ssm_state != nullptr && M2_OK(a.ssm_state + hs, 16, a.sp.ssm, &g_tc_errors))
     *reinterpret_cast<float4 *>(a.ssm_state + hs) = hc;
@@ -932,7 +973,7 @@ constexpr int kGroupThreads = 256;                 // threads of the operand / e
 // into other ranks) is 16-byte aligned; the static_asserts below check it.
 struct OutShared {
   // decay terms of the unit's heads (operand group)
-  alignas(16) float cum2[kMaxHeadsPerCta][kQ];   // cumsum * log2(e)
+  alignas(16) float cum2[2][kMaxHeadsPerCta][kQ];  // [unit parity] cumsum * log2(e) (also read by the epilogue)
   alignas(16) float dt[kMaxHeadsPerCta][kQ];
   alignas(16) float beta[kMaxHeadsPerCta][kQ];   // exp(cum_r - cum_s) dt_s, r = end of s's 32-token group
   alignas(16) float betad[kMaxHeadsPerCta][kQ];  // exp(cum_s0 - cum_s) dt_s, s0 = start of s's group
@@ -941,11 +982,13 @@ struct OutShared {
   alignas(16) float mine[kQ];                    // this CTA's per-token partial sums
   alignas(16) float part[2][16][kQ];             // [unit parity][rank] partial sums received
   alignas(16) float cbd[kQ];                     // C_t . B_t (fp32) of the unit's chunk and group
+  alignas(16) uint8_t scs[2][kMaxHeadsPerCta][32];  // [unit parity] exponents s of H_c's row-pair scales 2^s
+  alignas(16) float nw[kMaxHeadsPerCta][kHP];     // the unit's norm weights (epilogue group)
   int span_ok[kMaxHeadsPerCta][4];   // group's log2-decay span <= 60: factorise its diagonal
   float Dh[kMaxHeadsPerCta];
   uint64_t full_cb[2], b_free, c_free[2], full_xh[2], empty_xh[2], full_z[2], empty_z[2],
       a_ready[2], mma_done[2], mbar_cb, cb_free, t_free, y_free[kMaxHeadsPerCta], sums_ready[2],
-      mma_final;
+      mma_final, e1_done[2];
   uint32_t tmem_holder;
 };
 
@@ -953,6 +996,7 @@ static_assert(offsetof(OutShared, cum2) % 16 == 0 && offsetof(OutShared, dt) % 1
                   offsetof(OutShared, beta) % 16 == 0 && offsetof(OutShared, betad) % 16 == 0 &&
                   offsetof(OutShared, mine) % 16 == 0 &&
                   offsetof(OutShared, part) % 16 == 0 && offsetof(OutShared, cbd) % 16 == 0 &&
+                  offsetof(OutShared, scs) % 16 == 0 && offsetof(OutShared, nw) % 16 == 0 &&
                   offsetof(OutShared, full_cb) % 8 == 0,
               "16-byte accessed shared arrays must be 16-byte aligned");
 static_assert(kTcOutTiles % 1024 == 0, "OutShared starts 16-byte aligned");
@@ -1038,8 +1082,8 @@ __device__ __forceinline__ void out_unit(const Problem &pr, int nch, int ncl, in
 // four 16-byte chunks at column kc (0 or 32) of the 64-wide k-block at `at`:
 // zero above the diagonal group, factorised alpha_t beta_s below it, and on it
 // either factorised (decay span within 2^60) or with direct exponentials.
-__device__ __forceinline__ void build_a_group(const OutShared &sh, int j, int k, int q, int t,
-                                              uint32_t at, int kc, uint32_t tmem_cb) {
+__device__ __forceinline__ void build_a_group(const OutShared &sh, int par, int j, int k, int q,
+                                              int t, uint32_t at, int kc, uint32_t tmem_cb) {
   const int s0 = 32 * k;
   if (k > q) {
 #pragma unroll
@@ -1048,9 +1092,9 @@ __device__ __forceinline__ void build_a_group(const OutShared &sh, int j, int k,
   }
   float cb[32];
   tmem_ld32(tmem_cb + s0, cb);
-  const float c2t = sh.cum2[j][t];
+  const float c2t = sh.cum2[par][j][t];
   if (k < q) {
-    const float alpha = ex2_approx(c2t - sh.cum2[j][s0 + 31]);
+    const float alpha = ex2_approx(c2t - sh.cum2[par][j][s0 + 31]);
     const float4 *b4 = reinterpret_cast<const float4 *>(&sh.beta[j][s0]);
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) {
@@ -1070,7 +1114,7 @@ __device__ __forceinline__ void build_a_group(const OutShared &sh, int j, int k,
   if (sh.span_ok[j][k]) {
     // diagonal group, decay span <= 2^60: alpha_t = exp(cum_t - cum_s0) and
     // betad_s = exp(cum_s0 - cum_s) dt_s stay within [2^-60, 2^60]
-    const float alpha = ex2_approx(c2t - sh.cum2[j][s0]);
+    const float alpha = ex2_approx(c2t - sh.cum2[par][j][s0]);
     const float4 *b4 = reinterpret_cast<const float4 *>(&sh.betad[j][s0]);
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) {
@@ -1092,7 +1136,7 @@ __device__ __forceinline__ void build_a_group(const OutShared &sh, int j, int k,
       st_shared_v4(at + sw128_chunk(t, kc + 8 * qq), w4[0], w4[1], w4[2], w4[3]);
     }
   } else {
-    const float4 *c4 = reinterpret_cast<const float4 *>(&sh.cum2[j][s0]);
+    const float4 *c4 = reinterpret_cast<const float4 *>(&sh.cum2[par][j][s0]);
     const float4 *d4 = reinterpret_cast<const float4 *>(&sh.dt[j][s0]);
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) {
@@ -1123,7 +1167,7 @@ __device__ __forceinline__ void build_a_group(const OutShared &sh, int j, int k,
 __global__ void __launch_bounds__(kWsThreads, 1)
     tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps, int ncl) {
   if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA of every cluster alike
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  extern __shared__ __align__(16) unsigned char smem_raw[];  // aligned to 1024 below
   int cs, rank;
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs));
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
@@ -1151,6 +1195,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       mbar_init(&sh.empty_z[k], kGroupThreads);
       mbar_init(&sh.a_ready[k], kGroupThreads);
       mbar_init(&sh.mma_done[k], 1);
+      mbar_init(&sh.e1_done[k], kGroupThreads);  // the epilogue is done with a parity's cum2 / scs
       // the local arrival carries the bytes the ranks' partial sums complete;
       // units 0 and 1 are armed here, unit n + 2 once unit n's sums are read
       mbar_init(&sh.sums_ready[k], 1);
@@ -1173,6 +1218,69 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   const uint32_t tmem = sh.tmem_holder;
   constexpr uint32_t kTmemY = 128;                     // y_j at columns 128 + 64 j
 
+  // normalised bf16 output of head j of unit `un` by a thread of the epilogue group
+  // (row t = 32 (warp % 4) + lane, columns 32 ((warp / 4) % 2) .. +31 of the head);
+  // the head's TMEM columns go back to the MMA warp as soon as they are read
+  auto output_head = [&](int un, int j, float inv) {
+    const int q = warp & 3, eh = (warp >> 2) & 1, t = 32 * q + lane;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    int64_t obi;
+    int oc, og;
+    out_unit(pr, a.nch, ncl, cid, un, obi, oc, og);
+    const int h = og * hpg + lh0 + j;
+    const int64_t tok = (int64_t)oc * kQ + t;
+    const bool t_valid = tok < pr.L;
+    __nv_bfloat16 *yrow = a.y + (obi * pr.L + tok) * pr.d_inner + (int64_t)h * kHP + 32 * eh;
+    float v32[32];
+    tmem_ld32(tmem + lane_off + kTmemY + 64 * j + 32 * eh, v32);
+    tc_fence_before();
+    mbar_arrive(&sh.y_free[j]);
+    if (!t_valid) return;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float *v = v32 + 16 * hh;
+      if (pr.nbg) {
+        const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (obi * pr.L + tok) * a.ld_z +
+                                                          (int64_t)h * kHP + 32 * eh + 16 * hh);
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const uint4 raw = M2_OK(zp + qq, 16, a.sp.z, &g_tc_errors) ? __ldg(zp + qq)
+                                                                      : make_uint4(0, 0, 0, 0);
+          const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h2[i]);
+            v[8 * qq + 2 * i] *= silu_fast(f.x);
+            v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
+          }
+        }
+      }
+      const float4 *nw4 = reinterpret_cast<const float4 *>(&sh.nw[j][32 * eh + 16 * hh]);
+      uint32_t o[8];
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const float4 wA = nw4[2 * qq], wB = nw4[2 * qq + 1];
+        const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 8 * qq + 2 * e;
+          const __nv_bfloat162 b2 =
+              __floats2bfloat162_rn(v[i] * inv * ww[2 * e], v[i + 1] * inv * ww[2 * e + 1]);
+          o[4 * qq + e] = *reinterpret_cast<const uint32_t *>(&b2);
+        }
+      }
+      __nv_bfloat16 *yp = yrow + 16 * hh;  // 16 columns = 32 bytes
+      if (a.y32) {
+        if (M2_OK(yp, 16, a.sp.y, &g_tc_errors) && M2_OK(yp + 8, 16, a.sp.y, &g_tc_errors))
+          st_global_v8(yp, o);
+      } else {
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq)
+          if (M2_OK(yp + 8 * qq, 16, a.sp.y, &g_tc_errors))
+            st_global_v4(yp + 8 * qq, o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]);
+      }
+    }
+  };
   if (warp == 16) {
     // ---------------- producer
     if (lane == 0 && nh > 0) {
@@ -1229,7 +1337,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     if (lane == 0 && nh > 0) {
       const uint32_t idesc_cb = umma_idesc_f16(128, 128);
       const uint32_t idesc_mn = umma_idesc_f16(128, 64) | (1u << 16);  // B operand MN-major
-      const uint32_t idesc_t = umma_idesc_f16(128, 64);                 // both K-major
       int J = 0;
       bool ok = true;
       for (int n = 0; ok && n < n_units; ++n) {
@@ -1258,7 +1365,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           for (int ks = 0; ks < 8; ++ks)
             umma_f16(tmem + kTmemY + 64 * j, umma_desc_sw128(ab + (ks >> 2) * 16384 + (ks & 3) * 32),
                      umma_desc_sw128_mn(xt + ks * 2048, 16384), idesc_mn, ks > 0 ? 1u : 0u);
-          // T = C H_c^T : K = 64 (n), H_c [p][n] K-major; once the epilogue has read the
+          // T = C H_c^T : K = 64 (n), H_c [n][p] MN-major; once the epilogue has read the
           // previous head's T
           if (J > 0 && !mbar_wait_bounded(&sh.t_free, (uint32_t)((J - 1) & 1), &g_tc_errors)) {
             ok = false;
@@ -1266,8 +1373,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           }
           tc_fence_after();
           for (int kin = 0; kin < 4; ++kin)
-            umma_f16(tmem + kTmemT, umma_desc_sw128(ct + kin * 32), umma_desc_sw128(ht + kin * 32),
-                     idesc_t, kin > 0 ? 1u : 0u);
+            umma_f16(tmem + kTmemT, umma_desc_sw128(ct + kin * 32),
+                     umma_desc_sw128_mn(ht + kin * 2048, 8192), idesc_mn, kin > 0 ? 1u : 0u);
           umma_commit(&sh.mma_done[sl]);
           umma_commit(&sh.empty_xh[sl]);  // its x / H_c stage is free once they complete
         }
@@ -1289,6 +1396,14 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       int c, g;
       out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
       const int h0 = g * hpg + lh0;
+      const int par = n & 1;
+      // the epilogue reads this parity's exp(cum) and scales of unit n - 2 until it is done
+      // with that unit's gate pass
+      if (n >= 2) {
+        const bool got = mbar_wait_bounded(&sh.e1_done[par], (uint32_t)(((n - 2) >> 1) & 1), &g_tc_errors);
+        ok = group_all(1, got);
+        if (!ok) break;
+      }
       // decay terms of head j = warp (from the per-chunk dt and cumsum rows)
       if (warp < nh) {
         const int j = warp;
@@ -1303,7 +1418,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           c2[k] = cum4[k] * kLog2e;
-          sh.cum2[j][4 * lane + k] = c2[k];
+          sh.cum2[par][j][4 * lane + k] = c2[k];
           sh.dt[j][4 * lane + k] = dt4[k];
         }
         const float c2r = __shfl_sync(0xffffffffu, c2[3], (lane | 7));
@@ -1314,6 +1429,10 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           sh.betad[j][4 * lane + k] = ex2_approx(fminf(c2s0 - c2[k], 60.0f)) * dt4[k];
         }
         if ((lane & 7) == 7) sh.span_ok[j][lane >> 3] = (c2s0 - c2r) <= 60.0f;
+        // for the epilogue: the exponents of H_c's row-pair scales (powers of two >= 1)
+        const float *scp = a.hsc + row * 32 + lane;
+        const float scv = M2_OK(scp, 4, a.sp.hsc, &g_tc_errors) ? *scp : 1.0f;
+        sh.scs[par][j][lane] = (uint8_t)((__float_as_uint(scv) >> 23) - 127u);
         if (lane == 0)
           sh.Dh[j] = M2_OK(a.prm.D + h0 + j, 4, a.sp.D, &g_tc_errors) ? a.prm.D[h0 + j] : 0.0f;
       }
@@ -1332,8 +1451,8 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t at = base + kAbuf + sl * 32768 + blk * 16384;
-        build_a_group(sh, j, 2 * blk, q, t, at, 0, tmem + lane_off);
-        build_a_group(sh, j, 2 * blk + 1, q, t, at, 32, tmem + lane_off);
+        build_a_group(sh, par, j, 2 * blk, q, t, at, 0, tmem + lane_off);
+        build_a_group(sh, par, j, 2 * blk + 1, q, t, at, 32, tmem + lane_off);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sh.a_ready[sl]);
@@ -1350,71 +1469,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     bool ok = true;
     int J = 0;
-    // normalised bf16 output of head j of unit `un` (columns 32 blk .. +31 of row t);
-    // the head's TMEM columns go back to the MMA warp as soon as they are read
-    auto output_head = [&](int un, int j, float inv) {
-      int64_t obi;
-      int oc, og;
-      out_unit(pr, a.nch, ncl, cid, un, obi, oc, og);
-      const int h = og * hpg + lh0 + j;
-      const int64_t tok = (int64_t)oc * kQ + t;
-      const bool t_valid = tok < pr.L;
-      __nv_bfloat16 *yrow = a.y + (obi * pr.L + tok) * pr.d_inner + (int64_t)h * kHP + 32 * eh;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float v[16];
-        tmem_ld16(tmem + lane_off + kTmemY + 64 * j + 32 * eh + 16 * hh, v);
-        if (hh == 1) {
-          tc_fence_before();
-          mbar_arrive(&sh.y_free[j]);
-        }
-        if (!t_valid) continue;
-        if (pr.nbg) {
-          const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (obi * pr.L + tok) * a.ld_z +
-                                                            (int64_t)h * kHP + 32 * eh + 16 * hh);
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const uint4 raw = M2_OK(zp + qq, 16, a.sp.z, &g_tc_errors) ? __ldg(zp + qq)
-                                                                        : make_uint4(0, 0, 0, 0);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = __bfloat1622float2(h2[i]);
-              v[8 * qq + 2 * i] *= silu_fast(f.x);
-              v[8 * qq + 2 * i + 1] *= silu_fast(f.y);
-            }
-          }
-        }
-        const float4 *nw4 =
-            reinterpret_cast<const float4 *>(a.prm.norm_w + (int64_t)h * kHP + 32 * eh + 16 * hh);
-        uint32_t o[8];
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const bool wok = M2_OK(nw4 + 2 * qq, 16, a.sp.norm_w, &g_tc_errors) &&
-                           M2_OK(nw4 + 2 * qq + 1, 16, a.sp.norm_w, &g_tc_errors);
-          const float4 wA = wok ? __ldg(nw4 + 2 * qq) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 wB = wok ? __ldg(nw4 + 2 * qq + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float ww[8] = {wA.x, wA.y, wA.z, wA.w, wB.x, wB.y, wB.z, wB.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 8 * qq + 2 * e;
-            const __nv_bfloat162 b2 =
-                __floats2bfloat162_rn(v[i] * inv * ww[2 * e], v[i + 1] * inv * ww[2 * e + 1]);
-            o[4 * qq + e] = *reinterpret_cast<const uint32_t *>(&b2);
-          }
-        }
-        __nv_bfloat16 *yp = yrow + 16 * hh;  // 16 columns = 32 bytes
-        if (a.y32) {
-          if (M2_OK(yp, 16, a.sp.y, &g_tc_errors) && M2_OK(yp + 8, 16, a.sp.y, &g_tc_errors))
-            st_global_v8(yp, o);
-        } else {
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq)
-            if (M2_OK(yp + 8 * qq, 16, a.sp.y, &g_tc_errors))
-              st_global_v4(yp + 8 * qq, o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]);
-        }
-      }
-    };
     for (int n = 0; ok && n < n_units; ++n) {
       int64_t bi;
       int c, g;
@@ -1422,45 +1476,30 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       const int h0 = g * hpg + lh0;
       const int par = n & 1;
       float ss = 0.0f;
-      // cum_t of head j for this thread's token (the next head's is loaded while this
-      // one is worked on)
-      auto head_cum = [&](int j) -> float {
-        const int64_t row = (bi * a.nch + c) * pr.H + h0 + j;
-        const float *cp = a.cum + row * kQ + t;
-        return M2_OK(cp, 4, a.sp.cum, &g_tc_errors) ? *cp : 0.0f;
-      };
-      float cum_n = nh > 0 ? head_cum(0) : 0.0f;
       for (int j = 0; j < nh; ++j, ++J) {
         const int sl = J & 1;
-        const float ec = ex2_approx(cum_n * kLog2e);  // exp(cum_t)
-        if (j + 1 < nh) cum_n = head_cum(j + 1);
-        // the scales 2^s of H_c's rows p (pairs) that this thread's 32 columns use
-        const float4 *sp4 = reinterpret_cast<const float4 *>(
-            a.hsc + ((bi * a.nch + c) * pr.H + h0 + j) * 32 + 16 * eh);
-        float4 sc4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          sc4[i] = M2_OK(sp4 + i, 16, a.sp.hsc, &g_tc_errors) ? sp4[i]
-                                                            : make_float4(1.f, 1.f, 1.f, 1.f);
         ok = ok && mbar_wait_bounded(&sh.mma_done[sl], (uint32_t)((J >> 1) & 1), &g_tc_errors) &&
              mbar_wait_bounded(&sh.full_z[sl], (uint32_t)((J >> 1) & 1), &g_tc_errors);
         ok = __all_sync(0xffffffffu, ok) != 0;
         if (!ok) break;
         tc_fence_after();
+        const float ec = ex2_approx(sh.cum2[par][j][t]);  // exp(cum_t)
         const uint32_t ycol = tmem + lane_off + kTmemY + 64 * j + 32 * eh;
         const uint32_t zt = base + kZt + sl * 16384;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float v[16], w[16];
-          tmem_ld16(ycol + 16 * hh, v);
-          tmem_ld16(tmem + lane_off + kTmemT + 32 * eh + 16 * hh, w);
+          tmem_ld16x2(ycol + 16 * hh, v, tmem + lane_off + kTmemT + 32 * eh + 16 * hh, w);
           if (hh == 1) {
             tc_fence_before();
             mbar_arrive(&sh.t_free);  // the C H_c^T columns may take the next head's product
           }
-          const float scp[8] = {sc4[2 * hh].x, sc4[2 * hh].y, sc4[2 * hh].z, sc4[2 * hh].w,
-                                sc4[2 * hh + 1].x, sc4[2 * hh + 1].y, sc4[2 * hh + 1].z,
-                                sc4[2 * hh + 1].w};
+          // the scales 2^s of H_c's rows p (pairs) of these 16 columns, from their exponents
+          const uint2 se = *reinterpret_cast<const uint2 *>(&sh.scs[par][j][16 * eh + 8 * hh]);
+          float scp[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            scp[i] = __uint_as_float((127u + (((i < 4 ? se.x : se.y) >> (8 * (i & 3))) & 0xFFu)) << 23);
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = fmaf(ec * scp[i >> 1], w[i], v[i]);
           if (!pr.nbg) {
@@ -1478,9 +1517,22 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i) ss = fmaf(v[i], v[i], ss);
-          tmem_st16(ycol + 16 * hh, v);
+          tmem_st16_async(ycol + 16 * hh, v);
         }
         mbar_arrive(&sh.empty_z[sl]);
+      }
+      tmem_wait_st();  // the gated values are in TMEM before this thread reads them back
+      mbar_arrive(&sh.e1_done[par]);
+      // the unit's norm weights: loads issued now, stored to shared memory once the
+      // exchange below has been waited for (their latency overlaps it)
+      float nwv[2] = {0.0f, 0.0f};
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int idx = gt + kGroupThreads * r;
+        if (idx < nh * kHP) {
+          const float *wp = a.prm.norm_w + (int64_t)(h0 + idx / kHP) * kHP + idx % kHP;
+          nwv[r] = M2_OK(wp, 4, a.sp.norm_w, &g_tc_errors) ? __ldg(wp) : 0.0f;
+        }
       }
       // per-token sums of this CTA into part[par][rank][*] of every rank
       sh.half_ss[eh][t] = ss;
@@ -1501,6 +1553,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       float tot = 0.0f;
       for (int r = 0; r < cs; ++r) tot += sh.part[par][r][t];
       const float inv = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int idx = gt + kGroupThreads * r;
+        if (idx < nh * kHP) sh.nw[idx / kHP][idx % kHP] = nwv[r];
+      }
       ok = group_all(2, ok);
       // unit n + 2 uses this parity again; no rank sends it before this CTA has
       // sent unit n + 1's sums, which happens after this point
@@ -1556,7 +1613,7 @@ void out_choose(int hpg, int64_t units, int *cs, int *hpc, int *ncl) {
 }
 
 struct TcWorkspace {
-  float *S, *cum_end, *cum, *dtv, *hsc, *cbd;
+  float *S, *cum_end, *cum, *dtv, *hsc, *smax, *cbd;
   __half *Hc, *u;
 };
 
@@ -1577,6 +1634,8 @@ TcWorkspace tc_carve(const Problem &pr, char *base) {
   off += align_up(st * 2, 256);
   w.hsc = reinterpret_cast<float *>(base + off);
   off += align_up((size_t)pr.batch * nch * pr.H * 32 * 4, 256);
+  w.smax = reinterpret_cast<float *>(base + off);
+  off += align_up((size_t)pr.batch * nch * pr.H * 4, 256);
   w.cbd = reinterpret_cast<float *>(base + off);
   off += align_up((size_t)pr.batch * pr.G * nch * kQ * 4, 256);
   w.u = reinterpret_cast<__half *>(base + off);
@@ -1631,7 +1690,9 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank
 
 constexpr size_t kK1Smem = kK1Tiles + 1024;
 constexpr size_t kK3Smem = kTcOutTiles + sizeof(OutShared) + 1024;
-static_assert(kK1Smem <= 227 * 1024 && kK3Smem <= 227 * 1024, "shared memory per CTA");
+// (each kernel that uses tensor memory also holds 1 KB of static shared memory)
+static_assert(kK1Smem + 11 * 1024 <= 227 * 1024 && kK3Smem + 1024 <= 227 * 1024,
+              "shared memory per CTA");
 
 int out_max_clusters(int cs) {
   static int cache[64][17] = {};  // 0: not asked yet
@@ -1678,6 +1739,7 @@ size_t prefill_tc_workspace(const Problem &pr) {
   return align_up(st * 4, 256) + align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
          2 * align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256) + align_up(st * 2, 256) +
          align_up((size_t)pr.batch * nch * pr.H * 32 * 4, 256) +
+         align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
          align_up((size_t)pr.batch * pr.G * nch * kQ * 4, 256) +
          align_up((size_t)pr.batch * pr.L * pr.conv_dim * 2, 256);
 }
@@ -1719,6 +1781,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.dtv = w.dtv;
   a.Hc = w.Hc;
   a.hsc = w.hsc;
+  a.smax = w.smax;
   a.cbd = w.cbd;
   a.u = w.u;
   {
@@ -1736,6 +1799,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     a.sp.dtv = span_of(a.dtv, (size_t)pr.batch * nq * pr.H * kQ * 4);
     a.sp.Hc = span_of(a.Hc, st1 * 2);
     a.sp.hsc = span_of(a.hsc, (size_t)pr.batch * nq * pr.H * 32 * 4);
+    a.sp.smax = span_of(a.smax, (size_t)pr.batch * nq * pr.H * 4);
     a.sp.cbd = span_of(a.cbd, (size_t)pr.batch * pr.G * nq * kQ * 4);
     a.sp.u = span_of(a.u, (size_t)bl * pr.conv_dim * 2);
     a.sp.conv_w = span_of(a.prm.conv_w, (size_t)pr.conv_dim * 4 * 4);
@@ -1777,14 +1841,13 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   }
   stage_mark(st, 1);
   NvtxRange r2("tc_state_pass + tc_chunk_out");
-  dim3 g2((unsigned)(kPassBlocks + ceil_div(pr.conv_dim, 256)), (unsigned)pr.H,
-          (unsigned)pr.batch);
+  dim3 g2((unsigned)(pr.H * kPassBlocks + ceil_div(pr.conv_dim, kPassThreads)), (unsigned)pr.batch, 1);
   {
     // programmatic dependent launches: the state pass and the output kernel are
     // scheduled while their predecessor drains and wait for it on the device
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = g2;
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.blockDim = dim3(kPassThreads, 1, 1);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
