@@ -132,13 +132,51 @@ MAMBA2_API size_t mamba2_prefill_workspace_size(const mamba2_dims *dims);
  *          bytes, 256-byte aligned; contents on entry are ignored.
  *  stream  cudaStream_t as void*.
  * seqlen need not be a multiple of chunk_size.  seqlen == 0 copies or zeroes
- * the states and writes nothing else. */
+ * the states and writes nothing else.
+ * Range: bf16 I/O with headdim 64 and d_state 64 runs on the tensor cores with
+ * fp16 operands, so the post-conv activations x, B, C and the products
+ * x * dt * decay must stay below 2^15 in magnitude (larger values saturate);
+ * inputs of normal magnitude (|xBC| up to about 1e4) are far inside that.
+ * The carried SSM state has no such limit (its fp16 operand copy is scaled by
+ * a power of two per chunk and head; the returned state is fp32). */
 MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_params *params,
                                        const void *xBC, int64_t xBC_row_stride, const void *z,
                                        int64_t z_row_stride, const void *dt_raw,
                                        int64_t dt_row_stride, void *y, void *conv_state,
                                        float *ssm_state, int32_t states_in, void *workspace,
                                        size_t workspace_bytes, void *stream);
+
+/* Workspace bytes mamba2_conv_ssd_prefill_varlen needs for `dims` (batch =
+ * number of sequences, seqlen = total tokens); 0 if the dims are invalid or
+ * the call is not supported for them (see below). */
+MAMBA2_API size_t mamba2_prefill_varlen_workspace_size(const mamba2_dims *dims);
+
+/* Prefill of `batch` sequences of different lengths packed along the token
+ * axis, in one call (the chunked prefill of "Zamba2 hybrid architecture in
+ * Transformers", qwbw.cn, section 三 step 3, with a cache per sequence, for
+ * requests of different lengths served together as in the time-to-first-token
+ * scenario of the Zamba2-VL announcement, k7ail.com).  As
+ * mamba2_conv_ssd_prefill, except:
+ *  dims    batch = number of sequences, seqlen = L, the total token count.
+ *  xBC, z, dt_raw, y  as above for one row of L tokens: sequence s owns tokens
+ *          cu_seqlens[s] .. cu_seqlens[s + 1] - 1.  No chunk of the scan
+ *          spans two sequences, and no conv reaches across them.
+ *  cu_seqlens  device int32 [batch + 1], 4-byte aligned: 0, then the running
+ *          token counts, last = seqlen (empty sequences allowed).  Offsets
+ *          that break this are found on the device: the call then writes
+ *          nothing and mamba2_device_errors reports bit 2.
+ *  conv_state, ssm_state  per sequence ([batch, ...]), in and out as above;
+ *          a sequence of fewer than d_conv tokens shifts its conv state.
+ *  workspace   at least mamba2_prefill_varlen_workspace_size(dims) bytes.
+ * Supported on the tensor-core path only: bf16 I/O, headdim 64, d_state 64,
+ * at most 80 heads per group (MAMBA2_ERR_UNSUPPORTED otherwise).  The
+ * sequences' chunks are laid out on the device (one small kernel), so the
+ * host needs no copy of cu_seqlens. */
+MAMBA2_API int mamba2_conv_ssd_prefill_varlen(
+    const mamba2_dims *dims, const mamba2_params *params, const void *xBC,
+    int64_t xBC_row_stride, const void *z, int64_t z_row_stride, const void *dt_raw,
+    int64_t dt_row_stride, const int32_t *cu_seqlens, void *y, void *conv_state,
+    float *ssm_state, int32_t states_in, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Decode: advance every sequence by one token (qwbw.cn section 三 step 3,
  * the single-token recurrent update used when the cache holds the states and
@@ -169,7 +207,8 @@ MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *par
  * sets a flag and returns, leaving the context usable and the outputs of that
  * call undefined.  This call synchronises the current device, stores the
  * flags raised since the previous call in *flags (0 = none; bit 0 = a wait
- * ran out) and clears them.  Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG (flags
+ * ran out; bit 1 = the bounds-checked build skipped an access; bit 2 = a
+ * packed-sequence prefill got invalid cu_seqlens) and clears them.  Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG (flags
  * NULL) or MAMBA2_ERR_CUDA. */
 MAMBA2_API int mamba2_device_errors(unsigned int *flags);
 

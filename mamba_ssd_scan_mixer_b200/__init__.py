@@ -75,6 +75,11 @@ def lib() -> ctypes.CDLL:
         L.mamba2_conv_ssd_prefill.restype = ctypes.c_int
         L.mamba2_conv_ssd_prefill.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp, i32,
                                               vp, sz, vp]
+        L.mamba2_prefill_varlen_workspace_size.restype = sz
+        L.mamba2_prefill_varlen_workspace_size.argtypes = [pd]
+        L.mamba2_conv_ssd_prefill_varlen.restype = ctypes.c_int
+        L.mamba2_conv_ssd_prefill_varlen.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp,
+                                                     vp, vp, i32, vp, sz, vp]
         L.mamba2_conv_ssd_prefill_noalloc.restype = ctypes.c_int
         L.mamba2_conv_ssd_prefill_noalloc.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp,
                                                       vp, i32, vp]
@@ -184,6 +189,46 @@ def mamba2_conv_ssd_prefill(dims, params, xBC, z, dt_raw, y, conv_state=None, ss
         ws_bytes, _stream(stream))
     if st != 0:
         raise Mamba2Error(st, "mamba2_conv_ssd_prefill")
+
+
+def mamba2_prefill_varlen_workspace_size(dims: Mamba2Dims) -> int:
+    return int(lib().mamba2_prefill_varlen_workspace_size(ctypes.byref(dims)))
+
+
+def mamba2_conv_ssd_prefill_varlen(dims, params, xBC, z, dt_raw, cu_seqlens, y, conv_state=None,
+                                   ssm_state=None, states_in=False, workspace=None,
+                                   stream=None) -> None:
+    """Enqueue one prefill of dims.batch sequences packed along the token axis
+    (dims.seqlen = total tokens): xBC [T, conv_dim], z [T, d_inner], dt_raw [T, H]
+    (unit last stride, row strides passed through), y [T, d_inner] contiguous;
+    cu_seqlens: CUDA int32 [batch + 1] (0, running token counts, T); states per
+    sequence; workspace of mamba2_prefill_varlen_workspace_size(dims) bytes."""
+    lx = _rows(xBC, "xBC", None, 1, 0)
+    lz = _rows(z, "z", None, 1, 0)
+    ld = _rows(dt_raw, "dt_raw", None, 1, 0)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().mamba2_conv_ssd_prefill_varlen(
+        ctypes.byref(dims), ctypes.byref(params), _ptr(xBC), lx, _ptr(z), lz, _ptr(dt_raw), ld,
+        _ptr(cu_seqlens), _ptr(y), _ptr(conv_state), _ptr(ssm_state), int(bool(states_in)),
+        _ptr(workspace), ws_bytes, _stream(stream))
+    if st != 0:
+        raise Mamba2Error(st, "mamba2_conv_ssd_prefill_varlen")
+
+
+def prefill_varlen(dims, params, xBC, z, dt_raw, cu_seqlens, conv_state=None, ssm_state=None,
+                   states_in=False, workspace=None, y=None, stream=None):
+    """Allocate y (and the workspace if not given) and run a packed-sequence prefill.
+    Returns y [T, d_inner]; the states, if given, are updated in place."""
+    import torch
+    if y is None:
+        y = torch.empty(dims.seqlen, dims.nheads * dims.headdim, dtype=xBC.dtype,
+                        device=xBC.device)
+    if workspace is None:
+        workspace = torch.empty(max(1, mamba2_prefill_varlen_workspace_size(dims)),
+                                dtype=torch.uint8, device=xBC.device)
+    mamba2_conv_ssd_prefill_varlen(dims, params, xBC, z, dt_raw, cu_seqlens, y, conv_state,
+                                   ssm_state, states_in, workspace, stream)
+    return y
 
 
 def mamba2_conv_ssd_prefill_noalloc(dims, params, xBC, z, dt_raw, y, conv_state=None,

@@ -185,17 +185,19 @@ MAMBA2_API size_t mamba2_prefill_workspace_size(const mamba2_dims *dims) {
   return prefill_workspace(pr);
 }
 
-MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_params *params,
-                                       const void *xBC, int64_t xBC_row_stride, const void *z,
-                                       int64_t z_row_stride, const void *dt_raw,
-                                       int64_t dt_row_stride, void *y, void *conv_state,
-                                       float *ssm_state, int32_t states_in, void *workspace,
-                                       size_t workspace_bytes, void *stream) {
-  NvtxRange range("mamba2_conv_ssd_prefill");
-  DisarmOnExit disarm;
+namespace m2 {
+namespace {
+// The shared body of the fixed-length and the packed-sequence prefill: dims,
+// pointers and strides checked, the no-token case, then the launch.
+int prefill_entry(const mamba2_dims *dims, const mamba2_params *params, const void *xBC,
+                  int64_t xBC_row_stride, const void *z, int64_t z_row_stride,
+                  const void *dt_raw, int64_t dt_row_stride, const int32_t *cu_seqlens,
+                  void *y, void *conv_state, float *ssm_state, int32_t states_in,
+                  void *workspace, size_t workspace_bytes, void *stream) {
   Problem pr;
   int st = make_problem(dims, true, &pr);
   if (st != MAMBA2_OK) return st;
+  const bool varlen = cu_seqlens != nullptr;
   if (!params_ok(params)) return MAMBA2_ERR_INVALID_ARG;
   if (states_in != 0 && states_in != 1) return MAMBA2_ERR_INVALID_ARG;
   if (states_in && (conv_state == nullptr || ssm_state == nullptr)) return MAMBA2_ERR_INVALID_ARG;
@@ -212,7 +214,8 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
     if (xBC_row_stride % 8 != 0 || z_row_stride % 8 != 0) return MAMBA2_ERR_INVALID_ARG;
     if (!aligned(xBC, 16) || !aligned(z, 16) || !aligned(y, 16) || !aligned(dt_raw, esz))
       return MAMBA2_ERR_INVALID_ARG;
-    const size_t need = prefill_workspace(pr);
+    if (varlen && !prefill_tc_supported(pr, true)) return MAMBA2_ERR_UNSUPPORTED;
+    const size_t need = varlen ? prefill_tc_workspace(pr, true) : prefill_workspace(pr);
     if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
       return MAMBA2_ERR_WORKSPACE;
   } else {
@@ -244,8 +247,45 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
   a.states_in = states_in;
   a.ws = static_cast<char *>(workspace);
   a.stream = s;
-  return (use_tc(pr) ? prefill_tc(a) : prefill_simt(a)) == cudaSuccess ? MAMBA2_OK
-                                                                      : MAMBA2_ERR_CUDA;
+  a.cu_seqlens = cu_seqlens;
+  return (varlen || use_tc(pr) ? prefill_tc(a) : prefill_simt(a)) == cudaSuccess
+             ? MAMBA2_OK
+             : MAMBA2_ERR_CUDA;
+}
+}  // namespace
+}  // namespace m2
+
+MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_params *params,
+                                       const void *xBC, int64_t xBC_row_stride, const void *z,
+                                       int64_t z_row_stride, const void *dt_raw,
+                                       int64_t dt_row_stride, void *y, void *conv_state,
+                                       float *ssm_state, int32_t states_in, void *workspace,
+                                       size_t workspace_bytes, void *stream) {
+  NvtxRange range("mamba2_conv_ssd_prefill");
+  DisarmOnExit disarm;
+  return m2::prefill_entry(dims, params, xBC, xBC_row_stride, z, z_row_stride, dt_raw,
+                           dt_row_stride, nullptr, y, conv_state, ssm_state, states_in,
+                           workspace, workspace_bytes, stream);
+}
+
+MAMBA2_API size_t mamba2_prefill_varlen_workspace_size(const mamba2_dims *dims) {
+  Problem pr;
+  if (make_problem(dims, true, &pr) != MAMBA2_OK || pr.L < 1 || !prefill_tc_supported(pr, true))
+    return 0;
+  return prefill_tc_workspace(pr, true);
+}
+
+MAMBA2_API int mamba2_conv_ssd_prefill_varlen(
+    const mamba2_dims *dims, const mamba2_params *params, const void *xBC,
+    int64_t xBC_row_stride, const void *z, int64_t z_row_stride, const void *dt_raw,
+    int64_t dt_row_stride, const int32_t *cu_seqlens, void *y, void *conv_state,
+    float *ssm_state, int32_t states_in, void *workspace, size_t workspace_bytes, void *stream) {
+  NvtxRange range("mamba2_conv_ssd_prefill_varlen");
+  DisarmOnExit disarm;
+  if (cu_seqlens == nullptr || !m2::aligned(cu_seqlens, 4)) return MAMBA2_ERR_INVALID_ARG;
+  return m2::prefill_entry(dims, params, xBC, xBC_row_stride, z, z_row_stride, dt_raw,
+                           dt_row_stride, cu_seqlens, y, conv_state, ssm_state, states_in,
+                           workspace, workspace_bytes, stream);
 }
 
 MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *params,

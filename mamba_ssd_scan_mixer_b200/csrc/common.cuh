@@ -40,6 +40,9 @@ struct PrefillArgs {
   int states_in;
   char *ws;
   cudaStream_t stream;
+  // packed sequences of different lengths (batch = sequences, pr.L = total
+  // tokens): device [batch + 1] first token of each sequence; null otherwise
+  const int32_t *cu_seqlens = nullptr;
 };
 
 struct StepArgs {
@@ -253,6 +256,9 @@ __device__ __forceinline__ bool test_stall(const unsigned int *stall, unsigned i
 // (TMA) are bounded by their tensor maps and need no check.  In the ordinary
 // build the checks compile to nothing.
 constexpr unsigned int kErrBounds = 2u;
+// bit 2 of mamba2_device_errors: a packed-sequence prefill got sequence offsets
+// that do not start at 0, decrease, or do not end at the total token count
+constexpr unsigned int kErrSeqlens = 4u;
 struct Span {  // [lo, hi) byte addresses of one device buffer (lo == hi: none)
   unsigned long long lo, hi;
 };
@@ -471,8 +477,8 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
 }
 
 cudaError_t prefill_tc(const PrefillArgs &a);
-size_t prefill_tc_workspace(const Problem &pr);
-bool prefill_tc_supported(const Problem &pr);
+size_t prefill_tc_workspace(const Problem &pr, bool varlen = false);
+bool prefill_tc_supported(const Problem &pr, bool varlen = false);
 cudaError_t take_prefill_tc_errors(unsigned int *out);
 extern const char *const kPrefillTcStages[];
 extern const int kPrefillTcStageCount;

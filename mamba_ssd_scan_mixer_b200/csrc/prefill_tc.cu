@@ -33,6 +33,7 @@
 
 #include <algorithm>
 #include <cstddef>
+#include <cstring>
 
 #include "common.cuh"
 
@@ -83,7 +84,43 @@ struct TcArgs {
   __half *u;                     // [b][L][conv_dim] post-conv x | B | C, fp16
   int hpc;                       // max heads per CTA in tc_chunk_out
   int y32;                       // y is 32-byte aligned: rows are written in whole 32-byte sectors
+  // packed sequences of different lengths (batch = sequences, L = total tokens):
+  // chunk positions come from vl_chunks, written by tc_varlen_prep_kernel
+  int varlen;
+  const int4 *vl_chunks;         // [chunk capacity] {sequence, chunk in it, valid tokens, first token}
+  const int *vl_chunk0;          // [batch + 2] first global chunk of each sequence, the total,
+                                 // then 1 if the offsets were valid (0: the call does nothing)
+  const int *cu_seqlens;         // [batch + 1] first token of each sequence (last: L)
 };
+
+// Where global chunk gc lies: its sequence, its index in that sequence, its
+// valid tokens (1 .. 128) and its first token in the packed token order (row
+// r of a fixed-length batch starts at token r L).
+struct ChunkPos {
+  int seq, c, nv;
+  int64_t t0;
+};
+__device__ __forceinline__ ChunkPos chunk_pos(const TcArgs &a, int64_t gc) {
+  ChunkPos p;
+  if (a.varlen) {
+    const int4 e = a.vl_chunks[gc];
+    p.seq = e.x;
+    p.c = e.y;
+    p.nv = e.z;
+    p.t0 = (int64_t)(uint32_t)e.w;
+  } else {
+    p.seq = (int)(gc / a.nch);
+    p.c = (int)(gc - (int64_t)p.seq * a.nch);
+    p.t0 = (int64_t)p.seq * a.pr.L + (int64_t)p.c * 128;
+    p.nv = (int)min((int64_t)128, a.pr.L - (int64_t)p.c * 128);
+  }
+  return p;
+}
+// Chunks of the call: b * chunks per row, or (packed sequences) as counted by
+// the prep kernel.
+__device__ __forceinline__ int64_t total_chunks(const TcArgs &a) {
+  return a.varlen ? (int64_t)a.vl_chunk0[a.pr.batch] : a.pr.batch * (int64_t)a.nch;
+}
 
 // silu(v) = v * sigmoid(v) with sigmoid(v) = (1 + tanh(v / 2)) / 2, using the
 // hardware tanh approximation (one special-function op per element).
@@ -113,19 +150,20 @@ __device__ __forceinline__ float warp_scan(float v, int lane) {
   return v;
 }
 
-// Post-conv activations of 8 channels x 4 tokens -> u (fp16), tokens < L only.
-__device__ __forceinline__ void store_u(const TcArgs &a, int64_t bi, int64_t t0, int64_t ch,
+// Post-conv activations of 8 channels x 4 tokens (rows s0 .. s0 + 3 of the chunk
+// starting at token t0) -> u (fp16), the chunk's nv valid tokens only.
+__device__ __forceinline__ void store_u(const TcArgs &a, int64_t t0, int s0, int nv, int64_t ch,
                                         const float (&v)[4][8]) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const int64_t t = t0 + k;
-    if (t < a.pr.L) {
+    const int64_t t = t0 + s0 + k;
+    if (s0 + k < nv) {
       uint4 o;
       o.x = pack_half2(v[k][0], v[k][1]);
       o.y = pack_half2(v[k][2], v[k][3]);
       o.z = pack_half2(v[k][4], v[k][5]);
       o.w = pack_half2(v[k][6], v[k][7]);
-      uint4 *dst = reinterpret_cast<uint4 *>(a.u + (bi * a.pr.L + t) * a.pr.conv_dim + ch);
+      uint4 *dst = reinterpret_cast<uint4 *>(a.u + t * a.pr.conv_dim + ch);
       if (M2_OK(dst, 16, a.sp.u, &g_tc_errors)) *dst = o;
     }
   }
@@ -242,7 +280,8 @@ constexpr uint32_t kK1Ahi = kK1BC + 2 * kRawBytes, kK1Alo = kK1Ahi + kK1A, kK1Bh
                    kK1Blo = kK1Bhi + kK1B, kK1Tiles = kK1Blo + kK1B;
 
 struct K1Maps {
-  CUtensorMap xbc;  // [b][L][conv_dim] bf16 (row stride ld_x), box 64 ch x 136 tokens
+  CUtensorMap xbc;   // [b][L][conv_dim] bf16 (row stride ld_x), box 64 ch x 136 tokens
+  CUtensorMap xbc2;  // packed sequences: [L tokens][conv_dim], the same box
 };
 
 // conv1d + SiLU of the 8 channels in 16-byte column `cg` of a raw tile, for
@@ -282,25 +321,35 @@ __device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, cons
 }
 
 struct K1Item {
-  int bi;  // row (every index of the item fits in 32 bits)
-  int c, g, pair;
-  unsigned key;  // (row, chunk, group) index
+  int gc;        // global chunk (every index of the item fits in 32 bits)
+  int seq, c;    // its sequence (row) and chunk in the sequence
+  int nv;        // valid tokens of the chunk
+  int64_t t0;    // first token of the chunk
+  int g, pair;
+  unsigned key;  // (global chunk, group) index
   bool isC;
   bool freshB;  // B must be convolved (the CTA's previous item had another key)
 };
 
-// Item `it`, the k-th of its CTA.  Items are ordered (row, chunk, group, r) with
-// r = 0 .. pairs - 1 the head pairs and r = pairs the C item; every index fits
-// in 32 bits (the launch checks the item count).
-__device__ __forceinline__ K1Item k1_item(const Problem &pr, int nch, int pairs, int it, int k) {
+// Item `it`, the k-th of its CTA.  Items are ordered (global chunk, group, r)
+// with r = 0 .. pairs - 1 the head pairs and r = pairs the C item; every index
+// fits in 32 bits (the launch checks the item count).
+__device__ __forceinline__ bool k1_is_c(int pairs, int it) {
+  return it % (pairs + 1) == pairs;
+}
+__device__ __forceinline__ K1Item k1_item(const TcArgs &a, int pairs, int it, int k) {
   const unsigned key = (unsigned)it / (unsigned)(pairs + 1);
   const int r = it - (int)key * (pairs + 1);
-  const unsigned bc = key / (unsigned)pr.G;
+  const unsigned gc = key / (unsigned)a.pr.G;
   K1Item w;
   w.key = key;
-  w.g = (int)(key - bc * (unsigned)pr.G);
-  w.bi = (int)(bc / (unsigned)nch);
-  w.c = (int)(bc - (unsigned)w.bi * (unsigned)nch);
+  w.g = (int)(key - gc * (unsigned)a.pr.G);
+  w.gc = (int)gc;
+  const ChunkPos pos = chunk_pos(a, gc);
+  w.seq = pos.seq;
+  w.c = pos.c;
+  w.nv = pos.nv;
+  w.t0 = pos.t0;
   w.isC = r == pairs;
   w.pair = w.isC ? 0 : r;
   w.freshB = !w.isC && (k == 0 || r == 0);
@@ -325,8 +374,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                  sBlo = base + kK1Blo;
   const int hpg = pr.heads_per_group();
   const int pairs = (hpg + 1) / 2;
-  const int it0 = (int)((int64_t)n_items * blockIdx.x / gridDim.x),
-            it1 = (int)((int64_t)n_items * (blockIdx.x + 1) / gridDim.x);
+  // items past the call's chunks (packed sequences: n_items is a capacity) are void
+  const int n_real = (int)min((int64_t)n_items, total_chunks(a) * pr.G * (pairs + 1));
+  const int it0 = min(n_real, (int)((int64_t)n_items * blockIdx.x / gridDim.x)),
+            it1 = min(n_real, (int)((int64_t)n_items * (blockIdx.x + 1) / gridDim.x));
 
   if (warp == 0) tmem_alloc(&tmem_holder, 128);
   if (tid == 0) {
@@ -360,7 +411,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     bool ok = true;
     for (int it = it0; ok && it < it1; ++it, ++k) {
       const int st = k & 1;
-      const K1Item w = k1_item(pr, a.nch, pairs, it, k);
+      const K1Item w = k1_item(a, pairs, it, k);
       const bool useBC = w.isC || w.freshB;
       const int bcb = (int)(w.key & 1u);
       const int bc_use = !useBC ? 0 : (bcb ? bc_use1++ : bc_use0++);
@@ -394,9 +445,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int64_t tt = c0 + 4 * lane + q;
-          const __nv_bfloat16 *dp = a.dt_raw + (w.bi * pr.L + tt) * a.ld_dt + hA + half;
-          dtr[half][q] = (hv && tt < pr.L && M2_OK(dp, 2, a.sp.dt, &g_tc_errors))
+          const int li = 4 * lane + q;  // token of the chunk
+          const __nv_bfloat16 *dp = a.dt_raw + (w.t0 + li) * a.ld_dt + hA + half;
+          dtr[half][q] = (hv && li < w.nv && M2_OK(dp, 2, a.sp.dt, &g_tc_errors))
                              ? __bfloat162float(*dp)
                              : -INFINITY;
         }
@@ -435,7 +486,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             wsv[half][q] = expf(sfx[q]) * dt4[q];
           }
           if (hv) {
-            const int64_t row = ((int64_t)w.bi * a.nch + w.c) * pr.H + hA + half;
+            const int64_t row = (int64_t)w.gc * pr.H + hA + half;
             float4 *cp = reinterpret_cast<float4 *>(a.cum + row * kQ) + lane;
             float4 *dp = reinterpret_cast<float4 *>(a.dtv + row * kQ) + lane;
             if (M2_OK(cp, 16, a.sp.cum, &g_tc_errors)) *cp = make_float4(cq[0], cq[1], cq[2], cq[3]);
@@ -457,10 +508,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       }
       ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
       if (!ok) break;
-      // the first chunk of a sequence that continues from a carried conv state: its
-      // tiles land on a side barrier, then rows 0..2 (tokens -3 .. -1, read as zeros)
-      // are overwritten with that state before the stage is released
-      const bool halo = c0 == 0 && a.states_in;
+      // the first chunk of a sequence that continues from a carried conv state (or of
+      // a packed sequence, whose rows before it belong to the previous one): its
+      // tiles land on a side barrier, then rows 0..2 (tokens -3 .. -1) are
+      // overwritten with that state (or zeros) before the stage is released
+      const bool halo = w.c == 0 && (a.states_in || a.varlen);
       const uint32_t stage = base + st * kK1Stage;
       const uint32_t bcbuf = base + kK1BC + bcb * kRawBytes;
       const int64_t bc_ch = pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
@@ -469,15 +521,17 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         const uint32_t nbytes =
             (w.isC ? 1u : (1u + (hasB ? 1u : 0u))) * kRawBytes + (useBC ? kRawBytes : 0u);
         mbar_arrive_expect_tx(bar, nbytes);
-        if (w.isC)
-          tma_load_3d(stage, &maps.xbc, (int)(pr.d_inner + (int64_t)w.g * kNS), (int)c0 - 3,
-                      (int)w.bi, bar);
+        // raw rows c0 - 3 .. c0 + 132 of the item's channels starting at `ch`
+        auto load_raw = [&](uint32_t dst, int ch) {
+          if (a.varlen) tma_load_2d(dst, &maps.xbc2, ch, (int)(w.t0 - 3), bar);
+          else tma_load_3d(dst, &maps.xbc, ch, (int)c0 - 3, w.seq, bar);
+        };
+        if (w.isC) load_raw(stage, (int)(pr.d_inner + (int64_t)w.g * kNS));
         if (!w.isC) {
-          tma_load_3d(stage, &maps.xbc, hA * kHP, (int)c0 - 3, (int)w.bi, bar);
-          if (hasB)
-            tma_load_3d(stage + kRawBytes, &maps.xbc, (hA + 1) * kHP, (int)c0 - 3, (int)w.bi, bar);
+          load_raw(stage, hA * kHP);
+          if (hasB) load_raw(stage + kRawBytes, (hA + 1) * kHP);
         }
-        if (useBC) tma_load_3d(bcbuf, &maps.xbc, (int)bc_ch, (int)c0 - 3, (int)w.bi, bar);
+        if (useBC) load_raw(bcbuf, (int)bc_ch);
       }
       if (halo) {
         const int nh_used = st ? halo_use1++ : halo_use0++;
@@ -490,9 +544,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
           const int sl = idx / 192, r = (idx / 64) % 3, chn = idx % 64;
           if (!slot_on(sl)) continue;
           const int64_t ch = slot_ch(sl) + chn;
-          const __nv_bfloat16 *hp = a.conv_in + (w.bi * pr.conv_dim + ch) * 4 + 1 + r;
-          const __nv_bfloat16 v =
-              M2_OK(hp, 2, a.sp.conv, &g_tc_errors) ? *hp : __float2bfloat16(0.0f);
+          const __nv_bfloat16 *hp = a.conv_in + ((int64_t)w.seq * pr.conv_dim + ch) * 4 + 1 + r;
+          const __nv_bfloat16 v = a.states_in && M2_OK(hp, 2, a.sp.conv, &g_tc_errors)
+                                      ? *hp
+                                      : __float2bfloat16(0.0f);
           const uint32_t tile = sl < 2 ? stage + sl * kRawBytes : bcbuf;
           const uint32_t addr = tile + r * 128 + ((((chn >> 3) ^ r) & 7) << 4) + ((chn & 7) << 1);
           asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(v))
@@ -540,7 +595,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       const uint32_t As[3] = {sAhi, sAhi, sAlo}, Bs[3] = {sBhi, sBlo, sBhi};
       int np = 0;
       for (int it = it0; it < it1; ++it) {
-        if (k1_item(pr, a.nch, pairs, it, 1).isC) continue;
+        if (k1_is_c(pairs, it)) continue;
         if (!mbar_wait_bounded(&ops_ready, (uint32_t)(np & 1), &g_tc_errors)) break;
         if (np >= 2 &&
             !mbar_wait_bounded(&tmem_free[np & 1], (uint32_t)(((np - 2) >> 1) & 1), &g_tc_errors))
@@ -569,8 +624,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     // + lane (head half m / 64, lane p = m % 64), 16 columns per warp / 4; S is kept
     // [n/4][p][4] per head so that a warp's float4 stores are contiguous
     struct Pending {
-      int bi;
-      int c, hA;
+      int gc, hA;
       bool hasB;
     } pw{};
     auto store_states = [&](const Pending &q, int acc) {
@@ -587,11 +641,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (half == 0 || q.hasB) {
-        float *mp = a.smax + ((int64_t)q.bi * a.nch + q.c) * pr.H + q.hA + half;
+        float *mp = a.smax + (int64_t)q.gc * pr.H + q.hA + half;
         if (lane == 0 && M2_OK(mp, 4, a.sp.smax, &g_tc_errors))
           atomicMax(reinterpret_cast<int *>(mp), __float_as_int(mx));
         float4 *dst = reinterpret_cast<float4 *>(
-            a.S + (((int64_t)q.bi * a.nch + q.c) * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
+            a.S + ((int64_t)q.gc * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           if (M2_OK(dst + (4 * cb + i) * kHP + p, 16, a.sp.S, &g_tc_errors))
@@ -606,14 +660,13 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     for (int it = it0; ok && it < it1; ++it, ++k) {
       const int st = k & 1;
       const uint32_t stage = base + st * kK1Stage;
-      const K1Item w = k1_item(pr, a.nch, pairs, it, k);
+      const K1Item w = k1_item(a, pairs, it, k);
       const int bcb = (int)(w.key & 1u);
       {
         const bool got = mbar_wait_bounded(&full[st], (uint32_t)((k >> 1) & 1), &g_tc_errors);
         ok = __all_sync(0xffffffffu, got) != 0;
       }
       if (!ok) break;
-      const int64_t c0 = (int64_t)w.c * kQ;
       const int hA = w.g * hpg + 2 * w.pair;
       const bool hasB = 2 * w.pair + 1 < hpg;
       const uint32_t bcbuf = base + kK1BC + bcb * kRawBytes;
@@ -677,7 +730,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         if (warp < 8) {
           conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v);
           mbar_arrive(&bc_empty[bcb]);
-          store_u(a, w.bi, c0 + s0, bc_ch + cg * 8, v);
+          store_u(a, w.t0, s0, w.nv, bc_ch + cg * 8, v);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
@@ -721,7 +774,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             ok = __all_sync(0xffffffffu, got) != 0;
             if (ok && (lane & 3) == 0) {
               const float4 o = *reinterpret_cast<const float4 *>(&cbd_s[cpar][s0]);
-              float4 *dp = reinterpret_cast<float4 *>(a.cbd + (((int64_t)w.bi * pr.G + w.g) * a.nch + w.c) * kQ + s0);
+              float4 *dp = reinterpret_cast<float4 *>(a.cbd + ((int64_t)w.gc * pr.G + w.g) * kQ + s0);
               if (M2_OK(dp, 16, a.sp.cbd, &g_tc_errors))
                 *dp = make_float4(d4[0] + o.x, d4[1] + o.y, d4[2] + o.z, d4[3] + o.w);
             }
@@ -738,14 +791,14 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         if (!ok) break;
         if (warp < 8) {
           conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v);
-          if (w.pair == 0) store_u(a, w.bi, c0 + s0, bc_ch + cg * 8, v);
+          if (w.pair == 0) store_u(a, w.t0, s0, w.nv, bc_ch + cg * 8, v);
           put_operands(2, v, tile_weights(2));
           mbar_arrive(&bc_empty[bcb]);
         }
         if (sl == 1 && !hasB) zero_tile();
         else {
           conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
-          store_u(a, w.bi, c0 + s0, xch + cg * 8, v);
+          store_u(a, w.t0, s0, w.nv, xch + cg * 8, v);
           put_operands(sl, v, tile_weights(sl));
         }
         mbar_arrive(&empty[st]);
@@ -768,7 +821,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(&ops_ready);  // the MMA warp issues S = (x o w)^T B into accumulator np % 2
-        if (has_tile) store_u(a, w.bi, c0 + s0, xch + cg * 8, v);
+        if (has_tile) store_u(a, w.t0, s0, w.nv, xch + cg * 8, v);
       }
       if (w.freshB) {
         fence_proxy_async_smem();
@@ -776,8 +829,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       }
       // meanwhile: the previous pair item's chunk states out of its accumulator
       if (np >= 1) store_states(pw, (np - 1) & 1);
-      pw.bi = w.bi;
-      pw.c = w.c;
+      pw.gc = w.gc;
       pw.hA = hA;
       pw.hasB = hasB;
       ++np;
@@ -791,6 +843,71 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   __syncthreads();
   launch_dependents();
   if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+// ============================================================== packed sequences
+// One block: checks the sequence offsets (0 first, non-decreasing, the total
+// token count last), counts each sequence's chunks, scans the counts into
+// chunk0 and writes every chunk's position {sequence, chunk in it, valid tokens,
+// first token}; chunk0[nseq + 1] = 1.  Offsets that fail the check raise
+// kErrSeqlens and leave zero chunks and chunk0[nseq + 1] = 0, so that the
+// kernels after it do nothing.
+constexpr int kPrepThreads = 1024;
+__global__ void __launch_bounds__(kPrepThreads)
+    tc_varlen_prep_kernel(const int *cu, int nseq, int64_t L, int64_t cap, int4 *chunks,
+                          int *chunk0) {
+  __shared__ int bad;
+  __shared__ int wsum[kPrepThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) bad = (cu[0] != 0 || (int64_t)cu[nseq] != L) ? 1 : 0;
+  __syncthreads();
+  // thread tid takes sequences [s0, s1)
+  const int per = (nseq + kPrepThreads - 1) / kPrepThreads;
+  const int s0 = min(nseq, tid * per), s1 = min(nseq, s0 + per);
+  int local = 0;
+  for (int s = s0; s < s1; ++s) {
+    const int len = cu[s + 1] - cu[s];
+    if (len < 0) bad = 1;
+    local += len > 0 ? (len + kQ - 1) / kQ : 0;
+  }
+  // exclusive scan of the per-thread counts
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < kPrepThreads / 32 ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    if (lane < kPrepThreads / 32) wsum[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  const bool ok = bad == 0;
+  int run = incl - local + (warp > 0 ? wsum[warp - 1] : 0);  // chunks before s0
+  if (!ok || (int64_t)wsum[kPrepThreads / 32 - 1] > cap) {
+    if (tid == 0) atomicOr(&g_tc_errors, kErrSeqlens);
+    for (int s = tid; s <= nseq + 1; s += kPrepThreads) chunk0[s] = 0;
+    return;
+  }
+  for (int s = s0; s < s1; ++s) {
+    chunk0[s] = run;
+    const int len = cu[s + 1] - cu[s];
+    const int n = len > 0 ? (len + kQ - 1) / kQ : 0;
+    for (int c = 0; c < n; ++c)
+      chunks[run + c] = make_int4(s, c, min(kQ, len - c * kQ), cu[s] + c * kQ);
+    run += n;
+  }
+  if (tid == kPrepThreads - 1) {
+    chunk0[nseq] = wsum[kPrepThreads / 32 - 1];
+    chunk0[nseq + 1] = 1;
+  }
 }
 
 // ============================================================== state passing
@@ -828,7 +945,21 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
   grid_dependency_wait();  // the chunk-state kernel's results (launched early, see prefill_tc)
   launch_dependents();
   const Problem &pr = a.pr;
-  const int64_t bi = blockIdx.y;
+  const int64_t bi = blockIdx.y;  // sequence (row)
+  if (a.varlen && a.vl_chunk0[pr.batch + 1] == 0) return;  // invalid offsets: nothing to do
+  // its chunks [cb0, cb0 + nchs) and tokens [t0s, t0s + Ls)
+  int64_t cb0, nchs, t0s, Ls;
+  if (a.varlen) {
+    cb0 = a.vl_chunk0[bi];
+    nchs = a.vl_chunk0[bi + 1] - cb0;
+    t0s = a.cu_seqlens[bi];
+    Ls = a.cu_seqlens[bi + 1] - t0s;
+  } else {
+    cb0 = bi * a.nch;
+    nchs = a.nch;
+    t0s = bi * pr.L;
+    Ls = pr.L;
+  }
   const int nrb = pr.H * kPassBlocks;
   if ((int)blockIdx.x >= nrb) {
     if (cs == nullptr) return;
@@ -838,8 +969,8 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
     __nv_bfloat16 v[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int64_t tau = pr.L - 4 + k;
-      const __nv_bfloat16 *xp = a.xBC + (bi * pr.L + tau) * a.ld_x + ch;
+      const int64_t tau = Ls - 4 + k;
+      const __nv_bfloat16 *xp = a.xBC + (t0s + tau) * a.ld_x + ch;
       v[k] = __float2bfloat16(0.0f);
       if (tau >= 0) {
         if (M2_OK(xp, 2, a.sp.xbc, &g_tc_errors)) v[k] = *xp;
@@ -878,7 +1009,7 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
     for (int w = 0; w < kPassThreads / 32; ++w) bnd = fmaxf(bnd, red[w]);
   }
   const int64_t stride = (int64_t)pr.H * kHP * kNS;  // one chunk further
-  const int64_t c0h = bi * a.nch * pr.H + h;           // (row, chunk 0, head)
+  const int64_t c0h = cb0 * pr.H + h;                  // (first chunk, head)
   const float *S = a.S + c0h * (int64_t)(kHP * kNS) + 4 * j;
   __half *Hc = a.Hc + c0h * (int64_t)(kHP * kNS) + (4 * n4) * kHP + p;
   const float *ce = a.cum_end + c0h;
@@ -906,7 +1037,7 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
   // loads run 8 chunks ahead of the (sequential) recurrence
   constexpr int kAhead = 8;
   int c = 0;
-  for (; c + kAhead <= a.nch; c += kAhead) {
+  for (; c + kAhead <= nchs; c += kAhead) {
     float4 sv[kAhead];
     float d[kAhead], msv[kAhead];
 #pragma unroll
@@ -924,7 +1055,7 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
       step(sv[k], d[k], msv[k]);
     }
   }
-  for (; c < a.nch; ++c) {
+  for (; c < nchs; ++c) {
     put(c);
     const float *sp = S + c * stride;
     const int64_t r = (int64_t)c * pr.H;
@@ -1005,6 +1136,8 @@ struct OutMaps {
   CUtensorMap u;   // [b][L][conv_dim] fp16, box 64 ch x 128 tokens
   CUtensorMap z;   // [b][L][d_inner] bf16 (row stride ld_z), box 64 x 128
   CUtensorMap hc;  // [rows][64] fp16, box 64 x 64
+  CUtensorMap u2;  // packed sequences: u and z as [L tokens][channels], the same boxes
+  CUtensorMap z2;
 };
 
 // 16-byte asynchronous store into another rank's shared memory that completes
@@ -1068,14 +1201,12 @@ __device__ __forceinline__ void st_global_v8(void *p, const uint32_t (&v)[8]) {
                : "memory");
 }
 
-// Unit n of cluster `cid`: (row bi, chunk c, group g).
-__device__ __forceinline__ void out_unit(const Problem &pr, int nch, int ncl, int cid, int n,
-                                         int64_t &bi, int &c, int &g) {
+// Unit n of cluster `cid`: (global chunk gc, group g).
+__device__ __forceinline__ void out_unit(const Problem &pr, int ncl, int cid, int n, int64_t &gc,
+                                         int &g) {
   const int64_t u = cid + (int64_t)n * ncl;
   g = (int)(u % pr.G);
-  const int64_t bc = u / pr.G;
-  c = (int)(bc % nch);
-  bi = bc / nch;
+  gc = u / pr.G;
 }
 
 // One 32-column group k of row t of the decay operand A_j (j = head), written as
@@ -1167,7 +1298,7 @@ __device__ __forceinline__ void build_a_group(const OutShared &sh, int par, int 
 __global__ void __launch_bounds__(kWsThreads, 1)
     tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps, int ncl) {
   if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA of every cluster alike
-  extern __shared__ __align__(16) unsigned char smem_raw[];  // aligned to 1024 below
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   int cs, rank;
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs));
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
@@ -1180,7 +1311,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   const int hpg = pr.heads_per_group();
   const int lh0 = rank * a.hpc;
   const int nh = max(0, min(a.hpc, hpg - lh0));  // heads of this CTA in every unit
-  const int64_t n_all = pr.batch * (int64_t)a.nch * pr.G;
+  const int64_t n_all = total_chunks(a) * pr.G;
   const int n_units = n_all > cid ? (int)((n_all - cid + ncl - 1) / ncl) : 0;
   const uint32_t sum_bytes = (uint32_t)cs * kQ * 4;  // partial sums this CTA receives per unit
 
@@ -1224,13 +1355,14 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   auto output_head = [&](int un, int j, float inv) {
     const int q = warp & 3, eh = (warp >> 2) & 1, t = 32 * q + lane;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    int64_t obi;
-    int oc, og;
-    out_unit(pr, a.nch, ncl, cid, un, obi, oc, og);
+    int64_t ogc;
+    int og;
+    out_unit(pr, ncl, cid, un, ogc, og);
+    const ChunkPos pos = chunk_pos(a, ogc);
     const int h = og * hpg + lh0 + j;
-    const int64_t tok = (int64_t)oc * kQ + t;
-    const bool t_valid = tok < pr.L;
-    __nv_bfloat16 *yrow = a.y + (obi * pr.L + tok) * pr.d_inner + (int64_t)h * kHP + 32 * eh;
+    const int64_t tok = pos.t0 + t;
+    const bool t_valid = t < pos.nv;
+    __nv_bfloat16 *yrow = a.y + tok * pr.d_inner + (int64_t)h * kHP + 32 * eh;
     float v32[32];
     tmem_ld32(tmem + lane_off + kTmemY + 64 * j + 32 * eh, v32);
     tc_fence_before();
@@ -1240,7 +1372,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     for (int hh = 0; hh < 2; ++hh) {
       float *v = v32 + 16 * hh;
       if (pr.nbg) {
-        const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + (obi * pr.L + tok) * a.ld_z +
+        const uint4 *zp = reinterpret_cast<const uint4 *>(a.z + tok * a.ld_z +
                                                           (int64_t)h * kHP + 32 * eh + 16 * hh);
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
@@ -1286,40 +1418,48 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     if (lane == 0 && nh > 0) {
       bool ok = true;
       int J = 0, ncb = 0, nxh = 0, nz = 0;  // copies issued into each ring
+      // a [128 tokens][64 ch] tile of u or z for the unit at `pos`
+      auto load_tok = [&](uint32_t dst, const CUtensorMap *m3, const CUtensorMap *m2, int ch,
+                          const ChunkPos &pos, uint64_t *bar) {
+        if (a.varlen) tma_load_2d(dst, m2, ch, (int)pos.t0, bar);
+        else tma_load_3d(dst, m3, ch, pos.c * kQ, pos.seq, bar);
+      };
       auto load_cb = [&](int n) {  // C and B tiles of unit n
-        int64_t bi;
-        int c, g;
-        out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+        int64_t gc;
+        int g;
+        out_unit(pr, ncl, cid, n, gc, g);
+        const ChunkPos pos = chunk_pos(a, gc);
         const int cbuf = n & 1;
         if (n >= 2) ok = ok && mbar_wait_bounded(&sh.c_free[cbuf], (uint32_t)(((n - 2) >> 1) & 1), &g_tc_errors);
         if (n >= 1) ok = ok && mbar_wait_bounded(&sh.b_free, (uint32_t)((n - 1) & 1), &g_tc_errors);
         if (!ok) return;
         mbar_arrive_expect_tx(&sh.full_cb[cbuf], 2 * 16384);
-        tma_load_3d(base + kCt0 + cbuf * 16384, &maps.u,
-                    (int)(pr.d_inner + (int64_t)(pr.G + g) * kNS), c * kQ, (int)bi, &sh.full_cb[cbuf]);
-        tma_load_3d(base + kBt, &maps.u, (int)(pr.d_inner + (int64_t)g * kNS), c * kQ, (int)bi,
-                    &sh.full_cb[cbuf]);
+        load_tok(base + kCt0 + cbuf * 16384, &maps.u, &maps.u2,
+                 (int)(pr.d_inner + (int64_t)(pr.G + g) * kNS), pos, &sh.full_cb[cbuf]);
+        load_tok(base + kBt, &maps.u, &maps.u2, (int)(pr.d_inner + (int64_t)g * kNS), pos,
+                 &sh.full_cb[cbuf]);
         ++ncb;
       };
       load_cb(0);
       for (int n = 0; ok && n < n_units; ++n) {
-        int64_t bi;
-        int c, g;
-        out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+        int64_t gc;
+        int g;
+        out_unit(pr, ncl, cid, n, gc, g);
+        const ChunkPos pos = chunk_pos(a, gc);
         const int h0 = g * hpg + lh0;
         for (int j = 0; ok && j < nh; ++j, ++J) {
           const int h = h0 + j, sl = J & 1;
           if (J >= 2) ok = mbar_wait_bounded(&sh.empty_xh[sl], (uint32_t)(((J - 2) >> 1) & 1), &g_tc_errors);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.full_xh[sl], kXhBytes);
-          tma_load_3d(base + kXh + sl * kXhBytes, &maps.u, h * kHP, c * kQ, (int)bi, &sh.full_xh[sl]);
+          load_tok(base + kXh + sl * kXhBytes, &maps.u, &maps.u2, h * kHP, pos, &sh.full_xh[sl]);
           tma_load_2d(base + kXh + sl * kXhBytes + 16384, &maps.hc, 0,
-                      (int)(((bi * a.nch + c) * pr.H + h) * kHP), &sh.full_xh[sl]);
+                      (int)((gc * pr.H + h) * kHP), &sh.full_xh[sl]);
           ++nxh;
           if (J >= 2) ok = mbar_wait_bounded(&sh.empty_z[sl], (uint32_t)(((J - 2) >> 1) & 1), &g_tc_errors);
           if (!ok) break;
           mbar_arrive_expect_tx(&sh.full_z[sl], 16384);
-          tma_load_3d(base + kZt + sl * 16384, &maps.z, h * kHP, c * kQ, (int)bi, &sh.full_z[sl]);
+          load_tok(base + kZt + sl * 16384, &maps.z, &maps.z2, h * kHP, pos, &sh.full_z[sl]);
           ++nz;
           if (j == min(1, nh - 1) && n + 1 < n_units) load_cb(n + 1);
         }
@@ -1392,9 +1532,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     bool ok = true;
     int J = 0;
     for (int n = 0; ok && n < n_units && nh > 0; ++n) {
-      int64_t bi;
-      int c, g;
-      out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+      int64_t gc;
+      int g;
+      out_unit(pr, ncl, cid, n, gc, g);
       const int h0 = g * hpg + lh0;
       const int par = n & 1;
       // the epilogue reads this parity's exp(cum) and scales of unit n - 2 until it is done
@@ -1407,7 +1547,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       // decay terms of head j = warp (from the per-chunk dt and cumsum rows)
       if (warp < nh) {
         const int j = warp;
-        const int64_t row = (bi * a.nch + c) * pr.H + h0 + j;
+        const int64_t row = gc * pr.H + h0 + j;
         const float4 *cup = reinterpret_cast<const float4 *>(a.cum + row * kQ) + lane;
         const float4 *dvp = reinterpret_cast<const float4 *>(a.dtv + row * kQ) + lane;
         const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1437,7 +1577,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           sh.Dh[j] = M2_OK(a.prm.D + h0 + j, 4, a.sp.D, &g_tc_errors) ? a.prm.D[h0 + j] : 0.0f;
       }
       if (warp == 7) {  // the unit's fp32 diagonal C_t . B_t
-        const float4 *src = reinterpret_cast<const float4 *>(a.cbd + ((bi * pr.G + g) * a.nch + c) * kQ) + lane;
+        const float4 *src = reinterpret_cast<const float4 *>(a.cbd + (gc * pr.G + g) * kQ) + lane;
         reinterpret_cast<float4 *>(sh.cbd)[lane] =
             M2_OK(src, 16, a.sp.cbd, &g_tc_errors) ? *src : make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -1470,9 +1610,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     bool ok = true;
     int J = 0;
     for (int n = 0; ok && n < n_units; ++n) {
-      int64_t bi;
-      int c, g;
-      out_unit(pr, a.nch, ncl, cid, n, bi, c, g);
+      int64_t gc;
+      int g;
+      out_unit(pr, ncl, cid, n, gc, g);
       const int h0 = g * hpg + lh0;
       const int par = n & 1;
       float ss = 0.0f;
@@ -1615,31 +1755,41 @@ void out_choose(int hpg, int64_t units, int *cs, int *hpc, int *ncl) {
 struct TcWorkspace {
   float *S, *cum_end, *cum, *dtv, *hsc, *smax, *cbd;
   __half *Hc, *u;
+  int4 *vl_chunks;
+  int *vl_chunk0;
 };
 
-TcWorkspace tc_carve(const Problem &pr, char *base) {
-  const int64_t nch = ceil_div(pr.L, kQ);
-  const size_t st = (size_t)pr.batch * nch * pr.H * kHP * kNS;
-  TcWorkspace w;
+// Chunks the workspace holds: b * ceil(L / 128), or for packed sequences an
+// upper bound on the sum of their chunk counts, ceil(L / 128) + b.
+int64_t tc_chunk_cap(const Problem &pr, bool varlen) {
+  return varlen ? ceil_div(pr.L, kQ) + pr.batch : pr.batch * ceil_div(pr.L, kQ);
+}
+
+// Carves the workspace (or, with base null, measures it).
+size_t tc_carve(const Problem &pr, bool varlen, char *base, TcWorkspace *w) {
+  const size_t cap = (size_t)tc_chunk_cap(pr, varlen);
+  const size_t st = cap * pr.H * kHP * kNS;
   size_t off = 0;
-  w.S = reinterpret_cast<float *>(base + off);
-  off += align_up(st * 4, 256);
-  w.cum_end = reinterpret_cast<float *>(base + off);
-  off += align_up((size_t)pr.batch * nch * pr.H * 4, 256);
-  w.cum = reinterpret_cast<float *>(base + off);
-  off += align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256);
-  w.dtv = reinterpret_cast<float *>(base + off);
-  off += align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256);
-  w.Hc = reinterpret_cast<__half *>(base + off);
-  off += align_up(st * 2, 256);
-  w.hsc = reinterpret_cast<float *>(base + off);
-  off += align_up((size_t)pr.batch * nch * pr.H * 32 * 4, 256);
-  w.smax = reinterpret_cast<float *>(base + off);
-  off += align_up((size_t)pr.batch * nch * pr.H * 4, 256);
-  w.cbd = reinterpret_cast<float *>(base + off);
-  off += align_up((size_t)pr.batch * pr.G * nch * kQ * 4, 256);
-  w.u = reinterpret_cast<__half *>(base + off);
-  return w;
+  auto take = [&](size_t bytes) -> char * {
+    char *p = base == nullptr ? nullptr : base + off;
+    off += align_up(bytes, 256);
+    return p;
+  };
+  TcWorkspace t;
+  t.S = reinterpret_cast<float *>(take(st * 4));
+  t.cum_end = reinterpret_cast<float *>(take(cap * pr.H * 4));
+  t.cum = reinterpret_cast<float *>(take(cap * pr.H * kQ * 4));
+  t.dtv = reinterpret_cast<float *>(take(cap * pr.H * kQ * 4));
+  t.Hc = reinterpret_cast<__half *>(take(st * 2));
+  t.hsc = reinterpret_cast<float *>(take(cap * pr.H * 32 * 4));
+  t.smax = reinterpret_cast<float *>(take(cap * pr.H * 4));
+  t.cbd = reinterpret_cast<float *>(take(cap * pr.G * kQ * 4));
+  t.vl_chunks = varlen ? reinterpret_cast<int4 *>(take(cap * 16)) : nullptr;
+  t.vl_chunk0 = varlen ? reinterpret_cast<int *>(take((size_t)(pr.batch + 2) * 4)) : nullptr;
+  const size_t tokens = varlen ? (size_t)pr.L : (size_t)(pr.batch * pr.L);
+  t.u = reinterpret_cast<__half *>(take(tokens * pr.conv_dim * 2));
+  if (w != nullptr) *w = t;
+  return off;
 }
 
 // Number of SMs of the current device (cached per device).
@@ -1726,22 +1876,18 @@ int out_max_clusters(int cs) {
 const char *const kPrefillTcStages[] = {"tc_chunk_state", "tc_state_pass", "tc_chunk_out"};
 const int kPrefillTcStageCount = 3;
 
-bool prefill_tc_supported(const Problem &pr) {
-  const int64_t nch = ceil_div(pr.L, kQ);
+bool prefill_tc_supported(const Problem &pr, bool varlen) {
+  const int64_t nch = ceil_div(pr.L, kQ), cap = tc_chunk_cap(pr, varlen);
+  const int64_t pairs = (pr.heads_per_group() + 1) / 2;
   return pr.io == MAMBA2_BF16 && pr.P == kHP && pr.N == kNS && pr.K == 4 &&
-         pr.heads_per_group() <= 16 * kMaxHeadsPerCta && pr.L > 0 && nch <= 65535 &&
-         pr.L < ((int64_t)1 << 31) && pr.batch * nch * pr.H * kHP < ((int64_t)1 << 31);
+         pr.heads_per_group() <= 16 * kMaxHeadsPerCta && pr.L > 0 &&
+         (varlen || nch <= 65535) && pr.L < ((int64_t)1 << 31) &&
+         pr.batch * pr.L < ((int64_t)1 << 31) && cap * pr.H * kHP < ((int64_t)1 << 31) &&
+         cap * pr.G * (pairs + 1) < ((int64_t)1 << 31);
 }
 
-size_t prefill_tc_workspace(const Problem &pr) {
-  const int64_t nch = ceil_div(pr.L, kQ);
-  const size_t st = (size_t)pr.batch * nch * pr.H * kHP * kNS;
-  return align_up(st * 4, 256) + align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
-         2 * align_up((size_t)pr.batch * nch * pr.H * kQ * 4, 256) + align_up(st * 2, 256) +
-         align_up((size_t)pr.batch * nch * pr.H * 32 * 4, 256) +
-         align_up((size_t)pr.batch * nch * pr.H * 4, 256) +
-         align_up((size_t)pr.batch * pr.G * nch * kQ * 4, 256) +
-         align_up((size_t)pr.batch * pr.L * pr.conv_dim * 2, 256);
+size_t prefill_tc_workspace(const Problem &pr, bool varlen) {
+  return tc_carve(pr, varlen, nullptr, nullptr);
 }
 
 cudaError_t set_prefill_tc_stall(unsigned int v) {
@@ -1773,8 +1919,16 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.conv_in = static_cast<const __nv_bfloat16 *>(pa.conv_state);
   a.ssm_state = pa.ssm_state;
   a.states_in = pa.states_in;
+  const bool varlen = pa.cu_seqlens != nullptr;
   a.nch = (int)ceil_div(pr.L, kQ);
-  TcWorkspace w = tc_carve(pr, pa.ws);
+  TcWorkspace w;
+  tc_carve(pr, varlen, pa.ws, &w);
+  a.varlen = varlen ? 1 : 0;
+  a.vl_chunks = w.vl_chunks;
+  a.vl_chunk0 = w.vl_chunk0;
+  a.cu_seqlens = pa.cu_seqlens;
+  const int64_t cap = tc_chunk_cap(pr, varlen);    // chunks the workspace holds
+  const int64_t tokens = varlen ? pr.L : pr.batch * pr.L;
   a.S = w.S;
   a.cum_end = w.cum_end;
   a.cum = w.cum;
@@ -1785,8 +1939,8 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.cbd = w.cbd;
   a.u = w.u;
   {
-    const int64_t bl = pr.batch * pr.L, nq = a.nch;
-    const size_t st1 = (size_t)pr.batch * nq * pr.H * kHP * kNS;
+    const int64_t bl = tokens, nq = cap, nrow = 1;  // chunk arrays: cap chunks
+    const size_t st1 = (size_t)nrow * nq * pr.H * kHP * kNS;
     a.sp.xbc = span_of(a.xBC, (size_t)((bl - 1) * pa.ld_xbc + pr.conv_dim) * 2);
     a.sp.z = span_of(a.z, (size_t)((bl - 1) * pa.ld_z + pr.d_inner) * 2);
     a.sp.dt = span_of(a.dt_raw, (size_t)((bl - 1) * pa.ld_dt + pr.H) * 2);
@@ -1794,13 +1948,13 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     a.sp.conv = span_of(pa.conv_state, (size_t)pr.batch * pr.conv_dim * 4 * 2);
     a.sp.ssm = span_of(a.ssm_state, (size_t)pr.batch * pr.H * kHP * kNS * 4);
     a.sp.S = span_of(a.S, st1 * 4);
-    a.sp.cum_end = span_of(a.cum_end, (size_t)pr.batch * nq * pr.H * 4);
-    a.sp.cum = span_of(a.cum, (size_t)pr.batch * nq * pr.H * kQ * 4);
-    a.sp.dtv = span_of(a.dtv, (size_t)pr.batch * nq * pr.H * kQ * 4);
+    a.sp.cum_end = span_of(a.cum_end, (size_t)nq * pr.H * 4);
+    a.sp.cum = span_of(a.cum, (size_t)nq * pr.H * kQ * 4);
+    a.sp.dtv = span_of(a.dtv, (size_t)nq * pr.H * kQ * 4);
     a.sp.Hc = span_of(a.Hc, st1 * 2);
-    a.sp.hsc = span_of(a.hsc, (size_t)pr.batch * nq * pr.H * 32 * 4);
-    a.sp.smax = span_of(a.smax, (size_t)pr.batch * nq * pr.H * 4);
-    a.sp.cbd = span_of(a.cbd, (size_t)pr.batch * pr.G * nq * kQ * 4);
+    a.sp.hsc = span_of(a.hsc, (size_t)nq * pr.H * 32 * 4);
+    a.sp.smax = span_of(a.smax, (size_t)nq * pr.H * 4);
+    a.sp.cbd = span_of(a.cbd, (size_t)pr.G * nq * kQ * 4);
     a.sp.u = span_of(a.u, (size_t)bl * pr.conv_dim * 2);
     a.sp.conv_w = span_of(a.prm.conv_w, (size_t)pr.conv_dim * 4 * 4);
     a.sp.conv_b = span_of(a.prm.conv_b, (size_t)pr.conv_dim * 4);
@@ -1823,20 +1977,32 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     if (e != cudaSuccess) return e;
   }
   int cs = 1, hpc = 1, ncl = 1;
-  out_choose(hpg, pr.batch * a.nch * (int64_t)pr.G, &cs, &hpc, &ncl);
+  out_choose(hpg, cap * (int64_t)pr.G, &cs, &hpc, &ncl);
   a.hpc = hpc;
 
   stage_mark(st, 0);
-  const int64_t n_items = pr.batch * a.nch * (int64_t)pr.G * ((hpg + 1) / 2 + 1);
+  if (varlen) {  // the chunks of the packed sequences
+    tc_varlen_prep_kernel<<<1, kPrepThreads, 0, st>>>(pa.cu_seqlens, (int)pr.batch, pr.L, cap,
+                                                      w.vl_chunks, w.vl_chunk0);
+  }
+  const int64_t n_items = cap * (int64_t)pr.G * ((hpg + 1) / 2 + 1);
   const unsigned g1 = (unsigned)std::min<int64_t>(n_items, sm_count());
   {
     NvtxRange r1("tc_chunk_state");
     K1Maps m1;
-    const uint64_t dx[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
-    const uint64_t sx[2] = {(uint64_t)pa.ld_xbc * 2, (uint64_t)pr.L * pa.ld_xbc * 2};
+    std::memset(&m1, 0, sizeof(m1));
     const uint32_t bx[3] = {64, kRawRows, 1};
-    if (!make_map(&m1.xbc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xBC, 3, dx, sx, bx))
-      return cudaErrorInvalidValue;
+    if (varlen) {
+      const uint64_t dx[2] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L};
+      const uint64_t sx[1] = {(uint64_t)pa.ld_xbc * 2};
+      if (!make_map(&m1.xbc2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xBC, 2, dx, sx, bx))
+        return cudaErrorInvalidValue;
+    } else {
+      const uint64_t dx[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
+      const uint64_t sx[2] = {(uint64_t)pa.ld_xbc * 2, (uint64_t)pr.L * pa.ld_xbc * 2};
+      if (!make_map(&m1.xbc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.xBC, 3, dx, sx, bx))
+        return cudaErrorInvalidValue;
+    }
     tc_chunk_state_kernel<<<g1, kK1Threads, kK1Smem, st>>>(a, m1, (int)n_items);
   }
   stage_mark(st, 1);
@@ -1875,19 +2041,31 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     OutMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
     {
-      const uint64_t du[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
-      const uint64_t su[2] = {(uint64_t)pr.conv_dim * 2, (uint64_t)pr.L * pr.conv_dim * 2};
       const uint32_t bu[3] = {64, kQ, 1};
-      const uint64_t dz[3] = {(uint64_t)pr.d_inner, (uint64_t)pr.L, (uint64_t)pr.batch};
-      const uint64_t sz[2] = {(uint64_t)pa.ld_z * 2, (uint64_t)pr.L * pa.ld_z * 2};
-      const uint64_t dh[2] = {(uint64_t)kNS, (uint64_t)pr.batch * a.nch * pr.H * kHP};
+      const uint64_t dh[2] = {(uint64_t)kNS, (uint64_t)(cap * pr.H * kHP)};
       const uint64_t shc[1] = {(uint64_t)kNS * 2};
       const uint32_t bh[2] = {64, 64};
-      if (!make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.u, 3, du, su, bu) ||
-          !make_map(&maps.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.z, 3, dz, sz, bu) ||
-          !make_map(&maps.hc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Hc, 2, dh, shc, bh))
+      if (!make_map(&maps.hc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.Hc, 2, dh, shc, bh))
         return cudaErrorInvalidValue;
+      if (varlen) {
+        const uint64_t du[2] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L};
+        const uint64_t su[1] = {(uint64_t)pr.conv_dim * 2};
+        const uint64_t dz[2] = {(uint64_t)pr.d_inner, (uint64_t)pr.L};
+        const uint64_t sz[1] = {(uint64_t)pa.ld_z * 2};
+        if (!make_map(&maps.u2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.u, 2, du, su, bu) ||
+            !make_map(&maps.z2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.z, 2, dz, sz, bu))
+          return cudaErrorInvalidValue;
+      } else {
+        const uint64_t du[3] = {(uint64_t)pr.conv_dim, (uint64_t)pr.L, (uint64_t)pr.batch};
+        const uint64_t su[2] = {(uint64_t)pr.conv_dim * 2, (uint64_t)pr.L * pr.conv_dim * 2};
+        const uint64_t dz[3] = {(uint64_t)pr.d_inner, (uint64_t)pr.L, (uint64_t)pr.batch};
+        const uint64_t sz[2] = {(uint64_t)pa.ld_z * 2, (uint64_t)pr.L * pa.ld_z * 2};
+        if (!make_map(&maps.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.u, 3, du, su, bu) ||
+            !make_map(&maps.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.z, 3, dz, sz, bu))
+          return cudaErrorInvalidValue;
+      }
     }
     e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps, ncl);
     if (e != cudaSuccess) return e;

@@ -175,3 +175,52 @@ def test_noalloc_rejects_bad_dims_before_touching_the_device():
         st = lib.mamba2_conv_ssd_prefill_noalloc(ctypes.byref(d), ctypes.byref(p), A0, 5248,
                                                  A0, 5120, A0, 80, A0, None, None, 0, None)
         assert st == expect, kw
+
+
+# ---- packed-sequence prefill: validated on the host before any CUDA call
+
+def _call_varlen(d, **kw):
+    lib = m2.lib()
+    cd, di = d.nheads * d.headdim + 2 * d.ngroups * d.dstate, d.nheads * d.headdim
+    args = dict(params=_fake_params(), xBC=A0 + 0x10000, ld_x=cd, z=A0 + 0x20000, ld_z=di,
+                dt=A0 + 0x30000, ld_dt=d.nheads, cu=A0 + 0x70000, y=A0 + 0x40000,
+                cs=A0 + 0x50000, hs=A0 + 0x60000, states_in=0, ws=A0 + 0x100000,
+                ws_bytes=lib.mamba2_prefill_varlen_workspace_size(ctypes.byref(d)) or 1)
+    args.update(kw)
+    p = args["params"]
+    return lib.mamba2_conv_ssd_prefill_varlen(
+        ctypes.byref(d), ctypes.byref(p) if p is not None else None, args["xBC"], args["ld_x"],
+        args["z"], args["ld_z"], args["dt"], args["ld_dt"], args["cu"], args["y"], args["cs"],
+        args["hs"], args["states_in"], args["ws"], args["ws_bytes"], None)
+
+
+def test_varlen_workspace_size():
+    lib = m2.lib()
+    d = _dims(batch=7, seqlen=4096)  # 7 sequences, 4096 tokens in all
+    ws = lib.mamba2_prefill_varlen_workspace_size(ctypes.byref(d))
+    fixed = lib.mamba2_prefill_workspace_size(ctypes.byref(_dims(batch=1, seqlen=4096)))
+    # room for up to ceil(4096 / 128) + 7 chunks instead of 32
+    assert fixed < ws < fixed * (32 + 7 + 1) / 32
+    # the CUDA-core configurations have no packed-sequence path
+    assert lib.mamba2_prefill_varlen_workspace_size(ctypes.byref(_dims(io_dtype=0))) == 0
+    assert lib.mamba2_prefill_varlen_workspace_size(ctypes.byref(_dims(headdim=32))) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(cu=None), INVALID),                  # no offsets
+    (dict(cu=A0 + 0x70002), INVALID),          # offsets not 4-byte aligned
+    (dict(params=None), INVALID),
+    (dict(xBC=A0 + 0x10008), INVALID),
+    (dict(states_in=1, hs=None), INVALID),
+    (dict(ws=None), WORKSPACE),
+    (dict(ws_bytes=4096), WORKSPACE),
+])
+def test_varlen_rejects_bad_arguments(kw, expect):
+    assert _call_varlen(_dims(batch=3, seqlen=1000), **kw) == expect
+
+
+def test_varlen_unsupported_configurations():
+    for bad in (dict(io_dtype=0), dict(headdim=32), dict(dstate=128)):
+        d = _dims(batch=3, seqlen=1000, **bad)
+        assert _call_varlen(d, ld_x=d.nheads * d.headdim + 2 * d.ngroups * d.dstate,
+                            ld_z=d.nheads * d.headdim) == UNSUPPORTED, bad
