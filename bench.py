@@ -29,6 +29,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import itertools
 import json
 import os
 import statistics
@@ -386,6 +387,93 @@ def measure_prefill(name, args, dev, stream, seed, world, peaks, peak_src, m2, W
     return out
 
 
+# Packed-sequence prefill: eight requests of mixed lengths (4096 tokens in all,
+# from a single token to 1600, with chunk tails and an exact multiple of 128)
+# on the 2.7B-shaped mixer, each continuing from its own carried state.
+VARLEN_LENGTHS = (1, 3, 127, 129, 512, 700, 1024, 1600)
+
+
+def measure_varlen(args, dev, stream, seed, world, peaks, peak_src, m2, W, lib, steps, warmup):
+    """Device-timed packed-sequence prefills (mamba2_conv_ssd_prefill_varlen), L2
+    flushed (256 MB write) before every step, steps timed one by one."""
+    import torch
+    T, n = sum(VARLEN_LENGTHS), len(VARLEN_LENGTHS)
+    cfg1 = W.CONFIGS[PREFILL].with_(batch=1, seqlen=T)
+    cfg = cfg1.with_(batch=n)  # dims: batch = sequences, seqlen = total tokens
+    dims = m2.dims_from_config(cfg)
+    params = {k: v.to(dev) for k, v in W.make_params(cfg, seed).items()}
+    pp = m2.make_params(params["conv_w"], params["conv_b"], params["dt_bias"], params["A"],
+                        params["D"], params["norm_w"])
+    v = W.split_packed(cfg1, W.make_prefill_inputs(cfg1, seed)["zxbcdt"][0].to(dev))
+    st = W.make_states(cfg, seed)
+    cs0, hs0 = st["conv_state"].to(dev), st["ssm_state"].to(dev)
+    cs, hs = cs0.clone(), hs0.clone()
+    cu = torch.tensor([0] + list(itertools.accumulate(VARLEN_LENGTHS)), dtype=torch.int32,
+                      device=dev)
+    y = torch.empty(T, cfg.d_inner, dtype=cfg.torch_dtype, device=dev)
+    ws = torch.empty(max(1, m2.mamba2_prefill_varlen_workspace_size(dims)), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    names_arr = (ctypes.c_char_p * 16)()
+    nst = lib.mamba2_stage_names(0, ctypes.byref(dims), names_arr, 16)
+    stage_names = [names_arr[i].decode() for i in range(nst)]
+
+    def call(stage_events=None):
+        cs.copy_(cs0)  # every step continues from the same carried states
+        hs.copy_(hs0)
+        flush.fill_(1)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        if stage_events is not None:
+            arr = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
+            lib.mamba2_record_stage_events(arr, len(stage_events))
+        m2.mamba2_conv_ssd_prefill_varlen(dims, pp, v["xBC"], v["z"], v["dt_raw"], cu, y, cs, hs,
+                                          True, ws, stream)
+        b.record(stream)
+        return a, b
+
+    stage_ms, n_stage = [0.0] * nst, 0
+    for i in range(max(3, warmup)):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+        for ev in evs:
+            ev.record(stream)  # torch creates the CUDA event on its first record
+        call(evs)
+        torch.cuda.synchronize(dev)
+        if i >= 2:  # the first calls pay one-time costs
+            n_stage += 1
+            for j in range(nst):
+                stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
+    torch.cuda.synchronize(dev)
+    evs = [call() for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev) / steps
+    e = 2
+    states = 4 * cfg.nheads * cfg.headdim * cfg.dstate + e * cfg.conv_dim * cfg.d_conv
+    path_bytes = T * e * (cfg.conv_dim + 2 * cfg.d_inner + cfg.nheads) + n * 2 * states
+    path_flops = prefill_flops(cfg1)
+    t_roof = max(path_bytes / (peaks["hbm_gbs"] * 1e9), path_flops / (peaks["bf16_tflops"] * 1e12))
+    return {
+        "value": job_rate(T, steps, ms * steps, world), "unit": "tokens/s", "steps": steps,
+        "warmup": max(3, warmup), "ms_per_step": ms,
+        "config": {"workload": "zamba2_2p7b_varlen_prefill", "sequences": n,
+                   "lengths": list(VARLEN_LENGTHS), "tokens": T, "nheads": cfg.nheads,
+                   "headdim": cfg.headdim, "dstate": cfg.dstate, "ngroups": cfg.ngroups,
+                   "io_dtype": cfg.io_dtype, "chunk": 128, "states_in": True,
+                   "l2": "L2 flushed (256 MB write) before every step, steps timed one by one"},
+        # every input and carried state read once, y and the final states written once
+        "path_roofline": {"bytes": path_bytes, "flops": path_flops,
+                          "roofline_ms": t_roof * 1e3,
+                          "achieved_gbs": path_bytes / (ms * 1e-3) / 1e9,
+                          "frac": t_roof * 1e3 / ms, "peak_source": peak_src},
+        # (the first stage includes the small kernel that lays out the chunks)
+        "stages_ms_warmup_avg": {n: stage_ms[j] / max(1, n_stage)
+                                 for j, n in enumerate(stage_names)},
+        "gpu_launches": 4 * steps,
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import mamba_ssd_scan_mixer_b200 as m2
@@ -432,6 +520,10 @@ def run_ours(args, rank, world, local_rank):
                                 lib, steps=min(args.steps, 20), warmup=3, flush_l2=small)
             line["gpu_launches"] += o.pop("gpu_launches")
             other[name] = o
+        o = measure_varlen(args, dev, stream, seed, world, peaks, peak_src, m2, W, lib,
+                           steps=min(args.steps, 20), warmup=3)
+        line["gpu_launches"] += o.pop("gpu_launches")
+        other["zamba2_2p7b_varlen_prefill"] = o
         line["workloads"] = other
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, seconds=10.0)

@@ -291,13 +291,17 @@ struct K1Maps {
 // With h = pre / 2 (exact), silu(pre) = h + h tanh(h).
 // The 7 rows stay packed (2 bf16 per register) and are widened one channel at a
 // time, so that only 28 registers of inputs and one channel's taps are live.
+// hrows, if not 0, holds rows 0..2 (the 3 tokens before a sequence's first
+// chunk) in the tile's layout; they are read from there instead of the tile.
 __device__ __forceinline__ void conv8x4_smem(uint32_t tile, int s0, int cg, const float4 *wt,
-                                             const float *bs, float (&out)[4][8]) {
+                                             const float *bs, float (&out)[4][8],
+                                             uint32_t hrows = 0) {
   uint32_t raw[7][4];
 #pragma unroll
   for (int r = 0; r < 7; ++r) {
     const int R = s0 + r;
-    const uint4 q = ld_shared_v4(tile + R * 128 + (((cg ^ R) & 7) << 4));
+    const uint32_t src = (hrows != 0 && R < 3) ? hrows : tile;
+    const uint4 q = ld_shared_v4(src + R * 128 + (((cg ^ R) & 7) << 4));
     raw[r][0] = q.x;
     raw[r][1] = q.y;
     raw[r][2] = q.z;
@@ -364,7 +368,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   __shared__ float4 wts[2][3][64];                // [stage][slot x_A, x_B, B/C][channel] conv taps
   __shared__ __align__(16) float bss[2][3][64];   // [stage][slot][channel] conv bias
   __shared__ uint64_t full[2], empty[2], bc_empty[2], ops_ready, mma_done[2], tmem_free[2],
-      mma_final, halo_bar[2], cbd_bar, park_bar;
+      mma_final, cbd_bar, park_bar;
+  // rows 0..2 (the conv's left context) of a sequence's first chunk: per stage and
+  // x slot, and per B/C buffer; the tiles' own rows 0..2 are not read then
+  __shared__ __align__(16) unsigned char hrow_x[2][2][3 * 128];
+  __shared__ __align__(16) unsigned char hrow_bc[2][3 * 128];
   __shared__ __align__(16) float cbd_s[2][kQ];  // C-item parity: per-token partials of channel groups 4-7
   __shared__ uint32_t tmem_holder;
   const Problem &pr = a.pr;
@@ -374,10 +382,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                  sBlo = base + kK1Blo;
   const int hpg = pr.heads_per_group();
   const int pairs = (hpg + 1) / 2;
-  // items past the call's chunks (packed sequences: n_items is a capacity) are void
+  // the call's items (for packed sequences n_items is a capacity and the count
+  // comes from the chunk table), split evenly over the CTAs
   const int n_real = (int)min((int64_t)n_items, total_chunks(a) * pr.G * (pairs + 1));
-  const int it0 = min(n_real, (int)((int64_t)n_items * blockIdx.x / gridDim.x)),
-            it1 = min(n_real, (int)((int64_t)n_items * (blockIdx.x + 1) / gridDim.x));
+  const int it0 = (int)((int64_t)n_real * blockIdx.x / gridDim.x),
+            it1 = (int)((int64_t)n_real * (blockIdx.x + 1) / gridDim.x);
 
   if (warp == 0) tmem_alloc(&tmem_holder, 128);
   if (tid == 0) {
@@ -391,7 +400,6 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     }
     mbar_init(&ops_ready, kThreads);  // operands of a pair item written
     mbar_init(&mma_final, 1);
-    for (int k = 0; k < 2; ++k) mbar_init(&halo_bar[k], 1);  // a halo item's tiles landed
     mbar_init(&cbd_bar, 128);   // warps 12-15 have written a C item's diagonal partials
     mbar_init(&park_bar, 256);  // warps 0-7 have parked a C item's convolved C values
     fence_mbar_init();
@@ -407,7 +415,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     // uses of the two B/C buffers.
     const int mine = warp == kThreads / 32 ? 0 : 1;
     int k = 0;
-    int bc_use0 = 0, bc_use1 = 0, halo_use0 = 0, halo_use1 = 0;  // (scalars: no local memory)
+    int bc_use0 = 0, bc_use1 = 0;  // (scalars: no local memory)
     bool ok = true;
     for (int it = it0; ok && it < it1; ++it, ++k) {
       const int st = k & 1;
@@ -510,14 +518,14 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       if (!ok) break;
       // the first chunk of a sequence that continues from a carried conv state (or of
       // a packed sequence, whose rows before it belong to the previous one): its
-      // tiles land on a side barrier, then rows 0..2 (tokens -3 .. -1) are
-      // overwritten with that state (or zeros) before the stage is released
+      // left context (tokens -3 .. -1: that state, or zeros) goes to the side rows,
+      // which the compute warps read instead of the tiles' rows 0..2
       const bool halo = w.c == 0 && (a.states_in || a.varlen);
       const uint32_t stage = base + st * kK1Stage;
       const uint32_t bcbuf = base + kK1BC + bcb * kRawBytes;
       const int64_t bc_ch = pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
       if (lane == 0) {
-        uint64_t *bar = halo ? &halo_bar[st] : &full[st];
+        uint64_t *bar = &full[st];
         const uint32_t nbytes =
             (w.isC ? 1u : (1u + (hasB ? 1u : 0u))) * kRawBytes + (useBC ? kRawBytes : 0u);
         mbar_arrive_expect_tx(bar, nbytes);
@@ -534,11 +542,6 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         if (useBC) load_raw(bcbuf, (int)bc_ch);
       }
       if (halo) {
-        const int nh_used = st ? halo_use1++ : halo_use0++;
-        bool landed = lane == 0 ? mbar_wait_bounded(&halo_bar[st], (uint32_t)(nh_used & 1), &g_tc_errors)
-                                : true;
-        ok = __shfl_sync(0xffffffffu, landed ? 1 : 0, 0) != 0;
-        if (!ok) break;
         // slot x_A, x_B (if any) and the B/C tile: 3 rows x 64 channels each
         for (int idx = lane; idx < 3 * 3 * 64; idx += 32) {
           const int sl = idx / 192, r = (idx / 64) % 3, chn = idx % 64;
@@ -548,12 +551,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
           const __nv_bfloat16 v = a.states_in && M2_OK(hp, 2, a.sp.conv, &g_tc_errors)
                                       ? *hp
                                       : __float2bfloat16(0.0f);
-          const uint32_t tile = sl < 2 ? stage + sl * kRawBytes : bcbuf;
-          const uint32_t addr = tile + r * 128 + ((((chn >> 3) ^ r) & 7) << 4) + ((chn & 7) << 1);
+          const uint32_t rows = sl < 2 ? smem_u32(&hrow_x[st][sl][0]) : smem_u32(&hrow_bc[bcb][0]);
+          const uint32_t addr = rows + r * 128 + ((((chn >> 3) ^ r) & 7) << 4) + ((chn & 7) << 1);
           asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(v))
                        : "memory");
         }
-        if (lane == 0) mbar_arrive(&full[st]);  // stands for the tiles' transaction bytes
       }
       if (!w.isC) {
 #pragma unroll
@@ -644,6 +646,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         float *mp = a.smax + (int64_t)q.gc * pr.H + q.hA + half;
         if (lane == 0 && M2_OK(mp, 4, a.sp.smax, &g_tc_errors))
           atomicMax(reinterpret_cast<int *>(mp), __float_as_int(mx));
+
         float4 *dst = reinterpret_cast<float4 *>(
             a.S + ((int64_t)q.gc * pr.H + q.hA + half) * (int64_t)(kHP * kNS));
 #pragma unroll
@@ -671,6 +674,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       const bool hasB = 2 * w.pair + 1 < hpg;
       const uint32_t bcbuf = base + kK1BC + bcb * kRawBytes;
       const int64_t bc_ch = pr.d_inner + (int64_t)((w.isC ? pr.G : 0) + w.g) * kNS;
+      // a sequence's first chunk: its left context lives in the side rows
+      const bool halo = w.c == 0 && (a.states_in || a.varlen);
+      auto hx = [&](int sl) -> uint32_t { return halo ? smem_u32(&hrow_x[st][sl][0]) : 0u; };
+      const uint32_t hbc = halo ? smem_u32(&hrow_bc[bcb][0]) : 0u;
       // warp tile: 4 groups of 8 channels x 8 quads of tokens (lane = group lane % 4,
       // quad lane / 4); it reads the swizzled raw rows, stores u (64 contiguous bytes
       // per token) and, with the channel order of odd groups rotated by 4, stores the
@@ -728,7 +735,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         if (!ok) break;
         const uint32_t park = sBhi + (uint32_t)(((warp & 7) * 32 + lane) * 16);  // [8][256] float4
         if (warp < 8) {
-          conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v);
+          conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v, hbc);
           mbar_arrive(&bc_empty[bcb]);
           store_u(a, w.t0, s0, w.nv, bc_ch + cg * 8, v);
 #pragma unroll
@@ -741,7 +748,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
           mbar_arrive(&empty[st]);
           mbar_arrive(&park_bar);
         } else {
-          conv8x4_smem(stage, s0, cg, wts[st][0], bss[st][0], v);
+          conv8x4_smem(stage, s0, cg, wts[st][0], bss[st][0], v, hx(0));
           mbar_arrive(&empty[st]);
           {
             const bool got = mbar_wait_bounded(&park_bar, (uint32_t)(nc & 1), &g_tc_errors);
@@ -790,14 +797,14 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         if (np >= 1) wait_mma(np - 1);
         if (!ok) break;
         if (warp < 8) {
-          conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v);
+          conv8x4_smem(bcbuf, s0, cg, wts[st][2], bss[st][2], v, hbc);
           if (w.pair == 0) store_u(a, w.t0, s0, w.nv, bc_ch + cg * 8, v);
           put_operands(2, v, tile_weights(2));
           mbar_arrive(&bc_empty[bcb]);
         }
         if (sl == 1 && !hasB) zero_tile();
         else {
-          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
+          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v, hx(sl));
           store_u(a, w.t0, s0, w.nv, xch + cg * 8, v);
           put_operands(sl, v, tile_weights(sl));
         }
@@ -811,7 +818,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         if (np >= 1) wait_mma(np - 1);
         if (!ok) break;
         if (has_tile) {
-          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v);
+          conv8x4_smem(stage + sl * kRawBytes, s0, cg, wts[st][sl], bss[st][sl], v, hx(sl));
           const float4 wk4 = tile_weights(sl);
           mbar_arrive(&empty[st]);  // nothing of the stage is read after this
           put_operands(sl, v, wk4);
@@ -1840,8 +1847,9 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank
 
 constexpr size_t kK1Smem = kK1Tiles + 1024;
 constexpr size_t kK3Smem = kTcOutTiles + sizeof(OutShared) + 1024;
-// (each kernel that uses tensor memory also holds 1 KB of static shared memory)
-static_assert(kK1Smem + 11 * 1024 <= 227 * 1024 && kK3Smem + 1024 <= 227 * 1024,
+// (each kernel that uses tensor memory also holds 1 KB of static shared memory; the
+// chunk-state kernel's own static arrays take 12 KB more)
+static_assert(kK1Smem + 14 * 1024 <= 227 * 1024 && kK3Smem + 1024 <= 227 * 1024,
               "shared memory per CTA");
 
 int out_max_clusters(int cs) {

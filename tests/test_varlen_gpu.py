@@ -108,3 +108,14 @@ def test_varlen_invalid_offsets_are_reported_and_write_nothing():
     assert torch.all(got["y"] == 7.0)
     assert torch.all(got["conv_state"] == 7.0) and torch.all(got["ssm_state"] == 7.0)
     assert m2.device_errors() == 0
+
+
+def test_varlen_fullsize_request_mix():
+    # the benchmark's mix: eight requests of 1 .. 1600 tokens (4096 in all) on the
+    # 2.7B-shaped mixer (80 heads), each continuing from its own carried state
+    lengths = [1, 3, 127, 129, 512, 700, 1024, 1600]
+    cfg, params, inp = _packed(lengths, nheads=80, seed=35)
+    st = W.make_states(cfg.with_(batch=len(lengths)), 35)
+    got = _gpu_varlen(cfg, params, inp, lengths, states=st, states_in=True)
+    assert m2.device_errors() == 0
+    _check_against_oracle(cfg, params, inp, lengths, got, states=st)
