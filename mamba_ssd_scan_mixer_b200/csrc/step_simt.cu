@@ -52,6 +52,22 @@ __device__ __forceinline__ float conv4(const float *w, float b, T a0, T a1, T a2
   return b + w[0] * to_f(a0) + w[1] * to_f(a1) + w[2] * to_f(a2) + w[3] * to_f(a3);
 }
 
+// Bulk (non-tensor) shared -> global copy in this thread's bulk async-group, and
+// the waits for this thread's groups: until at most n are still reading their
+// shared-memory source, or until at most n are still in flight at all.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // barrier of the compute warps only (the producer warp never joins it)
 __device__ __forceinline__ void step_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -253,16 +269,32 @@ __global__ void __launch_bounds__(kStepBlock, 2)
   cluster_arrive_wait();
 
   if (threadIdx.x >= kStepThreads) {
-    // ---------------- producer warp
+    // ---------------- producer warp: streams each head's state in, and (once the
+    // compute warps have updated it in place) back out, both as bulk copies
     if (threadIdx.x == kStepThreads) {
+      auto head_state = [&](int64_t item) -> float * {  // global state of item (row, head)
+        const int64_t r = cid + (item / hpc) * nclusters;
+        return ssm + (r * H + h0 + (int)(item % hpc)) * (int64_t)head_floats;
+      };
+      // item j's updated state (buffer j % stages) back to global memory, once the
+      // compute warps are done with it; the buffer is free when the copy has read it
+      auto write_back = [&](int64_t j) -> bool {
+        const int s = (int)(j % stages);
+        if (!mbar_wait_bounded(&empty[s], (uint32_t)((j / stages) & 1), &g_step_errors))
+          return false;
+        float *dst = head_state(j);
+        if (M2_OK_BULK(dst, head_bytes, sp.ssm, &g_step_errors)) {
+          bulk_s2g(dst, sbuf + s * head_floats, head_bytes);
+          bulk_wait_read_all();
+        }
+        return true;
+      };
       int64_t np = 0;  // items issued
+      bool wb_ok = true;
       for (; np < n_items; ++np) {
         const int s = (int)(np % stages);
-        if (np >= stages &&
-            !mbar_wait_bounded(&empty[s], (uint32_t)((np / stages - 1) & 1), &g_step_errors))
-          break;
-        const int64_t r = cid + (np / hpc) * nclusters;
-        const float *src = ssm + (r * H + h0 + (int)(np % hpc)) * (int64_t)head_floats;
+        if (np >= stages && !(wb_ok = write_back(np - stages))) break;
+        const float *src = head_state(np);
         if (M2_OK_BULK(src, head_bytes, sp.ssm, &g_step_errors)) {
           mbar_arrive_expect_tx(&full[s], head_bytes);
           bulk_g2s(sbuf + s * head_floats, src, head_bytes, &full[s]);
@@ -270,9 +302,13 @@ __global__ void __launch_bounds__(kStepBlock, 2)
           mbar_arrive(&full[s]);  // nothing copied: the stage completes without bytes
         }
       }
-      // no copy may be in flight when the CTA exits (each stage's last copy)
+      // the last heads' write-backs; then no copy may be in flight when the CTA
+      // exits (each stage's last load, every store)
+      for (int64_t kk = std::max<int64_t>(0, np - stages); wb_ok && kk < np; ++kk)
+        wb_ok = write_back(kk);
       for (int64_t kk = std::max<int64_t>(0, np - stages); kk < np; ++kk)
         mbar_wait_bounded(&full[kk % stages], (uint32_t)((kk / stages) & 1), &g_step_errors);
+      bulk_wait_all();
     }
     __syncwarp();
     cluster_arrive_wait();
@@ -397,7 +433,6 @@ __global__ void __launch_bounds__(kStepBlock, 2)
                   ? to_f(dt_raw[(bi + nclusters) * ld_dt + h0 + tid])
                   : 0.0f;
     }
-    float *st_row = ssm + (bi * H + h0) * (int64_t)head_floats;
     float *ysr = ys + par * C;
     for (int j = 0; j < hpc; ++j, ++k) {
       const int s = (int)(k % stages);
@@ -409,8 +444,8 @@ __global__ void __launch_bounds__(kStepBlock, 2)
         const float4 b = reinterpret_cast<const float4 *>(ubc + g * N)[q];
         const float4 cc = reinterpret_cast<const float4 *>(ubc + GN + g * N)[q];
         const float dt = dts[j], dA = dAs[j], Dj = Dh[j];
-        const float4 *src = reinterpret_cast<const float4 *>(sbuf + s * head_floats);
-        float4 *dst = reinterpret_cast<float4 *>(st_row + (int64_t)j * head_floats);
+        // updated in place: the producer copies the buffer back to global memory
+        float4 *src = reinterpret_cast<float4 *>(sbuf + s * head_floats);
         // up to 4 rows per thread, independent: their reductions interleave
         constexpr int kPass = 4;
         float pt[kPass], xs[kPass];
@@ -426,7 +461,7 @@ __global__ void __launch_bounds__(kStepBlock, 2)
             v.y = fmaf(dA, v.y, xdt * b.y);
             v.z = fmaf(dA, v.z, xdt * b.z);
             v.w = fmaf(dA, v.w, xdt * b.w);
-            if (M2_OK(dst + idx, 16, sp.ssm, &g_step_errors)) dst[idx] = v;
+            src[idx] = v;
             pt[i] = fmaf(v.x, cc.x, fmaf(v.y, cc.y, fmaf(v.z, cc.z, v.w * cc.w)));
             xs[i] = xv;
           }
@@ -447,14 +482,16 @@ __global__ void __launch_bounds__(kStepBlock, 2)
           v.y = fmaf(dA, v.y, xdt * b.y);
           v.z = fmaf(dA, v.z, xdt * b.z);
           v.w = fmaf(dA, v.w, xdt * b.w);
-          if (M2_OK(dst + idx, 16, sp.ssm, &g_step_errors)) dst[idx] = v;
+          src[idx] = v;
           float t = fmaf(v.x, cc.x, fmaf(v.y, cc.y, fmaf(v.z, cc.z, v.w * cc.w)));
 #pragma unroll
           for (int o = NQ / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
           if (q == 0) ysr[j * P + p] = fmaf(Dj, xv, t);
         }
       }
-      mbar_arrive(&empty[s]);  // this thread is done with buffer s
+      // this thread is done with buffer s: its updates visible to the bulk copy out
+      fence_proxy_async_smem();
+      mbar_arrive(&empty[s]);
     }
     if (tid < hpc) dtr[(par ^ 1) * hpc + tid] = dtn;
     step_bar();  // y of the row complete
