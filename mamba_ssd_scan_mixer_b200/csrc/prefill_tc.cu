@@ -14,15 +14,16 @@
 //   tc_state_pass   H_{c+1} = exp(cum_end) H_c + S_c over chunks in fp32; the
 //                   state entering each chunk is kept as the fp16 MMA operand,
 //                   the final state in fp32.
-//   tc_chunk_out    persistent clusters; per (row, chunk, group) unit the
-//                   cluster's CTAs split the heads of the group:
+//   tc_chunk_out    persistent, one CTA per SM; the heads of a (row, chunk,
+//                   group) are split into blocks of up to 5 taken by different
+//                   CTAs in the same round; per block
 //                   CB = C B^T (M = N = 128, K = 64) once; per head the
 //                   operand CB o exp(cum_t - cum_s) dt_s (causal, D on the
 //                   diagonal) times x (K = 128) and C times H_c^T (K = 64, a
 //                   second accumulator scaled by exp(cum_t)) give y_pre in TMEM;
-//                   the silu(z) gate and sums of squares follow, the per-token
-//                   sums are exchanged through distributed shared memory, and
-//                   the normalised output is written in bf16.
+//                   the silu(z) gate and sums of squares follow, the blocks'
+//                   per-token sums are exchanged through global memory (L2),
+//                   and the normalised output is written in bf16.
 //
 // Operands are fp16 (11-bit significand; bf16's 8 bits cannot meet the output
 // tolerance on these workloads), accumulation is fp32.  The chunk-state
@@ -78,11 +79,15 @@ struct TcArgs {
   float *cbd;                    // [b][G][nch * 128] C_t . B_t in fp32 (the decay operand's diagonal)
   // byte ranges of every buffer, for the checked build (see M2_OK)
   struct Spans {
-    Span xbc, z, dt, y, conv, ssm, S, cum_end, cum, dtv, Hc, hsc, smax, cbd, u, conv_w, conv_b,
-        dt_bias, A, D, norm_w;
+    Span xbc, z, dt, y, conv, ssm, S, cum_end, cum, dtv, Hc, hsc, smax, cbd, u, xpart, xcnt,
+        conv_w, conv_b, dt_bias, A, D, norm_w;
   } sp;
   __half *u;                     // [b][L][conv_dim] post-conv x | B | C, fp16
-  int hpc;                       // max heads per CTA in tc_chunk_out
+  int hpc;                       // most heads of a head block in tc_chunk_out
+  int nhb;                       // head blocks per group in tc_chunk_out
+  float *xpart;                  // [b][nch][G][nhb][128] per-token sums of squares of each block
+  unsigned *xcnt;                // [b][nch][G] blocks that have published their sums
+  int64_t xkeys;                 // (chunk, group) pairs the workspace holds counters for
   int y32;                       // y is 32-byte aligned: rows are written in whole 32-byte sectors
   // packed sequences of different lengths (batch = sequences, L = total tokens):
   // chunk positions come from vl_chunks, written by tc_varlen_prep_kernel
@@ -227,15 +232,6 @@ __device__ __forceinline__ void grid_dependency_wait() {
 }
 __device__ __forceinline__ void launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Smem descriptor for an MN-major SW128 operand: 8-row (K) atoms of 64
 // elements (N) x 128 B, K atoms 1024 B apart (SBO), N atoms `lbo` apart.
@@ -952,6 +948,12 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
   grid_dependency_wait();  // the chunk-state kernel's results (launched early, see prefill_tc)
   launch_dependents();
   const Problem &pr = a.pr;
+  {  // the output kernel's exchange counters start from zero
+    const int64_t stride = (int64_t)gridDim.x * gridDim.y * blockDim.x;
+    for (int64_t i = ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
+         i < a.xkeys; i += stride)
+      if (M2_OK(a.xcnt + i, 4, a.sp.xcnt, &g_tc_errors)) a.xcnt[i] = 0u;
+  }
   const int64_t bi = blockIdx.y;  // sequence (row)
   if (a.varlen && a.vl_chunk0[pr.batch + 1] == 0) return;  // invalid offsets: nothing to do
   // its chunks [cb0, cb0 + nchs) and tokens [t0s, t0s + Ls)
@@ -1076,9 +1078,12 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
 }
 
 // ============================================================== chunk output
-// Persistent clusters: grid (cs, ncl, 1), cluster (cs, 1, 1).  Cluster k takes
-// the units (row, chunk, group) k, k + ncl, ...; its cs CTAs split the group's
-// heads (the same nh <= 5 heads of the group in every unit).  Per CTA:
+// Persistent grid of P CTAs, one per SM.  A unit is (row, chunk, group, head
+// block): the group's heads are cut into nhb blocks of at most 5 heads, and the
+// units are numbered with the head block fastest, so that the nhb units of one
+// (chunk, group) are neighbours.  CTA i takes units i, i + P, ...; P is a
+// multiple of nhb, so the blocks of one (chunk, group) are worked on in the same
+// round by nhb different CTAs.  Per CTA:
 //   warp 16      TMA producer: per unit the C and B tiles of u (C double-
 //                buffered, so the next unit's arrive during this one), per head
 //                the x and H_c tiles (ring of 2) and the z tile (ring of 2);
@@ -1091,12 +1096,19 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
 //                (its TMEM lane quarter) and columns 64 (w / 4) .. +63;
 //   warps 8-15   epilogue: y_j + exp(cum_t) 2^s T, gate by silu(z), per-token
 //                sums of squares, the gated value back into TMEM; after the
-//                unit's last head the per-token sums go to every CTA of the
-//                cluster (asynchronous DSMEM stores completing on the receiver's
-//                mbarrier), and each head is scaled by the norm and the norm
-//                weight and written to y (32-byte stores).  That output phase
-//                overlaps the next unit's operand builds and MMAs: a head's TMEM
-//                columns are handed back to the MMA warp one by one.
+//                unit's last head the per-token sums of the block go to global
+//                memory (row hb of the (chunk, group)'s exchange slot) and a
+//                counter of the (chunk, group) counts the blocks that have
+//                published.  Once it reaches nhb every block adds the nhb rows,
+//                in block order (the same sum, bit for bit, in every CTA and run),
+//                and each head is scaled by the norm and the norm weight and
+//                written to y (32-byte stores).  That output phase overlaps the
+//                next unit's operand builds and MMAs: a head's TMEM columns are
+//                handed back to the MMA warp one by one.
+// A CTA waits only for blocks of its own (chunk, group), which other CTAs reach
+// in the same round or, for a CTA that has more units, the next: with all P CTAs
+// resident (P <= SMs, one CTA per SM) every wait ends.  The counters are zeroed
+// by the state-pass kernel, which runs before this one.
 // All waits are bounded (they raise the error flag and the CTA leaves its loop).
 constexpr uint32_t kCt0 = 0;                       // C [2][128 t][64 n] fp16 (u), 2 x 16 KB
 constexpr uint32_t kBt = 2 * 16384;                // B [128 s][64 n] fp16 (u), 16 KB
@@ -1107,8 +1119,8 @@ constexpr uint32_t kAbuf = kZt + 2 * 16384;        // A [2][2 k-blocks][128 t][6
 constexpr uint32_t kTcOutTiles = kAbuf + 2 * 32768;  // 176 KB
 constexpr int kGroupThreads = 256;                 // threads of the operand / epilogue groups
 
-// Every array read or written with 16-byte accesses (float4 loads, st.async.v4
-// into other ranks) is 16-byte aligned; the static_asserts below check it.
+// Every array read or written with 16-byte accesses (float4 loads and stores) is
+// 16-byte aligned; the static_asserts below check it.
 struct OutShared {
   // decay terms of the unit's heads (operand group)
   alignas(16) float cum2[2][kMaxHeadsPerCta][kQ];  // [unit parity] cumsum * log2(e) (also read by the epilogue)
@@ -1117,23 +1129,20 @@ struct OutShared {
   alignas(16) float betad[kMaxHeadsPerCta][kQ];  // exp(cum_s0 - cum_s) dt_s, s0 = start of s's group
   // epilogue group
   alignas(16) float half_ss[2][kQ];              // per-token sums of squares of the two column halves
-  alignas(16) float mine[kQ];                    // this CTA's per-token partial sums
-  alignas(16) float part[2][16][kQ];             // [unit parity][rank] partial sums received
   alignas(16) float cbd[kQ];                     // C_t . B_t (fp32) of the unit's chunk and group
   alignas(16) uint8_t scs[2][kMaxHeadsPerCta][32];  // [unit parity] exponents s of H_c's row-pair scales 2^s
   alignas(16) float nw[kMaxHeadsPerCta][kHP];     // the unit's norm weights (epilogue group)
   int span_ok[kMaxHeadsPerCta][4];   // group's log2-decay span <= 60: factorise its diagonal
   float Dh[kMaxHeadsPerCta];
   uint64_t full_cb[2], b_free, c_free[2], full_xh[2], empty_xh[2], full_z[2], empty_z[2],
-      a_ready[2], mma_done[2], mbar_cb, cb_free, t_free, y_free[kMaxHeadsPerCta], sums_ready[2],
-      mma_final, e1_done[2];
+      a_ready[2], mma_done[2], mbar_cb, cb_free, t_free, y_free[kMaxHeadsPerCta], mma_final,
+      e1_done[2];
   uint32_t tmem_holder;
 };
 
 static_assert(offsetof(OutShared, cum2) % 16 == 0 && offsetof(OutShared, dt) % 16 == 0 &&
                   offsetof(OutShared, beta) % 16 == 0 && offsetof(OutShared, betad) % 16 == 0 &&
-                  offsetof(OutShared, mine) % 16 == 0 &&
-                  offsetof(OutShared, part) % 16 == 0 && offsetof(OutShared, cbd) % 16 == 0 &&
+                  offsetof(OutShared, cbd) % 16 == 0 &&
                   offsetof(OutShared, scs) % 16 == 0 && offsetof(OutShared, nw) % 16 == 0 &&
                   offsetof(OutShared, full_cb) % 8 == 0,
               "16-byte accessed shared arrays must be 16-byte aligned");
@@ -1147,34 +1156,21 @@ struct OutMaps {
   CUtensorMap z2;
 };
 
-// 16-byte asynchronous store into another rank's shared memory that completes
-// 16 transaction bytes on that rank's mbarrier
-__device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
-      "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)), "r"(__float_as_uint(v.z)),
-      "r"(__float_as_uint(v.w)), "r"(bar)
-      : "memory");
+// Release increment of a counter in global memory (gpu scope), and an acquire
+// read of it.
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t cluster_addr(const void *p, int r) {
-  uint32_t out;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(r));
-  return out;
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity) {
-  auto probe = [&]() {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-  };
-  if (probe()) return true;
+// Waits (bounded) until *cnt >= target; false (and the error flag) if it never gets there.
+__device__ __forceinline__ bool wait_count_bounded(const unsigned *cnt, unsigned target) {
+  if (ld_acquire(cnt) >= target) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (!probe()) {
+  while (ld_acquire(cnt) < target) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_tc_errors, kErrWaitTimeout);
       return false;
@@ -1182,6 +1178,7 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_
   }
   return true;
 }
+
 // Barriers over one 256-thread group (id 1: operand group, id 2: epilogue group);
 // the _and form also returns whether every thread of the group passed `v`.
 __device__ __forceinline__ void group_sync(int id) {
@@ -1208,12 +1205,27 @@ __device__ __forceinline__ void st_global_v8(void *p, const uint32_t (&v)[8]) {
                : "memory");
 }
 
-// Unit n of cluster `cid`: (global chunk gc, group g).
-__device__ __forceinline__ void out_unit(const Problem &pr, int ncl, int cid, int n, int64_t &gc,
-                                         int &g) {
-  const int64_t u = cid + (int64_t)n * ncl;
-  g = (int)(u % pr.G);
-  gc = u / pr.G;
+// Unit n of CTA `cid` in a grid of P: (global chunk gc, group g, head block hb);
+// key = gc G + g numbers the (chunk, group).  The group's hpg heads are split into
+// nhb blocks as evenly as possible: the first hpg % nhb blocks take one head more.
+// (Every index fits in 32 bits: the launch checks that the chunks times the
+// heads do.)
+struct OutUnit {
+  int gc, key, g, hb;
+  int lh0, nh;  // first head of the block within the group, and its heads
+};
+__device__ __forceinline__ OutUnit out_unit(const TcArgs &a, int P, int cid, int n) {
+  const unsigned u = (unsigned)cid + (unsigned)n * (unsigned)P;
+  const unsigned nhb = (unsigned)a.nhb, G = (unsigned)a.pr.G;
+  OutUnit o;
+  o.key = (int)(u / nhb);
+  o.hb = (int)(u - (unsigned)o.key * nhb);
+  o.gc = (int)((unsigned)o.key / G);
+  o.g = o.key - o.gc * (int)G;
+  const int hpg = a.pr.heads_per_group(), base = hpg / a.nhb, rem = hpg - base * a.nhb;
+  o.lh0 = o.hb * base + min(o.hb, rem);
+  o.nh = base + (o.hb < rem ? 1 : 0);
+  return o;
 }
 
 // One 32-column group k of row t of the decay operand A_j (j = head), written as
@@ -1303,24 +1315,18 @@ __device__ __forceinline__ void build_a_group(const OutShared &sh, int par, int 
 // (18 warps: one SM sub-partition holds 5 of them, and 5 x 32 x 96 registers is what
 // its quarter of the register file allows)
 __global__ void __launch_bounds__(kWsThreads, 1)
-    tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps, int ncl) {
-  if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA of every cluster alike
+    tc_chunk_out_kernel(TcArgs a, const __grid_constant__ OutMaps maps) {
+  if (test_stall(&g_tc_stall, &g_tc_errors)) return;  // every CTA alike
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  int cs, rank;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(cs));
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
   const Problem &pr = a.pr;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   OutShared &sh = *reinterpret_cast<OutShared *>(smem_raw + (base - smem_u32(smem_raw)) +
                                                  kTcOutTiles);
-  const int cid = blockIdx.y;
+  const int cid = blockIdx.x, P = gridDim.x;
   const int hpg = pr.heads_per_group();
-  const int lh0 = rank * a.hpc;
-  const int nh = max(0, min(a.hpc, hpg - lh0));  // heads of this CTA in every unit
-  const int64_t n_all = total_chunks(a) * pr.G;
-  const int n_units = n_all > cid ? (int)((n_all - cid + ncl - 1) / ncl) : 0;
-  const uint32_t sum_bytes = (uint32_t)cs * kQ * 4;  // partial sums this CTA receives per unit
+  const int64_t n_all = total_chunks(a) * pr.G * a.nhb;
+  const int n_units = n_all > cid ? (int)((n_all - cid + P - 1) / P) : 0;
 
   if (warp == 0) tmem_alloc(&sh.tmem_holder, 512);
   if (tid == 0) {
@@ -1334,10 +1340,6 @@ __global__ void __launch_bounds__(kWsThreads, 1)
       mbar_init(&sh.a_ready[k], kGroupThreads);
       mbar_init(&sh.mma_done[k], 1);
       mbar_init(&sh.e1_done[k], kGroupThreads);  // the epilogue is done with a parity's cum2 / scs
-      // the local arrival carries the bytes the ranks' partial sums complete;
-      // units 0 and 1 are armed here, unit n + 2 once unit n's sums are read
-      mbar_init(&sh.sums_ready[k], 1);
-      mbar_arrive_expect_tx(&sh.sums_ready[k], sum_bytes);
     }
     mbar_init(&sh.b_free, 1);
     mbar_init(&sh.mbar_cb, 1);
@@ -1350,23 +1352,17 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_arrive_relaxed();  // waited for before the first remote store
-  grid_dependency_wait();    // u, H_c, the scales and the dt rows are complete from here on
-  bool started = false;
+  grid_dependency_wait();  // u, H_c, the scales, the dt rows and the zeroed counters are ready
   const uint32_t tmem = sh.tmem_holder;
   constexpr uint32_t kTmemY = 128;                     // y_j at columns 128 + 64 j
 
   // normalised bf16 output of head j of unit `un` by a thread of the epilogue group
   // (row t = 32 (warp % 4) + lane, columns 32 ((warp / 4) % 2) .. +31 of the head);
   // the head's TMEM columns go back to the MMA warp as soon as they are read
-  auto output_head = [&](int un, int j, float inv) {
+  auto output_head = [&](int h0, const ChunkPos &pos, int j, float inv) {
     const int q = warp & 3, eh = (warp >> 2) & 1, t = 32 * q + lane;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    int64_t ogc;
-    int og;
-    out_unit(pr, ncl, cid, un, ogc, og);
-    const ChunkPos pos = chunk_pos(a, ogc);
-    const int h = og * hpg + lh0 + j;
+    const int h = h0 + j;
     const int64_t tok = pos.t0 + t;
     const bool t_valid = t < pos.nv;
     __nv_bfloat16 *yrow = a.y + tok * pr.d_inner + (int64_t)h * kHP + 32 * eh;
@@ -1422,7 +1418,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
   };
   if (warp == 16) {
     // ---------------- producer
-    if (lane == 0 && nh > 0) {
+    if (lane == 0) {
       bool ok = true;
       int J = 0, ncb = 0, nxh = 0, nz = 0;  // copies issued into each ring
       // a [128 tokens][64 ch] tile of u or z for the unit at `pos`
@@ -1432,9 +1428,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         else tma_load_3d(dst, m3, ch, pos.c * kQ, pos.seq, bar);
       };
       auto load_cb = [&](int n) {  // C and B tiles of unit n
-        int64_t gc;
-        int g;
-        out_unit(pr, ncl, cid, n, gc, g);
+        const OutUnit ou = out_unit(a, P, cid, n);
+        const int64_t gc = ou.gc;
+        const int g = ou.g;
         const ChunkPos pos = chunk_pos(a, gc);
         const int cbuf = n & 1;
         if (n >= 2) ok = ok && mbar_wait_bounded(&sh.c_free[cbuf], (uint32_t)(((n - 2) >> 1) & 1), &g_tc_errors);
@@ -1447,13 +1443,13 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                  &sh.full_cb[cbuf]);
         ++ncb;
       };
-      load_cb(0);
+      if (n_units > 0) load_cb(0);
       for (int n = 0; ok && n < n_units; ++n) {
-        int64_t gc;
-        int g;
-        out_unit(pr, ncl, cid, n, gc, g);
+        const OutUnit ou = out_unit(a, P, cid, n);
+        const int64_t gc = ou.gc;
+        const int nh = ou.nh;
         const ChunkPos pos = chunk_pos(a, gc);
-        const int h0 = g * hpg + lh0;
+        const int h0 = ou.g * hpg + ou.lh0;
         for (int j = 0; ok && j < nh; ++j, ++J) {
           const int h = h0 + j, sl = J & 1;
           if (J >= 2) ok = mbar_wait_bounded(&sh.empty_xh[sl], (uint32_t)(((J - 2) >> 1) & 1), &g_tc_errors);
@@ -1481,7 +1477,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     }
   } else if (warp == 17) {
     // ---------------- MMA issuer
-    if (lane == 0 && nh > 0) {
+    if (lane == 0) {
       const uint32_t idesc_cb = umma_idesc_f16(128, 128);
       const uint32_t idesc_mn = umma_idesc_f16(128, 64) | (1u << 16);  // B operand MN-major
       int J = 0;
@@ -1499,6 +1495,7 @@ __global__ void __launch_bounds__(kWsThreads, 1)
                    idesc_cb, kin > 0 ? 1u : 0u);
         umma_commit(&sh.mbar_cb);
         umma_commit(&sh.b_free);
+        const int nh = out_unit(a, P, cid, n).nh;
         for (int j = 0; j < nh; ++j, ++J) {
           const int sl = J & 1;
           ok = mbar_wait_bounded(&sh.a_ready[sl], (uint32_t)((J >> 1) & 1), &g_tc_errors) &&
@@ -1538,11 +1535,11 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     bool ok = true;
     int J = 0;
-    for (int n = 0; ok && n < n_units && nh > 0; ++n) {
-      int64_t gc;
-      int g;
-      out_unit(pr, ncl, cid, n, gc, g);
-      const int h0 = g * hpg + lh0;
+    for (int n = 0; ok && n < n_units; ++n) {
+      const OutUnit ou = out_unit(a, P, cid, n);
+      const int64_t gc = ou.gc;
+      const int g = ou.g, nh = ou.nh;
+      const int h0 = g * hpg + ou.lh0;
       const int par = n & 1;
       // the epilogue reads this parity's exp(cum) and scales of unit n - 2 until it is done
       // with that unit's gate pass
@@ -1617,10 +1614,9 @@ __global__ void __launch_bounds__(kWsThreads, 1)
     bool ok = true;
     int J = 0;
     for (int n = 0; ok && n < n_units; ++n) {
-      int64_t gc;
-      int g;
-      out_unit(pr, ncl, cid, n, gc, g);
-      const int h0 = g * hpg + lh0;
+      const OutUnit ou = out_unit(a, P, cid, n);
+      const int nh = ou.nh;
+      const int h0 = ou.g * hpg + ou.lh0;
       const int par = n & 1;
       float ss = 0.0f;
       for (int j = 0; j < nh; ++j, ++J) {
@@ -1633,14 +1629,16 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         const float ec = ex2_approx(sh.cum2[par][j][t]);  // exp(cum_t)
         const uint32_t ycol = tmem + lane_off + kTmemY + 64 * j + 32 * eh;
         const uint32_t zt = base + kZt + sl * 16384;
+        // this thread's 32 columns of C H_c^T first, together with the first 16 of
+        // y_j, so that the shared accumulator can take the next head's product early
+        float w32[32], v[16];
+        tmem_ld32x16(tmem + lane_off + kTmemT + 32 * eh, w32, ycol, v);
+        tc_fence_before();
+        mbar_arrive(&sh.t_free);  // the C H_c^T columns may take the next head's product
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          float v[16], w[16];
-          tmem_ld16x2(ycol + 16 * hh, v, tmem + lane_off + kTmemT + 32 * eh + 16 * hh, w);
-          if (hh == 1) {
-            tc_fence_before();
-            mbar_arrive(&sh.t_free);  // the C H_c^T columns may take the next head's product
-          }
+          if (hh == 1) tmem_ld16(ycol + 16, v);
+          const float *w = w32 + 16 * hh;
           // the scales 2^s of H_c's rows p (pairs) of these 16 columns, from their exponents
           const uint2 se = *reinterpret_cast<const uint2 *>(&sh.scs[par][j][16 * eh + 8 * hh]);
           float scp[8];
@@ -1681,24 +1679,37 @@ __global__ void __launch_bounds__(kWsThreads, 1)
           nwv[r] = M2_OK(wp, 4, a.sp.norm_w, &g_tc_errors) ? __ldg(wp) : 0.0f;
         }
       }
-      // per-token sums of this CTA into part[par][rank][*] of every rank
+      // the block's per-token sums into row hb of the (chunk, group)'s exchange slot
       sh.half_ss[eh][t] = ss;
       ok = group_all(2, ok);
       if (!ok) break;
-      if (gt < kQ) sh.mine[gt] = sh.half_ss[0][gt] + sh.half_ss[1][gt];
-      if (!started) {
-        cluster_wait();  // (arrived at the start) every CTA of the cluster is running
-        started = true;
+      float *xslot = a.xpart + (int64_t)ou.key * a.nhb * kQ;
+      unsigned *xcnt = a.xcnt + ou.key;
+      if (gt < kQ) {
+        float *dst = xslot + ou.hb * kQ + gt;
+        if (M2_OK(dst, 4, a.sp.xpart, &g_tc_errors)) __stcg(dst, sh.half_ss[0][gt] + sh.half_ss[1][gt]);
       }
-      group_sync(2);
-      for (int i = gt; i < cs * (kQ / 4); i += kGroupThreads) {
-        const int r = i / (kQ / 4), f = i % (kQ / 4);
-        st_async_v4(cluster_addr(&sh.part[par][rank][4 * f], r),
-                    reinterpret_cast<const float4 *>(sh.mine)[f], cluster_addr(&sh.sums_ready[par], r));
+      group_sync(2);  // every row of the block is written before it is counted
+      bool got = true;
+      if (gt == 0 && M2_OK(xcnt, 4, a.sp.xcnt, &g_tc_errors)) {
+        // (release: the rows the group wrote before the barrier are visible first)
+        red_release_add(xcnt, 1u);
+        got = wait_count_bounded(xcnt, (unsigned)a.nhb);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait_cluster_bounded(&sh.sums_ready[par], (uint32_t)((n >> 1) & 1))) != 0;
-      float tot = 0.0f;
-      for (int r = 0; r < cs; ++r) tot += sh.part[par][r][t];
+      ok = group_all(2, got);
+      if (!ok) break;
+      float tot = 0.0f;  // blocks in order: the same sum in every block's CTA
+      for (int r0 = 0; r0 < a.nhb; r0 += 16) {
+        float pv[16];  // (loads issued together, added in order)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float *src = xslot + (r0 + i) * kQ + t;
+          pv[i] = (r0 + i < a.nhb && M2_OK(src, 4, a.sp.xpart, &g_tc_errors)) ? __ldcg(src) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (r0 + i < a.nhb) tot += pv[i];
+      }
       const float inv = rsqrtf(tot / (float)(hpg * kHP) + pr.eps);
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
@@ -1706,61 +1717,56 @@ __global__ void __launch_bounds__(kWsThreads, 1)
         if (idx < nh * kHP) sh.nw[idx / kHP][idx % kHP] = nwv[r];
       }
       ok = group_all(2, ok);
-      // unit n + 2 uses this parity again; no rank sends it before this CTA has
-      // sent unit n + 1's sums, which happens after this point
-      if (gt == 0 && n + 2 < n_units) mbar_arrive_expect_tx(&sh.sums_ready[par], sum_bytes);
       if (!ok) break;
       // normalised bf16 output, head by head; each head's TMEM columns go back to the
-      // MMA warp (for the next unit) as soon as they are read
-      for (int j = 0; j < nh; ++j) output_head(n, j, inv);
+      // MMA warp (for the next unit) as soon as they are read.  Slots this unit
+      // leaves empty (a smaller head block) are handed back too, so that every
+      // slot's barrier completes once per unit
+      const ChunkPos pos = chunk_pos(a, ou.gc);
+      for (int j = 0; j < nh; ++j) output_head(h0, pos, j, inv);
+      for (int j = nh; j < a.hpc; ++j) mbar_arrive(&sh.y_free[j]);
     }
   }
-  // every thread: the cluster's start barrier (if not waited for yet), then one
-  // more: no CTA exits while another may still store into its shared memory
   __syncwarp();
-  if (!started) cluster_wait();
-  cluster_arrive_release();
-  cluster_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 
-// Heads per CTA and cluster size of tc_chunk_out for hpg heads per group.
-// Most clusters of `cs` output-kernel CTAs resident at once on the current
-// device (cached per device; -1 if the query fails).
-int out_max_clusters(int cs);
+// Most head blocks per group the output kernel uses (blocks of 2 heads or more,
+// unless a group has one head): the size of the exchange.
+int out_max_blocks(int hpg) { return hpg <= 1 ? 1 : (hpg + 1) / 2; }
 
-// Cluster size of the output kernel: every size from ceil(hpg / 6) to 16 whose
-// heads per CTA fit tensor memory is scored by the rounds of units its resident
-// clusters need times (heads per CTA + a per-unit cost of about 2.5 heads).
-void out_choose(int hpg, int64_t units, int *cs, int *hpc, int *ncl) {
-  const int lo = (hpg + kMaxHeadsPerCta - 1) / kMaxHeadsPerCta;
+// Head blocks of the output kernel for hpg heads per group and `keys` (chunk,
+// group) pairs on `sms` SMs: every block size h = 2 .. 5 (1 for a single head)
+// gives nhb = ceil(hpg / h) blocks and a grid of the largest multiple of nhb that
+// fits the SMs; the choice minimises the rounds of units times (heads per block +
+// a per-unit cost of about 2.5 heads).  False if no block size fits (more than
+// 5 x sms heads).
+bool out_choose(int hpg, int64_t keys, int sms, int *hpc, int *nhb, int *grid) {
   int64_t best = -1;
-  for (int c = std::max(lo, 1); c <= 16; ++c) {
-    const int h = (hpg + c - 1) / c;
-    if (h > kMaxHeadsPerCta) continue;
-    const int m = out_max_clusters(c);
-    if (m <= 0) continue;
-    const int64_t rounds = (units + m - 1) / m;
-    const int64_t score = rounds * (2 * h + 5);
+  for (int h = std::min(hpg, 2); h <= kMaxHeadsPerCta; ++h) {
+    const int nb = (hpg + h - 1) / h;
+    if (nb > sms) continue;
+    const int hh = (hpg + nb - 1) / nb;  // the largest block after evening out
+    const int64_t units = keys * nb;
+    const int64_t P = std::min<int64_t>((int64_t)(sms / nb) * nb, units);
+    const int64_t rounds = (units + P - 1) / P;
+    const int64_t score = rounds * (2 * hh + 5);
     if (best < 0 || score < best) {
       best = score;
-      *cs = c;
-      *hpc = h;
-      *ncl = (int)std::min<int64_t>(units, m);
+      *hpc = hh;
+      *nhb = nb;
+      *grid = (int)P;
     }
   }
-  if (best < 0) {  // no occupancy answer: the smallest cluster, one per unit
-    *cs = std::max(lo, 1);
-    *hpc = (hpg + *cs - 1) / *cs;
-    *ncl = (int)std::min<int64_t>(units, 65535);
-  }
+  return best >= 0;
 }
 
 struct TcWorkspace {
-  float *S, *cum_end, *cum, *dtv, *hsc, *smax, *cbd;
+  float *S, *cum_end, *cum, *dtv, *hsc, *smax, *cbd, *xpart;
+  unsigned *xcnt;
   __half *Hc, *u;
   int4 *vl_chunks;
   int *vl_chunk0;
@@ -1791,6 +1797,9 @@ size_t tc_carve(const Problem &pr, bool varlen, char *base, TcWorkspace *w) {
   t.hsc = reinterpret_cast<float *>(take(cap * pr.H * 32 * 4));
   t.smax = reinterpret_cast<float *>(take(cap * pr.H * 4));
   t.cbd = reinterpret_cast<float *>(take(cap * pr.G * kQ * 4));
+  // output-kernel exchange: at most hpg head blocks per (chunk, group)
+  t.xpart = reinterpret_cast<float *>(take(cap * pr.G * out_max_blocks(pr.heads_per_group()) * kQ * 4));
+  t.xcnt = reinterpret_cast<unsigned *>(take(cap * pr.G * 4));
   t.vl_chunks = varlen ? reinterpret_cast<int4 *>(take(cap * 16)) : nullptr;
   t.vl_chunk0 = varlen ? reinterpret_cast<int *>(take((size_t)(pr.batch + 2) * 4)) : nullptr;
   const size_t tokens = varlen ? (size_t)pr.L : (size_t)(pr.batch * pr.L);
@@ -1852,33 +1861,6 @@ constexpr size_t kK3Smem = kTcOutTiles + sizeof(OutShared) + 1024;
 static_assert(kK1Smem + 14 * 1024 <= 227 * 1024 && kK3Smem + 1024 <= 227 * 1024,
               "shared memory per CTA");
 
-int out_max_clusters(int cs) {
-  static int cache[64][17] = {};  // 0: not asked yet
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || cs < 1 || cs > 16) return -1;
-  int &m = cache[dev][cs];
-  if (m == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)cs, 1, 1);
-    cfg.blockDim = dim3(kWsThreads, 1, 1);
-    cfg.dynamicSmemBytes = kK3Smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int v = 0;
-    if (cudaOccupancyMaxActiveClusters(&v, tc_chunk_out_kernel, &cfg) != cudaSuccess) {
-      cudaGetLastError();  // clear the failed query
-      v = -1;
-    }
-    m = v > 0 ? v : -1;
-  }
-  return m;
-}
-
 }  // namespace
 
 const char *const kPrefillTcStages[] = {"tc_chunk_state", "tc_state_pass", "tc_chunk_out"};
@@ -1888,7 +1870,7 @@ bool prefill_tc_supported(const Problem &pr, bool varlen) {
   const int64_t nch = ceil_div(pr.L, kQ), cap = tc_chunk_cap(pr, varlen);
   const int64_t pairs = (pr.heads_per_group() + 1) / 2;
   return pr.io == MAMBA2_BF16 && pr.P == kHP && pr.N == kNS && pr.K == 4 &&
-         pr.heads_per_group() <= 16 * kMaxHeadsPerCta && pr.L > 0 &&
+         pr.heads_per_group() <= kMaxHeadsPerCta * 128 && pr.L > 0 &&
          (varlen || nch <= 65535) && pr.L < ((int64_t)1 << 31) &&
          pr.batch * pr.L < ((int64_t)1 << 31) && cap * pr.H * kHP < ((int64_t)1 << 31) &&
          cap * pr.G * (pairs + 1) < ((int64_t)1 << 31);
@@ -1946,6 +1928,9 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.smax = w.smax;
   a.cbd = w.cbd;
   a.u = w.u;
+  a.xpart = w.xpart;
+  a.xcnt = w.xcnt;
+  a.xkeys = cap * pr.G;
   {
     const int64_t bl = tokens, nq = cap, nrow = 1;  // chunk arrays: cap chunks
     const size_t st1 = (size_t)nrow * nq * pr.H * kHP * kNS;
@@ -1963,6 +1948,8 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     a.sp.hsc = span_of(a.hsc, (size_t)nq * pr.H * 32 * 4);
     a.sp.smax = span_of(a.smax, (size_t)nq * pr.H * 4);
     a.sp.cbd = span_of(a.cbd, (size_t)pr.G * nq * kQ * 4);
+    a.sp.xpart = span_of(a.xpart, (size_t)nq * pr.G * out_max_blocks(pr.heads_per_group()) * kQ * 4);
+    a.sp.xcnt = span_of(a.xcnt, (size_t)nq * pr.G * 4);
     a.sp.u = span_of(a.u, (size_t)bl * pr.conv_dim * 2);
     a.sp.conv_w = span_of(a.prm.conv_w, (size_t)pr.conv_dim * 4 * 4);
     a.sp.conv_b = span_of(a.prm.conv_b, (size_t)pr.conv_dim * 4);
@@ -1980,13 +1967,13 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kK3Smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_chunk_out_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                             1);
-    if (e != cudaSuccess) return e;
   }
-  int cs = 1, hpc = 1, ncl = 1;
-  out_choose(hpg, cap * (int64_t)pr.G, &cs, &hpc, &ncl);
+  // the output kernel's head blocks and grid (one CTA per SM, all resident at once)
+  int hpc = 1, nhb = 1, grid3 = 1;
+  if (!out_choose(hpg, cap * (int64_t)pr.G, sm_count(), &hpc, &nhb, &grid3))
+    return cudaErrorNotSupported;
   a.hpc = hpc;
+  a.nhb = nhb;
 
   stage_mark(st, 0);
   if (varlen) {  // the chunks of the packed sequences
@@ -2035,19 +2022,15 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   stage_mark(st, 2);
   {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)cs, (unsigned)ncl, 1);
+    cfg.gridDim = dim3((unsigned)grid3, 1, 1);
     cfg.blockDim = dim3(kWsThreads, 1, 1);
     cfg.dynamicSmemBytes = kK3Smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     OutMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     {
@@ -2075,7 +2058,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
           return cudaErrorInvalidValue;
       }
     }
-    e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps, ncl);
+    e = cudaLaunchKernelEx(&cfg, tc_chunk_out_kernel, a, maps);
     if (e != cudaSuccess) return e;
   }
   stage_mark(st, 3);

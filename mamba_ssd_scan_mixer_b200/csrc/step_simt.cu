@@ -341,8 +341,8 @@ __global__ void __launch_bounds__(kStepBlock, 2)
       else if (i < n2) src = reinterpret_cast<const char *>(xBC + bi * ld_x + (int64_t)h0 * P) + 16 * (i - n1);
       else if (i < n3) src = reinterpret_cast<const char *>(xBC + bi * ld_x + pr.d_inner) + 16 * (i - n2);
       else src = reinterpret_cast<const char *>(z + bi * ld_z + (int64_t)h0 * P) + 16 * (i - n3);
-      const Span &spn = i < n1 ? sp.conv : (i < n3 ? sp.xbc : sp.z);
-      if (M2_OK(src, 16, spn, &g_step_errors)) cp_async16(pb + 16 * i, src);
+      if (M2_OK(src, 16, i < n1 ? sp.conv : (i < n3 ? sp.xbc : sp.z), &g_step_errors))
+        cp_async16(pb + 16 * i, src);
     }
     cp_async_commit();
   };

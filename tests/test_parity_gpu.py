@@ -37,19 +37,22 @@ def test_tiny_f32_config():
     case("zamba2_2p7b_prefill", batch=1, seqlen=333, nheads=4, chunk_size=64),
     case("zamba2_2p7b_prefill", batch=3, seqlen=129, nheads=6, ngroups=3, chunk_size=128),
     case("zamba2_2p7b_prefill", batch=2, seqlen=300, nheads=4, norm_before_gate=True),
-    # head splits of the tensor-core output kernel: odd heads per group (a lone head in
-    # the last pair of the chunk-state kernel), 13 and 17 heads (uneven splits with a
-    # short last CTA), two groups of 16 heads, and 20 heads over 24 (row, chunk)
-    # units, more units than resident clusters
+    # head blocks of the tensor-core output kernel: odd heads per group (a lone head in
+    # the last pair of the chunk-state kernel), 13 and 17 heads (blocks of unequal
+    # size), two groups of 16 heads, and 20 heads over 24 (row, chunk) pairs
     case("zamba2_2p7b_prefill", batch=1, seqlen=300, nheads=6, ngroups=2),
     case("zamba2_2p7b_prefill", batch=1, seqlen=260, nheads=13),
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=17),
     case("zamba2_2p7b_prefill", batch=2, seqlen=256, nheads=32, ngroups=2),
     case("zamba2_2p7b_prefill", batch=3, seqlen=1000, nheads=20),
-    # 80 heads (16-CTA output clusters, several (chunk, group) units per cluster;
-    # several chunk-state items per CTA, crossing (row, chunk) keys)
+    # 80 heads (16 blocks of 5 per (chunk, group); several chunk-state items per CTA,
+    # crossing (row, chunk) keys), 64 heads (13 blocks of 4 or 5), 80 heads over 24
+    # (row, chunk) pairs (384 units: three rounds of the 144-CTA grid, blocks that
+    # change heads from unit to unit) and 96 heads in one group (20 blocks)
     case("zamba2_2p7b_prefill", batch=1, seqlen=1100, nheads=80),
     case("zamba2_2p7b_prefill", batch=2, seqlen=640, nheads=64),
+    case("zamba2_2p7b_prefill", batch=2, seqlen=1500, nheads=80),
+    case("zamba2_2p7b_prefill", batch=1, seqlen=400, nheads=96),
     case("zamba2_2p7b_prefill", batch=1, seqlen=257, nheads=4, headdim=32, dstate=128),
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=4, headdim=16, dstate=32),
     case("tiny_f32", batch=2, seqlen=517, nheads=6, ngroups=2, headdim=64, dstate=64,
