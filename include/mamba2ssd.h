@@ -259,9 +259,62 @@ MAMBA2_API int mamba2_conv_ssd_prefill_noalloc(const mamba2_dims *dims,
                                                float *ssm_state, int32_t states_in,
                                                void *stream);
 
+/* Workspace bytes mamba2_conv_ssd_prefill_backward needs for `dims` (0 if
+ * the dims are invalid).  It holds the SSM state after every token:
+ * batch * nheads * seqlen * headdim * dstate * 4 bytes of it (5.4 GB for one
+ * 4096-token sequence of 80 heads of 64 x 64), plus O(batch * seqlen *
+ * (conv_dim + nheads * dstate * 16)) bytes more. */
+MAMBA2_API size_t mamba2_prefill_backward_workspace_size(const mamba2_dims *dims);
+
+/* Backward pass of mamba2_conv_ssd_prefill, for training.  The pages give the
+ * Zamba2 layers gradient checkpointing ("Zamba2 hybrid architecture in
+ * Transformers", qwbw.cn, section 三): the forward is recomputed from the
+ * layer's inputs inside this call (nothing of a forward call is needed) and
+ * differentiated.  The gradients are those of
+ *     sum(y * dy) + sum(h_L * d_ssm_state_out)
+ * with respect to every input, parameter and initial state, y being the
+ * prefill's output and h_L its final SSM state.
+ *
+ *  dims, params, xBC, z, dt_raw and their row strides: as for the prefill
+ *          (the same validation; fixed-length rows, states_in given by the
+ *          state pointers below).
+ *  conv_state_in  [b, conv_dim, d_conv] io_dtype, contiguous, or NULL: the
+ *          carried conv state the prefill started from (NULL: zero context).
+ *  ssm_state_in   [b, nheads, headdim, dstate] fp32, contiguous, or NULL: the
+ *          initial SSM state (NULL: zero).
+ *  dy      [b, L, d_inner] io_dtype, contiguous: gradient of y.
+ *  d_ssm_state_out [b, nheads, headdim, dstate] fp32 or NULL (zero): gradient
+ *          of the returned final state.  (The final conv state's gradient is
+ *          taken as zero.)
+ * Outputs, overwritten (not accumulated):
+ *  d_xBC   [b, L, conv_dim] io_dtype, contiguous.
+ *  d_z     [b, L, d_inner] io_dtype, contiguous.
+ *  d_dt_raw [b, L, nheads] io_dtype, contiguous.
+ *  d_conv_w [conv_dim, d_conv], d_conv_b [conv_dim], d_dt_bias [nheads],
+ *          d_A [nheads], d_D [nheads], d_norm_w [d_inner]: fp32.
+ *  d_conv_state_in [b, conv_dim, d_conv] io_dtype or NULL (column 0, the
+ *          oldest input, never reaches y: its gradient is zero).
+ *  d_ssm_state_in  [b, nheads, headdim, dstate] fp32 or NULL.
+ *  workspace  >= mamba2_prefill_backward_workspace_size(dims) bytes, 256-byte
+ *          aligned.  stream: cudaStream_t as void*.
+ * Runs in fp32 on the CUDA cores for every supported shape.  The sums over
+ * tokens of the parameter gradients use atomic additions, so they may differ
+ * in the last bits between runs; the other gradients are deterministic.
+ * Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG (null or misaligned pointer, bad
+ * stride), MAMBA2_ERR_UNSUPPORTED, MAMBA2_ERR_WORKSPACE or MAMBA2_ERR_CUDA. */
+MAMBA2_API int mamba2_conv_ssd_prefill_backward(
+    const mamba2_dims *dims, const mamba2_params *params, const void *xBC,
+    int64_t xBC_row_stride, const void *z, int64_t z_row_stride, const void *dt_raw,
+    int64_t dt_row_stride, const void *conv_state_in, const float *ssm_state_in, const void *dy,
+    const float *d_ssm_state_out, void *d_xBC, void *d_z, void *d_dt_raw, float *d_conv_w,
+    float *d_conv_b, float *d_dt_bias, float *d_A, float *d_D, float *d_norm_w,
+    void *d_conv_state_in, float *d_ssm_state_in, void *workspace, size_t workspace_bytes,
+    void *stream);
+
 /* Profiling aid (no counterpart on the pages).  Arms the calling host thread
  * so that its NEXT call of mamba2_conv_ssd_prefill,
- * mamba2_conv_ssd_prefill_noalloc or mamba2_ssd_step records events[i]
+ * mamba2_conv_ssd_prefill_noalloc, mamba2_ssd_step or
+ * mamba2_conv_ssd_prefill_backward records events[i]
  * (cudaEvent_t passed as void*, created by the caller) on the call's stream
  * just before the call's kernel stage i, and events[S] after
  * its last stage, S being the stage count that mamba2_stage_names reports.
@@ -271,7 +324,8 @@ MAMBA2_API int mamba2_conv_ssd_prefill_noalloc(const mamba2_dims *dims,
  * MAMBA2_ERR_INVALID_ARG (bad count, or events NULL with n_events > 0). */
 MAMBA2_API int mamba2_record_stage_events(void *const *events, int n_events);
 
-/* Number of kernel stages a call of `kind` (0 = prefill, 1 = decode step)
+/* Number of kernel stages a call of `kind` (0 = prefill, 1 = decode step,
+ * 2 = prefill backward)
  * enqueues for `dims`, or MAMBA2_ERR_INVALID_ARG; writes up to max_names
  * static stage names to `names` (may be NULL).  A stage is one kernel launch
  * (a stage whose work is absent for a call, e.g. the conv-state write without

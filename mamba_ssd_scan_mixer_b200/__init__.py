@@ -21,7 +21,8 @@ __all__ = [
     "Mamba2Dims", "Mamba2Params", "Mamba2Error", "MAMBA2_F32", "MAMBA2_BF16", "lib",
     "library_path", "make_dims", "make_params", "mamba2_prefill_workspace_size",
     "mamba2_conv_ssd_prefill", "mamba2_conv_ssd_prefill_noalloc", "mamba2_ssd_step", "prefill",
-    "step", "status_string",
+    "step", "status_string", "mamba2_prefill_backward_workspace_size",
+    "mamba2_conv_ssd_prefill_backward", "prefill_backward",
 ]
 
 MAMBA2_F32, MAMBA2_BF16 = 0, 1
@@ -87,6 +88,11 @@ def lib() -> ctypes.CDLL:
         L.mamba2_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         L.mamba2_debug_stall_waits.restype = ctypes.c_int
         L.mamba2_debug_stall_waits.argtypes = [ctypes.c_int]
+        L.mamba2_prefill_backward_workspace_size.restype = sz
+        L.mamba2_prefill_backward_workspace_size.argtypes = [pd]
+        L.mamba2_conv_ssd_prefill_backward.restype = ctypes.c_int
+        L.mamba2_conv_ssd_prefill_backward.argtypes = ([pd, pp, vp, i64, vp, i64, vp, i64]
+                                                       + [vp] * 15 + [vp, sz, vp])
         L.mamba2_ssd_step.restype = ctypes.c_int
         L.mamba2_ssd_step.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp, vp]
         _lib = L
@@ -283,3 +289,61 @@ def step(dims, params, xBC, z, dt_raw, conv_state, ssm_state, y=None, stream=Non
                         device=xBC.device)
     mamba2_ssd_step(dims, params, xBC, z, dt_raw, y, conv_state, ssm_state, stream)
     return y
+
+
+def mamba2_prefill_backward_workspace_size(dims: Mamba2Dims) -> int:
+    return int(lib().mamba2_prefill_backward_workspace_size(ctypes.byref(dims)))
+
+
+def mamba2_conv_ssd_prefill_backward(dims, params, xBC, z, dt_raw, dy, grads, conv_state_in=None,
+                                     ssm_state_in=None, d_ssm_state_out=None, workspace=None,
+                                     stream=None) -> None:
+    """Enqueue the prefill's backward pass on `stream`.
+
+    xBC, z, dt_raw as for the prefill; dy [b, L, d_inner] contiguous; grads: a dict of
+    output tensors "xBC", "z", "dt_raw" (io dtype, contiguous), "conv_w", "conv_b",
+    "dt_bias", "A", "D", "norm_w" (fp32) and optionally "conv_state", "ssm_state" (the
+    initial states' gradients); workspace: a CUDA byte tensor of
+    mamba2_prefill_backward_workspace_size(dims) bytes."""
+    L = dims.seqlen
+    lx = _rows(xBC, "xBC", None, dims.batch, L)
+    lz = _rows(z, "z", None, dims.batch, L)
+    ld = _rows(dt_raw, "dt_raw", None, dims.batch, L)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    g = lambda k: _ptr(grads.get(k))
+    st = lib().mamba2_conv_ssd_prefill_backward(
+        ctypes.byref(dims), ctypes.byref(params), _ptr(xBC), lx, _ptr(z), lz, _ptr(dt_raw), ld,
+        _ptr(conv_state_in), _ptr(ssm_state_in), _ptr(dy), _ptr(d_ssm_state_out), g("xBC"),
+        g("z"), g("dt_raw"), g("conv_w"), g("conv_b"), g("dt_bias"), g("A"), g("D"), g("norm_w"),
+        g("conv_state"), g("ssm_state"), _ptr(workspace), ws_bytes, _stream(stream))
+    if st != 0:
+        raise Mamba2Error(st, "mamba2_conv_ssd_prefill_backward")
+
+
+def prefill_backward(dims, params, xBC, z, dt_raw, dy, conv_state_in=None, ssm_state_in=None,
+                     d_ssm_state_out=None, workspace=None, stream=None):
+    """Allocate the gradients (and the workspace if not given) and run the backward pass.
+    Returns the dict of gradients (initial-state gradients when those states are given)."""
+    import torch
+    dev, dt = xBC.device, xBC.dtype
+    b, L, H, P, N, G = (dims.batch, dims.seqlen, dims.nheads, dims.headdim, dims.dstate,
+                        dims.ngroups)
+    d_inner, conv_dim = H * P, H * P + 2 * G * N
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = {"xBC": torch.empty(b, L, conv_dim, dtype=dt, device=dev),
+             "z": torch.empty(b, L, d_inner, dtype=dt, device=dev),
+             "dt_raw": torch.empty(b, L, H, dtype=dt, device=dev),
+             "conv_w": torch.empty(conv_dim, dims.d_conv, **f32),
+             "conv_b": torch.empty(conv_dim, **f32), "dt_bias": torch.empty(H, **f32),
+             "A": torch.empty(H, **f32), "D": torch.empty(H, **f32),
+             "norm_w": torch.empty(d_inner, **f32)}
+    if conv_state_in is not None:
+        grads["conv_state"] = torch.empty_like(conv_state_in)
+    if ssm_state_in is not None:
+        grads["ssm_state"] = torch.empty_like(ssm_state_in)
+    if workspace is None:
+        workspace = torch.empty(max(1, mamba2_prefill_backward_workspace_size(dims)),
+                                dtype=torch.uint8, device=dev)
+    mamba2_conv_ssd_prefill_backward(dims, params, xBC, z, dt_raw, dy, grads, conv_state_in,
+                                     ssm_state_in, d_ssm_state_out, workspace, stream)
+    return grads

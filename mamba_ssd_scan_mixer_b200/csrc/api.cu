@@ -170,11 +170,17 @@ MAMBA2_API int mamba2_debug_stall_waits(int enable) {
 MAMBA2_API int mamba2_stage_names(int kind, const mamba2_dims *dims, const char **names,
                                   int max_names) {
   Problem pr;
-  if (make_problem(dims, kind == 0, &pr) != MAMBA2_OK) return MAMBA2_ERR_INVALID_ARG;
-  if (kind != 0 && kind != 1) return MAMBA2_ERR_INVALID_ARG;
+  if (kind != 0 && kind != 1 && kind != 2) return MAMBA2_ERR_INVALID_ARG;
+  if (make_problem(dims, kind != 1, &pr) != MAMBA2_OK) return MAMBA2_ERR_INVALID_ARG;
   const bool tc = kind == 0 && use_tc(pr);
-  const char *const *list = kind == 1 ? kStepSimtStages : tc ? kPrefillTcStages : kPrefillSimtStages;
-  const int n = kind == 1 ? kStepSimtStageCount : tc ? kPrefillTcStageCount : kPrefillSimtStageCount;
+  const char *const *list = kind == 2   ? kBackwardStages
+                            : kind == 1 ? kStepSimtStages
+                            : tc        ? kPrefillTcStages
+                                        : kPrefillSimtStages;
+  const int n = kind == 2   ? kBackwardStageCount
+                : kind == 1 ? kStepSimtStageCount
+                : tc        ? kPrefillTcStageCount
+                            : kPrefillSimtStageCount;
   for (int i = 0; names != nullptr && i < n && i < max_names; ++i) names[i] = list[i];
   return n;
 }
@@ -323,6 +329,75 @@ MAMBA2_API int mamba2_ssd_step(const mamba2_dims *dims, const mamba2_params *par
   a.ssm_state = ssm_state;
   a.stream = static_cast<cudaStream_t>(stream);
   return step_simt(a) == cudaSuccess ? MAMBA2_OK : MAMBA2_ERR_CUDA;
+}
+
+MAMBA2_API size_t mamba2_prefill_backward_workspace_size(const mamba2_dims *dims) {
+  Problem pr;
+  if (make_problem(dims, true, &pr) != MAMBA2_OK) return 0;
+  return backward_workspace(pr);
+}
+
+MAMBA2_API int mamba2_conv_ssd_prefill_backward(
+    const mamba2_dims *dims, const mamba2_params *params, const void *xBC,
+    int64_t xBC_row_stride, const void *z, int64_t z_row_stride, const void *dt_raw,
+    int64_t dt_row_stride, const void *conv_state_in, const float *ssm_state_in, const void *dy,
+    const float *d_ssm_state_out, void *d_xBC, void *d_z, void *d_dt_raw, float *d_conv_w,
+    float *d_conv_b, float *d_dt_bias, float *d_A, float *d_D, float *d_norm_w,
+    void *d_conv_state_in, float *d_ssm_state_in, void *workspace, size_t workspace_bytes,
+    void *stream) {
+  NvtxRange range("mamba2_conv_ssd_prefill_backward");
+  DisarmOnExit disarm;
+  Problem pr;
+  int st = make_problem(dims, true, &pr);
+  if (st != MAMBA2_OK) return st;
+  if (!params_ok(params)) return MAMBA2_ERR_INVALID_ARG;
+  if (d_conv_w == nullptr || d_conv_b == nullptr || d_dt_bias == nullptr || d_A == nullptr ||
+      d_D == nullptr || d_norm_w == nullptr)
+    return MAMBA2_ERR_INVALID_ARG;
+  const int64_t bl = pr.batch * pr.L;
+  if (bl > 0 && (xBC == nullptr || z == nullptr || dt_raw == nullptr || dy == nullptr ||
+                 d_xBC == nullptr || d_z == nullptr || d_dt_raw == nullptr))
+    return MAMBA2_ERR_INVALID_ARG;
+  const size_t esz = pr.io == MAMBA2_BF16 ? 2 : 4;
+  if (xBC_row_stride < pr.conv_dim || z_row_stride < pr.d_inner || dt_row_stride < pr.H)
+    return MAMBA2_ERR_INVALID_ARG;
+  const void *io_ptrs[] = {xBC, z, dt_raw, dy, d_xBC, d_z, d_dt_raw, conv_state_in,
+                           d_conv_state_in};  // element-aligned
+  const void *f32_ptrs[] = {ssm_state_in, d_ssm_state_out, d_ssm_state_in, d_conv_w,
+                            d_conv_b,     d_dt_bias,       d_A,            d_D, d_norm_w};
+  for (const void *q : io_ptrs)
+    if (!aligned(q, esz)) return MAMBA2_ERR_INVALID_ARG;
+  for (const void *q : f32_ptrs)
+    if (!aligned(q, 4)) return MAMBA2_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256)) return MAMBA2_ERR_WORKSPACE;
+  if (workspace_bytes < backward_workspace(pr)) return MAMBA2_ERR_WORKSPACE;
+  BackwardArgs a;
+  a.pr = pr;
+  a.prm = *params;
+  a.xBC = xBC;
+  a.ld_xbc = xBC_row_stride;
+  a.z = z;
+  a.ld_z = z_row_stride;
+  a.dt_raw = dt_raw;
+  a.ld_dt = dt_row_stride;
+  a.conv_state_in = conv_state_in;
+  a.ssm_state_in = ssm_state_in;
+  a.dy = dy;
+  a.d_ssm_state_out = d_ssm_state_out;
+  a.d_xBC = d_xBC;
+  a.d_z = d_z;
+  a.d_dt_raw = d_dt_raw;
+  a.d_conv_w = d_conv_w;
+  a.d_conv_b = d_conv_b;
+  a.d_dt_bias = d_dt_bias;
+  a.d_A = d_A;
+  a.d_D = d_D;
+  a.d_norm_w = d_norm_w;
+  a.d_conv_state_in = d_conv_state_in;
+  a.d_ssm_state_in = d_ssm_state_in;
+  a.ws = static_cast<char *>(workspace);
+  a.stream = static_cast<cudaStream_t>(stream);
+  return prefill_backward(a) == cudaSuccess ? MAMBA2_OK : MAMBA2_ERR_CUDA;
 }
 
 }  // extern "C"

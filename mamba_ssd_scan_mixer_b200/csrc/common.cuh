@@ -45,6 +45,28 @@ struct PrefillArgs {
   const int32_t *cu_seqlens = nullptr;
 };
 
+// One backward call of the prefill (device pointers checked by the C ABI).
+struct BackwardArgs {
+  Problem pr;
+  mamba2_params prm;
+  const void *xBC;
+  int64_t ld_xbc;
+  const void *z;
+  int64_t ld_z;
+  const void *dt_raw;
+  int64_t ld_dt;
+  const void *conv_state_in;      // or null (zero left context)
+  const float *ssm_state_in;      // or null (zero initial state)
+  const void *dy;                 // [b][L][d_inner]
+  const float *d_ssm_state_out;   // or null
+  void *d_xBC, *d_z, *d_dt_raw;   // [b][L][conv_dim], [b][L][d_inner], [b][L][H]
+  float *d_conv_w, *d_conv_b, *d_dt_bias, *d_A, *d_D, *d_norm_w;
+  void *d_conv_state_in;          // or null
+  float *d_ssm_state_in;          // or null
+  char *ws;
+  cudaStream_t stream;
+};
+
 struct StepArgs {
   Problem pr;
   mamba2_params prm;
@@ -128,6 +150,8 @@ extern const char *const kPrefillSimtStages[];
 extern const int kPrefillSimtStageCount;
 extern const char *const kStepSimtStages[];
 extern const int kStepSimtStageCount;
+extern const char *const kBackwardStages[];
+extern const int kBackwardStageCount;
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // MAMBA2_OK if `dims` describe a valid prefill problem, else the status the
@@ -138,6 +162,8 @@ int validate_prefill_dims(const mamba2_dims *dims);
 cudaError_t prefill_simt(const PrefillArgs &a);
 size_t prefill_simt_workspace(const Problem &pr);
 cudaError_t step_simt(const StepArgs &a);
+cudaError_t prefill_backward(const BackwardArgs &a);
+size_t backward_workspace(const Problem &pr);
 
 }  // namespace m2
 

@@ -224,3 +224,51 @@ def test_varlen_unsupported_configurations():
         d = _dims(batch=3, seqlen=1000, **bad)
         assert _call_varlen(d, ld_x=d.nheads * d.headdim + 2 * d.ngroups * d.dstate,
                             ld_z=d.nheads * d.headdim) == UNSUPPORTED, bad
+
+
+# ---- prefill backward: validated on the host before any CUDA call
+
+def _call_backward(d, **kw):
+    lib = m2.lib()
+    cd, di = d.nheads * d.headdim + 2 * d.ngroups * d.dstate, d.nheads * d.headdim
+    a = dict(params=_fake_params(), xBC=A0 + 0x10000, ld_x=cd, z=A0 + 0x20000, ld_z=di,
+             dt=A0 + 0x30000, ld_dt=d.nheads, cs=None, hs=None, dy=A0 + 0x40000, dhl=None,
+             dxbc=A0 + 0x50000, dz=A0 + 0x60000, ddt=A0 + 0x70000, dw=A0 + 0x80000,
+             db=A0 + 0x90000, ddtb=A0 + 0xa0000, dA=A0 + 0xb0000, dD=A0 + 0xc0000,
+             dnw=A0 + 0xd0000, dcs=None, dhs=None, ws=A0 + 0x100000,
+             ws_bytes=lib.mamba2_prefill_backward_workspace_size(ctypes.byref(d)) or 1)
+    a.update(kw)
+    p = a["params"]
+    return lib.mamba2_conv_ssd_prefill_backward(
+        ctypes.byref(d), ctypes.byref(p) if p is not None else None, a["xBC"], a["ld_x"], a["z"],
+        a["ld_z"], a["dt"], a["ld_dt"], a["cs"], a["hs"], a["dy"], a["dhl"], a["dxbc"], a["dz"],
+        a["ddt"], a["dw"], a["db"], a["ddtb"], a["dA"], a["dD"], a["dnw"], a["dcs"], a["dhs"],
+        a["ws"], a["ws_bytes"], None)
+
+
+def test_backward_workspace_size():
+    lib = m2.lib()
+    d = _dims(batch=1, seqlen=4096)
+    ws = lib.mamba2_prefill_backward_workspace_size(ctypes.byref(d))
+    states = 4096 * 80 * 64 * 64 * 4  # the state after every token
+    assert states < ws < 2 * states
+    assert lib.mamba2_prefill_backward_workspace_size(ctypes.byref(_dims(d_conv=2))) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(params=None), INVALID),
+    (dict(dy=None), INVALID),
+    (dict(dw=None), INVALID),
+    (dict(dxbc=A0 + 0x50001), INVALID),       # misaligned bf16 gradient
+    (dict(dhs=A0 + 0xe0002), INVALID),        # misaligned fp32 gradient
+    (dict(ld_x=8), INVALID),                  # row stride below conv_dim
+    (dict(ws=None), WORKSPACE),
+    (dict(ws_bytes=4096), WORKSPACE),
+])
+def test_backward_rejects_bad_arguments(kw, expect):
+    assert _call_backward(_dims(batch=2, seqlen=300), **kw) == expect
+
+
+def test_backward_unsupported_configurations():
+    for bad in (dict(d_conv=2), dict(dstate=256), dict(headdim=128)):
+        assert _call_backward(_dims(batch=2, seqlen=300, **bad)) == UNSUPPORTED, bad
