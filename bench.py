@@ -393,6 +393,82 @@ def measure_prefill(name, args, dev, stream, seed, world, peaks, peak_src, m2, W
 VARLEN_LENGTHS = (1, 3, 127, 129, 512, 700, 1024, 1600)
 
 
+def measure_backward(args, dev, stream, seed, world, peaks, peak_src, m2, W, lib, steps, warmup):
+    """Device-timed backward passes of the 2.7B prefill (mamba2_conv_ssd_prefill_backward:
+    forward recomputed, all gradients), carried states in and a final-state gradient,
+    steps timed one by one (each call writes and reads GBs: far beyond L2)."""
+    import torch
+    cfg = W.CONFIGS[PREFILL]
+    dims = m2.dims_from_config(cfg)
+    params = {k: v.to(dev) for k, v in W.make_params(cfg, seed).items()}
+    pp = m2.make_params(params["conv_w"], params["conv_b"], params["dt_bias"], params["A"],
+                        params["D"], params["norm_w"])
+    v = W.split_packed(cfg, W.make_prefill_inputs(cfg, seed)["zxbcdt"].to(dev))
+    st = W.make_states(cfg, seed)
+    cs, hs = st["conv_state"].to(dev), st["ssm_state"].to(dev)
+    g = torch.Generator(device=dev).manual_seed(2000 + seed)
+    dy = torch.randn(cfg.batch, cfg.seqlen, cfg.d_inner, generator=g, device=dev).to(
+        cfg.torch_dtype)
+    dhl = 0.1 * torch.randn(hs.shape, generator=g, device=dev)
+    ws = torch.empty(max(1, m2.mamba2_prefill_backward_workspace_size(dims)), dtype=torch.uint8,
+                     device=dev)
+    names_arr = (ctypes.c_char_p * 16)()
+    nst = lib.mamba2_stage_names(2, ctypes.byref(dims), names_arr, 16)
+    stage_names = [names_arr[i].decode() for i in range(nst)]
+    grads = None
+
+    def call(stage_events=None):
+        nonlocal grads
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        if stage_events is not None:
+            arr = (ctypes.c_void_p * len(stage_events))(*[e.cuda_event for e in stage_events])
+            lib.mamba2_record_stage_events(arr, len(stage_events))
+        grads = m2.prefill_backward(dims, pp, v["xBC"], v["z"], v["dt_raw"], dy, cs, hs, dhl,
+                                    ws, stream)
+        b.record(stream)
+        return a, b
+
+    stage_ms, n_stage = [0.0] * nst, 0
+    for i in range(max(3, warmup)):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+        for ev in evs:
+            ev.record(stream)
+        call(evs)
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            n_stage += 1
+            for j in range(nst):
+                stage_ms[j] += evs[j].elapsed_time(evs[j + 1])
+    evs = [call() for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev) / steps
+    T, e = cfg.batch * cfg.seqlen, 2
+    # compulsory bytes: the forward's inputs and dy read, the input gradients written
+    # (bf16); the states and their gradients (fp32 SSM, bf16 conv) read / written once
+    states = 4 * cfg.nheads * cfg.headdim * cfg.dstate + e * cfg.conv_dim * cfg.d_conv
+    io = cfg.conv_dim + cfg.d_inner + cfg.nheads
+    path_bytes = T * e * (io + cfg.d_inner + io) + cfg.batch * 3 * states
+    t_roof = path_bytes / (peaks["hbm_gbs"] * 1e9)
+    return {
+        "value": job_rate(T, steps, ms * steps, world), "unit": "tokens/s", "steps": steps,
+        "warmup": max(3, warmup), "ms_per_step": ms,
+        "config": {"workload": "zamba2_2p7b_prefill_backward", "batch": cfg.batch,
+                   "seqlen": cfg.seqlen, "nheads": cfg.nheads, "headdim": cfg.headdim,
+                   "dstate": cfg.dstate, "ngroups": cfg.ngroups, "io_dtype": cfg.io_dtype,
+                   "compute": "fp32 CUDA cores", "states_in": True,
+                   "workspace_bytes": ws.numel(),
+                   "l2": "each call writes and reads the per-token states (GBs)"},
+        "path_roofline": {"bytes": path_bytes, "roofline_ms": t_roof * 1e3,
+                          "achieved_gbs": path_bytes / (ms * 1e-3) / 1e9,
+                          "frac": t_roof * 1e3 / ms, "peak_source": peak_src},
+        "stages_ms_warmup_avg": {n: stage_ms[j] / max(1, n_stage)
+                                 for j, n in enumerate(stage_names)},
+        "gpu_launches": 9 * steps,
+    }
+
+
 def measure_varlen(args, dev, stream, seed, world, peaks, peak_src, m2, W, lib, steps, warmup):
     """Device-timed packed-sequence prefills (mamba2_conv_ssd_prefill_varlen), L2
     flushed (256 MB write) before every step, steps timed one by one."""
@@ -524,6 +600,10 @@ def run_ours(args, rank, world, local_rank):
                            steps=min(args.steps, 20), warmup=3)
         line["gpu_launches"] += o.pop("gpu_launches")
         other["zamba2_2p7b_varlen_prefill"] = o
+        o = measure_backward(args, dev, stream, seed, world, peaks, peak_src, m2, W, lib,
+                             steps=min(args.steps, 5), warmup=3)
+        line["gpu_launches"] += o.pop("gpu_launches")
+        other["zamba2_2p7b_prefill_backward"] = o
         line["workloads"] = other
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, seconds=10.0)

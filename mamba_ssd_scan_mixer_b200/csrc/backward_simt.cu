@@ -20,7 +20,7 @@
 //   bwd_conv        through the SiLU and the conv: dxBC, dconv_state, dw, db;
 //   col_sum         sums of the per-token terms over the tokens.
 // Everything is fp32 on CUDA cores.  The scan kernels give each warp of a
-// head's block rows p = warp, warp + 8, ... of the state and each lane the
+// head's block rows p = warp, warp + 16, ... of the state and each lane the
 // columns n = lane, lane + 32, ...: sums over n are warp shuffles, and the
 // sums over p that span warps are written per warp and added afterwards, so
 // no kernel synchronises a block inside its token loop.
@@ -31,8 +31,8 @@
 namespace m2 {
 namespace {
 
-constexpr int kScanWarps = 8;  // warps of a head's block in the scan kernels
-constexpr int kMaxRowsPerWarp = 8;   // P <= 64
+constexpr int kScanWarps = 16;  // warps of a head's block in the scan kernels
+constexpr int kMaxRowsPerWarp = 4;   // P <= 64
 constexpr int kMaxColsPerLane = 4;   // N <= 128
 
 __device__ __forceinline__ float sigmoid_f(float s) { return 1.0f / (1.0f + expf(-s)); }
@@ -78,8 +78,9 @@ __global__ void bwd_prologue_kernel(Problem pr, mamba2_params prm, const T *xBC,
 // The recurrence forward, one block of kScanWarps warps per (head, row); the
 // state after every token into hs [b][H][L][P][N]; ypre [b][L][d_inner].
 __global__ void __launch_bounds__(32 * kScanWarps)
-    bwd_scan_fwd_kernel(Problem pr, mamba2_params prm, const float *u, const float *dtv,
-                        const float *h0, float *hs, float *ypre) {
+    bwd_scan_fwd_kernel(Problem pr, mamba2_params prm, const float *__restrict__ u,
+                        const float *__restrict__ dtv, const float *__restrict__ h0,
+                        float *__restrict__ hs, float *__restrict__ ypre) {
   const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bi = blockIdx.y;
   const int P = pr.P, N = pr.N, g = h / pr.heads_per_group();
@@ -95,6 +96,7 @@ __global__ void __launch_bounds__(32 * kScanWarps)
       st[r][j] = (r < rows && j < cols && n < N && h0 != nullptr)
                      ? h0[(head * P + p) * N + n] : 0.0f;
     }
+#pragma unroll 2
   for (int64_t t = 0; t < pr.L; ++t) {
     const float *ut = u + (bi * pr.L + t) * pr.conv_dim;
     const float dt = dtv[(bi * pr.L + t) * pr.H + h], a = expf(dt * A);
@@ -175,9 +177,12 @@ __global__ void bwd_norm_kernel(Problem pr, mamba2_params prm, const float *ypre
 // pdt [b][H][warp][L] the warps' partial ddt; dA, dD by atomics; dh0 the
 // gradient of the initial state.
 __global__ void __launch_bounds__(32 * kScanWarps)
-    bwd_scan_rev_kernel(Problem pr, mamba2_params prm, const float *u, const float *dtv,
-                        const float *h0, const float *hs, const float *dypre, const float *dhL,
-                        float *du, float *pbc, float *pdt, float *dA, float *dD, float *dh0) {
+    bwd_scan_rev_kernel(Problem pr, mamba2_params prm, const float *__restrict__ u,
+                        const float *__restrict__ dtv, const float *__restrict__ h0,
+                        const float *__restrict__ hs, const float *__restrict__ dypre,
+                        const float *__restrict__ dhL, float *__restrict__ du,
+                        float *__restrict__ pbc, float *__restrict__ pdt, float *dA, float *dD,
+                        float *__restrict__ dh0) {
   const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bi = blockIdx.y;
   const int P = pr.P, N = pr.N, g = h / pr.heads_per_group();
@@ -194,6 +199,7 @@ __global__ void __launch_bounds__(32 * kScanWarps)
                      ? dhL[(head * P + p) * N + n] : 0.0f;
     }
   float dA_acc = 0.0f, dD_acc = 0.0f;
+#pragma unroll 2
   for (int64_t t = pr.L - 1; t >= 0; --t) {
     const float *ut = u + (bi * pr.L + t) * pr.conv_dim;
     const float dt = dtv[(bi * pr.L + t) * pr.H + h], a = expf(dt * A);
