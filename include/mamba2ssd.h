@@ -297,9 +297,10 @@ MAMBA2_API size_t mamba2_prefill_backward_workspace_size(const mamba2_dims *dims
  *  d_ssm_state_in  [b, nheads, headdim, dstate] fp32 or NULL.
  *  workspace  >= mamba2_prefill_backward_workspace_size(dims) bytes, 256-byte
  *          aligned.  stream: cudaStream_t as void*.
- * Runs in fp32 on the CUDA cores for every supported shape.  The sums over
- * tokens of the parameter gradients use atomic additions, so they may differ
- * in the last bits between runs; the other gradients are deterministic.
+ * Runs in fp32 on the CUDA cores for every supported shape.  The parameter
+ * gradients (sums over tokens) and the per-token sums over a head's state
+ * rows behind d_xBC's B and C channels and d_dt_raw use atomic additions, so
+ * those may differ in the last bits between runs.
  * Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG (null or misaligned pointer, bad
  * stride), MAMBA2_ERR_UNSUPPORTED, MAMBA2_ERR_WORKSPACE or MAMBA2_ERR_CUDA. */
 MAMBA2_API int mamba2_conv_ssd_prefill_backward(

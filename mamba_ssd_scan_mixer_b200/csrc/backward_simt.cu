@@ -14,8 +14,8 @@
 //   bwd_scan_fwd    h_t of every token kept in the workspace, and ypre;
 //   bwd_norm        dypre, dz, and the per-token terms of dnorm_w;
 //   bwd_scan_rev    reverse over tokens with dh in registers: dx, and per-warp
-//                   partial sums of dB, dC and ddt, dA, dD, dh_0;
-//   bwd_reduce_bc   dB, dC over the heads of a group and the warps of a head; ddt;
+//                   shares of dB, dC and ddt, dA, dD, dh_0;
+//   bwd_reduce_bc   dB, dC over the heads of a group and their warps; ddt;
 //   bwd_dt          ddt_raw and the per-token terms of ddt_bias;
 //   bwd_conv        through the SiLU and the conv: dxBC, dconv_state, dw, db;
 //   col_sum         sums of the per-token terms over the tokens.
@@ -23,17 +23,17 @@
 // head's block rows p = warp, warp + 16, ... of the state and each lane the
 // columns n = lane, lane + 32, ...: sums over n are warp shuffles, and the
 // sums over p that span warps are written per warp and added afterwards, so
-// no kernel synchronises a block inside its token loop.
+// no kernel synchronises a block inside its token loop (a block barrier per
+// token cost more than the separate sum).
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 
 namespace m2 {
 namespace {
 
-constexpr int kScanWarps = 16;  // warps of a head's block in the scan kernels
-constexpr int kMaxRowsPerWarp = 4;   // P <= 64
-constexpr int kMaxColsPerLane = 4;   // N <= 128
+constexpr int kScanWarps = 16;  // warps of a head's block in the scan kernels (P >= 16)
 
 __device__ __forceinline__ float sigmoid_f(float s) { return 1.0f / (1.0f + expf(-s)); }
 // d silu(s) / ds = sigmoid(s) (1 + s (1 - sigmoid(s)))
@@ -75,8 +75,41 @@ __global__ void bwd_prologue_kernel(Problem pr, mamba2_params prm, const T *xBC,
   }
 }
 
-// The recurrence forward, one block of kScanWarps warps per (head, row); the
-// state after every token into hs [b][H][L][P][N]; ypre [b][L][d_inner].
+// The per-token inputs of one head that a warp of the scan kernels reads: dt,
+// the lane's B and C columns, and x (and, backwards, dypre) of the warp's rows.
+template <int ROWS, int COLS>
+struct ScanTok {
+  float dt, bv[COLS], cv[COLS], x[ROWS], dy[ROWS];
+};
+template <int ROWS, int COLS>
+__device__ __forceinline__ void scan_load_tok(const Problem &pr, const float *__restrict__ u,
+                                              const float *__restrict__ dtv,
+                                              const float *__restrict__ dypre, int64_t bi,
+                                              int h, int g, int warp, int lane, int64_t t,
+                                              ScanTok<ROWS, COLS> &k) {
+  const int N = pr.N;
+  const float *ut = u + (bi * pr.L + t) * pr.conv_dim;
+  k.dt = dtv[(bi * pr.L + t) * pr.H + h];
+#pragma unroll
+  for (int j = 0; j < COLS; ++j) {
+    const int n = lane + 32 * j;
+    k.bv[j] = n < N ? ut[pr.d_inner + (int64_t)g * N + n] : 0.0f;
+    k.cv[j] = n < N ? ut[pr.d_inner + (int64_t)(pr.G + g) * N + n] : 0.0f;
+  }
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r) {
+    const int p = warp + kScanWarps * r;
+    k.x[r] = ut[(int64_t)h * pr.P + p];
+    k.dy[r] = dypre != nullptr ? dypre[(bi * pr.L + t) * pr.d_inner + (int64_t)h * pr.P + p]
+                               : 0.0f;
+  }
+}
+
+// The recurrence forward, one block of kScanWarps warps per (head, row), ROWS =
+// P / kScanWarps rows per warp, COLS = ceil(N / 32) columns per lane; the next
+// token's inputs are loaded while this one is computed.  The state after every
+// token into hs [b][H][L][P][N]; ypre [b][L][d_inner].
+template <int ROWS, int COLS>
 __global__ void __launch_bounds__(32 * kScanWarps)
     bwd_scan_fwd_kernel(Problem pr, mamba2_params prm, const float *__restrict__ u,
                         const float *__restrict__ dtv, const float *__restrict__ h0,
@@ -84,49 +117,38 @@ __global__ void __launch_bounds__(32 * kScanWarps)
   const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bi = blockIdx.y;
   const int P = pr.P, N = pr.N, g = h / pr.heads_per_group();
-  const int rows = P / kScanWarps, cols = (N + 31) / 32;
   const float A = prm.A[h], D = prm.D[h];
-  float st[kMaxRowsPerWarp][kMaxColsPerLane];
+  float st[ROWS][COLS];
   const int64_t head = bi * pr.H + h;
 #pragma unroll
-  for (int r = 0; r < kMaxRowsPerWarp; ++r)
+  for (int r = 0; r < ROWS; ++r)
 #pragma unroll
-    for (int j = 0; j < kMaxColsPerLane; ++j) {
+    for (int j = 0; j < COLS; ++j) {
       const int p = warp + kScanWarps * r, n = lane + 32 * j;
-      st[r][j] = (r < rows && j < cols && n < N && h0 != nullptr)
-                     ? h0[(head * P + p) * N + n] : 0.0f;
+      st[r][j] = (n < N && h0 != nullptr) ? h0[(head * P + p) * N + n] : 0.0f;
     }
-#pragma unroll 2
+  ScanTok<ROWS, COLS> cur, nxt;
+  if (pr.L > 0) scan_load_tok(pr, u, dtv, nullptr, bi, h, g, warp, lane, 0, cur);
   for (int64_t t = 0; t < pr.L; ++t) {
-    const float *ut = u + (bi * pr.L + t) * pr.conv_dim;
-    const float dt = dtv[(bi * pr.L + t) * pr.H + h], a = expf(dt * A);
-    float bv[kMaxColsPerLane], cv[kMaxColsPerLane];
-#pragma unroll
-    for (int j = 0; j < kMaxColsPerLane; ++j) {
-      const int n = lane + 32 * j;
-      const bool on = j < cols && n < N;
-      bv[j] = on ? ut[pr.d_inner + (int64_t)g * N + n] : 0.0f;
-      cv[j] = on ? ut[pr.d_inner + (int64_t)(pr.G + g) * N + n] : 0.0f;
-    }
+    if (t + 1 < pr.L) scan_load_tok(pr, u, dtv, nullptr, bi, h, g, warp, lane, t + 1, nxt);
+    const float a = expf(cur.dt * A);
     float *hst = hs + (head * pr.L + t) * (int64_t)(P * N);
 #pragma unroll
-    for (int r = 0; r < kMaxRowsPerWarp; ++r) {
-      if (r >= rows) break;
+    for (int r = 0; r < ROWS; ++r) {
       const int p = warp + kScanWarps * r;
-      const float x = ut[(int64_t)h * P + p], xdt = x * dt;
+      const float xdt = cur.x[r] * cur.dt;
       float acc = 0.0f;
 #pragma unroll
-      for (int j = 0; j < kMaxColsPerLane; ++j) {
+      for (int j = 0; j < COLS; ++j) {
         const int n = lane + 32 * j;
-        if (j < cols && n < N) {
-          st[r][j] = fmaf(a, st[r][j], xdt * bv[j]);
-          hst[p * N + n] = st[r][j];
-          acc = fmaf(st[r][j], cv[j], acc);
-        }
+        st[r][j] = fmaf(a, st[r][j], xdt * cur.bv[j]);
+        if (n < N) hst[p * N + n] = st[r][j];
+        acc = fmaf(st[r][j], cur.cv[j], acc);
       }
       acc = warp_sum(acc);
-      if (lane == 0) ypre[(bi * pr.L + t) * pr.d_inner + (int64_t)h * P + p] = acc + D * x;
+      if (lane == 0) ypre[(bi * pr.L + t) * pr.d_inner + (int64_t)h * P + p] = acc + D * cur.x[r];
     }
+    cur = nxt;
   }
 }
 
@@ -172,10 +194,14 @@ __global__ void bwd_norm_kernel(Problem pr, mamba2_params prm, const float *ypre
   }
 }
 
-// The recurrence backward, reverse over tokens, one block per (head, row).
-// du gets dx (x channels); pbc [b][H][warp][L][2][N] the warps' partial dB, dC;
-// pdt [b][H][warp][L] the warps' partial ddt; dA, dD by atomics; dh0 the
-// gradient of the initial state.
+// The recurrence backward, reverse over tokens, one block per (head, row),
+// with the warp layout of the forward kernel; the inputs and the stored states
+// of the next token (t - 1) are loaded while token t is computed.
+// du gets dx (x channels); each warp's shares of dB (times dt), dC and ddt of
+// every token go to pbc [b][L][2][H][warp][N] and pdt [b][L][H][warp] (token
+// major, so that the sums over a group's heads and warps read one contiguous
+// span per token); dA, dD by atomics; dh0 the gradient of the initial state.
+template <int ROWS, int COLS>
 __global__ void __launch_bounds__(32 * kScanWarps)
     bwd_scan_rev_kernel(Problem pr, mamba2_params prm, const float *__restrict__ u,
                         const float *__restrict__ dtv, const float *__restrict__ h0,
@@ -186,55 +212,61 @@ __global__ void __launch_bounds__(32 * kScanWarps)
   const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bi = blockIdx.y;
   const int P = pr.P, N = pr.N, g = h / pr.heads_per_group();
-  const int rows = P / kScanWarps, cols = (N + 31) / 32;
   const float A = prm.A[h], D = prm.D[h];
   const int64_t head = bi * pr.H + h;
-  float dh[kMaxRowsPerWarp][kMaxColsPerLane];
+  const int64_t PN = (int64_t)P * N;
+  // the state before token t (h_{t-1}): from hs, or the initial state (zero without one)
+  auto load_prev = [&](int64_t t, float (&hp)[ROWS][COLS]) {
+    const float *src = t > 0 ? hs + (head * pr.L + t - 1) * PN
+                             : (h0 != nullptr ? h0 + head * PN : nullptr);
 #pragma unroll
-  for (int r = 0; r < kMaxRowsPerWarp; ++r)
+    for (int r = 0; r < ROWS; ++r)
 #pragma unroll
-    for (int j = 0; j < kMaxColsPerLane; ++j) {
+      for (int j = 0; j < COLS; ++j) {
+        const int p = warp + kScanWarps * r, n = lane + 32 * j;
+        hp[r][j] = (src != nullptr && n < N) ? src[p * N + n] : 0.0f;
+      }
+  };
+  float dh[ROWS][COLS], hcur[ROWS][COLS], hprv[ROWS][COLS], hnx[ROWS][COLS];
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+    for (int j = 0; j < COLS; ++j) {
       const int p = warp + kScanWarps * r, n = lane + 32 * j;
-      dh[r][j] = (r < rows && j < cols && n < N && dhL != nullptr)
-                     ? dhL[(head * P + p) * N + n] : 0.0f;
+      dh[r][j] = (dhL != nullptr && n < N) ? dhL[(head * P + p) * N + n] : 0.0f;
     }
   float dA_acc = 0.0f, dD_acc = 0.0f;
-#pragma unroll 2
+  ScanTok<ROWS, COLS> cur, nxt;
+  if (pr.L > 0) {
+    scan_load_tok(pr, u, dtv, dypre, bi, h, g, warp, lane, pr.L - 1, cur);
+    load_prev(pr.L, hcur);      // h_{L-1}
+    load_prev(pr.L - 1, hprv);  // h_{L-2}
+  }
   for (int64_t t = pr.L - 1; t >= 0; --t) {
-    const float *ut = u + (bi * pr.L + t) * pr.conv_dim;
-    const float dt = dtv[(bi * pr.L + t) * pr.H + h], a = expf(dt * A);
-    float bv[kMaxColsPerLane], cv[kMaxColsPerLane], dbp[kMaxColsPerLane], dcp[kMaxColsPerLane];
+    if (t > 0) {  // token t - 1: its inputs and the state before it
+      scan_load_tok(pr, u, dtv, dypre, bi, h, g, warp, lane, t - 1, nxt);
+      load_prev(t - 1, hnx);
+    }
+    const float dt = cur.dt, a = expf(dt * A);
+    float dbp[COLS], dcp[COLS];
 #pragma unroll
-    for (int j = 0; j < kMaxColsPerLane; ++j) {
-      const int n = lane + 32 * j;
-      const bool on = j < cols && n < N;
-      bv[j] = on ? ut[pr.d_inner + (int64_t)g * N + n] : 0.0f;
-      cv[j] = on ? ut[pr.d_inner + (int64_t)(pr.G + g) * N + n] : 0.0f;
+    for (int j = 0; j < COLS; ++j) {
       dbp[j] = 0.0f;
       dcp[j] = 0.0f;
     }
-    const float *hst = hs + (head * pr.L + t) * (int64_t)(P * N);
-    const float *hpr = t > 0 ? hst - (int64_t)P * N : (h0 != nullptr ? h0 + head * P * N : nullptr);
     float ddt_dir = 0.0f, da = 0.0f;  // sum dh x B, sum dh h_{t-1}
 #pragma unroll
-    for (int r = 0; r < kMaxRowsPerWarp; ++r) {
-      if (r >= rows) break;
+    for (int r = 0; r < ROWS; ++r) {
       const int p = warp + kScanWarps * r;
-      const float x = ut[(int64_t)h * P + p];
-      const float dyp = dypre[(bi * pr.L + t) * pr.d_inner + (int64_t)h * P + p];
+      const float x = cur.x[r], dyp = cur.dy[r];
       float sb = 0.0f;
 #pragma unroll
-      for (int j = 0; j < kMaxColsPerLane; ++j) {
-        const int n = lane + 32 * j;
-        if (j < cols && n < N) {
-          const float ht = hst[p * N + n];
-          const float hp = hpr != nullptr ? hpr[p * N + n] : 0.0f;
-          dh[r][j] = fmaf(dyp, cv[j], dh[r][j]);   // y_t = h_t C_t + D x_t
-          dcp[j] = fmaf(dyp, ht, dcp[j]);
-          sb = fmaf(dh[r][j], bv[j], sb);
-          dbp[j] = fmaf(dh[r][j], x, dbp[j]);
-          da = fmaf(dh[r][j], hp, da);
-        }
+      for (int j = 0; j < COLS; ++j) {
+        dh[r][j] = fmaf(dyp, cur.cv[j], dh[r][j]);  // y_t = h_t C_t + D x_t
+        dcp[j] = fmaf(dyp, hcur[r][j], dcp[j]);
+        sb = fmaf(dh[r][j], cur.bv[j], sb);
+        dbp[j] = fmaf(dh[r][j], x, dbp[j]);
+        da = fmaf(dh[r][j], hprv[r][j], da);
       }
       sb = warp_sum(sb);
       ddt_dir = fmaf(x, sb, ddt_dir);
@@ -243,23 +275,33 @@ __global__ void __launch_bounds__(32 * kScanWarps)
         dD_acc = fmaf(dyp, x, dD_acc);
       }
 #pragma unroll
-      for (int j = 0; j < kMaxColsPerLane; ++j) dh[r][j] *= a;  // -> dL/dh_{t-1}
+      for (int j = 0; j < COLS; ++j) dh[r][j] *= a;  // -> dL/dh_{t-1}
     }
     da = warp_sum(da);
-    // partial dB (times dt) and dC of this warp's rows
-    float *pb = pbc + ((((head * kScanWarps + warp) * pr.L + t) * 2) * N);
+    // this warp's shares of dB (times dt) and dC, and of ddt
+    const int64_t bt = bi * pr.L + t;
+    float *pb = pbc + ((bt * 2 * pr.H + h) * kScanWarps + warp) * N;
+    const int64_t cstride = (int64_t)pr.H * kScanWarps * N;  // B -> C
 #pragma unroll
-    for (int j = 0; j < kMaxColsPerLane; ++j) {
+    for (int j = 0; j < COLS; ++j) {
       const int n = lane + 32 * j;
-      if (j < cols && n < N) {
+      if (n < N) {
         pb[n] = dt * dbp[j];
-        pb[N + n] = dcp[j];
+        pb[cstride + n] = dcp[j];
       }
     }
     if (lane == 0) {
-      pdt[(head * kScanWarps + warp) * pr.L + t] = ddt_dir + da * a * A;
+      pdt[(bt * pr.H + h) * kScanWarps + warp] = ddt_dir + da * a * A;
       dA_acc = fmaf(da * a, dt, dA_acc);
     }
+    cur = nxt;
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r)
+#pragma unroll
+      for (int j = 0; j < COLS; ++j) {
+        hcur[r][j] = hprv[r][j];
+        hprv[r][j] = hnx[r][j];
+      }
   }
   if (lane == 0) {
     atomicAdd(dA + h, dA_acc);
@@ -267,11 +309,11 @@ __global__ void __launch_bounds__(32 * kScanWarps)
   }
   if (dh0 != nullptr) {
 #pragma unroll
-    for (int r = 0; r < kMaxRowsPerWarp; ++r)
+    for (int r = 0; r < ROWS; ++r)
 #pragma unroll
-      for (int j = 0; j < kMaxColsPerLane; ++j) {
+      for (int j = 0; j < COLS; ++j) {
         const int p = warp + kScanWarps * r, n = lane + 32 * j;
-        if (r < rows && j < cols && n < N) dh0[(head * P + p) * N + n] = dh[r][j];
+        if (n < N) dh0[(head * P + p) * N + n] = dh[r][j];
       }
   }
 }
@@ -289,22 +331,19 @@ __global__ void bwd_reduce_bc_kernel(Problem pr, const float *pbc, const float *
     const int which = (int)(r % 2);  // 0: B, 1: C
     r /= 2;
     const int g = (int)(r % pr.G);
-    const int64_t bt = r / pr.G, t = bt % pr.L, bi = bt / pr.L;
+    const int64_t bt = r / pr.G;
+    // the group's heads and their warps: hpg * kScanWarps rows of N, contiguous
+    const float *src = pbc + ((bt * 2 + which) * pr.H + (int64_t)g * hpg) * kScanWarps * N + n;
     float s = 0.0f;
-    for (int hh = 0; hh < hpg; ++hh) {
-      const int64_t head = bi * pr.H + g * hpg + hh;
-      for (int w = 0; w < kScanWarps; ++w)
-        s += pbc[(((head * kScanWarps + w) * pr.L + t) * 2 + which) * N + n];
-    }
+    for (int k = 0; k < hpg * kScanWarps; ++k) s += src[(int64_t)k * N];
     du[bt * pr.conv_dim + pr.d_inner + (int64_t)(which * pr.G + g) * N + n] = s;
   }
   const int64_t nd = pr.batch * pr.L * pr.H;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nd;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t h = i % pr.H, bt = i / pr.H, t = bt % pr.L, bi = bt / pr.L;
-    const int64_t head = bi * pr.H + h;
     float s = 0.0f;
-    for (int w = 0; w < kScanWarps; ++w) s += pdt[(head * kScanWarps + w) * pr.L + t];
+#pragma unroll
+    for (int w = 0; w < kScanWarps; ++w) s += pdt[i * kScanWarps + w];
     ddt[i] = s;
   }
 }
@@ -391,6 +430,24 @@ __global__ void col_sum_kernel(const float *m, int64_t rows, int64_t cols, float
   if (r1 > r0) atomicAdd(out + c, s);
 }
 
+// Calls f(rows, cols) with the compile-time warp layout of the scan kernels for
+// P (16, 32, 64: rows P / 16 per warp) and N (16 .. 128: ceil(N / 32) per lane).
+template <typename F>
+void launch_scan(const Problem &pr, F f) {
+  auto with_rows = [&](auto cols) {
+    switch (pr.P / kScanWarps) {
+      case 1: f(std::integral_constant<int, 1>(), cols); break;
+      case 2: f(std::integral_constant<int, 2>(), cols); break;
+      default: f(std::integral_constant<int, 4>(), cols); break;
+    }
+  };
+  switch ((pr.N + 31) / 32) {
+    case 1: with_rows(std::integral_constant<int, 1>()); break;
+    case 2: with_rows(std::integral_constant<int, 2>()); break;
+    default: with_rows(std::integral_constant<int, 4>()); break;
+  }
+}
+
 struct BwdWorkspace {
   float *u, *dtv, *hs, *ypre, *dypre, *du, *pbc, *pdt, *ddt, *tok;
 };
@@ -410,7 +467,7 @@ size_t bwd_carve(const Problem &pr, char *base, BwdWorkspace *w) {
   t.ypre = take(bl * pr.d_inner);
   t.dypre = take(bl * pr.d_inner);
   t.du = take(bl * pr.conv_dim);
-  t.pbc = take(bl * pr.H * kScanWarps * 2 * pr.N);
+  t.pbc = take(bl * 2 * pr.H * kScanWarps * pr.N);
   t.pdt = take(bl * pr.H * kScanWarps);
   t.ddt = take(bl * pr.H);
   t.tok = take(bl * std::max<int64_t>(pr.d_inner, pr.H));  // per-token terms of a sum
@@ -460,8 +517,10 @@ cudaError_t run_backward(const BackwardArgs &a) {
                                                                       w.dtv);
   stage_mark(st, 1);
   const dim3 gh((unsigned)pr.H, (unsigned)pr.batch);
-  bwd_scan_fwd_kernel<<<gh, 32 * kScanWarps, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in,
-                                                      w.hs, w.ypre);
+  launch_scan(pr, [&](auto rows, auto cols) {
+    bwd_scan_fwd_kernel<decltype(rows)::value, decltype(cols)::value>
+        <<<gh, 32 * kScanWarps, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in, w.hs, w.ypre);
+  });
   stage_mark(st, 2);
   bwd_norm_kernel<T><<<(unsigned)bl, 256, 0, st>>>(pr, a.prm, w.ypre, z, a.ld_z, dy, w.dypre,
                                                    static_cast<T *>(a.d_z), w.tok);
@@ -469,10 +528,12 @@ cudaError_t run_backward(const BackwardArgs &a) {
   col_sum_kernel<<<dim3((unsigned)ceil_div(pr.d_inner, 256), 64), 256, 0, st>>>(
       w.tok, bl, pr.d_inner, a.d_norm_w);
   stage_mark(st, 4);
-  bwd_scan_rev_kernel<<<gh, 32 * kScanWarps, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in,
-                                                      w.hs, w.dypre, a.d_ssm_state_out, w.du,
-                                                      w.pbc, w.pdt, a.d_A, a.d_D,
-                                                      a.d_ssm_state_in);
+  launch_scan(pr, [&](auto rows, auto cols) {
+    bwd_scan_rev_kernel<decltype(rows)::value, decltype(cols)::value>
+        <<<gh, 32 * kScanWarps, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in, w.hs, w.dypre,
+                                         a.d_ssm_state_out, w.du, w.pbc, w.pdt, a.d_A, a.d_D,
+                                         a.d_ssm_state_in);
+  });
   stage_mark(st, 5);
   bwd_reduce_bc_kernel<<<grid_for(bl * pr.G * 2 * pr.N), 256, 0, st>>>(pr, w.pbc, w.pdt, w.du,
                                                                        w.ddt);
