@@ -85,8 +85,8 @@ template <int ROWS, int COLS>
 __device__ __forceinline__ void scan_load_tok(const Problem &pr, const float *__restrict__ u,
                                               const float *__restrict__ dtv,
                                               const float *__restrict__ dypre, int64_t bi,
-                                              int h, int g, int warp, int lane, int64_t t,
-                                              ScanTok<ROWS, COLS> &k) {
+                                              int h, int g, int gw, int nwh, int lane,
+                                              int64_t t, ScanTok<ROWS, COLS> &k) {
   const int N = pr.N;
   const float *ut = u + (bi * pr.L + t) * pr.conv_dim;
   k.dt = dtv[(bi * pr.L + t) * pr.H + h];
@@ -98,23 +98,30 @@ __device__ __forceinline__ void scan_load_tok(const Problem &pr, const float *__
   }
 #pragma unroll
   for (int r = 0; r < ROWS; ++r) {
-    const int p = warp + kScanWarps * r;
+    const int p = gw + nwh * r;
     k.x[r] = ut[(int64_t)h * pr.P + p];
     k.dy[r] = dypre != nullptr ? dypre[(bi * pr.L + t) * pr.d_inner + (int64_t)h * pr.P + p]
                                : 0.0f;
   }
 }
 
-// The recurrence forward, one block of kScanWarps warps per (head, row), ROWS =
-// P / kScanWarps rows per warp, COLS = ceil(N / 32) columns per lane; the next
-// token's inputs are loaded while this one is computed.  The state after every
-// token into hs [b][H][L][P][N]; ypre [b][L][d_inner].
-template <int ROWS, int COLS>
-__global__ void __launch_bounds__(32 * kScanWarps)
+// The warp layout of the scan kernels: a head's P / ROWS warps take rows p = gw,
+// gw + P / ROWS, ... (gw the warp's index in the head), split over blocks of
+// WARPS warps (grid.x = heads x blocks per head); each lane takes columns
+// n = lane, lane + 32, ... (COLS = ceil(N / 32)).
+//
+// The recurrence forward: every row is independent, so one row per warp and
+// several blocks per head keep all SMs busy; the next token's inputs are loaded
+// while this one is computed.  The state after every token into hs
+// [b][H][L][P][N]; ypre [b][L][d_inner].
+template <int ROWS, int COLS, int WARPS>
+__global__ void __launch_bounds__(32 * WARPS)
     bwd_scan_fwd_kernel(Problem pr, mamba2_params prm, const float *__restrict__ u,
                         const float *__restrict__ dtv, const float *__restrict__ h0,
                         float *__restrict__ hs, float *__restrict__ ypre) {
-  const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwh = pr.P / ROWS, bph = nwh / WARPS;
+  const int h = blockIdx.x / bph, gw = (blockIdx.x % bph) * WARPS + warp;
   const int64_t bi = blockIdx.y;
   const int P = pr.P, N = pr.N, g = h / pr.heads_per_group();
   const float A = prm.A[h], D = prm.D[h];
@@ -124,18 +131,18 @@ __global__ void __launch_bounds__(32 * kScanWarps)
   for (int r = 0; r < ROWS; ++r)
 #pragma unroll
     for (int j = 0; j < COLS; ++j) {
-      const int p = warp + kScanWarps * r, n = lane + 32 * j;
+      const int p = gw + nwh * r, n = lane + 32 * j;
       st[r][j] = (n < N && h0 != nullptr) ? h0[(head * P + p) * N + n] : 0.0f;
     }
   ScanTok<ROWS, COLS> cur, nxt;
-  if (pr.L > 0) scan_load_tok(pr, u, dtv, nullptr, bi, h, g, warp, lane, 0, cur);
+  if (pr.L > 0) scan_load_tok(pr, u, dtv, nullptr, bi, h, g, gw, nwh, lane, 0, cur);
   for (int64_t t = 0; t < pr.L; ++t) {
-    if (t + 1 < pr.L) scan_load_tok(pr, u, dtv, nullptr, bi, h, g, warp, lane, t + 1, nxt);
+    if (t + 1 < pr.L) scan_load_tok(pr, u, dtv, nullptr, bi, h, g, gw, nwh, lane, t + 1, nxt);
     const float a = expf(cur.dt * A);
     float *hst = hs + (head * pr.L + t) * (int64_t)(P * N);
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
-      const int p = warp + kScanWarps * r;
+      const int p = gw + nwh * r;
       const float xdt = cur.x[r] * cur.dt;
       float acc = 0.0f;
 #pragma unroll
@@ -194,22 +201,24 @@ __global__ void bwd_norm_kernel(Problem pr, mamba2_params prm, const float *ypre
   }
 }
 
-// The recurrence backward, reverse over tokens, one block per (head, row),
-// with the warp layout of the forward kernel; the inputs and the stored states
-// of the next token (t - 1) are loaded while token t is computed.
+// The recurrence backward, reverse over tokens, in the warp layout above with
+// kScanWarps warps per head (ROWS = P / kScanWarps); the inputs and the stored
+// states of the next token (t - 1) are loaded while token t is computed.
 // du gets dx (x channels); each warp's shares of dB (times dt), dC and ddt of
 // every token go to pbc [b][L][2][H][warp][N] and pdt [b][L][H][warp] (token
 // major, so that the sums over a group's heads and warps read one contiguous
 // span per token); dA, dD by atomics; dh0 the gradient of the initial state.
-template <int ROWS, int COLS>
-__global__ void __launch_bounds__(32 * kScanWarps)
+template <int ROWS, int COLS, int WARPS>
+__global__ void __launch_bounds__(32 * WARPS)
     bwd_scan_rev_kernel(Problem pr, mamba2_params prm, const float *__restrict__ u,
                         const float *__restrict__ dtv, const float *__restrict__ h0,
                         const float *__restrict__ hs, const float *__restrict__ dypre,
                         const float *__restrict__ dhL, float *__restrict__ du,
                         float *__restrict__ pbc, float *__restrict__ pdt, float *dA, float *dD,
                         float *__restrict__ dh0) {
-  const int h = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwh = pr.P / ROWS, bph = nwh / WARPS;  // nwh = kScanWarps
+  const int h = blockIdx.x / bph, gw = (blockIdx.x % bph) * WARPS + warp;
   const int64_t bi = blockIdx.y;
   const int P = pr.P, N = pr.N, g = h / pr.heads_per_group();
   const float A = prm.A[h], D = prm.D[h];
@@ -223,7 +232,7 @@ __global__ void __launch_bounds__(32 * kScanWarps)
     for (int r = 0; r < ROWS; ++r)
 #pragma unroll
       for (int j = 0; j < COLS; ++j) {
-        const int p = warp + kScanWarps * r, n = lane + 32 * j;
+        const int p = gw + nwh * r, n = lane + 32 * j;
         hp[r][j] = (src != nullptr && n < N) ? src[p * N + n] : 0.0f;
       }
   };
@@ -232,19 +241,19 @@ __global__ void __launch_bounds__(32 * kScanWarps)
   for (int r = 0; r < ROWS; ++r)
 #pragma unroll
     for (int j = 0; j < COLS; ++j) {
-      const int p = warp + kScanWarps * r, n = lane + 32 * j;
+      const int p = gw + nwh * r, n = lane + 32 * j;
       dh[r][j] = (dhL != nullptr && n < N) ? dhL[(head * P + p) * N + n] : 0.0f;
     }
   float dA_acc = 0.0f, dD_acc = 0.0f;
   ScanTok<ROWS, COLS> cur, nxt;
   if (pr.L > 0) {
-    scan_load_tok(pr, u, dtv, dypre, bi, h, g, warp, lane, pr.L - 1, cur);
+    scan_load_tok(pr, u, dtv, dypre, bi, h, g, gw, nwh, lane, pr.L - 1, cur);
     load_prev(pr.L, hcur);      // h_{L-1}
     load_prev(pr.L - 1, hprv);  // h_{L-2}
   }
   for (int64_t t = pr.L - 1; t >= 0; --t) {
     if (t > 0) {  // token t - 1: its inputs and the state before it
-      scan_load_tok(pr, u, dtv, dypre, bi, h, g, warp, lane, t - 1, nxt);
+      scan_load_tok(pr, u, dtv, dypre, bi, h, g, gw, nwh, lane, t - 1, nxt);
       load_prev(t - 1, hnx);
     }
     const float dt = cur.dt, a = expf(dt * A);
@@ -257,7 +266,7 @@ __global__ void __launch_bounds__(32 * kScanWarps)
     float ddt_dir = 0.0f, da = 0.0f;  // sum dh x B, sum dh h_{t-1}
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
-      const int p = warp + kScanWarps * r;
+      const int p = gw + nwh * r;
       const float x = cur.x[r], dyp = cur.dy[r];
       float sb = 0.0f;
 #pragma unroll
@@ -280,7 +289,7 @@ __global__ void __launch_bounds__(32 * kScanWarps)
     da = warp_sum(da);
     // this warp's shares of dB (times dt) and dC, and of ddt
     const int64_t bt = bi * pr.L + t;
-    float *pb = pbc + ((bt * 2 * pr.H + h) * kScanWarps + warp) * N;
+    float *pb = pbc + ((bt * 2 * pr.H + h) * kScanWarps + gw) * N;
     const int64_t cstride = (int64_t)pr.H * kScanWarps * N;  // B -> C
 #pragma unroll
     for (int j = 0; j < COLS; ++j) {
@@ -291,7 +300,7 @@ __global__ void __launch_bounds__(32 * kScanWarps)
       }
     }
     if (lane == 0) {
-      pdt[(bt * pr.H + h) * kScanWarps + warp] = ddt_dir + da * a * A;
+      pdt[(bt * pr.H + h) * kScanWarps + gw] = ddt_dir + da * a * A;
       dA_acc = fmaf(da * a, dt, dA_acc);
     }
     cur = nxt;
@@ -312,7 +321,7 @@ __global__ void __launch_bounds__(32 * kScanWarps)
     for (int r = 0; r < ROWS; ++r)
 #pragma unroll
       for (int j = 0; j < COLS; ++j) {
-        const int p = warp + kScanWarps * r, n = lane + 32 * j;
+        const int p = gw + nwh * r, n = lane + 32 * j;
         if (n < N) dh0[(head * P + p) * N + n] = dh[r][j];
       }
   }
@@ -516,10 +525,10 @@ cudaError_t run_backward(const BackwardArgs &a) {
                                                                       dt_raw, a.ld_dt, cs, w.u,
                                                                       w.dtv);
   stage_mark(st, 1);
-  const dim3 gh((unsigned)pr.H, (unsigned)pr.batch);
-  launch_scan(pr, [&](auto rows, auto cols) {
-    bwd_scan_fwd_kernel<decltype(rows)::value, decltype(cols)::value>
-        <<<gh, 32 * kScanWarps, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in, w.hs, w.ypre);
+  launch_scan(pr, [&](auto, auto cols) {  // one row per warp, 16-warp blocks
+    const dim3 grid((unsigned)(pr.H * (pr.P / 16)), (unsigned)pr.batch);
+    bwd_scan_fwd_kernel<1, decltype(cols)::value, 16>
+        <<<grid, 32 * 16, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in, w.hs, w.ypre);
   });
   stage_mark(st, 2);
   bwd_norm_kernel<T><<<(unsigned)bl, 256, 0, st>>>(pr, a.prm, w.ypre, z, a.ld_z, dy, w.dypre,
@@ -528,11 +537,12 @@ cudaError_t run_backward(const BackwardArgs &a) {
   col_sum_kernel<<<dim3((unsigned)ceil_div(pr.d_inner, 256), 64), 256, 0, st>>>(
       w.tok, bl, pr.d_inner, a.d_norm_w);
   stage_mark(st, 4);
-  launch_scan(pr, [&](auto rows, auto cols) {
-    bwd_scan_rev_kernel<decltype(rows)::value, decltype(cols)::value>
-        <<<gh, 32 * kScanWarps, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in, w.hs, w.dypre,
-                                         a.d_ssm_state_out, w.du, w.pbc, w.pdt, a.d_A, a.d_D,
-                                         a.d_ssm_state_in);
+  launch_scan(pr, [&](auto rows, auto cols) {  // kScanWarps warps per head, 4-warp blocks
+    const dim3 grid((unsigned)(pr.H * (kScanWarps / 4)), (unsigned)pr.batch);
+    bwd_scan_rev_kernel<decltype(rows)::value, decltype(cols)::value, 4>
+        <<<grid, 32 * 4, 0, st>>>(pr, a.prm, w.u, w.dtv, a.ssm_state_in, w.hs, w.dypre,
+                                  a.d_ssm_state_out, w.du, w.pbc, w.pdt, a.d_A, a.d_D,
+                                  a.d_ssm_state_in);
   });
   stage_mark(st, 5);
   bwd_reduce_bc_kernel<<<grid_for(bl * pr.G * 2 * pr.N), 256, 0, st>>>(pr, w.pbc, w.pdt, w.du,
