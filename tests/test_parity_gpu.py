@@ -151,8 +151,8 @@ def test_tc_large_dt(bias):
 @pytest.mark.parametrize("mag", [1e5, 3e7])
 def test_tc_large_carried_state(mag):
     # a carried SSM state far beyond the fp16 range: the output kernel's operand
-    # holds each (chunk, head, 16-column) block of the state divided by a power
-    # of two, so y and the final state still match the oracle
+    # holds each (chunk, head) state divided by a power of two and multiplies
+    # C H_c^T back by it, so y and the final state still match the oracle
     cfg, params, inp, st = _tc_case(24)
     st = dict(st, ssm_state=st["ssm_state"] * (mag / 0.1))
     got = gpu_prefill(cfg, inp, params, states={k: v.clone() for k, v in st.items()},
