@@ -936,11 +936,11 @@ __global__ void __launch_bounds__(kPrepThreads)
 constexpr int kPassBlocks = 4;     // blocks per head
 constexpr int kPassThreads = 256;  // 1024 float4 slots of a head's 64 x 64 state
 
-// 2^s with s = max(0, floor(log2 m) - 13), so that m / 2^s < 2^14.
-__device__ __forceinline__ float state_scale(float m) {
+// s = max(0, floor(log2 m) - 13), so that m / 2^s < 2^14; 2^s and 2^-s are then
+// built from their exponent bits (both normal: s <= 100).
+__device__ __forceinline__ int state_shift(float m) {
   const int e = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;  // floor(log2 m) for normal m
-  const int s = min(max(e - 13, 0), 100);
-  return __uint_as_float((uint32_t)(127 + s) << 23);
+  return min(max(e - 13, 0), 100);
 }
 
 __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, __nv_bfloat16 *cs) {
@@ -1017,61 +1017,73 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
 #pragma unroll
     for (int w = 0; w < kPassThreads / 32; ++w) bnd = fmaxf(bnd, red[w]);
   }
+  // The chain issues more instructions than it moves bytes, so each chunk's step
+  // is kept short: pointers advance by one chunk, 2^-s comes from its exponent
+  // bits, and the decay factor is one ex2.approx of cum_end log2(e).
   const int64_t stride = (int64_t)pr.H * kHP * kNS;  // one chunk further
   const int64_t c0h = cb0 * pr.H + h;                  // (first chunk, head)
   const float *S = a.S + c0h * (int64_t)(kHP * kNS) + 4 * j;
   __half *Hc = a.Hc + c0h * (int64_t)(kHP * kNS) + (4 * n4) * kHP + p;
   const float *ce = a.cum_end + c0h;
   const float *sm = a.smax + c0h;
+  float *hp = a.hsc + c0h * 32 + lane;
+  const int64_t hstep = (int64_t)pr.H * 32;
   const bool scale_writer = q == 0 && warp == 0;  // the head's 32 scale entries per chunk
   // H_c / 2^s into the operand (4 coalesced 2-byte stores), 2^s into the scale table
-  auto put = [&](int64_t c) {
-    const float sc = state_scale(bnd), inv = 1.0f / sc;  // powers of two: exact
-    __half *o = Hc + c * stride;
-    if (M2_OK(o, 2, a.sp.Hc, &g_tc_errors) && M2_OK(o + 3 * kHP, 2, a.sp.Hc, &g_tc_errors)) {
-      o[0] = __float2half_rn(hc.x * inv);
-      o[kHP] = __float2half_rn(hc.y * inv);
-      o[2 * kHP] = __float2half_rn(hc.z * inv);
-      o[3 * kHP] = __float2half_rn(hc.w * inv);
+  auto put = [&]() {
+    const uint32_t sh = (uint32_t)state_shift(bnd);
+    const float inv = __uint_as_float((127u - sh) << 23);  // 2^-s, exact
+    if (M2_OK(Hc, 2, a.sp.Hc, &g_tc_errors) && M2_OK(Hc + 3 * kHP, 2, a.sp.Hc, &g_tc_errors)) {
+      Hc[0] = __float2half_rn(hc.x * inv);
+      Hc[kHP] = __float2half_rn(hc.y * inv);
+      Hc[2 * kHP] = __float2half_rn(hc.z * inv);
+      Hc[3 * kHP] = __float2half_rn(hc.w * inv);
     }
-    float *hp = a.hsc + (c0h + c * pr.H) * 32 + lane;
-    if (scale_writer && M2_OK(hp, 4, a.sp.hsc, &g_tc_errors)) *hp = sc;
+    if (scale_writer && M2_OK(hp, 4, a.sp.hsc, &g_tc_errors))
+      *hp = __uint_as_float((127u + sh) << 23);  // 2^s
   };
   auto step = [&](float4 sv, float d, float msv) {
-    const float f = expf(d);
+    const float f = ex2_approx(d * kLog2e);
     hc = make_float4(fmaf(f, hc.x, sv.x), fmaf(f, hc.y, sv.y), fmaf(f, hc.z, sv.z),
                      fmaf(f, hc.w, sv.w));
     bnd = fmaf(f, bnd, msv);
   };
   // loads run 8 chunks ahead of the (sequential) recurrence
   constexpr int kAhead = 8;
-  int c = 0;
+  int64_t c = 0;
   for (; c + kAhead <= nchs; c += kAhead) {
     float4 sv[kAhead];
     float d[kAhead], msv[kAhead];
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
-      const float *sp = S + (c + k) * stride;
-      const int64_t r = (int64_t)(c + k) * pr.H;
+      const float *sp = S + k * stride;
       sv[k] = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-      d[k] = M2_OK(ce + r, 4, a.sp.cum_end, &g_tc_errors) ? ce[r] : 0.0f;
-      msv[k] = M2_OK(sm + r, 4, a.sp.smax, &g_tc_errors) ? sm[r] : 0.0f;
+      d[k] = M2_OK(ce + k * pr.H, 4, a.sp.cum_end, &g_tc_errors) ? ce[k * pr.H] : 0.0f;
+      msv[k] = M2_OK(sm + k * pr.H, 4, a.sp.smax, &g_tc_errors) ? sm[k * pr.H] : 0.0f;
     }
+    S += kAhead * stride;
+    ce += kAhead * pr.H;
+    sm += kAhead * pr.H;
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
-      put(c + k);
+      put();
       step(sv[k], d[k], msv[k]);
+      Hc += stride;
+      hp += hstep;
     }
   }
   for (; c < nchs; ++c) {
-    put(c);
-    const float *sp = S + c * stride;
-    const int64_t r = (int64_t)c * pr.H;
-    step(M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
-                                             : make_float4(0.f, 0.f, 0.f, 0.f),
-         M2_OK(ce + r, 4, a.sp.cum_end, &g_tc_errors) ? ce[r] : 0.0f,
-         M2_OK(sm + r, 4, a.sp.smax, &g_tc_errors) ? sm[r] : 0.0f);
+    put();
+    step(M2_OK(S, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(S)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f),
+         M2_OK(ce, 4, a.sp.cum_end, &g_tc_errors) ? *ce : 0.0f,
+         M2_OK(sm, 4, a.sp.smax, &g_tc_errors) ? *sm : 0.0f);
+    S += stride;
+    ce += pr.H;
+    sm += pr.H;
+    Hc += stride;
+    hp += hstep;
   }
   if (a.ssm_state != nullptr && M2_OK(a.ssm_state + hs, 16, a.sp.ssm, &g_tc_errors))
     *reinterpret_cast<float4 *>(a.ssm_state + hs) = hc;
