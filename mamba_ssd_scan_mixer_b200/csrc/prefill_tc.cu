@@ -914,11 +914,14 @@ __global__ void __launch_bounds__(kPrepThreads)
 }
 
 // ============================================================== state passing
-// grid (H * 4 + conv-state blocks, b) of 256-thread blocks.  Block 4 h + q runs
-// the recurrence H_{c+1} = exp(cum_end_c) H_c + S_c in fp32 for the float4 slots
-// j = 256 q + thread of head h's chunk states ([n/4][p][4]: columns n = 4 (j / 64)
-// .. +3 of row p = j % 64), sequential over chunks, with loads issued 8 chunks at
-// a time: a warp reads 512 contiguous bytes per chunk and writes the fp16 state
+// grid (H * 8 + conv-state blocks, b) of 128-thread blocks, five per SM, so that
+// a launch is one wave.  Block 8 h + q runs the recurrence
+// H_{c+1} = exp(cum_end_c) H_c + S_c in fp32 for the float4 slots j = 128 q +
+// thread of head h's chunk states ([n/4][p][4]: columns n = 4 (j / 64) .. +3 of
+// row p = j % 64), sequential over chunks.  The chain waits on memory, so loads
+// are issued 16 chunks at a time (one round trip per 16 chunks; the batch's
+// scalars come through shared memory to leave the registers to the states): a
+// warp reads 512 contiguous bytes per chunk and writes the fp16 state
 // entering each chunk as H_c [n][p] (the output kernel's MN-major operand), four
 // coalesced 64-byte rows.
 // H_c is stored divided by 2^s, one power of two per (chunk, head), so that fp16
@@ -933,8 +936,9 @@ __global__ void __launch_bounds__(kPrepThreads)
 // Blocks 4 H and up write the final conv state instead: the last 4 raw inputs of
 // [old state | new tokens], in place (the chunk-state kernel, which reads the old
 // state, has finished by now).
-constexpr int kPassBlocks = 4;     // blocks per head
-constexpr int kPassThreads = 256;  // 1024 float4 slots of a head's 64 x 64 state
+constexpr int kPassBlocks = 8;     // blocks per head
+constexpr int kPassThreads = 128;  // x 8 = the 1024 float4 slots of a head's 64 x 64 state
+constexpr int kPassAhead = 16;     // chunks whose loads are in flight together
 
 // s = max(0, floor(log2 m) - 13), so that m / 2^s < 2^14; 2^s and 2^-s are then
 // built from their exponent bits (both normal: s <= 100).
@@ -943,7 +947,7 @@ __device__ __forceinline__ int state_shift(float m) {
   return min(max(e - 13, 0), 100);
 }
 
-__global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, __nv_bfloat16 *cs) {
+__global__ void __launch_bounds__(kPassThreads, 5) tc_state_pass_kernel(TcArgs a, __nv_bfloat16 *cs) {
   __shared__ float red[kPassThreads / 32];
   grid_dependency_wait();  // the chunk-state kernel's results (launched early, see prefill_tc)
   launch_dependents();
@@ -1048,27 +1052,38 @@ __global__ void __launch_bounds__(kPassThreads) tc_state_pass_kernel(TcArgs a, _
                      fmaf(f, hc.w, sv.w));
     bnd = fmaf(f, bnd, msv);
   };
-  // loads run 8 chunks ahead of the (sequential) recurrence
-  constexpr int kAhead = 8;
+  // loads run kPassAhead chunks ahead of the (sequential) recurrence; the batch's
+  // decay and bound scalars, the same for the whole block, are loaded by warp 0
+  // (lanes 0-15 cum_end, 16-31 smax) and shared through a double buffer
+  constexpr int kAhead = kPassAhead;
+  static_assert(2 * kAhead == 32, "one lane of warp 0 per scalar of a batch");
+  __shared__ float s_dm[2][2 * kAhead];
   int64_t c = 0;
   for (; c + kAhead <= nchs; c += kAhead) {
+    const int par = (int)((c / kAhead) & 1);
+    float sl = 0.0f;
+    if (warp == 0) {
+      const float *src = lane < kAhead ? ce + lane * pr.H : sm + (lane - kAhead) * pr.H;
+      const bool okp = lane < kAhead ? M2_OK(src, 4, a.sp.cum_end, &g_tc_errors)
+                                     : M2_OK(src, 4, a.sp.smax, &g_tc_errors);
+      sl = okp ? *src : 0.0f;
+    }
     float4 sv[kAhead];
-    float d[kAhead], msv[kAhead];
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
       const float *sp = S + k * stride;
       sv[k] = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-      d[k] = M2_OK(ce + k * pr.H, 4, a.sp.cum_end, &g_tc_errors) ? ce[k * pr.H] : 0.0f;
-      msv[k] = M2_OK(sm + k * pr.H, 4, a.sp.smax, &g_tc_errors) ? sm[k * pr.H] : 0.0f;
     }
     S += kAhead * stride;
     ce += kAhead * pr.H;
     sm += kAhead * pr.H;
+    if (warp == 0) s_dm[par][lane] = sl;
+    __syncthreads();  // (the buffer written here was last read two batches ago)
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
       put();
-      step(sv[k], d[k], msv[k]);
+      step(sv[k], s_dm[par][k], s_dm[par][kAhead + k]);
       Hc += stride;
       hp += hstep;
     }
