@@ -1021,9 +1021,9 @@ __global__ void __launch_bounds__(kPassThreads, 5) tc_state_pass_kernel(TcArgs a
 #pragma unroll
     for (int w = 0; w < kPassThreads / 32; ++w) bnd = fmaxf(bnd, red[w]);
   }
-  // The chain issues more instructions than it moves bytes, so each chunk's step
-  // is kept short: pointers advance by one chunk, 2^-s comes from its exponent
-  // bits, and the decay factor is one ex2.approx of cum_end log2(e).
+  // Each chunk's step is kept short: pointers advance by one chunk, 2^-s comes
+  // from its exponent bits, and the decay factor is one ex2.approx of
+  // cum_end log2(e).
   const int64_t stride = (int64_t)pr.H * kHP * kNS;  // one chunk further
   const int64_t c0h = cb0 * pr.H + h;                  // (first chunk, head)
   const float *S = a.S + c0h * (int64_t)(kHP * kNS) + 4 * j;
@@ -1058,11 +1058,12 @@ __global__ void __launch_bounds__(kPassThreads, 5) tc_state_pass_kernel(TcArgs a
   constexpr int kAhead = kPassAhead;
   static_assert(2 * kAhead == 32, "one lane of warp 0 per scalar of a batch");
   __shared__ float s_dm[2][2 * kAhead];
-  int64_t c = 0;
-  for (; c + kAhead <= nchs; c += kAhead) {
+  // chunks [c, c + nb) of the chain, nb <= kAhead (a constant in the main loop, so
+  // that only the last, shorter batch carries the predicates)
+  auto run_batch = [&](int64_t c, int nb) {
     const int par = (int)((c / kAhead) & 1);
     float sl = 0.0f;
-    if (warp == 0) {
+    if (warp == 0 && (lane & (kAhead - 1)) < nb) {
       const float *src = lane < kAhead ? ce + lane * pr.H : sm + (lane - kAhead) * pr.H;
       const bool okp = lane < kAhead ? M2_OK(src, 4, a.sp.cum_end, &g_tc_errors)
                                      : M2_OK(src, 4, a.sp.smax, &g_tc_errors);
@@ -1072,8 +1073,9 @@ __global__ void __launch_bounds__(kPassThreads, 5) tc_state_pass_kernel(TcArgs a
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
       const float *sp = S + k * stride;
-      sv[k] = M2_OK(sp, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(sp)
-                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      sv[k] = (k < nb && M2_OK(sp, 16, a.sp.S, &g_tc_errors))
+                  ? *reinterpret_cast<const float4 *>(sp)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     S += kAhead * stride;
     ce += kAhead * pr.H;
@@ -1082,24 +1084,17 @@ __global__ void __launch_bounds__(kPassThreads, 5) tc_state_pass_kernel(TcArgs a
     __syncthreads();  // (the buffer written here was last read two batches ago)
 #pragma unroll
     for (int k = 0; k < kAhead; ++k) {
-      put();
-      step(sv[k], s_dm[par][k], s_dm[par][kAhead + k]);
-      Hc += stride;
-      hp += hstep;
+      if (k < nb) {
+        put();
+        step(sv[k], s_dm[par][k], s_dm[par][kAhead + k]);
+        Hc += stride;
+        hp += hstep;
+      }
     }
-  }
-  for (; c < nchs; ++c) {
-    put();
-    step(M2_OK(S, 16, a.sp.S, &g_tc_errors) ? *reinterpret_cast<const float4 *>(S)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f),
-         M2_OK(ce, 4, a.sp.cum_end, &g_tc_errors) ? *ce : 0.0f,
-         M2_OK(sm, 4, a.sp.smax, &g_tc_errors) ? *sm : 0.0f);
-    S += stride;
-    ce += pr.H;
-    sm += pr.H;
-    Hc += stride;
-    hp += hstep;
-  }
+  };
+  int64_t c = 0;
+  for (; c + kAhead <= nchs; c += kAhead) run_batch(c, kAhead);
+  if (c < nchs) run_batch(c, (int)(nchs - c));
   if (a.ssm_state != nullptr && M2_OK(a.ssm_state + hs, 16, a.sp.ssm, &g_tc_errors))
     *reinterpret_cast<float4 *>(a.ssm_state + hs) = hc;
 }
