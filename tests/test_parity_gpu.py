@@ -53,6 +53,10 @@ def test_tiny_f32_config():
     case("zamba2_2p7b_prefill", batch=2, seqlen=640, nheads=64),
     case("zamba2_2p7b_prefill", batch=2, seqlen=1500, nheads=80),
     case("zamba2_2p7b_prefill", batch=1, seqlen=400, nheads=96),
+    # state-pass chains longer than one 16-chunk batch of loads, with a shorter
+    # last batch (21 and 17 chunks, the last one ragged)
+    case("zamba2_2p7b_prefill", batch=2, seqlen=2600, nheads=16),
+    case("zamba2_2p7b_prefill", batch=1, seqlen=2100, nheads=8, ngroups=2),
     case("zamba2_2p7b_prefill", batch=1, seqlen=257, nheads=4, headdim=32, dstate=128),
     case("zamba2_2p7b_prefill", batch=1, seqlen=200, nheads=4, headdim=16, dstate=32),
     case("tiny_f32", batch=2, seqlen=517, nheads=6, ngroups=2, headdim=64, dstate=64,

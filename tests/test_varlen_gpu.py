@@ -83,6 +83,17 @@ def test_varlen_two_groups():
     _check_against_oracle(cfg, params, inp, lengths, got, states=st)
 
 
+def test_varlen_long_and_short_chains():
+    # one sequence of 19 chunks (a full 16-chunk batch of state-pass loads and a
+    # ragged 3-chunk remainder) beside sequences of one and two chunks
+    lengths = [5, 2400, 129]
+    cfg, params, inp = _packed(lengths, seed=34)
+    st = W.make_states(cfg.with_(batch=len(lengths)), 34)
+    got = _gpu_varlen(cfg, params, inp, lengths, states=st, states_in=True)
+    assert m2.device_errors() == 0
+    _check_against_oracle(cfg, params, inp, lengths, got, states=st)
+
+
 @pytest.mark.parametrize("lengths", [[700], [384, 384]])
 def test_varlen_equals_fixed_length_path_bitwise(lengths):
     # equal lengths: the packed call must reproduce the batched call exactly
