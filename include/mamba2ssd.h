@@ -146,6 +146,48 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
                                        float *ssm_state, int32_t states_in, void *workspace,
                                        size_t workspace_bytes, void *stream);
 
+/* Bytes of DEVICE workspace that mamba2_conv_ssd_prefill_host needs for `dims`
+ * (0 if dims are invalid): two staged input pieces, two output pieces, the
+ * carried states and one piece's prefill workspace (about a quarter of the
+ * whole-sequence input and output, for long sequences). */
+MAMBA2_API size_t mamba2_prefill_host_workspace_size(const mamba2_dims *dims);
+
+/* Prefill with every input and output in HOST memory: the same computation as
+ * mamba2_conv_ssd_prefill (qwbw.cn section 三 steps 2-4) on host buffers, with
+ * the copies overlapped with the work.  The sequence is cut into pieces of
+ * whole chunks (a multiple of 256 tokens, about an eighth of L); piece i + 1 is
+ * copied in and piece i - 1's y copied out while piece i runs, each piece
+ * continuing from the states the previous one left (the chunked prefill of
+ * section 三 step 3), so the result equals the one-call prefill up to rounding.
+ *
+ *  xBC, z, dt_raw  HOST, layout and row strides as for mamba2_conv_ssd_prefill
+ *          (strides in elements, >= the widths; no alignment needed).
+ *  y       HOST [b, L, d_inner] io_dtype, contiguous.  Output.
+ *  conv_state, ssm_state  HOST or NULL, layouts as for mamba2_conv_ssd_prefill;
+ *          read when states_in = 1, overwritten with the final states.
+ *  workspace  DEVICE, >= mamba2_prefill_host_workspace_size(dims) bytes,
+ *          256-byte aligned; contents on entry are ignored.
+ *  stream  the caller's cudaStream_t (as void*): the call begins after the
+ *          work already enqueued on it, and work enqueued on it afterwards
+ *          begins after the call's last copy.  The call returns once its work
+ *          is enqueued: synchronise the stream before reading y or the states.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister): the
+ * copies of pageable memory are correct but neither asynchronous nor
+ * overlapped.  The call creates two streams and eight events of its own (so it
+ * cannot be captured into a CUDA graph) and releases them when their work is
+ * done.  Stage events (mamba2_record_stage_events) are not recorded.
+ * Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG (null pointer, stride below a
+ * width, states_in without states), MAMBA2_ERR_UNSUPPORTED (as for
+ * mamba2_conv_ssd_prefill), MAMBA2_ERR_WORKSPACE or MAMBA2_ERR_CUDA. */
+MAMBA2_API int mamba2_conv_ssd_prefill_host(const mamba2_dims *dims,
+                                            const mamba2_params *params, const void *xBC,
+                                            int64_t xBC_row_stride, const void *z,
+                                            int64_t z_row_stride, const void *dt_raw,
+                                            int64_t dt_row_stride, void *y, void *conv_state,
+                                            float *ssm_state, int32_t states_in,
+                                            void *workspace, size_t workspace_bytes,
+                                            void *stream);
+
 /* Workspace bytes mamba2_conv_ssd_prefill_varlen needs for `dims` (batch =
  * number of sequences, seqlen = total tokens); 0 if the dims are invalid or
  * the call is not supported for them (see below). */

@@ -23,6 +23,7 @@ __all__ = [
     "mamba2_conv_ssd_prefill", "mamba2_conv_ssd_prefill_noalloc", "mamba2_ssd_step", "prefill",
     "step", "status_string", "mamba2_prefill_backward_workspace_size",
     "mamba2_conv_ssd_prefill_backward", "prefill_backward",
+    "mamba2_prefill_host_workspace_size", "mamba2_conv_ssd_prefill_host", "prefill_host",
 ]
 
 MAMBA2_F32, MAMBA2_BF16 = 0, 1
@@ -76,6 +77,11 @@ def lib() -> ctypes.CDLL:
         L.mamba2_conv_ssd_prefill.restype = ctypes.c_int
         L.mamba2_conv_ssd_prefill.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp, i32,
                                               vp, sz, vp]
+        L.mamba2_prefill_host_workspace_size.restype = sz
+        L.mamba2_prefill_host_workspace_size.argtypes = [pd]
+        L.mamba2_conv_ssd_prefill_host.restype = ctypes.c_int
+        L.mamba2_conv_ssd_prefill_host.argtypes = [pd, pp, vp, i64, vp, i64, vp, i64, vp, vp, vp,
+                                                   i32, vp, sz, vp]
         L.mamba2_prefill_varlen_workspace_size.restype = sz
         L.mamba2_prefill_varlen_workspace_size.argtypes = [pd]
         L.mamba2_conv_ssd_prefill_varlen.restype = ctypes.c_int
@@ -195,6 +201,53 @@ def mamba2_conv_ssd_prefill(dims, params, xBC, z, dt_raw, y, conv_state=None, ss
         ws_bytes, _stream(stream))
     if st != 0:
         raise Mamba2Error(st, "mamba2_conv_ssd_prefill")
+
+
+def mamba2_prefill_host_workspace_size(dims: Mamba2Dims) -> int:
+    return int(lib().mamba2_prefill_host_workspace_size(ctypes.byref(dims)))
+
+
+def mamba2_conv_ssd_prefill_host(dims, params, xBC, z, dt_raw, y, conv_state=None,
+                                 ssm_state=None, states_in=False, workspace=None,
+                                 stream=None) -> None:
+    """Enqueue one prefill whose inputs, y and states are CPU tensors (page-locked
+    for overlapped copies); layouts as mamba2_conv_ssd_prefill; workspace: a CUDA
+    byte tensor of mamba2_prefill_host_workspace_size(dims) bytes.  Synchronise
+    the stream before reading y or the states."""
+    for name, t in (("xBC", xBC), ("z", z), ("dt_raw", dt_raw), ("y", y),
+                    ("conv_state", conv_state), ("ssm_state", ssm_state)):
+        if t is not None and t.is_cuda:
+            raise ValueError(f"{name}: the host entry takes CPU tensors")
+    L = dims.seqlen
+    lx = _rows(xBC, "xBC", None, dims.batch, L)
+    lz = _rows(z, "z", None, dims.batch, L)
+    ld = _rows(dt_raw, "dt_raw", None, dims.batch, L)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().mamba2_conv_ssd_prefill_host(
+        ctypes.byref(dims), ctypes.byref(params), _ptr(xBC), lx, _ptr(z), lz, _ptr(dt_raw), ld,
+        _ptr(y), _ptr(conv_state), _ptr(ssm_state), int(bool(states_in)), _ptr(workspace),
+        ws_bytes, _stream(stream))
+    if st != 0:
+        raise Mamba2Error(st, "mamba2_conv_ssd_prefill_host")
+
+
+def prefill_host(dims, params, xBC, z, dt_raw, conv_state=None, ssm_state=None,
+                 states_in=False, workspace=None, y=None, stream=None, device=None):
+    """Allocate y (page-locked) and the device workspace if not given, run a
+    host-buffer prefill and wait for it.  Returns y [b, L, d_inner] on the CPU;
+    the states, if given, are updated in place."""
+    import torch
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    if y is None:
+        y = torch.empty(dims.batch, dims.seqlen, dims.nheads * dims.headdim, dtype=xBC.dtype,
+                        pin_memory=True)
+    if workspace is None:
+        workspace = torch.empty(max(1, mamba2_prefill_host_workspace_size(dims)),
+                                dtype=torch.uint8, device=dev)
+    mamba2_conv_ssd_prefill_host(dims, params, xBC, z, dt_raw, y, conv_state, ssm_state,
+                                 states_in, workspace, stream)
+    torch.cuda.synchronize(dev)
+    return y
 
 
 def mamba2_prefill_varlen_workspace_size(dims: Mamba2Dims) -> int:

@@ -2,6 +2,7 @@
 // include/mamba2ssd.h for the contract of every entry point.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -272,6 +273,224 @@ MAMBA2_API int mamba2_conv_ssd_prefill(const mamba2_dims *dims, const mamba2_par
   return m2::prefill_entry(dims, params, xBC, xBC_row_stride, z, z_row_stride, dt_raw,
                            dt_row_stride, nullptr, y, conv_state, ssm_state, states_in,
                            workspace, workspace_bytes, stream);
+}
+
+namespace m2 {
+namespace {
+// Device memory of the host-buffer prefill: two staged input pieces, two output
+// pieces, the carried states and the prefill workspace of one piece.
+struct HostPlan {
+  int64_t Lp, ldx, ldz, ldd;  // tokens per piece; staged row strides (elements)
+  size_t x, z, d, in, y, cs, hs, ws, total;
+};
+size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+bool host_plan(const mamba2_dims *dims, const Problem &pr, HostPlan *o) {
+  // pieces of whole chunks for every chunk size (multiples of 256 tokens), about
+  // an eighth of the sequence each, so that the copies of the first and last
+  // pieces, which nothing overlaps, are short
+  const int64_t eighth = (pr.L + 7) / 8;
+  o->Lp = std::min<int64_t>(std::max<int64_t>((eighth + 255) / 256 * 256, 256),
+                            std::max<int64_t>(pr.L, 1));
+  const size_t esz = pr.io == MAMBA2_BF16 ? 2 : 4;
+  o->ldx = (pr.conv_dim + 7) / 8 * 8;
+  o->ldz = (pr.d_inner + 7) / 8 * 8;
+  o->ldd = (pr.H + 7) / 8 * 8;
+  const size_t rows = (size_t)pr.batch * (size_t)o->Lp;
+  o->x = up256(rows * o->ldx * esz);
+  o->z = up256(rows * o->ldz * esz);
+  o->d = up256(rows * o->ldd * esz);
+  o->in = o->x + o->z + o->d;
+  o->y = up256(rows * pr.d_inner * esz);
+  o->cs = up256((size_t)pr.batch * pr.conv_dim * pr.K * esz);
+  o->hs = up256((size_t)pr.batch * pr.H * pr.P * pr.N * 4);
+  mamba2_dims dp = *dims;
+  dp.seqlen = (int32_t)o->Lp;
+  Problem pp;
+  if (make_problem(&dp, true, &pp) != MAMBA2_OK) return false;
+  o->ws = up256(prefill_workspace(pp));
+  o->total = 2 * o->in + 2 * o->y + o->cs + o->hs + o->ws;
+  return true;
+}
+}  // namespace
+}  // namespace m2
+
+MAMBA2_API size_t mamba2_prefill_host_workspace_size(const mamba2_dims *dims) {
+  Problem pr;
+  m2::HostPlan plan;
+  if (make_problem(dims, true, &pr) != MAMBA2_OK || !m2::host_plan(dims, pr, &plan)) return 0;
+  return plan.total;
+}
+
+MAMBA2_API int mamba2_conv_ssd_prefill_host(
+    const mamba2_dims *dims, const mamba2_params *params, const void *xBC,
+    int64_t xBC_row_stride, const void *z, int64_t z_row_stride, const void *dt_raw,
+    int64_t dt_row_stride, void *y, void *conv_state, float *ssm_state, int32_t states_in,
+    void *workspace, size_t workspace_bytes, void *stream) {
+  NvtxRange range("mamba2_conv_ssd_prefill_host");
+  g_stage_events.n = 0;  // stage events are not recorded by this entry
+  DisarmOnExit disarm;
+  Problem pr;
+  int st = make_problem(dims, true, &pr);
+  if (st != MAMBA2_OK) return st;
+  if (!params_ok(params)) return MAMBA2_ERR_INVALID_ARG;
+  if (states_in != 0 && states_in != 1) return MAMBA2_ERR_INVALID_ARG;
+  if (states_in && (conv_state == nullptr || ssm_state == nullptr)) return MAMBA2_ERR_INVALID_ARG;
+  if (pr.batch == 0) return MAMBA2_OK;
+  if (pr.L > 0 && (xBC == nullptr || z == nullptr || dt_raw == nullptr || y == nullptr))
+    return MAMBA2_ERR_INVALID_ARG;
+  if (pr.L > 0 &&
+      (xBC_row_stride < pr.conv_dim || z_row_stride < pr.d_inner || dt_row_stride < pr.H))
+    return MAMBA2_ERR_INVALID_ARG;
+  m2::HostPlan pl;
+  if (!m2::host_plan(dims, pr, &pl)) return MAMBA2_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < pl.total || !aligned(workspace, 256))
+    return MAMBA2_ERR_WORKSPACE;
+  const size_t esz = pr.io == MAMBA2_BF16 ? 2 : 4;
+  char *w = static_cast<char *>(workspace);
+  char *in[2] = {w, w + pl.in};
+  char *yb[2] = {w + 2 * pl.in, w + 2 * pl.in + pl.y};
+  char *cs_d = w + 2 * pl.in + 2 * pl.y;
+  float *hs_d = reinterpret_cast<float *>(cs_d + pl.cs);
+  char *ws_d = cs_d + pl.cs + pl.hs;
+  const size_t cs_bytes = (size_t)pr.batch * pr.conv_dim * pr.K * esz;
+  const size_t hs_bytes = (size_t)pr.batch * pr.H * pr.P * pr.N * 4;
+  cudaStream_t cs_ = static_cast<cudaStream_t>(stream);
+  // The usual layout, the three views side by side in one packed row (an in_proj
+  // output): copy each row's span once and point the staged views into it, which
+  // avoids copies of narrow rows (dt_raw's are a few hundred bytes).  Needs one
+  // row stride, the device entry's alignments at the views' offsets in the row,
+  // and a staged row that fits the slot.
+  const char *hx = static_cast<const char *>(xBC), *hz = static_cast<const char *>(z),
+             *hd = static_cast<const char *>(dt_raw);
+  const char *base = std::min(hx, std::min(hz, hd));
+  const char *span_end = std::max(hx + pr.conv_dim * esz,
+                                  std::max(hz + pr.d_inner * esz, hd + pr.H * esz));
+  const int64_t S = xBC_row_stride;
+  const bool packed = pr.L > 0 && z_row_stride == S && dt_row_stride == S && S % 8 == 0 &&
+                      span_end - base <= S * (int64_t)esz &&
+                      (size_t)S <= (size_t)(pl.ldx + pl.ldz + pl.ldd) &&
+                      (hx - base) % 16 == 0 && (hz - base) % 16 == 0 && (hd - base) % esz == 0;
+
+  // Copies in on one stream, the prefill of each piece on the caller's stream,
+  // copies out on a third: piece i + 1 arrives and piece i - 1 leaves while piece
+  // i runs.  Two staging slots per direction; every reuse waits for its reader.
+  cudaStream_t upl = nullptr, dnl = nullptr;
+  cudaEvent_t ev[8] = {};  // start, in_ready[2], comp_done[2], out_free[2], done
+  bool ok = cudaStreamCreateWithFlags(&upl, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&dnl, cudaStreamNonBlocking) == cudaSuccess;
+  for (int i = 0; ok && i < 8; ++i)
+    ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+  cudaEvent_t start = ev[0], done = ev[7];
+  cudaEvent_t *in_ready = ev + 1, *comp_done = ev + 3, *out_free = ev + 5;
+  int rc = MAMBA2_OK;
+  auto chk = [&](cudaError_t e) {
+    if (e != cudaSuccess && rc == MAMBA2_OK) rc = MAMBA2_ERR_CUDA;
+    return rc == MAMBA2_OK;
+  };
+  if (ok) {
+    // nothing of this call starts before the caller's earlier work on its stream
+    chk(cudaEventRecord(start, cs_));
+    chk(cudaStreamWaitEvent(upl, start, 0));
+    chk(cudaStreamWaitEvent(dnl, start, 0));
+    const int64_t np = pr.L > 0 ? (pr.L + pl.Lp - 1) / pl.Lp : 0;
+    if (states_in && np > 0) {
+      chk(cudaMemcpyAsync(cs_d, conv_state, cs_bytes, cudaMemcpyHostToDevice, upl));
+      chk(cudaMemcpyAsync(hs_d, ssm_state, hs_bytes, cudaMemcpyHostToDevice, upl));
+    }
+    if (np == 0 && !states_in) {  // no tokens and no carried states: they start at zero
+      chk(cudaMemsetAsync(cs_d, 0, cs_bytes, dnl));
+      chk(cudaMemsetAsync(hs_d, 0, hs_bytes, dnl));
+    }
+    for (int64_t i = 0; i < np && rc == MAMBA2_OK; ++i) {
+      const int s = (int)(i & 1);
+      const int64_t t0 = i * pl.Lp, Li = std::min<int64_t>(pl.Lp, pr.L - t0);
+      char *xs = in[s], *zs = in[s] + pl.x, *ds = in[s] + pl.x + pl.z;
+      int64_t lx = pl.ldx, lz = pl.ldz, ld = pl.ldd;
+      if (packed) {
+        xs = in[s] + (hx - base);
+        zs = in[s] + (hz - base);
+        ds = in[s] + (hd - base);
+        lx = lz = ld = S;
+      }
+      if (i >= 2) chk(cudaStreamWaitEvent(upl, comp_done[s], 0));  // slot s read by piece i - 2
+      if (packed) {  // rows bi L + t0 .. + Li of every batch row: their spans
+        const size_t row = (size_t)S * esz, span = (size_t)(span_end - base);
+        for (int64_t bi = 0; bi < pr.batch && rc == MAMBA2_OK; ++bi) {
+          const size_t r0 = (size_t)(bi * pr.L + t0), d0 = (size_t)(bi * pl.Lp);
+          if (span == row)
+            chk(cudaMemcpyAsync(in[s] + d0 * row, base + r0 * row, (size_t)Li * row,
+                                cudaMemcpyHostToDevice, upl));
+          else
+            chk(cudaMemcpy2DAsync(in[s] + d0 * row, row, base + r0 * row, row, span, Li,
+                                  cudaMemcpyHostToDevice, upl));
+        }
+      }
+      for (int64_t bi = 0; !packed && bi < pr.batch && rc == MAMBA2_OK; ++bi) {
+        const size_t r0 = (size_t)(bi * pr.L + t0), d0 = (size_t)(bi * pl.Lp);
+        chk(cudaMemcpy2DAsync(xs + d0 * pl.ldx * esz, pl.ldx * esz,
+                              static_cast<const char *>(xBC) + r0 * xBC_row_stride * esz,
+                              xBC_row_stride * esz, pr.conv_dim * esz, Li,
+                              cudaMemcpyHostToDevice, upl));
+        chk(cudaMemcpy2DAsync(zs + d0 * pl.ldz * esz, pl.ldz * esz,
+                              static_cast<const char *>(z) + r0 * z_row_stride * esz,
+                              z_row_stride * esz, pr.d_inner * esz, Li, cudaMemcpyHostToDevice,
+                              upl));
+        chk(cudaMemcpy2DAsync(ds + d0 * pl.ldd * esz, pl.ldd * esz,
+                              static_cast<const char *>(dt_raw) + r0 * dt_row_stride * esz,
+                              dt_row_stride * esz, pr.H * esz, Li, cudaMemcpyHostToDevice, upl));
+      }
+      chk(cudaEventRecord(in_ready[s], upl));
+      chk(cudaStreamWaitEvent(cs_, in_ready[s], 0));
+      if (i >= 2) chk(cudaStreamWaitEvent(cs_, out_free[s], 0));  // y slot s copied out
+      if (rc != MAMBA2_OK) break;
+      // the piece's batch rows are Lp apart in the staging slot: one batch row at
+      // a time when the last piece is shorter, else all rows in one call
+      mamba2_dims di = *dims;
+      di.seqlen = (int32_t)Li;
+      const int32_t sin = (i > 0 || states_in) ? 1 : 0;
+      if (Li == pl.Lp || pr.batch == 1) {
+        rc = m2::prefill_entry(&di, params, xs, lx, zs, lz, ds, ld, nullptr, yb[s], cs_d, hs_d,
+                               sin, ws_d, pl.ws, cs_);
+      } else {
+        di.batch = 1;
+        for (int64_t bi = 0; bi < pr.batch && rc == MAMBA2_OK; ++bi) {
+          const size_t d0 = (size_t)(bi * pl.Lp);
+          rc = m2::prefill_entry(&di, params, xs + d0 * lx * esz, lx, zs + d0 * lz * esz, lz,
+                                 ds + d0 * ld * esz, ld, nullptr, yb[s] + d0 * pr.d_inner * esz,
+                                 cs_d + (size_t)bi * pr.conv_dim * pr.K * esz,
+                                 hs_d + (size_t)bi * pr.H * pr.P * pr.N, sin, ws_d, pl.ws, cs_);
+        }
+      }
+      if (rc != MAMBA2_OK) break;
+      chk(cudaEventRecord(comp_done[s], cs_));
+      chk(cudaStreamWaitEvent(dnl, comp_done[s], 0));
+      // y rows of the piece: batch row bi of the slot at bi Lp rows
+      chk(cudaMemcpy2DAsync(static_cast<char *>(y) + (size_t)t0 * pr.d_inner * esz,
+                            (size_t)pr.L * pr.d_inner * esz, yb[s],
+                            (size_t)pl.Lp * pr.d_inner * esz, (size_t)Li * pr.d_inner * esz,
+                            pr.batch, cudaMemcpyDeviceToHost, dnl));
+      chk(cudaEventRecord(out_free[s], dnl));
+    }
+    if (rc == MAMBA2_OK && (np > 0 || !states_in)) {  // (no tokens: carried states unchanged)
+      if (conv_state != nullptr)
+        chk(cudaMemcpyAsync(conv_state, cs_d, cs_bytes, cudaMemcpyDeviceToHost, dnl));
+      if (ssm_state != nullptr)
+        chk(cudaMemcpyAsync(ssm_state, hs_d, hs_bytes, cudaMemcpyDeviceToHost, dnl));
+    }
+    // the caller's stream resumes after everything this call enqueued
+    cudaEventRecord(in_ready[0], upl);
+    cudaEventRecord(done, dnl);
+    cudaStreamWaitEvent(cs_, in_ready[0], 0);
+    cudaStreamWaitEvent(cs_, done, 0);
+  } else {
+    rc = MAMBA2_ERR_CUDA;
+  }
+  // released once their work is complete
+  for (int i = 0; i < 8; ++i)
+    if (ev[i] != nullptr) cudaEventDestroy(ev[i]);
+  if (upl != nullptr) cudaStreamDestroy(upl);
+  if (dnl != nullptr) cudaStreamDestroy(dnl);
+  return rc;
 }
 
 MAMBA2_API size_t mamba2_prefill_varlen_workspace_size(const mamba2_dims *dims) {

@@ -272,3 +272,51 @@ def test_backward_rejects_bad_arguments(kw, expect):
 def test_backward_unsupported_configurations():
     for bad in (dict(d_conv=2), dict(dstate=256), dict(headdim=128)):
         assert _call_backward(_dims(batch=2, seqlen=300, **bad)) == UNSUPPORTED, bad
+
+
+def test_host_workspace_size():
+    lib = m2.lib()
+    d = _dims()  # b1 L4096: eight pieces of 512 tokens
+    ws = lib.mamba2_prefill_host_workspace_size(ctypes.byref(d))
+    piece = lib.mamba2_prefill_workspace_size(ctypes.byref(_dims(seqlen=512)))
+    whole = lib.mamba2_prefill_workspace_size(ctypes.byref(d))
+    # one piece's workspace plus two staged pieces each way and the states
+    assert piece < ws < whole
+    assert lib.mamba2_prefill_host_workspace_size(ctypes.byref(_dims(ngroups=3))) == 0
+
+
+def _call_host(d, **kw):
+    lib = m2.lib()
+    cd, di = d.nheads * d.headdim + 2 * d.ngroups * d.dstate, d.nheads * d.headdim
+    args = dict(params=_fake_params(), xBC=A0 + 0x10000, ld_x=cd, z=A0 + 0x20000, ld_z=di,
+                dt=A0 + 0x30000, ld_dt=d.nheads, y=A0 + 0x40000, cs=A0 + 0x50000,
+                hs=A0 + 0x60000, states_in=0, ws=A0 + 0x100000,
+                ws_bytes=lib.mamba2_prefill_host_workspace_size(ctypes.byref(d)) or 1)
+    args.update(kw)
+    p = args["params"]
+    return lib.mamba2_conv_ssd_prefill_host(
+        ctypes.byref(d), ctypes.byref(p) if p is not None else None, args["xBC"], args["ld_x"],
+        args["z"], args["ld_z"], args["dt"], args["ld_dt"], args["y"], args["cs"], args["hs"],
+        args["states_in"], args["ws"], args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(params=None), INVALID),
+    (dict(xBC=None), INVALID),
+    (dict(y=None), INVALID),
+    (dict(ld_z=5), INVALID),                   # row stride below the width
+    (dict(states_in=1, cs=None), INVALID),
+    (dict(states_in=2), INVALID),
+    (dict(ws=None), WORKSPACE),
+    (dict(ws=A0 + 0x100010), WORKSPACE),       # device workspace not 256-byte aligned
+    (dict(ws_bytes=4096), WORKSPACE),
+])
+def test_host_entry_rejects_bad_arguments(kw, expect):
+    # host pointers need no alignment; everything here is rejected before CUDA
+    assert _call_host(_dims(batch=2, seqlen=1000), **kw) == expect
+
+
+def test_host_entry_empty_batch_and_bad_dims():
+    assert _call_host(_dims(batch=0)) == OK
+    assert _call_host(_dims(ngroups=3)) == INVALID
+    assert _call_host(_dims(d_conv=3)) == UNSUPPORTED
