@@ -140,12 +140,17 @@ def load_peaks():
 
 
 def source_hash() -> str:
+    """Hash of the kernel sources: the files that define kernels and the headers
+    they include (the host-only ABI code does not change what a kernel reads or
+    writes, so DRAM counters taken before an edit there still hold)."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "mamba_ssd_scan_mixer_b200", "csrc")
     for f in sorted(os.listdir(d)):
         with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+            text = fh.read()
+        if f.endswith(".cuh") or b"__global__" in text:
+            h.update(f.encode() + text)
     return h.hexdigest()[:16]
 
 

@@ -173,9 +173,11 @@ MAMBA2_API size_t mamba2_prefill_host_workspace_size(const mamba2_dims *dims);
  *          is enqueued: synchronise the stream before reading y or the states.
  * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister): the
  * copies of pageable memory are correct but neither asynchronous nor
- * overlapped.  The call creates two streams and eight events of its own (so it
- * cannot be captured into a CUDA graph) and releases them when their work is
- * done.  Stage events (mamba2_record_stage_events) are not recorded.
+ * overlapped.  The call uses two streams and eight events of its own, made on
+ * a host thread's first call on a device and kept for the thread's lifetime
+ * (so it cannot be captured into a CUDA graph; calls from one thread are
+ * ordered by the caller's stream as usual).  Stage events
+ * (mamba2_record_stage_events) are not recorded.
  * Returns MAMBA2_OK, MAMBA2_ERR_INVALID_ARG (null pointer, stride below a
  * width, states_in without states), MAMBA2_ERR_UNSUPPORTED (as for
  * mamba2_conv_ssd_prefill), MAMBA2_ERR_WORKSPACE or MAMBA2_ERR_CUDA. */

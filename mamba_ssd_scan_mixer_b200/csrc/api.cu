@@ -287,9 +287,10 @@ size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 bool host_plan(const mamba2_dims *dims, const Problem &pr, HostPlan *o) {
   // pieces of whole chunks for every chunk size (multiples of 256 tokens), about
   // an eighth of the sequence each, so that the copies of the first and last
-  // pieces, which nothing overlaps, are short
-  const int64_t eighth = (pr.L + 7) / 8;
-  o->Lp = std::min<int64_t>(std::max<int64_t>((eighth + 255) / 256 * 256, 256),
+  // pieces, which nothing overlaps, are short (sixteenths were measured slower:
+  // the per-piece launches and waits add up)
+  const int64_t part = (pr.L + 7) / 8;
+  o->Lp = std::min<int64_t>(std::max<int64_t>((part + 255) / 256 * 256, 256),
                             std::max<int64_t>(pr.L, 1));
   const size_t esz = pr.io == MAMBA2_BF16 ? 2 : 4;
   o->ldx = (pr.conv_dim + 7) / 8 * 8;
@@ -309,6 +310,50 @@ bool host_plan(const mamba2_dims *dims, const Problem &pr, HostPlan *o) {
   if (make_problem(&dp, true, &pp) != MAMBA2_OK) return false;
   o->ws = up256(prefill_workspace(pp));
   o->total = 2 * o->in + 2 * o->y + o->cs + o->hs + o->ws;
+  return true;
+}
+// The two streams and eight events of the host-buffer prefill, kept per host
+// thread and device for the thread's lifetime; a context that was destroyed and
+// created again gets new ones (the old handles died with it).  Without a
+// context id they are made for the call and released after it (owned).
+struct HostPipe {
+  unsigned long long ctx = 0;
+  cudaStream_t up = nullptr, dn = nullptr;
+  cudaEvent_t ev[8] = {};
+};
+bool make_pipe(HostPipe *p) {
+  *p = HostPipe{};
+  bool ok = cudaStreamCreateWithFlags(&p->up, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p->dn, cudaStreamNonBlocking) == cudaSuccess;
+  for (int i = 0; ok && i < 8; ++i)
+    ok = cudaEventCreateWithFlags(&p->ev[i], cudaEventDisableTiming) == cudaSuccess;
+  return ok;
+}
+void release_pipe(HostPipe *p) {  // once their work is complete
+  for (int i = 0; i < 8; ++i)
+    if (p->ev[i] != nullptr) cudaEventDestroy(p->ev[i]);
+  if (p->up != nullptr) cudaStreamDestroy(p->up);
+  if (p->dn != nullptr) cudaStreamDestroy(p->dn);
+  *p = HostPipe{};
+}
+bool host_pipe(HostPipe *call_owned, HostPipe **out, bool *owned) {
+  thread_local HostPipe pipes[64];
+  int dev = 0;
+  const unsigned long long id = current_context_id();
+  *owned = id == 0 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64;
+  if (*owned) {
+    *out = call_owned;
+    return make_pipe(call_owned);
+  }
+  HostPipe &p = pipes[dev];
+  if (p.ctx != id) {
+    if (!make_pipe(&p)) {
+      release_pipe(&p);
+      return false;
+    }
+    p.ctx = id;
+  }
+  *out = &p;
   return true;
 }
 }  // namespace
@@ -374,12 +419,15 @@ MAMBA2_API int mamba2_conv_ssd_prefill_host(
   // Copies in on one stream, the prefill of each piece on the caller's stream,
   // copies out on a third: piece i + 1 arrives and piece i - 1 leaves while piece
   // i runs.  Two staging slots per direction; every reuse waits for its reader.
-  cudaStream_t upl = nullptr, dnl = nullptr;
-  cudaEvent_t ev[8] = {};  // start, in_ready[2], comp_done[2], out_free[2], done
-  bool ok = cudaStreamCreateWithFlags(&upl, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaStreamCreateWithFlags(&dnl, cudaStreamNonBlocking) == cudaSuccess;
-  for (int i = 0; ok && i < 8; ++i)
-    ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+  m2::HostPipe own, *pipe = nullptr;
+  bool owned = false;
+  const bool ok = m2::host_pipe(&own, &pipe, &owned);
+  if (!ok) {
+    if (owned) m2::release_pipe(&own);
+    return MAMBA2_ERR_CUDA;
+  }
+  cudaStream_t upl = pipe->up, dnl = pipe->dn;
+  cudaEvent_t *ev = pipe->ev;  // start, in_ready[2], comp_done[2], out_free[2], done
   cudaEvent_t start = ev[0], done = ev[7];
   cudaEvent_t *in_ready = ev + 1, *comp_done = ev + 3, *out_free = ev + 5;
   int rc = MAMBA2_OK;
@@ -485,11 +533,7 @@ MAMBA2_API int mamba2_conv_ssd_prefill_host(
   } else {
     rc = MAMBA2_ERR_CUDA;
   }
-  // released once their work is complete
-  for (int i = 0; i < 8; ++i)
-    if (ev[i] != nullptr) cudaEventDestroy(ev[i]);
-  if (upl != nullptr) cudaStreamDestroy(upl);
-  if (dnl != nullptr) cudaStreamDestroy(dnl);
+  if (owned) m2::release_pipe(&own);
   return rc;
 }
 

@@ -38,7 +38,7 @@ def _host(cfg, inp, params, states=None, states_in=False):
     (case("zamba2_2p7b_prefill", batch=2, seqlen=1000, nheads=8, ngroups=2), False),
     # one piece shorter than a chunk; fp32 I/O (CUDA-core path)
     (case("tiny_f32", batch=2, seqlen=37, nheads=4, headdim=16, dstate=16), True),
-    # 3 pieces of 512 over three rows, norm before the gate
+    # 6 pieces of 256 over three rows (the last 20 tokens), norm before the gate
     (case("zamba2_2p7b_prefill", batch=3, seqlen=1300, nheads=4, norm_before_gate=True), True),
 ], ids=lambda c: getattr(c, "name", str(c)))
 def test_host_entry_matches_oracle(cfg, states_in):
