@@ -80,7 +80,7 @@ struct TcArgs {
   // byte ranges of every buffer, for the checked build (see M2_OK)
   struct Spans {
     Span xbc, z, dt, y, conv, ssm, S, cum_end, cum, dtv, Hc, hsc, smax, cbd, u, xpart, xcnt,
-        conv_w, conv_b, dt_bias, A, D, norm_w;
+        conv_w, conv_b, dt_bias, A, D, norm_w, h0max;
   } sp;
   __half *u;                     // [b][L][conv_dim] post-conv x | B | C, fp16
   int hpc;                       // most heads of a head block in tc_chunk_out
@@ -96,6 +96,8 @@ struct TcArgs {
   const int *vl_chunk0;          // [batch + 2] first global chunk of each sequence, the total,
                                  // then 1 if the offsets were valid (0: the call does nothing)
   const int *cu_seqlens;         // [batch + 1] first token of each sequence (last: L)
+  const float *vl_h0max;         // [batch][H] max |initial state| of each (sequence, head) when
+                                 // states_in, else null (the state pass reduces it itself)
 };
 
 // Where global chunk gc lies: its sequence, its index in that sequence, its
@@ -855,13 +857,37 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 // first token}; chunk0[nseq + 1] = 1.  Offsets that fail the check raise
 // kErrSeqlens and leave zero chunks and chunk0[nseq + 1] = 0, so that the
 // kernels after it do nothing.
-constexpr int kPrepThreads = 1024;
+// With carried states, blocks 1 .. nseq H each reduce one (sequence, head)'s
+// initial state to max |h0| (the state pass's first bound B_0), once, instead of
+// every state-pass block of the head reading the whole state again: the packed
+// sequences' many short chains then start without that round trip.
+constexpr int kPrepThreads = 1024;  // = the 4096 floats of a 64 x 64 state, as float4
 __global__ void __launch_bounds__(kPrepThreads)
     tc_varlen_prep_kernel(const int *cu, int nseq, int64_t L, int64_t cap, int4 *chunks,
-                          int *chunk0) {
+                          int *chunk0, const float *ssm, float *h0max, Span ssm_span) {
   __shared__ int bad;
   __shared__ int wsum[kPrepThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (blockIdx.x > 0) {
+    const int64_t pair = blockIdx.x - 1;  // sequence * H + head
+    const float4 *src = reinterpret_cast<const float4 *>(ssm + pair * (int64_t)(kHP * kNS)) + tid;
+    float m = 0.0f;
+    if (M2_OK(src, 16, ssm_span, &g_tc_errors)) {
+      const float4 v = *src;
+      m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ float red[kPrepThreads / 32];
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (tid == 0) {
+      float r = 0.0f;
+      for (int w = 0; w < kPrepThreads / 32; ++w) r = fmaxf(r, red[w]);
+      h0max[pair] = r;
+    }
+    return;
+  }
   if (tid == 0) bad = (cu[0] != 0 || (int64_t)cu[nseq] != L) ? 1 : 0;
   __syncthreads();
   // thread tid takes sequences [s0, s1)
@@ -1006,7 +1032,10 @@ __global__ void __launch_bounds__(kPassThreads, 5) tc_state_pass_kernel(TcArgs a
                   : make_float4(0.f, 0.f, 0.f, 0.f);
   // B_0: max |initial state| over the whole head (each block of the head alike)
   float bnd = 0.0f;
-  if (a.states_in) {
+  if (a.states_in && a.vl_h0max != nullptr) {
+    // (packed sequences: reduced once per (sequence, head) by the prep kernel)
+    bnd = M2_OK(a.vl_h0max + head, 4, a.sp.h0max, &g_tc_errors) ? a.vl_h0max[head] : 0.0f;
+  } else if (a.states_in) {
     const float4 *h0 = reinterpret_cast<const float4 *>(a.ssm_state + head * (int64_t)(kHP * kNS));
     float m = 0.0f;
     for (int i = tid; i < kHP * kNS / 4; i += kPassThreads) {
@@ -1792,6 +1821,7 @@ struct TcWorkspace {
   __half *Hc, *u;
   int4 *vl_chunks;
   int *vl_chunk0;
+  float *vl_h0max;
 };
 
 // Chunks the workspace holds: b * ceil(L / 128), or for packed sequences an
@@ -1824,6 +1854,7 @@ size_t tc_carve(const Problem &pr, bool varlen, char *base, TcWorkspace *w) {
   t.xcnt = reinterpret_cast<unsigned *>(take(cap * pr.G * 4));
   t.vl_chunks = varlen ? reinterpret_cast<int4 *>(take(cap * 16)) : nullptr;
   t.vl_chunk0 = varlen ? reinterpret_cast<int *>(take((size_t)(pr.batch + 2) * 4)) : nullptr;
+  t.vl_h0max = varlen ? reinterpret_cast<float *>(take((size_t)pr.batch * pr.H * 4)) : nullptr;
   const size_t tokens = varlen ? (size_t)pr.L : (size_t)(pr.batch * pr.L);
   t.u = reinterpret_cast<__half *>(take(tokens * pr.conv_dim * 2));
   if (w != nullptr) *w = t;
@@ -1938,6 +1969,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
   a.varlen = varlen ? 1 : 0;
   a.vl_chunks = w.vl_chunks;
   a.vl_chunk0 = w.vl_chunk0;
+  a.vl_h0max = varlen && pa.states_in ? w.vl_h0max : nullptr;
   a.cu_seqlens = pa.cu_seqlens;
   const int64_t cap = tc_chunk_cap(pr, varlen);    // chunks the workspace holds
   const int64_t tokens = varlen ? pr.L : pr.batch * pr.L;
@@ -1979,6 +2011,7 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
     a.sp.A = span_of(a.prm.A, (size_t)pr.H * 4);
     a.sp.D = span_of(a.prm.D, (size_t)pr.H * 4);
     a.sp.norm_w = span_of(a.prm.norm_w, (size_t)pr.d_inner * 4);
+    a.sp.h0max = span_of(a.vl_h0max, (size_t)pr.batch * pr.H * 4);
   }
   const int hpg = pr.heads_per_group();
   cudaError_t e;
@@ -1999,8 +2032,10 @@ cudaError_t prefill_tc(const PrefillArgs &pa) {
 
   stage_mark(st, 0);
   if (varlen) {  // the chunks of the packed sequences
-    tc_varlen_prep_kernel<<<1, kPrepThreads, 0, st>>>(pa.cu_seqlens, (int)pr.batch, pr.L, cap,
-                                                      w.vl_chunks, w.vl_chunk0);
+    const unsigned gp = 1u + (a.vl_h0max != nullptr ? (unsigned)(pr.batch * pr.H) : 0u);
+    tc_varlen_prep_kernel<<<gp, kPrepThreads, 0, st>>>(pa.cu_seqlens, (int)pr.batch, pr.L, cap,
+                                                       w.vl_chunks, w.vl_chunk0, pa.ssm_state,
+                                                       w.vl_h0max, a.sp.ssm);
   }
   const int64_t n_items = cap * (int64_t)pr.G * ((hpg + 1) / 2 + 1);
   const unsigned g1 = (unsigned)std::min<int64_t>(n_items, sm_count());
