@@ -170,6 +170,18 @@ size_t backward_workspace(const Problem &pr);
 // ---------------------------------------------------------------- async copies
 namespace m2 {
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream drains;
+// grid_dependency_wait blocks until that kernel has completed and its memory
+// operations are visible.  launch_dependents lets the next kernel's CTAs be
+// scheduled once every CTA of this one has called it (or exited).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Each translation unit that waits on mbarriers keeps its own error word (a
 // file-scope __device__ variable, so no relocatable device code is needed),
 // passes its address to mbar_wait_bounded, and exposes a host function that

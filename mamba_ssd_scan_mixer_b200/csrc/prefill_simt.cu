@@ -55,6 +55,8 @@ __global__ void conv_silu_kernel(Problem pr, const T *__restrict__ xBC, int64_t 
                                  const T *__restrict__ cs, int states_in,
                                  const float *__restrict__ w, const float *__restrict__ bias,
                                  float *__restrict__ u) {
+  grid_dependency_wait();  // (launched as a dependent of the previous kernel)
+  launch_dependents();
   const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= pr.conv_dim) return;
   const int64_t bi = blockIdx.z, t0 = (int64_t)blockIdx.y * kConvTokens;
@@ -83,6 +85,8 @@ __global__ void conv_silu_kernel(Problem pr, const T *__restrict__ xBC, int64_t 
 template <typename T>
 __global__ void conv_state_out_kernel(Problem pr, const T *__restrict__ xBC, int64_t ld, T *cs,
                                       int states_in) {
+  grid_dependency_wait();  // (launched as a dependent of the previous kernel)
+  launch_dependents();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= pr.batch * pr.conv_dim) return;
   const int64_t bi = i / pr.conv_dim, c = i % pr.conv_dim;
@@ -104,6 +108,8 @@ template <typename T>
 __global__ void dt_cumsum_kernel(Problem pr, const T *__restrict__ dt_raw, int64_t ld,
                                  const float *__restrict__ dt_bias, const float *__restrict__ A,
                                  float *__restrict__ dt_out, float *__restrict__ cum_out) {
+  grid_dependency_wait();  // (launched as a dependent of the previous kernel)
+  launch_dependents();
   __shared__ float warp_tot[32];
   const int h = blockIdx.y;
   const int64_t bi = blockIdx.z, t = (int64_t)blockIdx.x * pr.Q + threadIdx.x;
@@ -134,6 +140,8 @@ __global__ void dt_cumsum_kernel(Problem pr, const T *__restrict__ dt_raw, int64
 __global__ void chunk_state_kernel(Problem pr, const float *__restrict__ u,
                                    const float *__restrict__ dtw, const float *__restrict__ cum,
                                    float *__restrict__ states) {
+  grid_dependency_wait();  // (launched as a dependent of the previous kernel)
+  launch_dependents();
   extern __shared__ float smem[];
   const int P = pr.P, N = pr.N;
   float *xs = smem;                 // [kTileS][P]
@@ -190,6 +198,8 @@ __global__ void chunk_state_kernel(Problem pr, const float *__restrict__ u,
 __global__ void state_pass_kernel(Problem pr, float *__restrict__ states,
                                   const float *__restrict__ cum, float *ssm_state,
                                   int states_in) {
+  grid_dependency_wait();  // (launched as a dependent of the previous kernel)
+  launch_dependents();
   const int nout = pr.P * pr.N;
   const int o = blockIdx.x * blockDim.x + threadIdx.x;
   if (o >= nout) return;
@@ -215,6 +225,8 @@ __global__ void chunk_out_kernel(Problem pr, const float *__restrict__ u,
                                  const float *__restrict__ dtw, const float *__restrict__ cum,
                                  const float *__restrict__ states, const float *__restrict__ Dp,
                                  float *__restrict__ ypre) {
+  grid_dependency_wait();  // (launched as a dependent of the previous kernel)
+  launch_dependents();
   extern __shared__ float smem[];
   const int P = pr.P, N = pr.N, NP = N + 1;
   float *Cs = smem;                   // [kTileT][N+1]
@@ -324,6 +336,8 @@ template <typename T>
 __global__ void gated_norm_kernel(Problem pr, const float *__restrict__ ypre,
                                   const T *__restrict__ z, int64_t ld_z,
                                   const float *__restrict__ w, T *__restrict__ y) {
+  grid_dependency_wait();  // (launched as a dependent of the previous kernel)
+  launch_dependents();
   __shared__ float red[33];
   const int64_t t = blockIdx.x, bi = blockIdx.y;
   const int64_t row = bi * pr.L + t;
@@ -359,6 +373,25 @@ size_t chunk_state_smem(const Problem &pr) {
   return sizeof(float) * (size_t)(kTileS * pr.P + kTileS * pr.N + kTileS);
 }
 
+// Launch of a kernel that may start while the previous one on the stream drains
+// (programmatic dependent launch): each kernel waits for its predecessor before
+// its first memory access, so only the launch latency overlaps.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
+
 template <typename T>
 cudaError_t run(const PrefillArgs &a) {
   const Problem &pr = a.pr;
@@ -372,29 +405,40 @@ cudaError_t run(const PrefillArgs &a) {
   stage_mark(st, 0);
   conv_silu_kernel<T><<<g1, 128, 0, st>>>(pr, xBC, a.ld_xbc, cs, a.states_in, a.prm.conv_w,
                                           a.prm.conv_b, w.u);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   stage_mark(st, 1);
   if (cs != nullptr) {
     const int64_t n = pr.batch * pr.conv_dim;
-    conv_state_out_kernel<T><<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(pr, xBC, a.ld_xbc, cs,
-                                                                        a.states_in);
+    e = launch_dependent(conv_state_out_kernel<T>, dim3((unsigned)ceil_div(n, 256)), dim3(256), 0,
+                         st, pr, xBC, a.ld_xbc, cs, a.states_in);
+    if (e != cudaSuccess) return e;
   }
   dim3 g2((unsigned)pr.nchunks, pr.H, (unsigned)pr.batch);
   stage_mark(st, 2);
-  dt_cumsum_kernel<T><<<g2, pr.Q, 0, st>>>(pr, static_cast<const T *>(a.dt_raw), a.ld_dt,
-                                           a.prm.dt_bias, a.prm.A, w.dt, w.cum);
+  e = launch_dependent(dt_cumsum_kernel<T>, g2, dim3(pr.Q), 0, st, pr,
+                       static_cast<const T *>(a.dt_raw), a.ld_dt, a.prm.dt_bias, a.prm.A, w.dt,
+                       w.cum);
+  if (e != cudaSuccess) return e;
   stage_mark(st, 3);
-  chunk_state_kernel<<<g2, 256, chunk_state_smem(pr), st>>>(pr, w.u, w.dt, w.cum, w.states);
+  e = launch_dependent(chunk_state_kernel, g2, dim3(256), chunk_state_smem(pr), st, pr, w.u, w.dt,
+                       w.cum, w.states);
+  if (e != cudaSuccess) return e;
   dim3 g3((unsigned)ceil_div(pr.P * pr.N, 256), pr.H, (unsigned)pr.batch);
   stage_mark(st, 4);
-  state_pass_kernel<<<g3, 256, 0, st>>>(pr, w.states, w.cum, a.ssm_state, a.states_in);
+  e = launch_dependent(state_pass_kernel, g3, dim3(256), 0, st, pr, w.states, w.cum, a.ssm_state,
+                       a.states_in);
+  if (e != cudaSuccess) return e;
   dim3 g4((unsigned)ceil_div(pr.L, kTileT), pr.H, (unsigned)pr.batch);
   stage_mark(st, 5);
-  chunk_out_kernel<<<g4, 256, chunk_out_smem(pr), st>>>(pr, w.u, w.dt, w.cum, w.states, a.prm.D,
-                                                        w.ypre);
+  e = launch_dependent(chunk_out_kernel, g4, dim3(256), chunk_out_smem(pr), st, pr, w.u, w.dt,
+                       w.cum, w.states, a.prm.D, w.ypre);
+  if (e != cudaSuccess) return e;
   dim3 g5((unsigned)pr.L, (unsigned)pr.batch);
   stage_mark(st, 6);
-  gated_norm_kernel<T><<<g5, 256, 0, st>>>(pr, w.ypre, static_cast<const T *>(a.z), a.ld_z,
-                                           a.prm.norm_w, static_cast<T *>(a.y));
+  e = launch_dependent(gated_norm_kernel<T>, g5, dim3(256), 0, st, pr, w.ypre,
+                       static_cast<const T *>(a.z), a.ld_z, a.prm.norm_w, static_cast<T *>(a.y));
+  if (e != cudaSuccess) return e;
   stage_mark(st, 7);
   return cudaGetLastError();
 }

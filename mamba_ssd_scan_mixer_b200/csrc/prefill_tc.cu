@@ -224,17 +224,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
-// Programmatic dependent launch: a kernel launched with programmatic stream
-// serialization may start while the previous kernel of the stream drains;
-// grid_dependency_wait blocks until that kernel has completed and its memory
-// operations are visible.  launch_dependents lets the next kernel's CTAs be
-// scheduled once every CTA of this one has called it (or exited).
-__device__ __forceinline__ void grid_dependency_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 // Smem descriptor for an MN-major SW128 operand: 8-row (K) atoms of 64
 // elements (N) x 128 B, K atoms 1024 B apart (SBO), N atoms `lbo` apart.
 __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
